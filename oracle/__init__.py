@@ -1,0 +1,232 @@
+"""CPU oracle of the MSA forward pass -- TEST INFRASTRUCTURE ONLY.
+
+Only the tests, the smoke check and the benchmark's CPU-baseline leg may
+import this package.  The product path (the CUDA library and its binding)
+never loads it, and this package never loads the CUDA library.
+
+The arithmetic lives in ``msa_oracle.c`` (plain C, fp64 sums, OpenMP threads
+over rows), compiled here with gcc on first use.  Each function cites the
+equation of the MSA pages it follows (xllm-io review, "核心公式" section:
+Eq. 1, 4, 6, 7, 8, 12; chlience notes, section 5.1.1).  Arrays of bf16 values
+are numpy ``uint16`` bit patterns.
+
+Pins (tests/test_oracle_pins.py): planted block maxima with a hand-derived
+selection, brute-force subset enumeration, numpy stable argsort, rescale
+invariance, dense equivalence with torch's scaled_dot_product_attention,
+block-diagonal causal attention for k = 1, softmax weights summing to one,
+the LSE split/merge identity and the Eq. 12 closed form (28.4x at 1M).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+from typing import Optional, Tuple
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "msa_oracle.c")
+_HDR = os.path.join(_HERE, "msa_oracle.h")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile msa_oracle.c into liboracle.so (gcc, -O2, no fast-math)."""
+    newest = max(os.path.getmtime(_SRC), os.path.getmtime(_HDR))
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < newest:
+        tmp = _LIB + f".{os.getpid()}.tmp"
+        cmd = ["gcc", "-std=c11", "-O2", "-fno-fast-math", "-ffp-contract=off", "-fopenmp",
+               "-fPIC", "-shared", "-Wall", "-Wextra", "-o", tmp, _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            P = ctypes.c_void_p
+            I64, I32, D = ctypes.c_int64, ctypes.c_int, ctypes.c_double
+            lib.oracle_max_threads.restype = I32
+            lib.oracle_block_scores.argtypes = [P, P, I64, I32, I32, I64, P]
+            lib.oracle_index_topk.argtypes = [P, P, I64, I32, I32, I32, I32, P, I64, P, P, P, I32]
+            lib.oracle_sparse_attn.argtypes = [P, P, P, P, I64, I32, I32, I32, I32, I32, D, P, I64,
+                                               P, P, I32]
+            lib.oracle_dense_attn.argtypes = [P, P, P, I64, I32, I32, I32, D, P, I64, P, P, I32]
+            lib.oracle_flops.argtypes = [D] * 7 + [P, P, P]
+            for f in ("oracle_block_scores", "oracle_index_topk", "oracle_sparse_attn",
+                      "oracle_dense_attn"):
+                getattr(lib, f).restype = I32
+            lib.oracle_flops.restype = None
+            _lib = lib
+    return _lib
+
+
+def _c(a: np.ndarray, dtype) -> np.ndarray:
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def _p(a: Optional[np.ndarray]):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _check(rc: int, what: str) -> None:
+    if rc != 0:
+        raise ValueError(f"oracle {what} rejected its arguments (code {rc})")
+
+
+def max_threads() -> int:
+    return int(_load().oracle_max_threads())
+
+
+def block_scores(q_idx_row: np.ndarray, k_idx: np.ndarray, B_k: int, i: int) -> np.ndarray:
+    """Eq. 6: M[b] for b = 0..i//B_k of one index-query row (float64)."""
+    q = _c(q_idx_row, np.uint16).reshape(-1)
+    kk = _c(k_idx, np.uint16)
+    out = np.empty(i // B_k + 1, dtype=np.float64)
+    _check(_load().oracle_block_scores(_p(q), _p(kk), kk.shape[0], q.size, B_k, i, _p(out)),
+           "block_scores")
+    return out
+
+
+def index_topk(q_idx: np.ndarray, k_idx: np.ndarray, B_k: int, k: int,
+               rows: Optional[np.ndarray] = None, threads: int = 0
+               ) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """Eq. 6-7 for ``rows`` (default: all).  q_idx [N,H_kv,d_idx], k_idx [N,d_idx].
+
+    Returns idx [n,H_kv,k] int32 (ascending, -1 padded), cut and next [n,H_kv]
+    float64 (tie-band bounds).
+    """
+    kk = _c(k_idx, np.uint16)
+    N, d_idx = kk.shape
+    H_kv = q_idx.shape[1]
+    rows = np.arange(N, dtype=np.int64) if rows is None else _c(rows, np.int64)
+    qr = _c(np.asarray(q_idx)[rows], np.uint16)
+    idx = np.empty((rows.size, H_kv, k), dtype=np.int32)
+    cut = np.empty((rows.size, H_kv), dtype=np.float64)
+    nxt = np.empty((rows.size, H_kv), dtype=np.float64)
+    _check(_load().oracle_index_topk(_p(qr), _p(kk), N, H_kv, d_idx, B_k, k, _p(rows), rows.size,
+                                     _p(idx), _p(cut), _p(nxt), threads), "index_topk")
+    return idx, cut, nxt
+
+
+def index_topk_rows(q_idx_rows: np.ndarray, k_idx: np.ndarray, N: int, B_k: int, k: int,
+                    rows: np.ndarray, threads: int = 0
+                    ) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """As ``index_topk`` but with the index queries of the rows given directly
+    (q_idx_rows [n,H_kv,d_idx]) and the first N rows of k_idx as the keys."""
+    kk = _c(k_idx, np.uint16)
+    d_idx = kk.shape[1]
+    rows = _c(rows, np.int64)
+    qr = _c(q_idx_rows, np.uint16)
+    H_kv = qr.shape[1]
+    idx = np.empty((rows.size, H_kv, k), dtype=np.int32)
+    cut = np.empty((rows.size, H_kv), dtype=np.float64)
+    nxt = np.empty((rows.size, H_kv), dtype=np.float64)
+    _check(_load().oracle_index_topk(_p(qr), _p(kk), N, H_kv, d_idx, B_k, k, _p(rows), rows.size,
+                                     _p(idx), _p(cut), _p(nxt), threads), "index_topk")
+    return idx, cut, nxt
+
+
+def sparse_attn(q_rows: np.ndarray, k: np.ndarray, v: np.ndarray, idx_rows: np.ndarray,
+                B_k: int, rows: np.ndarray, N: Optional[int] = None,
+                scale: Optional[float] = None, threads: int = 0
+                ) -> Tuple[np.ndarray, np.ndarray]:
+    """Eq. 8 for the listed rows.  q_rows [n,H_q,d_h] (the rows' queries),
+    k/v [>=N,H_kv,d_h], idx_rows [n,H_kv,kk].  Returns O [n,H_q,d_h] and
+    LSE [n,H_q] (float64, natural log)."""
+    qr = _c(q_rows, np.uint16)
+    kk_ = _c(k, np.uint16)
+    vv = _c(v, np.uint16)
+    ir = _c(idx_rows, np.int32)
+    rows = _c(rows, np.int64)
+    n, H_q, d_h = qr.shape
+    H_kv = kk_.shape[1]
+    N = kk_.shape[0] if N is None else N
+    scale = 1.0 / np.sqrt(d_h) if scale is None else scale
+    o = np.empty((n, H_q, d_h), dtype=np.float64)
+    lse = np.empty((n, H_q), dtype=np.float64)
+    _check(_load().oracle_sparse_attn(_p(qr), _p(kk_), _p(vv), _p(ir), N, H_q, H_kv, d_h, B_k,
+                                      ir.shape[2], float(scale), _p(rows), n, _p(o), _p(lse),
+                                      threads), "sparse_attn")
+    return o, lse
+
+
+def dense_attn(q_rows: np.ndarray, k: np.ndarray, v: np.ndarray, rows: np.ndarray,
+               N: Optional[int] = None, scale: Optional[float] = None, threads: int = 0
+               ) -> Tuple[np.ndarray, np.ndarray]:
+    """Eq. 1 dense causal GQA for the listed rows (same layouts as sparse_attn)."""
+    qr = _c(q_rows, np.uint16)
+    kk_ = _c(k, np.uint16)
+    vv = _c(v, np.uint16)
+    rows = _c(rows, np.int64)
+    n, H_q, d_h = qr.shape
+    H_kv = kk_.shape[1]
+    N = kk_.shape[0] if N is None else N
+    scale = 1.0 / np.sqrt(d_h) if scale is None else scale
+    o = np.empty((n, H_q, d_h), dtype=np.float64)
+    lse = np.empty((n, H_q), dtype=np.float64)
+    _check(_load().oracle_dense_attn(_p(qr), _p(kk_), _p(vv), N, H_q, H_kv, d_h, float(scale),
+                                     _p(rows), n, _p(o), _p(lse), threads), "dense_attn")
+    return o, lse
+
+
+def forward(inp: dict, B_k: int, k: int, rows: Optional[np.ndarray] = None,
+            idx_rows: Optional[np.ndarray] = None, threads: int = 0) -> dict:
+    """Whole forward pass (Eq. 6-8) for ``rows``: selection, then attention.
+
+    If ``idx_rows`` is given it replaces the oracle's own selection in the
+    attention step (so a selection made elsewhere can be checked on its own).
+    """
+    N = inp["k_idx"].shape[0]
+    rows = np.arange(N, dtype=np.int64) if rows is None else np.asarray(rows, dtype=np.int64)
+    idx, cut, nxt = index_topk(inp["q_idx"], inp["k_idx"], B_k, k, rows, threads)
+    use = idx if idx_rows is None else idx_rows
+    o, lse = sparse_attn(inp["q"][rows], inp["k"], inp["v"], use, B_k, rows, N=N,
+                         threads=threads)
+    return {"idx": idx, "cut": cut, "next": nxt, "o": o, "lse": lse, "rows": rows}
+
+
+def decode_reference(state: dict, step_in: dict, B_k: int, k: int, seqs=None,
+                     idx_rows: Optional[np.ndarray] = None, threads: int = 0) -> dict:
+    """One decode step for the listed sequences, on host copies of the caches.
+
+    Appends the new rows at position L_s (the query attends to itself, Eq. 1's
+    i <= t), then runs Eq. 6-8 for the single query at i = L_s (new length
+    L_s + 1).  The caches in ``state`` are not modified.
+    """
+    S = state["seq_len"].shape[0]
+    seqs = range(S) if seqs is None else seqs
+    outs = {"idx": [], "cut": [], "next": [], "o": [], "lse": []}
+    for n, s in enumerate(seqs):
+        L = int(state["seq_len"][s])
+        kc = state["k_cache"][s, : L + 1].copy()
+        vc = state["v_cache"][s, : L + 1].copy()
+        kic = state["k_idx_cache"][s, : L + 1].copy()
+        kc[L] = step_in["k_new"][s]
+        vc[L] = step_in["v_new"][s]
+        kic[L] = step_in["k_idx_new"][s]
+        row = np.array([L], dtype=np.int64)
+        idx, cut, nxt = index_topk_rows(step_in["q_idx"][s][None], kic, L + 1, B_k, k, row,
+                                        threads)
+        use = idx if idx_rows is None else idx_rows[n][None]
+        o, lse = sparse_attn(step_in["q"][s][None], kc, vc, use, B_k, row, N=L + 1,
+                             threads=threads)
+        for key, val in (("idx", idx), ("cut", cut), ("next", nxt), ("o", o), ("lse", lse)):
+            outs[key].append(val[0])
+    return {key: np.stack(val) for key, val in outs.items()}
+
+
+def flops(N: float, H_q: int, H_kv: int, d_h: int, d_idx: int, B_k: int, k: int) -> dict:
+    """Eq. 12: F_GQA, F_MSA index term, F_MSA main term (FLOPs)."""
+    g, fi, fm = ctypes.c_double(), ctypes.c_double(), ctypes.c_double()
+    _load().oracle_flops(float(N), H_q, H_kv, d_h, d_idx, B_k, k, ctypes.byref(g),
+                         ctypes.byref(fi), ctypes.byref(fm))
+    return {"gqa": g.value, "index": fi.value, "main": fm.value,
+            "msa": fi.value + fm.value, "ratio": g.value / (fi.value + fm.value)}

@@ -1,0 +1,361 @@
+/*
+ * msa_oracle.c -- plain CPU oracle for the MiniMax Sparse Attention (MSA)
+ * forward pass.  TEST INFRASTRUCTURE ONLY: nothing on the product path may
+ * link, load or call this file; only the tests, the smoke check and the
+ * benchmark's CPU-baseline leg do.
+ *
+ * Sources (web pages about arXiv:2606.13392, "MiniMax Sparse Attention"):
+ *   [xllm]  xllm-io paper review, section "核心公式": Eq. 1 (causal GQA),
+ *           Eq. 4 (block partition), Eq. 6 (index score + block max-pool),
+ *           Eq. 7 (Top-k, local block always kept), Eq. 8 (main branch).
+ *   [chl]   chlience paper-archive notes, section 5.1 and its sub-section
+ *           5.1.1 (the four selection steps: token scoring, block max
+ *           pooling, local block reservation, remaining Top-k).
+ *
+ * Arithmetic: bf16 inputs are widened exactly to double and every sum is a
+ * plain left-to-right loop in double (fp64).  The only float32 step is the
+ * Top-k decision itself: a block's max-pooled score M (Eq. 6) is rounded to
+ * float32 before ranking, because the GPU kernel ranks in float32 and an
+ * integer result decided by floating point must be decided in the same
+ * precision on both sides.  Ties in that float32 value go to the lower
+ * block index.
+ *
+ * Indexing is 0-based throughout: block b holds tokens
+ * [b*B_k, min((b+1)*B_k, N)); query i lives in block b_i = i / B_k.
+ *
+ * Threads: one OpenMP thread per core, each owning whole (row, group)
+ * problems; no blocking or reordering of any sum.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#include "msa_oracle.h"
+
+/* bf16 -> double: bf16 is the top half of an IEEE float32, so the widening
+ * is exact. */
+static double bf(uint16_t h)
+{
+    uint32_t u = ((uint32_t)h) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+static void set_threads(int n_threads)
+{
+#ifdef _OPENMP
+    if (n_threads > 0) omp_set_num_threads(n_threads);
+#else
+    (void)n_threads;
+#endif
+}
+
+int oracle_max_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/* ------------------------------------------------------------------ */
+/* Index Branch: Eq. 6 (token score and causal block max-pool).        */
+/* ------------------------------------------------------------------ */
+
+/*
+ * Block scores of one (query, group) row, Eq. 6 [xllm]; step 1 and 2 of
+ * [chl] 5.1.1:
+ *   S[j] = <q_idx, K_idx[j]> / sqrt(d_idx)          for every key j <= i
+ *   M[b] = max_{j in block b, j <= i} S[j]           for b = 0 .. b_i
+ * Blocks after b_i see no token and are -inf; they are not written.
+ * q_row points at the d_idx values of this row's index query.
+ */
+static void block_scores_row(const uint16_t *q_row, const uint16_t *k_idx,
+                             int64_t i, int d_idx, int B_k, double *M)
+{
+    const double scale = 1.0 / sqrt((double)d_idx);
+    const int64_t b_i = i / B_k;
+    for (int64_t b = 0; b <= b_i; ++b) M[b] = -INFINITY;
+    for (int64_t j = 0; j <= i; ++j) {
+        const uint16_t *kr = k_idx + j * (int64_t)d_idx;
+        double dot = 0.0;
+        for (int d = 0; d < d_idx; ++d) dot += bf(q_row[d]) * bf(kr[d]);
+        const double s = dot * scale;
+        const int64_t b = j / B_k;
+        if (s > M[b]) M[b] = s;
+    }
+}
+
+int oracle_block_scores(const uint16_t *q_idx_row, const uint16_t *k_idx,
+                        int64_t N, int d_idx, int B_k, int64_t i, double *M_out)
+{
+    if (!q_idx_row || !k_idx || !M_out || i < 0 || i >= N || d_idx <= 0 || B_k <= 0)
+        return -1;
+    block_scores_row(q_idx_row, k_idx, i, d_idx, B_k, M_out);
+    return 0;
+}
+
+typedef struct {
+    float m32; /* the decision value: M rounded to float32 */
+    int64_t b;
+} cand_t;
+
+/* Order used by Eq. 7's TopK: higher score first, equal scores -> lower
+ * block index first. */
+static int cand_cmp(const void *pa, const void *pb)
+{
+    const cand_t *a = (const cand_t *)pa, *c = (const cand_t *)pb;
+    if (a->m32 > c->m32) return -1;
+    if (a->m32 < c->m32) return 1;
+    return (a->b < c->b) ? -1 : (a->b > c->b) ? 1 : 0;
+}
+
+static int int_cmp(const void *pa, const void *pb)
+{
+    const int32_t a = *(const int32_t *)pa, c = *(const int32_t *)pb;
+    return (a > c) - (a < c);
+}
+
+/*
+ * Eq. 7 [xllm] with steps 3 and 4 of [chl] 5.1.1 for one row:
+ *   the local block b_i is reserved and takes one of the k slots; the other
+ *   k-1 slots go to the best of the visible non-local blocks 0 .. b_i-1.
+ *   Fewer visible blocks than k: all of them, remaining slots = -1.
+ *   Output ascending by block index.
+ * cut  = M (double) of the worst selected non-local block (NaN if none),
+ * next = M (double) of the best visible non-local block left out (NaN if
+ *        none); together they bound the tie band a comparison may allow.
+ */
+static void select_row(const double *M, int64_t b_i, int k, cand_t *scratch,
+                       int32_t *out, double *cut, double *next)
+{
+    int n = 0;
+    for (int64_t b = 0; b < b_i; ++b) {
+        scratch[n].m32 = (float)M[b];
+        scratch[n].b = b;
+        ++n;
+    }
+    qsort(scratch, (size_t)n, sizeof(cand_t), cand_cmp);
+    const int take = (n < k - 1) ? n : k - 1;
+    int w = 0;
+    out[w++] = (int32_t)b_i;
+    for (int t = 0; t < take; ++t) out[w++] = (int32_t)scratch[t].b;
+    qsort(out, (size_t)w, sizeof(int32_t), int_cmp);
+    for (; w < k; ++w) out[w] = -1;
+    *cut = take > 0 ? M[scratch[take - 1].b] : NAN;
+    *next = take < n ? M[scratch[take].b] : NAN;
+}
+
+int oracle_index_topk(const uint16_t *q_idx_rows, const uint16_t *k_idx,
+                      int64_t N, int H_kv, int d_idx, int B_k, int k,
+                      const int64_t *rows, int64_t n_rows,
+                      int32_t *idx_out, double *cut_out, double *next_out,
+                      int n_threads)
+{
+    if (!q_idx_rows || !k_idx || !rows || !idx_out || N <= 0 || H_kv <= 0 ||
+        d_idx <= 0 || B_k <= 0 || k <= 0 || n_rows < 0)
+        return -1;
+    for (int64_t t = 0; t < n_rows; ++t)
+        if (rows[t] < 0 || rows[t] >= N) return -2;
+    const int64_t B = (N + B_k - 1) / B_k;
+    set_threads(n_threads);
+    int err = 0;
+#pragma omp parallel
+    {
+        double *M = (double *)malloc(sizeof(double) * (size_t)B);
+        cand_t *scratch = (cand_t *)malloc(sizeof(cand_t) * (size_t)B);
+        if (!M || !scratch) {
+#pragma omp atomic write
+            err = -3;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int64_t p = 0; p < n_rows * H_kv; ++p) {
+                const int64_t t = p / H_kv;
+                const int r = (int)(p % H_kv);
+                const int64_t i = rows[t];
+                const uint16_t *q_row = q_idx_rows + (t * H_kv + r) * (int64_t)d_idx;
+                block_scores_row(q_row, k_idx, i, d_idx, B_k, M);
+                double cut, next;
+                select_row(M, i / B_k, k, scratch, idx_out + p * k, &cut, &next);
+                if (cut_out) cut_out[p] = cut;
+                if (next_out) next_out[p] = next;
+            }
+        }
+        free(M);
+        free(scratch);
+    }
+    return err;
+}
+
+/* ------------------------------------------------------------------ */
+/* Main Branch: Eq. 8 over the selected blocks, Eq. 1 dense.           */
+/* ------------------------------------------------------------------ */
+
+/*
+ * Softmax attention of one query head over an explicit key list (Eq. 1 /
+ * Eq. 8): two passes, plain sums in double.
+ *   s_j  = <q, k_j> / sqrt(d_h)
+ *   m    = max_j s_j,  l = sum_j exp(s_j - m)
+ *   o    = sum_j exp(s_j - m) v_j / l,   lse = m + log l   (natural log)
+ * keys[] lists token positions; kv_stride is the distance between two
+ * tokens' rows of the same KV head.
+ */
+static void attend(const uint16_t *q, const uint16_t *K, const uint16_t *V,
+                   const int64_t *keys, int64_t n_keys, int64_t kv_stride,
+                   int d_h, double scale, double *s, double *o, double *lse)
+{
+    double m = -INFINITY;
+    for (int64_t t = 0; t < n_keys; ++t) {
+        const uint16_t *kr = K + keys[t] * kv_stride;
+        double dot = 0.0;
+        for (int d = 0; d < d_h; ++d) dot += bf(q[d]) * bf(kr[d]);
+        s[t] = dot * scale;
+        if (s[t] > m) m = s[t];
+    }
+    double l = 0.0;
+    for (int d = 0; d < d_h; ++d) o[d] = 0.0;
+    for (int64_t t = 0; t < n_keys; ++t) {
+        const double p = exp(s[t] - m);
+        l += p;
+        const uint16_t *vr = V + keys[t] * kv_stride;
+        for (int d = 0; d < d_h; ++d) o[d] += p * bf(vr[d]);
+    }
+    for (int d = 0; d < d_h; ++d) o[d] /= l;
+    *lse = m + log(l);
+}
+
+/*
+ * Eq. 8 [xllm], [chl] 5.1: for each requested query row i and head h
+ * (group r = h / G, adjacent heads share one KV head, Eq. 1 note) attend to
+ * the tokens of the blocks in idx[row, r, :] (entries < 0 are empty slots),
+ * keeping only tokens j <= i (the causal rule of Eq. 1/2 inside the local
+ * block).  q_rows: [n_rows, H_q, d_h]; K, V: [N, H_kv, d_h];
+ * idx: [n_rows, H_kv, k]; o_out: [n_rows, H_q, d_h]; lse_out: [n_rows, H_q].
+ */
+int oracle_sparse_attn(const uint16_t *q_rows, const uint16_t *K, const uint16_t *V,
+                       const int32_t *idx, int64_t N, int H_q, int H_kv, int d_h,
+                       int B_k, int k, double scale, const int64_t *rows,
+                       int64_t n_rows, double *o_out, double *lse_out, int n_threads)
+{
+    if (!q_rows || !K || !V || !idx || !rows || !o_out || N <= 0 || H_q <= 0 ||
+        H_kv <= 0 || H_q % H_kv != 0 || d_h <= 0 || B_k <= 0 || k <= 0 || n_rows < 0)
+        return -1;
+    const int G = H_q / H_kv;
+    const int64_t B = (N + B_k - 1) / B_k;
+    for (int64_t t = 0; t < n_rows; ++t) {
+        if (rows[t] < 0 || rows[t] >= N) return -2;
+        for (int r = 0; r < H_kv; ++r)
+            for (int s = 0; s < k; ++s) {
+                const int32_t b = idx[(t * H_kv + r) * k + s];
+                if (b >= B || b < -1) return -4;
+            }
+    }
+    const int64_t kv_stride = (int64_t)H_kv * d_h;
+    set_threads(n_threads);
+    int err = 0;
+#pragma omp parallel
+    {
+        const int64_t cap = (int64_t)k * B_k;
+        int64_t *keys = (int64_t *)malloc(sizeof(int64_t) * (size_t)cap);
+        double *s = (double *)malloc(sizeof(double) * (size_t)cap);
+        if (!keys || !s) {
+#pragma omp atomic write
+            err = -3;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int64_t p = 0; p < n_rows * H_q; ++p) {
+                const int64_t t = p / H_q;
+                const int h = (int)(p % H_q);
+                const int r = h / G;
+                const int64_t i = rows[t];
+                int64_t n = 0;
+                for (int sl = 0; sl < k; ++sl) {
+                    const int32_t b = idx[(t * H_kv + r) * k + sl];
+                    if (b < 0) continue;
+                    const int64_t j0 = (int64_t)b * B_k;
+                    int64_t j1 = j0 + B_k;
+                    if (j1 > N) j1 = N;
+                    for (int64_t j = j0; j < j1 && j <= i; ++j) keys[n++] = j;
+                }
+                double lse = NAN;
+                double *o = o_out + p * d_h;
+                if (n > 0) {
+                    attend(q_rows + p * d_h, K + (int64_t)r * d_h, V + (int64_t)r * d_h,
+                           keys, n, kv_stride, d_h, scale, s, o, &lse);
+                } else {
+                    for (int d = 0; d < d_h; ++d) o[d] = NAN;
+                }
+                if (lse_out) lse_out[p] = lse;
+            }
+        }
+        free(keys);
+        free(s);
+    }
+    return err;
+}
+
+/*
+ * Eq. 1 [xllm]: dense causal GQA attention, every token j <= i.  Written
+ * separately from the sparse path so the special case "every visible block
+ * selected" can be checked against it.
+ */
+int oracle_dense_attn(const uint16_t *q_rows, const uint16_t *K, const uint16_t *V,
+                      int64_t N, int H_q, int H_kv, int d_h, double scale,
+                      const int64_t *rows, int64_t n_rows, double *o_out,
+                      double *lse_out, int n_threads)
+{
+    if (!q_rows || !K || !V || !rows || !o_out || N <= 0 || H_q <= 0 || H_kv <= 0 ||
+        H_q % H_kv != 0 || d_h <= 0 || n_rows < 0)
+        return -1;
+    for (int64_t t = 0; t < n_rows; ++t)
+        if (rows[t] < 0 || rows[t] >= N) return -2;
+    const int G = H_q / H_kv;
+    const int64_t kv_stride = (int64_t)H_kv * d_h;
+    set_threads(n_threads);
+    int err = 0;
+#pragma omp parallel
+    {
+        int64_t *keys = (int64_t *)malloc(sizeof(int64_t) * (size_t)N);
+        double *s = (double *)malloc(sizeof(double) * (size_t)N);
+        if (!keys || !s) {
+#pragma omp atomic write
+            err = -3;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int64_t p = 0; p < n_rows * H_q; ++p) {
+                const int64_t t = p / H_q;
+                const int h = (int)(p % H_q);
+                const int r = h / G;
+                const int64_t i = rows[t];
+                for (int64_t j = 0; j <= i; ++j) keys[j] = j;
+                double lse;
+                attend(q_rows + p * d_h, K + (int64_t)r * d_h, V + (int64_t)r * d_h,
+                       keys, i + 1, kv_stride, d_h, scale, s, o_out + p * d_h, &lse);
+                if (lse_out) lse_out[p] = lse;
+            }
+        }
+        free(keys);
+        free(s);
+    }
+    return err;
+}
+
+/* ------------------------------------------------------------------ */
+/* Eq. 12: FLOP model.                                                 */
+/* ------------------------------------------------------------------ */
+
+/* F_GQA(N) = 2 H_q d_h N^2;  F_MSA(N) = H_kv d_idx N^2 + 4 H_q d_h N k B_k
+ * ([xllm] Eq. 12; [chl] 5.3). */
+void oracle_flops(double N, double H_q, double H_kv, double d_h, double d_idx,
+                  double B_k, double k, double *f_gqa, double *f_index, double *f_main)
+{
+    if (f_gqa) *f_gqa = 2.0 * H_q * d_h * N * N;
+    if (f_index) *f_index = H_kv * d_idx * N * N;
+    if (f_main) *f_main = 4.0 * H_q * d_h * N * k * B_k;
+}

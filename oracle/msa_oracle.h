@@ -1,0 +1,53 @@
+/*
+ * msa_oracle.h -- plain CPU oracle of the MSA forward pass (test
+ * infrastructure only; see msa_oracle.c for the equations each function
+ * follows).  bf16 arrays are passed as their raw 16-bit patterns.
+ * Every function returns 0 on success and a negative code on bad arguments.
+ */
+#ifndef MSA_ORACLE_H
+#define MSA_ORACLE_H
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+int oracle_max_threads(void);
+
+/* Eq. 6 block scores (double) of query i against blocks 0..i/B_k.
+ * q_idx_row: [d_idx]; k_idx: [N, d_idx]; M_out: [i/B_k + 1]. */
+int oracle_block_scores(const uint16_t *q_idx_row, const uint16_t *k_idx,
+                        int64_t N, int d_idx, int B_k, int64_t i, double *M_out);
+
+/* Eq. 6-7 for the listed query rows.
+ * q_idx_rows: [n_rows, H_kv, d_idx] (the index queries of those rows);
+ * k_idx: [N, d_idx]; idx_out: [n_rows, H_kv, k], ascending, -1 padded;
+ * cut_out / next_out: [n_rows, H_kv] or NULL (tie-band bounds, NaN if none). */
+int oracle_index_topk(const uint16_t *q_idx_rows, const uint16_t *k_idx,
+                      int64_t N, int H_kv, int d_idx, int B_k, int k,
+                      const int64_t *rows, int64_t n_rows,
+                      int32_t *idx_out, double *cut_out, double *next_out,
+                      int n_threads);
+
+/* Eq. 8 for the listed rows with the given selection.
+ * q_rows: [n_rows, H_q, d_h]; K, V: [N, H_kv, d_h]; idx: [n_rows, H_kv, k];
+ * o_out: [n_rows, H_q, d_h]; lse_out: [n_rows, H_q] or NULL. */
+int oracle_sparse_attn(const uint16_t *q_rows, const uint16_t *K, const uint16_t *V,
+                       const int32_t *idx, int64_t N, int H_q, int H_kv, int d_h,
+                       int B_k, int k, double scale, const int64_t *rows,
+                       int64_t n_rows, double *o_out, double *lse_out, int n_threads);
+
+/* Eq. 1 dense causal GQA for the listed rows (same layouts, no idx). */
+int oracle_dense_attn(const uint16_t *q_rows, const uint16_t *K, const uint16_t *V,
+                      int64_t N, int H_q, int H_kv, int d_h, double scale,
+                      const int64_t *rows, int64_t n_rows, double *o_out,
+                      double *lse_out, int n_threads);
+
+/* Eq. 12 FLOP model. */
+void oracle_flops(double N, double H_q, double H_kv, double d_h, double d_idx,
+                  double B_k, double k, double *f_gqa, double *f_index, double *f_main);
+
+#ifdef __cplusplus
+}
+#endif
+#endif
