@@ -1,0 +1,348 @@
+"""Benchmark of the MSA forward hot path on B200.
+
+One step = the whole prefill forward (Index Branch kernel + inverse index +
+KV-outer attention + merge) over one 131072-token sequence shaped like the
+pages' setting (H_q=32, H_kv=4, d_h=128, d_idx=64, B_k=128, k=16; seeded
+synthetic inputs with a sink block and retrieval blocks).  Inputs (Q alone is
+1.07 GB) are larger than the 126 MB L2, so no flush is needed between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl msa|reference]
+                    [--workload 128k|32k|1m|decode]
+
+For N > 1 each rank runs an independent replica (its own sequence): the path
+has no exchange step, so there is no collective on the data path; timing is
+the max over ranks and ``value`` is the tokens of all ranks per second.
+``--impl reference`` times the CPU oracle on a bounded row sample instead.
+Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return PEAKS_FALLBACK, "fallback"
+
+
+def dist_init():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+class Clocks:
+    """nvidia-smi sampling during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                p = [x.strip() for x in line.split(",")]
+                if len(p) >= 9:
+                    rows.append(p)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[j] for r in rows for j in range(4) if r[5 + j].lower() == "active"})
+        hi = [x for x in sm if mx and x > 0.5 * max(mx)] or sm
+        return {"sm_mhz": statistics.median(hi) if hi else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def workload(name: str):
+    from block_sparse_gqa_idx_b200 import inputs
+
+    return inputs.CONFIGS[name]
+
+
+def flops_of(cfg):
+    """Eq. 12 (xllm-io review): index term H_kv*d_idx*N^2, main term 4*N*H_q*k*B_k*d_h."""
+    f_idx = cfg.H_kv * cfg.d_idx * float(cfg.N) ** 2
+    f_main = 4.0 * cfg.N * cfg.H_q * cfg.k * cfg.B_k * cfg.d_h
+    return f_idx, f_main
+
+
+# ------------------------------------------------------------ reference arm --
+def run_reference(args, cfg, rank, world):
+    if rank != 0:
+        return 0
+    import oracle
+    from block_sparse_gqa_idx_b200 import inputs
+
+    inp = inputs.prefill_inputs(cfg)
+    rng = np.random.default_rng(7)
+    n_rows = args.ref_rows
+    times = []
+    for it in range(args.warmup + args.steps):
+        rows = np.sort(rng.choice(cfg.N, size=n_rows, replace=False))
+        t0 = time.perf_counter()
+        oracle.forward(inp, cfg.B_k, cfg.k, rows=rows)
+        dt = time.perf_counter() - t0
+        if it >= args.warmup:
+            times.append(dt)
+    tps = n_rows / statistics.mean(times)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": tps, "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * statistics.mean(times), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": cfg.name, "N": cfg.N, "rows_per_step": n_rows},
+        "cpu_baseline": {"value": tps, "unit": "tokens/s", "cores": oracle.max_threads(),
+                         "kind": "oracle",
+                         "sample": f"{n_rows} uniformly drawn query rows per step of the {cfg.name} "
+                                   f"workload (full causal prefix each)"},
+        "e2e": {"value": tps, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+METRIC = "MSA fwd prefill tokens/s @128K"
+
+
+# ----------------------------------------------------------------- msa arm --
+def run_msa(args, cfg, rank, world, local):
+    import torch
+    import torch.distributed as dist
+
+    import block_sparse_gqa_idx_b200 as msa
+    from block_sparse_gqa_idx_b200 import inputs
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+
+    # every replica gets its own seeded sequence
+    inp = inputs.prefill_inputs(cfg, seed=cfg.seed + 1000 * rank)
+    host = {k: torch.from_numpy(np.ascontiguousarray(v).view(np.int16)).view(torch.bfloat16)
+            for k, v in inp.items()}
+    d = {k: v.to(dev) for k, v in host.items()}
+    N, H_q, H_kv, d_h, d_idx, B_k, kk = cfg.N, cfg.H_q, cfg.H_kv, cfg.d_h, cfg.d_idx, cfg.B_k, cfg.k
+    idx = torch.empty((N, H_kv, kk), dtype=torch.int32, device=dev)
+    o = torch.empty((N, H_q, d_h), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((N, H_q), dtype=torch.float32, device=dev)
+    dims = msa.dims(N, H_q, H_kv, d_h, d_idx, B_k, kk)
+    ws = torch.empty(max(msa.sparse_attn_fwd_workspace_size(dims),
+                         msa.index_topk_workspace_size(dims)), dtype=torch.uint8, device=dev)
+
+    def step(src):
+        msa.index_topk(src["q_idx"], src["k_idx"], B_k, kk, idx_out=idx, workspace=ws,
+                       stream=stream)
+        msa.sparse_attn_fwd(src["q"], src["k"], src["v"], idx, B_k, o=o, lse=lse, workspace=ws,
+                            stream=stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step(d)
+    torch.cuda.synchronize()
+    code, where = msa.device_status(ws)
+    if code != 0:
+        raise RuntimeError(f"device status {code} at {where} after warm-up")
+
+    clocks = Clocks(local)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    msa.profile_enable(True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step(d)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    msa.profile_enable(False)
+    clk = clocks.stop()
+    prof = msa.profile_read()
+    ms = e0.elapsed_time(e1) / args.steps
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    value = world * N / (ms * 1e-3)
+
+    # ---- end to end: pinned host inputs -> device -> forward -> host result
+    pinned = {k: v.pin_memory() for k, v in host.items()}
+    o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    idx_host = torch.empty(idx.shape, dtype=idx.dtype).pin_memory()
+    e2e_steps = max(1, min(args.steps, 3))
+    h2d = sum(v.numel() * v.element_size() for v in pinned.values())
+    d2h = o_host.numel() * o_host.element_size() + idx_host.numel() * idx_host.element_size()
+
+    def e2e_step():
+        for k, v in pinned.items():
+            d[k].copy_(v, non_blocking=True)
+        step(d)
+        o_host.copy_(o, non_blocking=True)
+        idx_host.copy_(idx, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    f1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = f0.elapsed_time(f1) / e2e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    barrier()
+
+    if rank != 0:
+        return 0
+
+    # ---- roofline of the dominant kernel (live CUDA-event durations)
+    pk, pk_kind = peaks()
+    f_idx, f_main = flops_of(cfg)
+    total_ms = sum(v[1] for v in prof.values())
+    dom = max(prof, key=lambda n: prof[n][1])
+    launches, dom_ms = prof[dom]
+    per_launch_ms = dom_ms / launches
+    if dom == "index_topk":
+        work, unit, bound = f_idx, "TFLOP/s", "tensor"
+        achieved = work / (per_launch_ms * 1e-3) / 1e12
+        peak = pk["bf16_tflops"]
+    elif dom == "attn_phase1":
+        # one launch per query chunk and step: the Main Branch FLOPs of a chunk
+        work = f_main / (launches / args.steps)
+        unit, bound = "TFLOP/s", "tensor"
+        achieved = work / (per_launch_ms * 1e-3) / 1e12
+        peak = pk["bf16_tflops"]
+    else:
+        unit, bound = "GB/s", "hbm"
+        achieved, peak = None, pk["hbm_gbs"]
+    roofline = {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+                "frac": (achieved / peak) if achieved else None, "traffic": None,
+                "peak_kind": f"{pk_kind} burst",
+                "share": dom_ms / total_ms if total_ms else None}
+
+    # ---- CPU oracle on a bounded sample (rank 0, N=1 only)
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        import oracle
+
+        rng = np.random.default_rng(11)
+        rows = np.sort(rng.choice(N, size=args.cpu_rows, replace=False))
+        t0 = time.perf_counter()
+        oracle.forward(inp, B_k, kk, rows=rows)
+        dt = time.perf_counter() - t0
+        cpu = {"value": args.cpu_rows / dt, "unit": "tokens/s", "cores": oracle.max_threads(),
+               "kind": "oracle",
+               "sample": f"{args.cpu_rows} uniformly drawn query rows of the {cfg.name} workload "
+                         f"(index + attention, full causal prefix), {dt:.1f} s"}
+
+    kernels = {n: {"launches": v[0], "ms_per_step": v[1] / args.steps,
+                   "share": v[1] / total_ms if total_ms else None} for n, v in prof.items()}
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": cfg.name, "N": N, "H_q": H_q, "H_kv": H_kv, "d_h": d_h,
+                   "d_idx": d_idx, "B_k": B_k, "k": kk, "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (Q alone 1.07 GB); no flush"},
+        "tc_frac_eq12": (f_idx + f_main) / (ms * 1e-3) / 1e12 / pk["bf16_tflops"],
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": {"value": world * N / (e2e_ms * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": sum(v[0] for v in prof.values()),
+        "kernels": kernels,
+        "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="msa", choices=["msa", "reference"])
+    ap.add_argument("--workload", default="128k")
+    ap.add_argument("--cpu-rows", type=int, default=256)
+    ap.add_argument("--ref-rows", type=int, default=32)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    world, rank, local = dist_init()
+    cfg = workload(args.workload)
+    if args.impl == "reference":
+        return run_reference(args, cfg, rank, world)
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        return run_msa(args, cfg, rank, world, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

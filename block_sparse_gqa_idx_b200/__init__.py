@@ -1,0 +1,28 @@
+"""MiniMax Sparse Attention (MSA) forward path for B200 (sm_100a).
+
+The compute lives in ``libmsa_b200.so`` (hand-written CUDA behind the C ABI
+of ``include/msa.h``); this package is its thin Python binding:
+
+* ``index_topk``      Index Branch, Eq. 6-7 (fused scores, block max, Top-k)
+* ``sparse_attn_fwd`` Main Branch, Eq. 8 (KV-outer sparse attention + merge)
+* ``forward``         both, for one prefill sequence
+* ``sparse_decode``   one decode step for a batch of sequences
+
+``inputs`` holds the seeded synthetic workload generators.  The binding is
+loaded on first use of one of the names above and raises if the CUDA library
+has not been built (``python -m block_sparse_gqa_idx_b200.build``).
+"""
+_CAPI = ("index_topk", "sparse_attn_fwd", "forward", "sparse_decode", "device_status",
+         "version", "MSAError", "dims", "decode_dims", "index_topk_workspace_size",
+         "sparse_attn_fwd_workspace_size", "sparse_decode_workspace_size", "EXPORTS", "LIB_PATH",
+         "profile_enable", "profile_read")
+
+__all__ = list(_CAPI) + ["inputs"]
+
+
+def __getattr__(name):
+    if name in _CAPI:
+        from . import _capi
+
+        return getattr(_capi, name)
+    raise AttributeError(f"module {__name__!r} has no attribute {name!r}")

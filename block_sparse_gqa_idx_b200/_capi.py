@@ -1,0 +1,262 @@
+"""ctypes binding of ``include/msa.h`` (libmsa_b200.so).
+
+Argument marshalling only: every step of the MSA path runs in the CUDA
+library.  Tensors are torch CUDA tensors (PyTorch provides device memory and
+streams); the binding checks dtype, shape, device and contiguity, allocates
+outputs/workspaces with torch when the caller does not pass them, and passes
+raw pointers plus the current CUDA stream.  If the library is missing this
+module raises at import: there is no other implementation to fall back to.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmsa_b200.so")
+
+
+class MSAError(RuntimeError):
+    def __init__(self, what: str, status: int, text: str):
+        super().__init__(f"{what}: {text} (status {status})")
+        self.status = status
+
+
+class msa_dims(ctypes.Structure):
+    _fields_ = [("N", ctypes.c_int64), ("H_q", ctypes.c_int32), ("H_kv", ctypes.c_int32),
+                ("d_h", ctypes.c_int32), ("d_idx", ctypes.c_int32), ("B_k", ctypes.c_int32),
+                ("k", ctypes.c_int32), ("attn_scale", ctypes.c_float),
+                ("idx_scale", ctypes.c_float)]
+
+
+class msa_decode_dims(ctypes.Structure):
+    _fields_ = [("S", ctypes.c_int32), ("L_max", ctypes.c_int64), ("H_q", ctypes.c_int32),
+                ("H_kv", ctypes.c_int32), ("d_h", ctypes.c_int32), ("d_idx", ctypes.c_int32),
+                ("B_k", ctypes.c_int32), ("k", ctypes.c_int32), ("attn_scale", ctypes.c_float),
+                ("idx_scale", ctypes.c_float)]
+
+
+class msa_kernel_time(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char * 48), ("launches", ctypes.c_int32),
+                ("total_ms", ctypes.c_double)]
+
+
+# every symbol include/msa.h declares
+EXPORTS = ("msa_index_topk_workspace", "msa_index_topk", "msa_sparse_attn_fwd_workspace",
+           "msa_sparse_attn_fwd", "msa_sparse_decode_workspace", "msa_sparse_decode",
+           "msa_get_device_status", "msa_profile_enable", "msa_profile_read",
+           "msa_status_string", "msa_version")
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build the CUDA library first "
+            "(python -m block_sparse_gqa_idx_b200.build); there is no fallback path")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, Z, I32 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
+    D, DD = ctypes.POINTER(msa_dims), ctypes.POINTER(msa_decode_dims)
+    lib.msa_index_topk_workspace.argtypes = [D]
+    lib.msa_index_topk_workspace.restype = Z
+    lib.msa_index_topk.argtypes = [D, P, P, P, P, Z, P]
+    lib.msa_index_topk.restype = I32
+    lib.msa_sparse_attn_fwd_workspace.argtypes = [D]
+    lib.msa_sparse_attn_fwd_workspace.restype = Z
+    lib.msa_sparse_attn_fwd.argtypes = [D, P, P, P, P, P, P, P, Z, P]
+    lib.msa_sparse_attn_fwd.restype = I32
+    lib.msa_sparse_decode_workspace.argtypes = [DD]
+    lib.msa_sparse_decode_workspace.restype = Z
+    lib.msa_sparse_decode.argtypes = [DD] + [P] * 12 + [Z, P]
+    lib.msa_sparse_decode.restype = I32
+    lib.msa_get_device_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_int32),
+                                          ctypes.POINTER(ctypes.c_int32)]
+    lib.msa_get_device_status.restype = I32
+    lib.msa_profile_enable.argtypes = [ctypes.c_int32]
+    lib.msa_profile_enable.restype = I32
+    lib.msa_profile_read.argtypes = [ctypes.POINTER(msa_kernel_time), ctypes.c_int32]
+    lib.msa_profile_read.restype = ctypes.c_int32
+    lib.msa_status_string.argtypes = [I32]
+    lib.msa_status_string.restype = ctypes.c_char_p
+    lib.msa_version.argtypes = []
+    lib.msa_version.restype = ctypes.c_char_p
+    return lib
+
+
+LIB = _load()
+
+
+def version() -> str:
+    return LIB.msa_version().decode()
+
+
+def _raise(what: str, st: int) -> None:
+    if st != 0:
+        raise MSAError(what, st, LIB.msa_status_string(st).decode())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _want(t: torch.Tensor, name: str, dtype, shape) -> None:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def dims(N, H_q, H_kv, d_h, d_idx, B_k, k, attn_scale=0.0, idx_scale=0.0) -> msa_dims:
+    return msa_dims(int(N), int(H_q), int(H_kv), int(d_h), int(d_idx), int(B_k), int(k),
+                    float(attn_scale), float(idx_scale))
+
+
+def decode_dims(S, L_max, H_q, H_kv, d_h, d_idx, B_k, k, attn_scale=0.0,
+                idx_scale=0.0) -> msa_decode_dims:
+    return msa_decode_dims(int(S), int(L_max), int(H_q), int(H_kv), int(d_h), int(d_idx),
+                           int(B_k), int(k), float(attn_scale), float(idx_scale))
+
+
+def _workspace(nbytes: int, device, ws: Optional[torch.Tensor]) -> torch.Tensor:
+    if ws is None:
+        return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+    if ws.dtype != torch.uint8 or not ws.is_cuda or ws.numel() < nbytes:
+        raise ValueError(f"workspace must be a CUDA uint8 tensor of >= {nbytes} bytes")
+    return ws
+
+
+def index_topk_workspace_size(d: msa_dims) -> int:
+    return int(LIB.msa_index_topk_workspace(ctypes.byref(d)))
+
+
+def sparse_attn_fwd_workspace_size(d: msa_dims) -> int:
+    return int(LIB.msa_sparse_attn_fwd_workspace(ctypes.byref(d)))
+
+
+def sparse_decode_workspace_size(d: msa_decode_dims) -> int:
+    return int(LIB.msa_sparse_decode_workspace(ctypes.byref(d)))
+
+
+def index_topk(q_idx: torch.Tensor, k_idx: torch.Tensor, B_k: int, k: int,
+               idx_out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+               stream=None) -> torch.Tensor:
+    """Eq. 6-7: q_idx [N,H_kv,d_idx] bf16, k_idx [N,d_idx] bf16 -> idx [N,H_kv,k] int32."""
+    N, H_kv, d_idx = q_idx.shape
+    _want(q_idx, "q_idx", torch.bfloat16, (N, H_kv, d_idx))
+    _want(k_idx, "k_idx", torch.bfloat16, (N, d_idx))
+    if idx_out is None:
+        idx_out = torch.empty((N, H_kv, k), dtype=torch.int32, device=q_idx.device)
+    _want(idx_out, "idx_out", torch.int32, (N, H_kv, k))
+    d = dims(N, H_kv, H_kv, 64, d_idx, B_k, k)
+    ws = _workspace(index_topk_workspace_size(d), q_idx.device, workspace)
+    _raise("msa_index_topk", LIB.msa_index_topk(ctypes.byref(d), _ptr(q_idx), _ptr(k_idx),
+                                                _ptr(idx_out), _ptr(ws), ws.numel(),
+                                                _stream(stream)))
+    return idx_out
+
+
+def sparse_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, idx: torch.Tensor,
+                    B_k: int, attn_scale: float = 0.0, o: Optional[torch.Tensor] = None,
+                    lse: Optional[torch.Tensor] = None, want_lse: bool = True,
+                    workspace: Optional[torch.Tensor] = None, stream=None
+                    ) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Eq. 8: q [N,H_q,d_h], k/v [N,H_kv,d_h] bf16, idx [N,H_kv,kk] int32 ->
+    o [N,H_q,d_h] bf16 and lse [N,H_q] fp32."""
+    N, H_q, d_h = q.shape
+    H_kv = k.shape[1]
+    kk = idx.shape[2]
+    _want(q, "q", torch.bfloat16, (N, H_q, d_h))
+    _want(k, "k", torch.bfloat16, (N, H_kv, d_h))
+    _want(v, "v", torch.bfloat16, (N, H_kv, d_h))
+    _want(idx, "idx", torch.int32, (N, H_kv, kk))
+    if o is None:
+        o = torch.empty((N, H_q, d_h), dtype=torch.bfloat16, device=q.device)
+    _want(o, "o", torch.bfloat16, (N, H_q, d_h))
+    if lse is None and want_lse:
+        lse = torch.empty((N, H_q), dtype=torch.float32, device=q.device)
+    if lse is not None:
+        _want(lse, "lse", torch.float32, (N, H_q))
+    d = dims(N, H_q, H_kv, d_h, 64, B_k, kk, attn_scale)
+    ws = _workspace(sparse_attn_fwd_workspace_size(d), q.device, workspace)
+    _raise("msa_sparse_attn_fwd",
+           LIB.msa_sparse_attn_fwd(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(idx), _ptr(o),
+                                   _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)))
+    return o, lse
+
+
+def forward(q, k, v, q_idx, k_idx, B_k: int, kk: int, attn_scale: float = 0.0, stream=None,
+            workspace: Optional[torch.Tensor] = None):
+    """Whole MSA forward (Eq. 6-8): returns (o, lse, idx)."""
+    idx = index_topk(q_idx, k_idx, B_k, kk, workspace=workspace, stream=stream)
+    o, lse = sparse_attn_fwd(q, k, v, idx, B_k, attn_scale, workspace=workspace, stream=stream)
+    return o, lse, idx
+
+
+def sparse_decode(q, q_idx, k_new, v_new, k_idx_new, k_cache, v_cache, k_idx_cache,
+                  seq_len, B_k: int, kk: int, attn_scale: float = 0.0,
+                  o: Optional[torch.Tensor] = None, idx_out: Optional[torch.Tensor] = None,
+                  workspace: Optional[torch.Tensor] = None, stream=None):
+    """One decode step (append + Eq. 6-8 for the new token of each sequence).
+    Returns (o [S,H_q,d_h] bf16, idx_out or None); seq_len is incremented."""
+    S, H_q, d_h = q.shape
+    H_kv, d_idx = q_idx.shape[1], q_idx.shape[2]
+    L_max = k_cache.shape[1]
+    _want(q, "q", torch.bfloat16, (S, H_q, d_h))
+    _want(q_idx, "q_idx", torch.bfloat16, (S, H_kv, d_idx))
+    _want(k_new, "k_new", torch.bfloat16, (S, H_kv, d_h))
+    _want(v_new, "v_new", torch.bfloat16, (S, H_kv, d_h))
+    _want(k_idx_new, "k_idx_new", torch.bfloat16, (S, d_idx))
+    _want(k_cache, "k_cache", torch.bfloat16, (S, L_max, H_kv, d_h))
+    _want(v_cache, "v_cache", torch.bfloat16, (S, L_max, H_kv, d_h))
+    _want(k_idx_cache, "k_idx_cache", torch.bfloat16, (S, L_max, d_idx))
+    _want(seq_len, "seq_len", torch.int32, (S,))
+    if o is None:
+        o = torch.empty((S, H_q, d_h), dtype=torch.bfloat16, device=q.device)
+    _want(o, "o", torch.bfloat16, (S, H_q, d_h))
+    if idx_out is not None:
+        _want(idx_out, "idx_out", torch.int32, (S, H_kv, kk))
+    d = decode_dims(S, L_max, H_q, H_kv, d_h, d_idx, B_k, kk, attn_scale)
+    ws = _workspace(sparse_decode_workspace_size(d), q.device, workspace)
+    _raise("msa_sparse_decode",
+           LIB.msa_sparse_decode(ctypes.byref(d), _ptr(q), _ptr(q_idx), _ptr(k_new), _ptr(v_new),
+                                 _ptr(k_idx_new), _ptr(k_cache), _ptr(v_cache), _ptr(k_idx_cache),
+                                 _ptr(seq_len), _ptr(o), _ptr(idx_out), _ptr(ws), ws.numel(),
+                                 _stream(stream)))
+    return o, idx_out
+
+
+def profile_enable(on: bool) -> None:
+    """Start (clearing earlier records) or stop per-kernel event timing."""
+    LIB.msa_profile_enable(1 if on else 0)
+
+
+def profile_read() -> dict:
+    """{kernel name: (launches, total milliseconds)} recorded since enable."""
+    buf = (msa_kernel_time * 64)()
+    n = LIB.msa_profile_read(buf, 64)
+    if n < 0:
+        raise MSAError("msa_profile_read", 4, "CUDA error")
+    return {buf[j].name.decode(): (int(buf[j].launches), float(buf[j].total_ms))
+            for j in range(min(n, 64))}
+
+
+def device_status(workspace: torch.Tensor, stream=None) -> Tuple[int, int]:
+    """(code, where) of the workspace's device status word; syncs the stream."""
+    code, where = ctypes.c_int32(0), ctypes.c_int32(0)
+    LIB.msa_get_device_status(_ptr(workspace), _stream(stream), ctypes.byref(code),
+                              ctypes.byref(where))
+    return int(code.value), int(where.value)

@@ -1,0 +1,609 @@
+// decode.cu -- one MSA decode step for S independent sequences.
+//
+// Per sequence s with L = seq_len[s]:
+//   append   k/v/k_idx of the new token at row L (Eq. 1: the query sees i <= t,
+//            itself included)
+//   scan     Eq. 6 for the single query i = L over the full blocks 0..b_i-1
+//            (b_i = L / B_k; the local block b_i is forced and needs no score):
+//            block maxima of the H_kv index-query dots, streamed from the K_idx
+//            cache.  HBM-bound: 2*d_idx bytes per cached token.
+//   top-k    Eq. 7: one warp per (s, r) keeps per-lane sorted candidate lists
+//            and merges them in k-1 warp-argmax rounds (ties -> lower block).
+//   attend   Eq. 8: one CTA per (s, r, slot) gathers that block's K/V rows
+//            (TMA), S = q K^T and O = P V on mma.sync, causal mask j <= L in
+//            the local block; writes a normalised partial and its LSE.
+//   merge    LSE-weighted combine of the <= k partials per head; seq_len += 1.
+//
+// Source: xllm-io paper review, "核心公式" Eq. 1, 6, 7, 8; chlience notes
+// 5.1.1 (selection steps) and 5.4 (exp-free selection on raw scores).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "msa_internal.h"
+
+namespace msa {
+namespace {
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+struct DecBufs {
+  int32_t* Lcur;    // [S] this step's length before the append, -1 = skipped
+  float* M;         // [S, H_kv, Bmax] block maxima (raw dots)
+  int32_t* sel;     // [S, H_kv, k]
+  float* part_o;    // [S, H_kv, k, G, d_h] normalised partial outputs
+  float* part_lse;  // [S, H_kv, k, G]
+};
+
+DecBufs carve(void* ws, int S, int64_t L_max, int H_q, int H_kv, int d_h, int B_k, int kk,
+              size_t* total) {
+  DecBufs b;
+  uint8_t* p = static_cast<uint8_t*>(ws);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    uint8_t* r = p ? p + off : nullptr;
+    off += align256(bytes);
+    return r;
+  };
+  const int64_t Bmax = (L_max + B_k - 1) / B_k + 1;
+  const int G = H_q / H_kv;
+  b.Lcur = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * S));
+  b.M = reinterpret_cast<float*>(take(sizeof(float) * S * H_kv * Bmax));
+  b.sel = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * S * H_kv * kk));
+  b.part_o = reinterpret_cast<float*>(take(sizeof(float) * S * H_kv * kk * G * d_h));
+  b.part_lse = reinterpret_cast<float*>(take(sizeof(float) * S * H_kv * kk * G));
+  *total = off;
+  return b;
+}
+
+struct DecParams {
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* q_idx;
+  const __nv_bfloat16* k_new;
+  const __nv_bfloat16* v_new;
+  const __nv_bfloat16* k_idx_new;
+  __nv_bfloat16* k_cache;
+  __nv_bfloat16* v_cache;
+  __nv_bfloat16* k_idx_cache;
+  int32_t* seq_len;
+  __nv_bfloat16* o;
+  int32_t* idx_out;
+  int S;
+  int64_t L_max, Bmax;
+  int H_q, H_kv, d_h, d_idx, B_k, kk, G;
+  float scale_log2, scale;
+  DecBufs w;
+  DevStatus* status;
+};
+
+// ------------------------------------------------------------------ append --
+__global__ void dec_append_kernel(const DecParams p) {
+  const int s = blockIdx.x;
+  const int64_t L = p.seq_len[s];
+  if (L < 0 || L >= p.L_max) {
+    if (threadIdx.x == 0) {
+      p.w.Lcur[s] = -1;
+      report(p.status, DEV_ERR_CACHE_FULL, 80, s, static_cast<int>(L));
+    }
+    return;
+  }
+  if (threadIdx.x == 0) p.w.Lcur[s] = static_cast<int32_t>(L);
+  const int kv16 = p.H_kv * p.d_h / 8;  // 16-byte pieces per K (or V) row
+  const int ki16 = p.d_idx / 8;
+  const uint4* kn = reinterpret_cast<const uint4*>(p.k_new + static_cast<int64_t>(s) * p.H_kv * p.d_h);
+  const uint4* vn = reinterpret_cast<const uint4*>(p.v_new + static_cast<int64_t>(s) * p.H_kv * p.d_h);
+  const uint4* kin = reinterpret_cast<const uint4*>(p.k_idx_new + static_cast<int64_t>(s) * p.d_idx);
+  uint4* kc = reinterpret_cast<uint4*>(p.k_cache + (s * p.L_max + L) * p.H_kv * p.d_h);
+  uint4* vc = reinterpret_cast<uint4*>(p.v_cache + (s * p.L_max + L) * p.H_kv * p.d_h);
+  uint4* kic = reinterpret_cast<uint4*>(p.k_idx_cache + (s * p.L_max + L) * p.d_idx);
+  for (int t = threadIdx.x; t < kv16; t += blockDim.x) {
+    kc[t] = kn[t];
+    vc[t] = vn[t];
+  }
+  for (int t = threadIdx.x; t < ki16; t += blockDim.x) kic[t] = kin[t];
+}
+
+// -------------------------------------------------------------------- scan --
+__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
+                                               uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// One warp scores one 128-key block at a time (B_k = 128: 8 row tiles of 16
+// keys; B_k = 64: 4).  MMA rows = keys, columns = index-query heads (padded
+// to 8), reduction over d_idx.  The d axis is consumed in a per-thread order
+// (thread t of a quad owns d in [t*D/4, (t+1)*D/4)), applied identically to
+// the A rows (keys, loaded straight from global memory with 16-byte loads)
+// and to the B columns (index queries), so every dot product is complete.
+template <int D_IDX, int BK>
+__global__ void __launch_bounds__(256) dec_scan_kernel(const DecParams p, int nsplit) {
+  constexpr int DT = D_IDX / 4;       // d elements per thread and key row
+  constexpr int NMMA = D_IDX / 16;    // MMAs per 16-key tile
+  constexpr int NV = DT / 8;          // 16-byte loads per key row
+  const int s = blockIdx.y;
+  const int64_t L = p.w.Lcur[s];
+  if (L < 0) return;
+  const int64_t b_i = L / p.B_k;  // candidate blocks 0 .. b_i-1
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
+  // B fragments: column n = g (index-query head), k-slots follow the d order.
+  uint32_t bq[NMMA][2];
+  {
+    const __nv_bfloat16* qr = p.q_idx + (static_cast<int64_t>(s) * p.H_kv + (g < p.H_kv ? g : 0)) * D_IDX;
+#pragma unroll
+    for (int j = 0; j < NMMA; ++j) {
+      const int d0 = t * DT + 4 * j;
+      uint32_t lo = *reinterpret_cast<const uint32_t*>(qr + d0);
+      uint32_t hi = *reinterpret_cast<const uint32_t*>(qr + d0 + 2);
+      bq[j][0] = g < p.H_kv ? lo : 0u;
+      bq[j][1] = g < p.H_kv ? hi : 0u;
+    }
+  }
+  const __nv_bfloat16* kbase = p.k_idx_cache + static_cast<int64_t>(s) * p.L_max * D_IDX;
+  const int wstride = nsplit * 8;
+  for (int64_t b = blockIdx.x * 8 + warp; b < b_i; b += wstride) {
+    float mx0 = -INFINITY, mx1 = -INFINITY;  // columns 2t, 2t+1
+#pragma unroll
+    for (int tile = 0; tile < BK / 16; ++tile) {
+      const __nv_bfloat16* r0 = kbase + (b * BK + tile * 16 + g) * D_IDX + t * DT;
+      const __nv_bfloat16* r1 = r0 + 8 * D_IDX;
+      uint4 v0[NV], v1[NV];
+#pragma unroll
+      for (int u = 0; u < NV; ++u) {
+        v0[u] = __ldg(reinterpret_cast<const uint4*>(r0) + u);
+        v1[u] = __ldg(reinterpret_cast<const uint4*>(r1) + u);
+      }
+      const uint32_t* w0 = reinterpret_cast<const uint32_t*>(v0);
+      const uint32_t* w1 = reinterpret_cast<const uint32_t*>(v1);
+      float c[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int j = 0; j < NMMA; ++j) {
+        // k-slots 2t,2t+1 <- d0,d0+1 ; 2t+8,2t+9 <- d0+2,d0+3 (d0 = t*DT + 4j)
+        const uint32_t a[4] = {w0[2 * j], w1[2 * j], w0[2 * j + 1], w1[2 * j + 1]};
+        mma_bf16_16816(c, a, bq[j][0], bq[j][1]);
+      }
+      mx0 = fmax3(mx0, c[0], c[2]);
+      mx1 = fmax3(mx1, c[1], c[3]);
+    }
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xFFFFFFFFu, mx0, o));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xFFFFFFFFu, mx1, o));
+    }
+    if (g == 0) {
+      const int r0 = 2 * t, r1 = 2 * t + 1;
+      float* Mrow = p.w.M + static_cast<int64_t>(s) * p.H_kv * p.Bmax;
+      if (r0 < p.H_kv) Mrow[r0 * p.Bmax + b] = mx0;
+      if (r1 < p.H_kv) Mrow[r1 * p.Bmax + b] = mx1;
+    }
+  }
+}
+
+// ------------------------------------------------------------------- top-k --
+__device__ __forceinline__ uint64_t pack_key(float v, int b) {
+  uint32_t u = __float_as_uint(v);
+  u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  return (static_cast<uint64_t>(u) << 32) | (0xFFFFFFFFu - static_cast<uint32_t>(b));
+}
+
+__global__ void __launch_bounds__(256) dec_topk_kernel(const DecParams p) {
+  extern __shared__ uint64_t lists[];  // [8 warps][k-1 slots][32 lanes]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int pair = blockIdx.x * 8 + warp;
+  if (pair >= p.S * p.H_kv) return;
+  const int s = pair / p.H_kv, r = pair - s * p.H_kv;
+  const int64_t L = p.w.Lcur[s];
+  if (L < 0) return;
+  const int b_i = static_cast<int>(L / p.B_k);
+  const int HS = p.kk - 1;
+  uint64_t* my = lists + static_cast<size_t>(warp) * (HS > 0 ? HS : 1) * 32;
+  const float* Mrow = p.w.M + (static_cast<int64_t>(s) * p.H_kv + r) * p.Bmax;
+  int cnt = 0;
+  uint64_t worst = 0;  // smallest kept key once the list is full
+  for (int b = lane; b < b_i && HS > 0; b += 32) {
+    const uint64_t key = pack_key(Mrow[b], b);
+    if (cnt == HS && key <= worst) continue;
+    // insert into the lane's descending list
+    int pos = cnt < HS ? cnt : HS - 1;
+    while (pos > 0 && my[(pos - 1) * 32 + lane] < key) {
+      my[pos * 32 + lane] = my[(pos - 1) * 32 + lane];
+      --pos;
+    }
+    my[pos * 32 + lane] = key;
+    if (cnt < HS) ++cnt;
+    worst = my[(cnt - 1) * 32 + lane];
+  }
+  // k-1 rounds of warp argmax over the lanes' list heads
+  int head = 0;
+  int32_t mine = -1;  // lane j keeps the j-th winner
+  const int rounds = HS < b_i ? HS : b_i;
+  for (int round = 0; round < rounds; ++round) {
+    const uint64_t cand = head < cnt ? my[head * 32 + lane] : 0ull;
+    uint64_t best = cand;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const uint64_t other = __shfl_xor_sync(0xFFFFFFFFu, best, o);
+      best = other > best ? other : best;
+    }
+    if (cand == best && cand != 0ull) ++head;
+    if (lane == round) mine = static_cast<int32_t>(0xFFFFFFFFu - static_cast<uint32_t>(best));
+  }
+  if (lane == rounds) mine = b_i;  // the local block (Eq. 7: always kept)
+  // ascending order: rank of each lane's block among the valid ones
+  const int nsel = rounds + 1;
+  int rank = 0;
+  for (int j = 0; j < nsel; ++j) {
+    const int32_t x = __shfl_sync(0xFFFFFFFFu, mine, j);
+    if (lane < nsel && x < mine) ++rank;
+  }
+  int32_t* dst = p.w.sel + (static_cast<int64_t>(s) * p.H_kv + r) * p.kk;
+  if (lane < nsel) dst[rank] = mine;
+  else if (lane < p.kk) dst[lane] = -1;
+  if (p.idx_out != nullptr) {
+    int32_t* d2 = p.idx_out + (static_cast<int64_t>(s) * p.H_kv + r) * p.kk;
+    if (lane < nsel) d2[rank] = mine;
+    else if (lane < p.kk) d2[lane] = -1;
+  }
+}
+
+// ------------------------------------------------------------------ attend --
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                        uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                          uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// Byte address of (row, 16-byte chunk c) in a TMA tile of 128-byte rows with
+// 128-byte swizzle (chunks XOR row mod 8), split in 64-element column boxes.
+template <int BK>
+__device__ __forceinline__ uint32_t sw_addr(uint32_t base, int row, int d) {
+  const int box = d >> 6, c = (d >> 3) & 7;
+  return base + box * BK * 128 + row * 128 + ((c ^ (row & 7)) << 4);
+}
+
+// One CTA (4 warps) per (sequence, group, slot).  Rows of the MMA are the
+// group's query heads (G <= 16, padded to 16); warp w owns keys
+// [w*BK/4, (w+1)*BK/4) of the block; the four partial softmax states are
+// merged through shared memory.
+template <int D_H, int BK>
+__global__ void __launch_bounds__(128) dec_attend_kernel(const __grid_constant__ CUtensorMap tm_k,
+                                                         const __grid_constant__ CUtensorMap tm_v,
+                                                         const DecParams p) {
+  constexpr int KW = BK / 4;          // keys per warp
+  constexpr int NT = KW / 8;          // S n-tiles per warp
+  constexpr int DT = D_H / 8;         // O n-tiles
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sK = smem;
+  uint8_t* sV = smem + BK * D_H * 2;
+  float* red = reinterpret_cast<float*>(sV + BK * D_H * 2);  // [4][16] m, [4][16] l
+  float* obuf = red + 128;                                    // [4][16][D_H]
+  uint64_t* bar = reinterpret_cast<uint64_t*>(obuf + 4 * 16 * D_H);
+
+  const int item = blockIdx.x;  // (s, r, slot)
+  const int slot = item % p.kk;
+  const int r = (item / p.kk) % p.H_kv;
+  const int s = item / (p.kk * p.H_kv);
+  const int64_t L = p.w.Lcur[s];
+  if (L < 0) return;
+  const int b = p.w.sel[(static_cast<int64_t>(s) * p.H_kv + r) * p.kk + slot];
+  if (b < 0) return;
+  const int64_t last = L;  // the new token's position: keys j <= last
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    mbar_arrive_expect_tx(bar, 2 * BK * D_H * 2);
+    const int row0 = static_cast<int>(s * p.L_max + static_cast<int64_t>(b) * BK);
+    for (int c = 0; c < D_H / 64; ++c) {
+      tma_load_3d(sK + c * BK * 128, &tm_k, bar, c * 64, r, row0);
+      tma_load_3d(sV + c * BK * 128, &tm_v, bar, c * 64, r, row0);
+    }
+  }
+  // Q fragments (rows = heads, zero beyond G) while the tiles land.
+  uint32_t qa[D_H / 16][4];
+  {
+    const __nv_bfloat16* qb = p.q + (static_cast<int64_t>(s) * p.H_q + r * p.G) * D_H;
+#pragma unroll
+    for (int ks = 0; ks < D_H / 16; ++ks) {
+      const int d = ks * 16 + 2 * t;
+      qa[ks][0] = g < p.G ? *reinterpret_cast<const uint32_t*>(qb + g * D_H + d) : 0u;
+      qa[ks][1] = g + 8 < p.G ? *reinterpret_cast<const uint32_t*>(qb + (g + 8) * D_H + d) : 0u;
+      qa[ks][2] = g < p.G ? *reinterpret_cast<const uint32_t*>(qb + g * D_H + d + 8) : 0u;
+      qa[ks][3] = g + 8 < p.G ? *reinterpret_cast<const uint32_t*>(qb + (g + 8) * D_H + d + 8) : 0u;
+    }
+  }
+  bool ok = mbar_wait(bar, 0, nullptr, p.status, 90);
+  const int kw0 = warp * KW;  // first key (within the block) of this warp
+  float sacc[NT][4];
+#pragma unroll
+  for (int n = 0; n < NT; ++n) sacc[n][0] = sacc[n][1] = sacc[n][2] = sacc[n][3] = 0.f;
+  if (ok) {
+    const uint32_t kb = smem_u32(sK);
+#pragma unroll
+    for (int ks = 0; ks < D_H / 16; ++ks) {
+#pragma unroll
+      for (int n2 = 0; n2 < NT / 2; ++n2) {
+        // matrices: (keys 0-7, d lo), (keys 0-7, d hi), (keys 8-15, d lo), (keys 8-15, d hi)
+        const int mi = lane >> 3, rr = lane & 7;
+        const int key = kw0 + n2 * 16 + (mi >> 1) * 8 + rr;
+        const int d = ks * 16 + (mi & 1) * 8;
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(sw_addr<BK>(kb, key, d), b0, b1, b2, b3);
+        mma_bf16_16816(sacc[2 * n2], qa[ks], b0, b1);
+        mma_bf16_16816(sacc[2 * n2 + 1], qa[ks], b2, b3);
+      }
+    }
+  }
+  // scale, causal mask (only the block holding the new token), row max / sum
+  const int64_t j0 = static_cast<int64_t>(b) * BK + kw0;
+  float m_lo = -INFINITY, m_hi = -INFINITY;
+#pragma unroll
+  for (int n = 0; n < NT; ++n) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int64_t j = j0 + n * 8 + 2 * t + (e & 1);
+      float x = sacc[n][e] * p.scale_log2;
+      if (j > last) x = -INFINITY;
+      sacc[n][e] = x;
+    }
+    m_lo = fmax3(m_lo, sacc[n][0], sacc[n][1]);
+    m_hi = fmax3(m_hi, sacc[n][2], sacc[n][3]);
+  }
+#pragma unroll
+  for (int o = 1; o < 4; o <<= 1) {
+    m_lo = fmaxf(m_lo, __shfl_xor_sync(0xFFFFFFFFu, m_lo, o));
+    m_hi = fmaxf(m_hi, __shfl_xor_sync(0xFFFFFFFFu, m_hi, o));
+  }
+  const float ms_lo = m_lo == -INFINITY ? 0.f : m_lo;
+  const float ms_hi = m_hi == -INFINITY ? 0.f : m_hi;
+  float l_lo = 0.f, l_hi = 0.f;
+  uint32_t pa[NT / 2][4];
+#pragma unroll
+  for (int n = 0; n < NT; ++n) {
+    const float e0 = exp2f(sacc[n][0] - ms_lo), e1 = exp2f(sacc[n][1] - ms_lo);
+    const float e2 = exp2f(sacc[n][2] - ms_hi), e3 = exp2f(sacc[n][3] - ms_hi);
+    l_lo += e0 + e1;
+    l_hi += e2 + e3;
+    // A fragment of P for k-step n/2: n even -> regs 0,1 ; n odd -> regs 2,3
+    pa[n >> 1][(n & 1) * 2 + 0] = pack_bf16(e0, e1);
+    pa[n >> 1][(n & 1) * 2 + 1] = pack_bf16(e2, e3);
+  }
+#pragma unroll
+  for (int o = 1; o < 4; o <<= 1) {
+    l_lo += __shfl_xor_sync(0xFFFFFFFFu, l_lo, o);
+    l_hi += __shfl_xor_sync(0xFFFFFFFFu, l_hi, o);
+  }
+  float oacc[DT][4];
+#pragma unroll
+  for (int n = 0; n < DT; ++n) oacc[n][0] = oacc[n][1] = oacc[n][2] = oacc[n][3] = 0.f;
+  if (ok) {
+    const uint32_t vb = smem_u32(sV);
+#pragma unroll
+    for (int ks = 0; ks < NT / 2; ++ks) {
+#pragma unroll
+      for (int n2 = 0; n2 < DT / 2; ++n2) {
+        // matrices: (keys 0-7, d lo), (keys 8-15, d lo), (keys 0-7, d hi), (keys 8-15, d hi)
+        const int mi = lane >> 3, rr = lane & 7;
+        const int key = kw0 + ks * 16 + (mi & 1) * 8 + rr;
+        const int d = n2 * 16 + (mi >> 1) * 8;
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(sw_addr<BK>(vb, key, d), b0, b1, b2, b3);
+        mma_bf16_16816(oacc[2 * n2], pa[ks], b0, b1);
+        mma_bf16_16816(oacc[2 * n2 + 1], pa[ks], b2, b3);
+      }
+    }
+  }
+  // merge the four warps' (m, l, O) through shared memory (log2 domain)
+  if (t == 0) {
+    red[warp * 16 + g] = m_lo;
+    red[warp * 16 + g + 8] = m_hi;
+    red[64 + warp * 16 + g] = l_lo;
+    red[64 + warp * 16 + g + 8] = l_hi;
+  }
+#pragma unroll
+  for (int n = 0; n < DT; ++n) {
+    float* o0 = obuf + (warp * 16 + g) * D_H + n * 8 + 2 * t;
+    float* o1 = obuf + (warp * 16 + g + 8) * D_H + n * 8 + 2 * t;
+    o0[0] = oacc[n][0];
+    o0[1] = oacc[n][1];
+    o1[0] = oacc[n][2];
+    o1[1] = oacc[n][3];
+  }
+  __syncthreads();
+  // thread -> (head row, d slice): 16 rows x 8 threads
+  const int hr = threadIdx.x >> 3, part = threadIdx.x & 7;
+  if (hr < p.G) {
+    float M = -INFINITY;
+    for (int w = 0; w < 4; ++w) M = fmaxf(M, red[w * 16 + hr]);
+    const float Ms = M == -INFINITY ? 0.f : M;
+    float wsum = 0.f, wt[4];
+    for (int w = 0; w < 4; ++w) {
+      const float mw = red[w * 16 + hr];
+      wt[w] = mw == -INFINITY ? 0.f : exp2f(mw - Ms);
+      wsum += wt[w] * red[64 + w * 16 + hr];
+    }
+    const int64_t pslot = ((static_cast<int64_t>(s) * p.H_kv + r) * p.kk + slot) * p.G + hr;
+    float* dst = p.w.part_o + pslot * D_H;
+    const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+    for (int d = part; d < D_H; d += 8) {
+      float acc = 0.f;
+      for (int w = 0; w < 4; ++w) acc += wt[w] * obuf[(w * 16 + hr) * D_H + d];
+      dst[d] = acc * inv;
+    }
+    if (part == 0)
+      p.w.part_lse[pslot] = wsum > 0.f ? (M + log2f(wsum)) * 0.6931471805599453f : -INFINITY;
+  }
+}
+
+// ------------------------------------------------------------------- merge --
+template <int D_H>
+__global__ void __launch_bounds__(256) dec_merge_kernel(const DecParams p) {
+  constexpr int PER = D_H / 32;
+  const int lane = threadIdx.x & 31;
+  const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;  // (s, h)
+  if (row >= p.S * p.H_q) return;
+  const int s = row / p.H_q, h = row - s * p.H_q;
+  const int r = h / p.G, g = h - r * p.G;
+  const int64_t L = p.w.Lcur[s];
+  if (L < 0) return;
+  const int32_t* sel = p.w.sel + (static_cast<int64_t>(s) * p.H_kv + r) * p.kk;
+  const unsigned use = __ballot_sync(0xFFFFFFFFu, lane < p.kk && sel[lane < p.kk ? lane : 0] >= 0);
+  float m = -INFINITY, wsum = 0.f, acc[PER];
+#pragma unroll
+  for (int e = 0; e < PER; ++e) acc[e] = 0.f;
+  unsigned rest = use;
+  while (rest) {
+    const int sl = __ffs(rest) - 1;
+    rest &= rest - 1;
+    const int64_t pslot = ((static_cast<int64_t>(s) * p.H_kv + r) * p.kk + sl) * p.G + g;
+    const float ls = p.w.part_lse[pslot];
+    if (ls == -INFINITY) continue;
+    const float* src = p.w.part_o + pslot * D_H + lane * PER;
+    const float mn = fmaxf(m, ls);
+    const float a_old = __expf(m - mn), a_new = __expf(ls - mn);
+#pragma unroll
+    for (int e = 0; e < PER; ++e) acc[e] = acc[e] * a_old + src[e] * a_new;
+    wsum = wsum * a_old + a_new;
+    m = mn;
+  }
+  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+  __nv_bfloat16* dst = p.o + (static_cast<int64_t>(s) * p.H_q + h) * D_H + lane * PER;
+#pragma unroll
+  for (int e = 0; e < PER; e += 2)
+    *reinterpret_cast<__nv_bfloat162*>(dst + e) = __floats2bfloat162_rn(acc[e] * inv, acc[e + 1] * inv);
+  // seq_len is read only by the append kernel; the rest of the step uses Lcur
+  if (h == 0 && lane == 0) p.seq_len[s] = static_cast<int32_t>(L + 1);
+}
+
+template <int D_H, int BK>
+size_t attend_smem() {
+  return 1024 + 2 * BK * D_H * 2 + 128 * 4 + 4 * 16 * D_H * 4 + 16;
+}
+
+template <int D_H, int BK>
+cudaError_t launch_attend(const DecParams& p, cudaStream_t stream) {
+  CUtensorMap tk, tv;
+  const uint64_t dims[3] = {static_cast<uint64_t>(D_H), static_cast<uint64_t>(p.H_kv),
+                            static_cast<uint64_t>(p.S) * static_cast<uint64_t>(p.L_max)};
+  const uint64_t strides[2] = {static_cast<uint64_t>(D_H) * 2,
+                               static_cast<uint64_t>(p.H_kv) * D_H * 2};
+  const uint32_t box[3] = {64, 1, static_cast<uint32_t>(BK)};
+  if (!make_tmap_bf16(&tk, p.k_cache, 3, dims, strides, box, 128)) return cudaErrorInvalidValue;
+  if (!make_tmap_bf16(&tv, p.v_cache, 3, dims, strides, box, 128)) return cudaErrorInvalidValue;
+  const size_t smem = attend_smem<D_H, BK>();
+  cudaError_t e = cudaFuncSetAttribute(dec_attend_kernel<D_H, BK>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  prof_begin("dec_attend", stream);
+  dec_attend_kernel<D_H, BK><<<p.S * p.H_kv * p.kk, 128, smem, stream>>>(tk, tv, p);
+  prof_end(stream);
+  return cudaGetLastError();
+}
+
+template <int D_IDX>
+cudaError_t launch_scan(const DecParams& p, cudaStream_t stream) {
+  const int nsplit = p.S >= 64 ? 8 : (p.S >= 16 ? 32 : 64);
+  dim3 grid(nsplit, p.S);
+  prof_begin("dec_scan", stream);
+  if (p.B_k == 128) dec_scan_kernel<D_IDX, 128><<<grid, 256, 0, stream>>>(p, nsplit);
+  else dec_scan_kernel<D_IDX, 64><<<grid, 256, 0, stream>>>(p, nsplit);
+  prof_end(stream);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t decode_workspace_bytes(int S, int64_t L_max, int H_q, int H_kv, int d_h, int B_k, int kk) {
+  size_t total = 0;
+  carve(nullptr, S, L_max, H_q, H_kv, d_h, B_k, kk, &total);
+  return total;
+}
+
+cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t stream) {
+  DecParams p;
+  p.q = static_cast<const __nv_bfloat16*>(a.q);
+  p.q_idx = static_cast<const __nv_bfloat16*>(a.q_idx);
+  p.k_new = static_cast<const __nv_bfloat16*>(a.k_new);
+  p.v_new = static_cast<const __nv_bfloat16*>(a.v_new);
+  p.k_idx_new = static_cast<const __nv_bfloat16*>(a.k_idx_new);
+  p.k_cache = static_cast<__nv_bfloat16*>(a.k_cache);
+  p.v_cache = static_cast<__nv_bfloat16*>(a.v_cache);
+  p.k_idx_cache = static_cast<__nv_bfloat16*>(a.k_idx_cache);
+  p.seq_len = a.seq_len;
+  p.o = static_cast<__nv_bfloat16*>(a.o);
+  p.idx_out = a.idx_out;
+  p.S = a.S;
+  p.L_max = a.L_max;
+  p.Bmax = (a.L_max + a.B_k - 1) / a.B_k + 1;
+  p.H_q = a.H_q;
+  p.H_kv = a.H_kv;
+  p.d_h = a.d_h;
+  p.d_idx = a.d_idx;
+  p.B_k = a.B_k;
+  p.kk = a.kk;
+  p.G = a.H_q / a.H_kv;
+  p.scale = a.scale;
+  p.scale_log2 = a.scale * 1.4426950408889634f;
+  size_t need = 0;
+  p.w = carve(a.ws, a.S, a.L_max, a.H_q, a.H_kv, a.d_h, a.B_k, a.kk, &need);
+  if (need > a.ws_bytes) return cudaErrorInvalidValue;
+  p.status = a.status;
+
+  prof_begin("dec_append", stream);
+  dec_append_kernel<<<a.S, 128, 0, stream>>>(p);
+  prof_end(stream);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  switch (a.d_idx) {
+    case 32: e = launch_scan<32>(p, stream); break;
+    case 64: e = launch_scan<64>(p, stream); break;
+    case 128: e = launch_scan<128>(p, stream); break;
+    default: return cudaErrorInvalidValue;
+  }
+  if (e != cudaSuccess) return e;
+  const int hs = a.kk - 1 > 0 ? a.kk - 1 : 1;
+  const size_t topk_smem = 8 * hs * 32 * sizeof(uint64_t);
+  e = cudaFuncSetAttribute(dec_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(topk_smem));
+  if (e != cudaSuccess) return e;
+  prof_begin("dec_topk", stream);
+  dec_topk_kernel<<<(a.S * a.H_kv + 7) / 8, 256, topk_smem, stream>>>(p);
+  prof_end(stream);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  if (a.d_h == 128 && a.B_k == 128) e = launch_attend<128, 128>(p, stream);
+  else if (a.d_h == 128 && a.B_k == 64) e = launch_attend<128, 64>(p, stream);
+  else if (a.d_h == 64 && a.B_k == 128) e = launch_attend<64, 128>(p, stream);
+  else e = launch_attend<64, 64>(p, stream);
+  if (e != cudaSuccess) return e;
+  const int rows = a.S * a.H_q;
+  prof_begin("dec_merge", stream);
+  if (a.d_h == 128) dec_merge_kernel<128><<<(rows * 32 + 255) / 256, 256, 0, stream>>>(p);
+  else dec_merge_kernel<64><<<(rows * 32 + 255) / 256, 256, 0, stream>>>(p);
+  prof_end(stream);
+  return cudaGetLastError();
+}
+
+}  // namespace msa

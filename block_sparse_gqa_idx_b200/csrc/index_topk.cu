@@ -1,0 +1,421 @@
+// index_topk.cu -- fused Index Branch kernel: Eq. 6 scores on tcgen05, causal
+// block max-pool in registers, Eq. 7 Top-k with the local block forced.
+//
+// Source: xllm-io paper review, "核心公式" (Eq. 6-7) and "4.1 Index & TopK
+// Kernel"; chlience notes 5.1.1 (local block takes one slot) and 5.4
+// (exp-free selection: rank raw scores).
+//
+// Design (sm_100a):
+//   * Rows of the MMA are (query, group) pairs: Q_idx is [N, H_kv, d_idx], so
+//     128 consecutive rows of the [N*H_kv, d_idx] view are 128/H_kv queries x
+//     all H_kv groups, and they all share the one index key head (Eq. 5).  A
+//     work unit is two such 128-row M-tiles; every 128-key K_idx tile streamed
+//     by TMA feeds two 128x128xd_idx UMMAs (A = Q_idx rows, B = K_idx rows,
+//     both K-major, fp32 accumulators in TMEM).
+//   * All queries of an M-tile live in one block c (128/H_kv divides B_k), so
+//     the non-local candidates are exactly blocks 0..c-1: every key tile is
+//     fully visible and needs no causal mask.  The local block is forced and
+//     needs no score at all.
+//   * Epilogue: one TMEM lane (= one row) per thread.  tcgen05.ld pulls the
+//     row's 128 scores, a 3-input max tree pools them per block, and a
+//     per-row min-heap of k-1 packed keys (score bits, inverted block index)
+//     in shared memory keeps the running Top-(k-1).  The root's score is
+//     cached in a register, so a block costs one compare unless it enters.
+//     The scale 1/sqrt(d_idx) is positive and is not applied: the order of
+//     the raw dot products is the order of Eq. 6's scores.
+//   * Warp roles: warp 0 = TMA producer, warp 1 = MMA issuer (and TMEM
+//     owner), warps 2..9 = epilogue (4 per M-tile; warp w reads TMEM lanes
+//     32*(w%4) .. +31).  TMEM holds 2 accumulator stages x 2 M-tiles x 128
+//     columns = 512 columns.
+//   * Persistent grid of one CTA per SM; units are visited longest-first in a
+//     snake order over CTAs to balance the causal triangle.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "msa_internal.h"
+
+namespace msa {
+namespace {
+
+constexpr int kThreads = 320;
+constexpr int kRows = 128;         // rows per M-tile (UMMA M)
+constexpr int kKeys = 128;         // keys per K_idx tile (UMMA N)
+constexpr int kEpiThreads = 256;   // 2 M-tiles x 128 rows
+constexpr uint32_t kTmemCols = 512;
+
+struct IndexParams {
+  int64_t N;
+  int H_kv, B_k, k;
+  int n_mtiles;
+  int n_units;
+  int32_t* idx_out;
+  DevStatus* status;
+};
+
+template <int D_IDX>
+struct IndexShape {
+  static constexpr int SWB = (D_IDX * 2 < 128) ? D_IDX * 2 : 128;  // swizzle span (bytes)
+  static constexpr int CH = D_IDX * 2 / SWB;                       // K chunks
+  static constexpr int CHE = SWB / 2;                              // elements per chunk
+  static constexpr int KSTEPS = SWB / 32;                          // UMMA K=16 steps per chunk
+  static constexpr uint32_t SWZ = (SWB == 128) ? SW_128B : SW_64B;
+  static constexpr int SBO = 8 * SWB;                              // 8-row atom
+  static constexpr int A_BYTES = kRows * D_IDX * 2;                // one M-tile
+  static constexpr int B_BYTES = kKeys * D_IDX * 2;                // one key tile
+  static constexpr int STAGES = (D_IDX == 128) ? 3 : 6;
+};
+
+__device__ __forceinline__ int unit_of(int round, int cta, int nctas) {
+  return round * nctas + ((round & 1) ? (nctas - 1 - cta) : cta);
+}
+
+// Number of 128-key tiles holding blocks 0..c-1 of an M-tile (0 if absent).
+__device__ __forceinline__ int mtile_ntiles(const IndexParams& p, int m, int* c_out) {
+  if (m >= p.n_mtiles) {
+    *c_out = 0;
+    return 0;
+  }
+  const int64_t i0 = (static_cast<int64_t>(m) * kRows) / p.H_kv;
+  const int c = static_cast<int>(i0 / p.B_k);
+  *c_out = c;
+  return static_cast<int>((static_cast<int64_t>(c) * p.B_k + kKeys - 1) / kKeys);
+}
+
+__device__ __forceinline__ uint32_t order_bits(float f) {
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float unorder_key(uint64_t key) {
+  if (key == 0) return -INFINITY;  // empty slot
+  const uint32_t o = static_cast<uint32_t>(key >> 32);
+  return __uint_as_float((o & 0x80000000u) ? (o & 0x7FFFFFFFu) : ~o);
+}
+
+template <int D_IDX>
+__global__ void __launch_bounds__(kThreads, 1)
+    index_topk_kernel(const __grid_constant__ CUtensorMap tm_q,
+                      const __grid_constant__ CUtensorMap tm_k, const IndexParams p) {
+  using S = IndexShape<D_IDX>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;                                   // 2 x A_BYTES
+  uint8_t* sB = sA + 2 * S::A_BYTES;                    // STAGES x B_BYTES
+  uint64_t* heap = reinterpret_cast<uint64_t*>(sB + S::STAGES * S::B_BYTES);
+  const int HS = p.k - 1;                               // heap size per row
+  uint64_t* bars = heap + static_cast<size_t>(kEpiThreads) * (HS > 0 ? HS : 1);
+  uint64_t* a_full = bars;
+  uint64_t* a_empty = bars + 1;
+  uint64_t* b_full = bars + 2;
+  uint64_t* b_empty = b_full + S::STAGES;
+  uint64_t* acc_full = b_empty + S::STAGES;
+  uint64_t* acc_empty = acc_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(a_full, 1);
+    mbar_init(a_empty, 1);
+    for (int s = 0; s < S::STAGES; ++s) {
+      mbar_init(&b_full[s], 1);
+      mbar_init(&b_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&acc_full[s], 1);
+      mbar_init(&acc_empty[s], 8);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int nctas = gridDim.x;
+  const int cta = blockIdx.x;
+
+  if (warp == 0) {
+    // ------------------------------------------------------- TMA producer --
+    if (lane == 0) {
+      uint32_t g = 0, ua = 0;
+      for (int round = 0;; ++round) {
+        const int u = unit_of(round, cta, nctas);
+        if (u >= p.n_units || *abort_flag) break;
+        const int v = p.n_units - 1 - u;  // longest first
+        int c0, c1;
+        const int nt0 = mtile_ntiles(p, 2 * v, &c0);
+        const int nt1 = mtile_ntiles(p, 2 * v + 1, &c1);
+        const int nt = nt0 > nt1 ? nt0 : nt1;
+        if (nt == 0) continue;
+        if (!mbar_wait(a_empty, (ua & 1) ^ 1, abort_flag, p.status, 10)) break;
+        mbar_arrive_expect_tx(a_full, 2 * S::A_BYTES);
+        for (int mt = 0; mt < 2; ++mt)
+          for (int c = 0; c < S::CH; ++c)
+            tma_load_2d(sA + mt * S::A_BYTES + c * kRows * S::SWB, &tm_q, a_full, c * S::CHE,
+                        (2 * v + mt) * kRows);
+        ++ua;
+        bool ok = true;
+        for (int t = 0; t < nt; ++t, ++g) {
+          const uint32_t st = g % S::STAGES;
+          if (!mbar_wait(&b_empty[st], ((g / S::STAGES) & 1) ^ 1, abort_flag, p.status, 11)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&b_full[st], S::B_BYTES);
+          for (int c = 0; c < S::CH; ++c)
+            tma_load_2d(sB + st * S::B_BYTES + c * kKeys * S::SWB, &tm_k, &b_full[st],
+                        c * S::CHE, t * kKeys);
+        }
+        if (!ok) break;
+      }
+    }
+  } else if (warp == 1) {
+    // -------------------------------------------------------- MMA issuer --
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(kRows, kKeys, 0, 0);
+      uint32_t g = 0, acnt = 0, ua = 0;
+      for (int round = 0;; ++round) {
+        const int u = unit_of(round, cta, nctas);
+        if (u >= p.n_units || *abort_flag) break;
+        const int v = p.n_units - 1 - u;
+        int c0, c1;
+        const int nt0 = mtile_ntiles(p, 2 * v, &c0);
+        const int nt1 = mtile_ntiles(p, 2 * v + 1, &c1);
+        const int nt = nt0 > nt1 ? nt0 : nt1;
+        if (nt == 0) continue;
+        if (!mbar_wait(a_full, ua & 1, abort_flag, p.status, 20)) break;
+        tc_fence_after();
+        bool ok = true;
+        for (int t = 0; t < nt; ++t, ++g, ++acnt) {
+          const uint32_t st = g % S::STAGES;
+          if (!mbar_wait(&b_full[st], (g / S::STAGES) & 1, abort_flag, p.status, 21)) {
+            ok = false;
+            break;
+          }
+          const uint32_t acc = acnt & 1;
+          if (!mbar_wait(&acc_empty[acc], ((acnt >> 1) & 1) ^ 1, abort_flag, p.status, 22)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          for (int mt = 0; mt < 2; ++mt) {
+            if (t >= (mt == 0 ? nt0 : nt1)) continue;
+            const uint32_t d_tmem = tmem_base + acc * 256 + mt * 128;
+            const uint32_t a_base = smem_u32(sA + mt * S::A_BYTES);
+            const uint32_t b_base = smem_u32(sB + st * S::B_BYTES);
+#pragma unroll
+            for (int c = 0; c < S::CH; ++c) {
+#pragma unroll
+              for (int s = 0; s < S::KSTEPS; ++s) {
+                const uint64_t ad =
+                    umma_desc(a_base + c * kRows * S::SWB + s * 32, 16, S::SBO, S::SWZ);
+                const uint64_t bd =
+                    umma_desc(b_base + c * kKeys * S::SWB + s * 32, 16, S::SBO, S::SWZ);
+                umma_bf16(d_tmem, ad, bd, idesc, (c | s) != 0);
+              }
+            }
+          }
+          umma_commit(&b_empty[st]);
+          umma_commit(&acc_full[acc]);
+        }
+        if (!ok) break;
+        umma_commit(a_empty);
+        ++ua;
+      }
+    }
+  } else {
+    // ---------------------------------------------------------- epilogue --
+    const int e = warp - 2;
+    const int mt = e >> 2;
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;      // TMEM lane = row of the M-tile
+    const int hrow = mt * kRows + row;        // heap column
+    const int per_tile = kKeys / p.B_k;       // blocks per key tile (1 or 2)
+    uint32_t acnt = 0;
+    for (int round = 0;; ++round) {
+      const int u = unit_of(round, cta, nctas);
+      if (u >= p.n_units || *abort_flag) break;
+      const int v = p.n_units - 1 - u;
+      int c0, c1;
+      const int nt0 = mtile_ntiles(p, 2 * v, &c0);
+      const int nt1 = mtile_ntiles(p, 2 * v + 1, &c1);
+      const int nt = nt0 > nt1 ? nt0 : nt1;
+      const int my_nt = mt == 0 ? nt0 : nt1;
+      const int my_c = mt == 0 ? c0 : c1;
+      for (int s = 0; s < HS; ++s) heap[s * kEpiThreads + hrow] = 0ull;
+      float root = HS > 0 ? -INFINITY : INFINITY;
+      bool ok = true;
+      for (int t = 0; t < nt; ++t, ++acnt) {
+        const uint32_t acc = acnt & 1;
+        if (!mbar_wait(&acc_full[acc], (acnt >> 1) & 1, abort_flag, p.status, 30)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t r0[32], r1[32], r2[32], r3[32];
+        const bool active = t < my_nt;
+        if (active) {
+          const uint32_t ta = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                              acc * 256 + mt * 128;
+          tmem_ld32(ta + 0, r0);
+          tmem_ld32(ta + 32, r1);
+          tmem_ld32(ta + 64, r2);
+          tmem_ld32(ta + 96, r3);
+          tmem_wait_ld();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[acc]);
+        if (!active) continue;
+        float m[2];
+        {
+          float x0 = __uint_as_float(r0[0]), x1 = __uint_as_float(r1[0]);
+          float x2 = __uint_as_float(r2[0]), x3 = __uint_as_float(r3[0]);
+#pragma unroll
+          for (int j = 1; j < 31; j += 2) {
+            x0 = fmax3(x0, __uint_as_float(r0[j]), __uint_as_float(r0[j + 1]));
+            x1 = fmax3(x1, __uint_as_float(r1[j]), __uint_as_float(r1[j + 1]));
+            x2 = fmax3(x2, __uint_as_float(r2[j]), __uint_as_float(r2[j + 1]));
+            x3 = fmax3(x3, __uint_as_float(r3[j]), __uint_as_float(r3[j + 1]));
+          }
+          x0 = fmaxf(x0, __uint_as_float(r0[31]));
+          x1 = fmaxf(x1, __uint_as_float(r1[31]));
+          x2 = fmaxf(x2, __uint_as_float(r2[31]));
+          x3 = fmaxf(x3, __uint_as_float(r3[31]));
+          if (per_tile == 1) {
+            m[0] = fmax3(x0, x1, fmaxf(x2, x3));
+            m[1] = -INFINITY;
+          } else {
+            m[0] = fmaxf(x0, x1);
+            m[1] = fmaxf(x2, x3);
+          }
+        }
+        for (int h = 0; h < per_tile; ++h) {
+          const int b = t * per_tile + h;
+          if (b >= my_c || !(m[h] > root)) continue;
+          // replace the root (worst kept) and sift down; ties -> lower block
+          const uint64_t key = (static_cast<uint64_t>(order_bits(m[h])) << 32) |
+                               static_cast<uint64_t>(0xFFFFFFFFu - static_cast<uint32_t>(b));
+          int pos = 0;
+          while (true) {
+            const int c1i = 2 * pos + 1;
+            if (c1i >= HS) break;
+            uint64_t km = heap[c1i * kEpiThreads + hrow];
+            int cm = c1i;
+            if (c1i + 1 < HS) {
+              const uint64_t k2 = heap[(c1i + 1) * kEpiThreads + hrow];
+              if (k2 < km) {
+                km = k2;
+                cm = c1i + 1;
+              }
+            }
+            if (km >= key) break;
+            heap[pos * kEpiThreads + hrow] = km;
+            pos = cm;
+          }
+          heap[pos * kEpiThreads + hrow] = key;
+          root = unorder_key(heap[hrow]);
+        }
+      }
+      if (!ok) break;
+      // -------------------------------------------------- write the row --
+      const int m_glob = 2 * v + mt;
+      const int64_t row_glob = static_cast<int64_t>(m_glob) * kRows + row;
+      if (m_glob < p.n_mtiles && row_glob < p.N * p.H_kv) {
+        int sel[32];
+        int n = 0;
+        sel[n++] = my_c;  // the local block (Eq. 7: always kept)
+        for (int s = 0; s < HS; ++s) {
+          const uint64_t key = heap[s * kEpiThreads + hrow];
+          if (key != 0ull) sel[n++] = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(key));
+        }
+        for (int a = 1; a < n; ++a) {  // ascending
+          const int x = sel[a];
+          int b = a - 1;
+          while (b >= 0 && sel[b] > x) {
+            sel[b + 1] = sel[b];
+            --b;
+          }
+          sel[b + 1] = x;
+        }
+        int32_t* out = p.idx_out + row_glob * p.k;
+        for (int s = 0; s < p.k; ++s) out[s] = s < n ? sel[s] : -1;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+template <int D_IDX>
+size_t index_smem_bytes(int k) {
+  using S = IndexShape<D_IDX>;
+  const int hs = k - 1 > 0 ? k - 1 : 1;
+  return 1024 + 2 * S::A_BYTES + S::STAGES * S::B_BYTES + static_cast<size_t>(kEpiThreads) * hs * 8 +
+         (4 + 2 * S::STAGES + 2) * 8 + 16;
+}
+
+template <int D_IDX>
+cudaError_t launch_typed(const IndexLaunch& a, cudaStream_t stream) {
+  using S = IndexShape<D_IDX>;
+  CUtensorMap tq, tk;
+  {
+    const uint64_t dims[2] = {static_cast<uint64_t>(D_IDX), static_cast<uint64_t>(a.N) * a.H_kv};
+    const uint64_t strides[1] = {static_cast<uint64_t>(D_IDX) * 2};
+    const uint32_t box[2] = {static_cast<uint32_t>(S::CHE), static_cast<uint32_t>(kRows)};
+    if (!make_tmap_bf16(&tq, a.q_idx, 2, dims, strides, box, S::SWB)) return cudaErrorInvalidValue;
+  }
+  {
+    const uint64_t dims[2] = {static_cast<uint64_t>(D_IDX), static_cast<uint64_t>(a.N)};
+    const uint64_t strides[1] = {static_cast<uint64_t>(D_IDX) * 2};
+    const uint32_t box[2] = {static_cast<uint32_t>(S::CHE), static_cast<uint32_t>(kKeys)};
+    if (!make_tmap_bf16(&tk, a.k_idx, 2, dims, strides, box, S::SWB)) return cudaErrorInvalidValue;
+  }
+  IndexParams p;
+  p.N = a.N;
+  p.H_kv = a.H_kv;
+  p.B_k = a.B_k;
+  p.k = a.k;
+  p.n_mtiles = static_cast<int>((a.N * a.H_kv + kRows - 1) / kRows);
+  p.n_units = (p.n_mtiles + 1) / 2;
+  p.idx_out = a.idx_out;
+  p.status = a.status;
+  const size_t smem = index_smem_bytes<D_IDX>(a.k);
+  cudaError_t e = cudaFuncSetAttribute(index_topk_kernel<D_IDX>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  int grid = num_sms();
+  if (grid > p.n_units) grid = p.n_units;
+  if (grid < 1) grid = 1;
+  prof_begin("index_topk", stream);
+  index_topk_kernel<D_IDX><<<grid, kThreads, smem, stream>>>(tq, tk, p);
+  prof_end(stream);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_index_topk(const IndexLaunch& a, cudaStream_t s) {
+  switch (a.d_idx) {
+    case 32: return launch_typed<32>(a, s);
+    case 64: return launch_typed<64>(a, s);
+    case 128: return launch_typed<128>(a, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace msa

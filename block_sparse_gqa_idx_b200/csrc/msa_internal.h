@@ -1,0 +1,72 @@
+// msa_internal.h -- launchers shared between the C-ABI layer and the kernels.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "msa_common.cuh"
+
+namespace msa {
+
+// Host: encode a 2D/3D bf16 tiled tensor map (dims/strides innermost first).
+bool make_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                    const uint64_t* strides_bytes, const uint32_t* box, int swizzle_bytes);
+
+int num_sms();
+
+// Optional per-kernel timing (msa_profile_enable): when on, prof_begin/prof_end
+// record a CUDA event pair around each kernel launch on its stream.
+void prof_begin(const char* name, cudaStream_t s);
+void prof_end(cudaStream_t s);
+
+struct IndexLaunch {
+  const void* q_idx;
+  const void* k_idx;
+  int32_t* idx_out;
+  int64_t N;
+  int H_kv, d_idx, B_k, k;
+  DevStatus* status;
+};
+cudaError_t launch_index_topk(const IndexLaunch& a, cudaStream_t s);
+
+struct AttnLaunch {
+  const void* q;
+  const void* k;
+  const void* v;
+  const int32_t* idx;
+  void* o;
+  float* lse;
+  int64_t N;
+  int H_q, H_kv, d_h, B_k, kk;
+  float scale;
+  void* ws;  // device workspace after the status word
+  size_t ws_bytes;
+  DevStatus* status;
+};
+size_t attn_workspace_bytes(int64_t N, int H_q, int H_kv, int d_h, int B_k, int kk);
+cudaError_t launch_sparse_attn(const AttnLaunch& a, cudaStream_t s);
+
+struct DecodeLaunch {
+  const void* q;
+  const void* q_idx;
+  const void* k_new;
+  const void* v_new;
+  const void* k_idx_new;
+  void* k_cache;
+  void* v_cache;
+  void* k_idx_cache;
+  int32_t* seq_len;
+  void* o;
+  int32_t* idx_out;
+  int S;
+  int64_t L_max;
+  int H_q, H_kv, d_h, d_idx, B_k, kk;
+  float scale;
+  void* ws;
+  size_t ws_bytes;
+  DevStatus* status;
+};
+size_t decode_workspace_bytes(int S, int64_t L_max, int H_q, int H_kv, int d_h, int B_k, int kk);
+cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t s);
+
+}  // namespace msa

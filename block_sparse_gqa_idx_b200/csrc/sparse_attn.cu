@@ -1,0 +1,678 @@
+// sparse_attn.cu -- Main Branch (Eq. 8 with the causal rule of Eq. 1) as a
+// KV-outer block-sparse attention on tcgen05, in three steps per query chunk:
+//
+//   1. inverse index: for every (group r, block b) the list of selection slots
+//      (query i, slot s) that chose b -- count, exclusive scan, scatter.  The
+//      scan also cuts each list into tiles of Tq queries (Tq * rows-per-query
+//      = 128 MMA rows), so hot blocks are split over many CTAs with every
+//      output slot fixed in advance: no atomics on the outputs.
+//   2. phase 1: one tile = one KV block (K_b, V_b by TMA) and the gathered
+//      query rows that selected it (one TMA box per query: its group's heads).
+//      S = Q K_b^T (UMMA, fp32 in TMEM) -> causal mask (only rows whose own
+//      block is b) -> softmax in registers (one row per thread, exp2) -> P
+//      (bf16) to shared memory -> O = P V_b (UMMA) -> O / l written as an fp16
+//      partial with its natural-log LSE into the row's slot.
+//   3. merge: per (query, head), LSE-weighted sum of its partials (split-K
+//      softmax normalisation), bf16 output + fp32 LSE.
+//
+// Source: xllm-io paper review, "核心公式" Eq. 8 and "4.2 Sparse Attention
+// Kernel" (KV-outer with query gather, two-phase forward: partial outputs
+// then a combine pass); chlience notes 5.4 (pre-scheduled tile chunking,
+// slots assigned ahead, two-phase combine).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "msa_internal.h"
+
+namespace msa {
+namespace {
+
+constexpr int kThreads = 320;
+constexpr int kRowsPerTile = 128;
+constexpr int kMaxChunk = 1 << 17;  // queries per chunk (bounds the partial buffer)
+
+// Rows per query inside an MMA tile: the group's G heads, or 8 heads (one
+// 128-byte swizzle atom) when G < 8 (the extra heads are computed and dropped).
+inline int rows_per_query(int G) { return G >= 8 ? G : 8; }
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+struct ChunkBufs {
+  int32_t* counts;    // [nkeys]
+  int32_t* offsets;   // [nkeys + 1]
+  int32_t* tile_off;  // [nkeys + 1]
+  int32_t* cursor;    // [nkeys]
+  int32_t* n_tiles;   // [1]
+  uint32_t* entries;  // [Nc * H_kv * k]
+  __half* part_o;     // [Nc * H_kv * k, G, d_h]
+  float* part_lse;    // [Nc * H_kv * k, G]
+};
+
+ChunkBufs carve(void* ws, int64_t Nc, int H_q, int H_kv, int d_h, int kk, int64_t nkeys,
+                size_t* total) {
+  ChunkBufs c;
+  uint8_t* p = static_cast<uint8_t*>(ws);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    uint8_t* r = p ? p + off : nullptr;
+    off += align256(bytes);
+    return r;
+  };
+  const int G = H_q / H_kv;
+  const int64_t slots = Nc * H_kv * kk;
+  c.counts = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * nkeys));
+  c.cursor = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * nkeys));
+  c.offsets = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * (nkeys + 1)));
+  c.tile_off = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * (nkeys + 1)));
+  c.n_tiles = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * 4));
+  c.entries = reinterpret_cast<uint32_t*>(take(sizeof(uint32_t) * slots));
+  c.part_lse = reinterpret_cast<float*>(take(sizeof(float) * slots * G));
+  c.part_o = reinterpret_cast<__half*>(take(sizeof(__half) * slots * G * d_h));
+  *total = off;
+  return c;
+}
+
+int64_t chunk_len(int64_t N, int B_k) {
+  int64_t c = N < kMaxChunk ? N : kMaxChunk;
+  return (c + B_k - 1) / B_k * B_k;
+}
+
+// ------------------------------------------------------------------ step 1 --
+struct InvParams {
+  const int32_t* idx;
+  int64_t q0, nq;  // chunk [q0, q0 + nq)
+  int H_kv, B_k, kk;
+  int64_t B;
+  int Tq;
+  ChunkBufs c;
+  DevStatus* status;
+};
+
+// Thread order: slot-major, then group, then query, so lanes of a warp read the
+// same slot of consecutive queries -- hot blocks (a sink, the previous block)
+// collapse into one aggregated atomic per warp.
+template <bool SCATTER>
+__global__ void inv_index_kernel(const InvParams p) {
+  const int64_t total = p.nq * p.H_kv * p.kk;
+  for (int64_t t = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; t - threadIdx.x < total;
+       t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    int key = -1;
+    uint32_t slot = 0;
+    if (t < total) {
+      const int s = static_cast<int>(t / (p.nq * p.H_kv));
+      const int64_t rem = t % (p.nq * p.H_kv);
+      const int r = static_cast<int>(rem / p.nq);
+      const int64_t il = rem % p.nq;
+      const int64_t i = p.q0 + il;
+      const int32_t b = p.idx[(i * p.H_kv + r) * p.kk + s];
+      const int64_t b_i = i / p.B_k;
+      if (b < -1 || b >= p.B) {
+        if (!SCATTER) report(p.status, DEV_ERR_BAD_INDEX, 40, static_cast<int>(i), b);
+      } else if (b >= 0 && b <= b_i) {
+        key = r * static_cast<int>(p.B) + b;
+        slot = static_cast<uint32_t>((il * p.H_kv + r) * p.kk + s);
+      }
+    }
+    const unsigned active = __ballot_sync(0xFFFFFFFFu, key >= 0);
+    if (key >= 0) {
+      const unsigned peers = __match_any_sync(active, key);
+      const int leader = __ffs(peers) - 1;
+      const int lane = threadIdx.x & 31;
+      const int rank = __popc(peers & ((1u << lane) - 1));
+      if (!SCATTER) {
+        if (lane == leader) atomicAdd(&p.c.counts[key], __popc(peers));
+      } else {
+        int base = 0;
+        if (lane == leader) base = atomicAdd(&p.c.cursor[key], __popc(peers));
+        base = __shfl_sync(peers, base, leader);
+        p.c.entries[base + rank] = slot;
+      }
+    }
+  }
+}
+
+// Single CTA: exclusive scans of the counts and of the per-key tile counts.
+__global__ void __launch_bounds__(1024) inv_scan_kernel(const InvParams p) {
+  __shared__ int32_t warp_sum[2][32];
+  const int64_t nkeys = p.H_kv * p.B;
+  const int per = static_cast<int>((nkeys + blockDim.x - 1) / blockDim.x);
+  const int64_t beg = static_cast<int64_t>(threadIdx.x) * per;
+  int32_t s_cnt = 0, s_til = 0;
+  for (int j = 0; j < per; ++j) {
+    const int64_t e = beg + j;
+    if (e < nkeys) {
+      const int32_t c = p.c.counts[e];
+      s_cnt += c;
+      s_til += (c + p.Tq - 1) / p.Tq;
+    }
+  }
+  // block-wide exclusive scan of (s_cnt, s_til)
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  int32_t a = s_cnt, b = s_til;
+  for (int o = 1; o < 32; o <<= 1) {
+    const int32_t ya = __shfl_up_sync(0xFFFFFFFFu, a, o);
+    const int32_t yb = __shfl_up_sync(0xFFFFFFFFu, b, o);
+    if (lane >= o) {
+      a += ya;
+      b += yb;
+    }
+  }
+  if (lane == 31) {
+    warp_sum[0][w] = a;
+    warp_sum[1][w] = b;
+  }
+  __syncthreads();
+  if (w == 0) {
+    int32_t x = lane < static_cast<int>(blockDim.x >> 5) ? warp_sum[0][lane] : 0;
+    int32_t y = lane < static_cast<int>(blockDim.x >> 5) ? warp_sum[1][lane] : 0;
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t yx = __shfl_up_sync(0xFFFFFFFFu, x, o);
+      const int32_t yy = __shfl_up_sync(0xFFFFFFFFu, y, o);
+      if (lane >= o) {
+        x += yx;
+        y += yy;
+      }
+    }
+    warp_sum[0][lane] = x;
+    warp_sum[1][lane] = y;
+  }
+  __syncthreads();
+  int32_t run_cnt = a - s_cnt + (w > 0 ? warp_sum[0][w - 1] : 0);
+  int32_t run_til = b - s_til + (w > 0 ? warp_sum[1][w - 1] : 0);
+  for (int j = 0; j < per; ++j) {
+    const int64_t e = beg + j;
+    if (e < nkeys) {
+      const int32_t c = p.c.counts[e];
+      p.c.offsets[e] = run_cnt;
+      p.c.cursor[e] = run_cnt;
+      p.c.tile_off[e] = run_til;
+      run_cnt += c;
+      run_til += (c + p.Tq - 1) / p.Tq;
+    }
+  }
+  if (threadIdx.x == blockDim.x - 1) {
+    p.c.offsets[nkeys] = run_cnt;
+    p.c.tile_off[nkeys] = run_til;
+    p.c.n_tiles[0] = run_til;
+  }
+}
+
+// ------------------------------------------------------------------ step 2 --
+struct P1Params {
+  int64_t q0;
+  int H_q, H_kv, B_k, kk, G, R, Tq;
+  int64_t nkeys;
+  float scale_log2;  // softmax scale * log2(e)
+  float scale;
+  ChunkBufs c;
+  DevStatus* status;
+};
+
+template <int D_H, int B_K>
+struct P1Shape {
+  static constexpr int QP_BYTES = kRowsPerTile * (D_H > B_K ? D_H : B_K) * 2;  // Q, later P
+  static constexpr int K_BYTES = B_K * D_H * 2;
+  static constexpr int V_BYTES = B_K * D_H * 2;
+  static constexpr int STAGE_BYTES = QP_BYTES + K_BYTES + V_BYTES;
+  static constexpr int DCH = D_H / 64;  // 128-byte chunks along d
+  static constexpr int PCH = B_K / 64;  // 128-byte chunks along keys (P)
+  static constexpr uint32_t TM_S = 0, TM_O = 128;  // column offsets inside a stage
+};
+
+struct TileInfo {
+  int r, b, len;
+  int pad;
+  uint32_t slot[128];
+};
+
+__device__ __forceinline__ int find_key(const int32_t* tile_off, int64_t nkeys, int t) {
+  int64_t lo = 0, hi = nkeys;  // tile_off[lo] <= t < tile_off[hi]
+  while (hi - lo > 1) {
+    const int64_t mid = (lo + hi) >> 1;
+    if (tile_off[mid] <= t) lo = mid;
+    else hi = mid;
+  }
+  return static_cast<int>(lo);
+}
+
+template <int D_H, int B_K>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_phase1_kernel(const __grid_constant__ CUtensorMap tm_q,
+                       const __grid_constant__ CUtensorMap tm_k,
+                       const __grid_constant__ CUtensorMap tm_v, const P1Params p) {
+  using SH = P1Shape<D_H, B_K>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  TileInfo* info = reinterpret_cast<TileInfo*>(smem + 2 * SH::STAGE_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(info + 2);
+  uint64_t* full = bars;          // [2] TMA landed
+  uint64_t* empty = bars + 2;     // [2] stage smem free (O MMA done)
+  uint64_t* s_full = bars + 4;    // [2] S in TMEM
+  uint64_t* p_full = bars + 6;    // [2] P in smem (S read)
+  uint64_t* o_full = bars + 8;    // [2] O in TMEM
+  uint64_t* o_empty = bars + 10;  // [2] O read
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+      mbar_init(&s_full[s], 1);
+      mbar_init(&p_full[s], 4);
+      mbar_init(&o_full[s], 1);
+      mbar_init(&o_empty[s], 4);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int n_tiles = p.c.n_tiles[0];
+  const int nctas = gridDim.x;
+
+  if (warp == 0) {
+    // ------------------------------------------------------- TMA producer --
+    if (lane == 0) {
+      prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_v);
+      int n = 0;
+      for (int t = blockIdx.x; t < n_tiles; t += nctas, ++n) {
+        const int st = n & 1;
+        if (!mbar_wait(&empty[st], ((n >> 1) & 1) ^ 1, abort_flag, p.status, 50)) break;
+        const int key = find_key(p.c.tile_off, p.nkeys, t);
+        const int lt = t - p.c.tile_off[key];
+        const int cnt = p.c.offsets[key + 1] - p.c.offsets[key];
+        const int len = min(p.Tq, cnt - lt * p.Tq);
+        const int r = key / static_cast<int>(p.nkeys / p.H_kv);
+        const int b = key - r * static_cast<int>(p.nkeys / p.H_kv);
+        TileInfo& ti = info[st];
+        ti.r = r;
+        ti.b = b;
+        ti.len = len;
+        const uint32_t* ent = p.c.entries + p.c.offsets[key] + lt * p.Tq;
+        for (int q = 0; q < len; ++q) ti.slot[q] = ent[q];
+        uint8_t* sQ = smem + st * SH::STAGE_BYTES;
+        uint8_t* sK = sQ + SH::QP_BYTES;
+        uint8_t* sV = sK + SH::K_BYTES;
+        mbar_arrive_expect_tx(&full[st], SH::K_BYTES + SH::V_BYTES + len * p.R * D_H * 2);
+        const int h0 = p.G >= 8 ? r * p.G : (r * p.G / 8) * 8;
+        for (int c = 0; c < SH::DCH; ++c) {
+          tma_load_3d(sK + c * B_K * 128, &tm_k, &full[st], c * 64, r, b * B_K);
+          tma_load_3d(sV + c * B_K * 128, &tm_v, &full[st], c * 64, r, b * B_K);
+        }
+        const int per_q = p.H_kv * p.kk;
+        for (int q = 0; q < len; ++q) {
+          const int i = static_cast<int>(p.q0 + ti.slot[q] / per_q);
+          for (int c = 0; c < SH::DCH; ++c)
+            tma_load_3d(sQ + c * kRowsPerTile * 128 + q * p.R * 128, &tm_q, &full[st], c * 64,
+                        h0, i);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // -------------------------------------------------------- MMA issuer --
+    // Software-pipelined: S of tile n+1 is issued before waiting for the
+    // softmax of tile n, so the tensor core works while P is being built.
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, B_K, 0, 0);
+      constexpr uint32_t idesc_o = idesc_bf16_f32(128, D_H, 0, 1);
+      auto issue_s = [&](int n) -> bool {
+        const int st = n & 1;
+        if (!mbar_wait(&full[st], (n >> 1) & 1, abort_flag, p.status, 60)) return false;
+        tc_fence_after();
+        uint8_t* sQ = smem + st * SH::STAGE_BYTES;
+        const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sQ + SH::QP_BYTES);
+        const uint32_t tS = tmem_base + st * 256 + SH::TM_S;
+#pragma unroll
+        for (int c = 0; c < SH::DCH; ++c)
+#pragma unroll
+          for (int s = 0; s < 4; ++s) {
+            const uint64_t ad =
+                umma_desc(q_base + c * kRowsPerTile * 128 + s * 32, 16, 1024, SW_128B);
+            const uint64_t bd = umma_desc(k_base + c * B_K * 128 + s * 32, 16, 1024, SW_128B);
+            umma_bf16(tS, ad, bd, idesc_s, (c | s) != 0);
+          }
+        umma_commit(&s_full[st]);
+        return true;
+      };
+      const int my_tiles = blockIdx.x < n_tiles ? (n_tiles - 1 - blockIdx.x) / nctas + 1 : 0;
+      bool ok = my_tiles == 0 || issue_s(0);
+      for (int n = 0; ok && n < my_tiles; ++n) {
+        const int st = n & 1;
+        const uint32_t ph = (n >> 1) & 1;
+        // the S accumulator of stage (n+1)&1 was last read by the softmax of
+        // tile n-1, whose p_full was waited for in the previous iteration
+        if (n + 1 < my_tiles && !issue_s(n + 1)) break;
+        if (!mbar_wait(&p_full[st], ph, abort_flag, p.status, 61)) break;
+        if (!mbar_wait(&o_empty[st], ph ^ 1, abort_flag, p.status, 62)) break;
+        tc_fence_after();
+        uint8_t* sQ = smem + st * SH::STAGE_BYTES;
+        const uint32_t q_base = smem_u32(sQ);
+        const uint32_t v_base = smem_u32(sQ + SH::QP_BYTES + SH::K_BYTES);
+        const uint32_t tO = tmem_base + st * 256 + SH::TM_O;
+#pragma unroll
+        for (int c = 0; c < SH::PCH; ++c)
+#pragma unroll
+          for (int s = 0; s < 4; ++s) {
+            // P: K-major (keys contiguous), chunk c = keys [64c, 64c+64)
+            const uint64_t ad =
+                umma_desc(q_base + c * kRowsPerTile * 128 + s * 32, 16, 1024, SW_128B);
+            // V: MN-major (d contiguous); 16 keys = two 8-key groups = 2048 B
+            const uint64_t bd = umma_desc(v_base + (c * 4 + s) * 2048, B_K * 128, 1024, SW_128B);
+            umma_bf16(tO, ad, bd, idesc_o, (c | s) != 0);
+          }
+        umma_commit(&o_full[st]);
+        umma_commit(&empty[st]);
+      }
+    }
+  } else {
+    // ------------------------------------------ softmax + epilogue groups --
+    const int grp = (warp - 2) >> 2;  // handles local tiles n with n % 2 == grp
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const int q_local = row / p.R;
+    const int hrow = row - q_local * p.R;
+    const int per_q = p.H_kv * p.kk;
+    int n = grp;
+    for (int t = blockIdx.x + grp * nctas; t < n_tiles; t += 2 * nctas, n += 2) {
+      const int st = grp;
+      const uint32_t ph = (n >> 1) & 1;
+      uint8_t* sP = smem + st * SH::STAGE_BYTES;
+      const uint32_t tS = tmem_base + st * 256 + SH::TM_S + (static_cast<uint32_t>(quarter * 32) << 16);
+      const uint32_t tO = tmem_base + st * 256 + SH::TM_O + (static_cast<uint32_t>(quarter * 32) << 16);
+      if (!mbar_wait(&s_full[st], ph, abort_flag, p.status, 70)) break;
+      // full[st] cannot advance before this group's p_full, so this wait
+      // returns at once; it orders the producer's TileInfo writes before reads
+      if (!mbar_wait(&full[st], ph, abort_flag, p.status, 72)) break;
+      tc_fence_after();
+      const int ti_r = info[st].r, ti_b = info[st].b, ti_len = info[st].len;
+      const bool live = q_local < ti_len;
+      const uint32_t slot = live ? info[st].slot[q_local] : 0u;
+      const int64_t i = p.q0 + slot / per_q;
+      // ---- softmax over the block's keys (exp2 with the scale folded in)
+      float sv[B_K];
+#pragma unroll
+      for (int c = 0; c < B_K / 32; ++c) {
+        uint32_t r32[32];
+        tmem_ld32(tS + c * 32, r32);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) sv[c * 32 + j] = __uint_as_float(r32[j]);
+      }
+      const int64_t j0 = static_cast<int64_t>(ti_b) * B_K;
+      if (j0 + B_K - 1 > i) {  // the query's own block: causal rule j <= i
+#pragma unroll
+        for (int j = 0; j < B_K; ++j)
+          if (j0 + j > i) sv[j] = -INFINITY;
+      }
+      float mx = sv[0];
+#pragma unroll
+      for (int j = 1; j + 1 < B_K; j += 2) mx = fmax3(mx, sv[j], sv[j + 1]);
+      mx = fmaxf(mx, sv[B_K - 1]);
+      const float mscaled = mx * p.scale_log2;
+      float l = 0.0f;
+#pragma unroll
+      for (int j = 0; j < B_K; ++j) {
+        const float e = exp2f(fmaf(sv[j], p.scale_log2, -mscaled));
+        sv[j] = e;
+        l += e;
+      }
+      // P (bf16) into the stage's Q buffer, K-major 128B-swizzled rows
+#pragma unroll
+      for (int c = 0; c < B_K / 8; ++c) {
+        uint4 w;
+        __nv_bfloat162 h0 = __floats2bfloat162_rn(sv[c * 8 + 0], sv[c * 8 + 1]);
+        __nv_bfloat162 h1 = __floats2bfloat162_rn(sv[c * 8 + 2], sv[c * 8 + 3]);
+        __nv_bfloat162 h2 = __floats2bfloat162_rn(sv[c * 8 + 4], sv[c * 8 + 5]);
+        __nv_bfloat162 h3 = __floats2bfloat162_rn(sv[c * 8 + 6], sv[c * 8 + 7]);
+        w.x = *reinterpret_cast<uint32_t*>(&h0);
+        w.y = *reinterpret_cast<uint32_t*>(&h1);
+        w.z = *reinterpret_cast<uint32_t*>(&h2);
+        w.w = *reinterpret_cast<uint32_t*>(&h3);
+        const int kc = c >> 3, j16 = c & 7;
+        uint8_t* dst = sP + kc * kRowsPerTile * 128 + row * 128 + ((j16 ^ (row & 7)) << 4);
+        *reinterpret_cast<uint4*>(dst) = w;
+      }
+      fence_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[st]);
+      // ---- O = P V; write O / l as an fp16 partial and lse into the slot
+      if (!mbar_wait(&o_full[st], ph, abort_flag, p.status, 71)) break;
+      tc_fence_after();
+      const int goff = p.G >= 8 ? 0 : (ti_r * p.G) % 8;  // group's first head in the box
+      const bool useful = live && hrow >= goff && hrow < goff + p.G;
+      const int g = hrow - goff;
+      __half* dst = p.c.part_o + (static_cast<int64_t>(slot) * p.G + g) * D_H;
+      const float inv_l = 1.0f / l;
+#pragma unroll
+      for (int c = 0; c < D_H / 32; ++c) {
+        uint32_t r32[32];
+        tmem_ld32(tO + c * 32, r32);
+        tmem_wait_ld();
+        if (useful) {
+#pragma unroll
+          for (int j = 0; j < 32; j += 8) {
+            uint4 w;
+            __half2 a0 = __floats2half2_rn(__uint_as_float(r32[j + 0]) * inv_l, __uint_as_float(r32[j + 1]) * inv_l);
+            __half2 a1 = __floats2half2_rn(__uint_as_float(r32[j + 2]) * inv_l, __uint_as_float(r32[j + 3]) * inv_l);
+            __half2 a2 = __floats2half2_rn(__uint_as_float(r32[j + 4]) * inv_l, __uint_as_float(r32[j + 5]) * inv_l);
+            __half2 a3 = __floats2half2_rn(__uint_as_float(r32[j + 6]) * inv_l, __uint_as_float(r32[j + 7]) * inv_l);
+            w.x = *reinterpret_cast<uint32_t*>(&a0);
+            w.y = *reinterpret_cast<uint32_t*>(&a1);
+            w.z = *reinterpret_cast<uint32_t*>(&a2);
+            w.w = *reinterpret_cast<uint32_t*>(&a3);
+            *reinterpret_cast<uint4*>(dst + c * 32 + j) = w;
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&o_empty[st]);
+      if (useful) p.c.part_lse[static_cast<int64_t>(slot) * p.G + g] = mx * p.scale + logf(l);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+// ------------------------------------------------------------------ step 3 --
+struct MergeParams {
+  const int32_t* idx;
+  __nv_bfloat16* o;
+  float* lse;
+  int64_t q0, nq;
+  int H_q, H_kv, kk, G, B_k;
+  ChunkBufs c;
+};
+
+// One warp per (query, head): LSE-weighted merge of the row's partials.
+template <int D_H>
+__global__ void __launch_bounds__(256) attn_merge_kernel(const MergeParams p) {
+  constexpr int PER = D_H / 32;  // elements per lane
+  const int lane = threadIdx.x & 31;
+  const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  if (row >= p.nq * p.H_q) return;
+  const int64_t il = row / p.H_q;
+  const int h = static_cast<int>(row - il * p.H_q);
+  const int r = h / p.G, g = h - r * p.G;
+  const int64_t i = p.q0 + il;
+  const int64_t b_i = i / p.B_k;
+  int32_t myb = -1;
+  if (lane < p.kk) myb = p.idx[(i * p.H_kv + r) * p.kk + lane];
+  const unsigned use = __ballot_sync(0xFFFFFFFFu, lane < p.kk && myb >= 0 && myb <= b_i);
+  float m = -INFINITY, wsum = 0.0f;
+  float acc[PER];
+#pragma unroll
+  for (int e = 0; e < PER; ++e) acc[e] = 0.0f;
+  unsigned rest = use;
+  while (rest) {
+    const int s = __ffs(rest) - 1;
+    rest &= rest - 1;
+    const int64_t slot = (il * p.H_kv + r) * p.kk + s;
+    const float ls = p.c.part_lse[slot * p.G + g];
+    const __half* src = p.c.part_o + (slot * p.G + g) * D_H + lane * PER;
+    float x[PER];
+#pragma unroll
+    for (int e = 0; e < PER; e += 2) {
+      const float2 a = __half22float2(*reinterpret_cast<const __half2*>(src + e));
+      x[e] = a.x;
+      x[e + 1] = a.y;
+    }
+    const float mn = fmaxf(m, ls);
+    const float a_old = __expf(m - mn);
+    const float a_new = __expf(ls - mn);
+#pragma unroll
+    for (int e = 0; e < PER; ++e) acc[e] = acc[e] * a_old + x[e] * a_new;
+    wsum = wsum * a_old + a_new;
+    m = mn;
+  }
+  __nv_bfloat16* dst = p.o + (i * p.H_q + h) * static_cast<int64_t>(D_H) + lane * PER;
+  const float inv = wsum > 0.0f ? 1.0f / wsum : 0.0f;
+#pragma unroll
+  for (int e = 0; e < PER; e += 2)
+    *reinterpret_cast<__nv_bfloat162*>(dst + e) = __floats2bfloat162_rn(acc[e] * inv, acc[e + 1] * inv);
+  if (p.lse != nullptr && lane == 0) p.lse[i * p.H_q + h] = use ? m + logf(wsum) : -INFINITY;
+}
+
+template <int D_H, int B_K>
+size_t p1_smem_bytes() {
+  using SH = P1Shape<D_H, B_K>;
+  return 1024 + 2 * SH::STAGE_BYTES + 2 * sizeof(TileInfo) + 12 * 8 + 16;
+}
+
+template <int D_H, int B_K>
+cudaError_t launch_typed(const AttnLaunch& a, cudaStream_t stream) {
+  const int G = a.H_q / a.H_kv;
+  const int R = rows_per_query(G);
+  const int Tq = kRowsPerTile / R;
+  const int64_t B = (a.N + a.B_k - 1) / a.B_k;
+  const int64_t nkeys = a.H_kv * B;
+  const int64_t Nc = chunk_len(a.N, a.B_k);
+  size_t need = 0;
+  ChunkBufs c = carve(a.ws, Nc, a.H_q, a.H_kv, a.d_h, a.kk, nkeys, &need);
+  if (need > a.ws_bytes) return cudaErrorInvalidValue;
+
+  CUtensorMap tq, tk, tv;
+  {
+    const uint64_t dims[3] = {static_cast<uint64_t>(D_H), static_cast<uint64_t>(a.H_q),
+                              static_cast<uint64_t>(a.N)};
+    const uint64_t strides[2] = {static_cast<uint64_t>(D_H) * 2,
+                                 static_cast<uint64_t>(a.H_q) * D_H * 2};
+    const uint32_t box[3] = {64, static_cast<uint32_t>(R), 1};
+    if (!make_tmap_bf16(&tq, a.q, 3, dims, strides, box, 128)) return cudaErrorInvalidValue;
+  }
+  {
+    const uint64_t dims[3] = {static_cast<uint64_t>(D_H), static_cast<uint64_t>(a.H_kv),
+                              static_cast<uint64_t>(a.N)};
+    const uint64_t strides[2] = {static_cast<uint64_t>(D_H) * 2,
+                                 static_cast<uint64_t>(a.H_kv) * D_H * 2};
+    const uint32_t box[3] = {64, 1, static_cast<uint32_t>(B_K)};
+    if (!make_tmap_bf16(&tk, a.k, 3, dims, strides, box, 128)) return cudaErrorInvalidValue;
+    if (!make_tmap_bf16(&tv, a.v, 3, dims, strides, box, 128)) return cudaErrorInvalidValue;
+  }
+  const size_t smem = p1_smem_bytes<D_H, B_K>();
+  cudaError_t e = cudaFuncSetAttribute(attn_phase1_kernel<D_H, B_K>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  const int sms = num_sms();
+
+  for (int64_t q0 = 0; q0 < a.N; q0 += Nc) {
+    const int64_t nq = (a.N - q0) < Nc ? (a.N - q0) : Nc;
+    e = cudaMemsetAsync(c.counts, 0, sizeof(int32_t) * nkeys, stream);
+    if (e != cudaSuccess) return e;
+    InvParams ip;
+    ip.idx = a.idx;
+    ip.q0 = q0;
+    ip.nq = nq;
+    ip.H_kv = a.H_kv;
+    ip.B_k = a.B_k;
+    ip.kk = a.kk;
+    ip.B = B;
+    ip.Tq = Tq;
+    ip.c = c;
+    ip.status = a.status;
+    const int64_t total = nq * a.H_kv * a.kk;
+    int blocks = static_cast<int>((total + 255) / 256);
+    if (blocks > sms * 16) blocks = sms * 16;
+    prof_begin("inv_count", stream);
+    inv_index_kernel<false><<<blocks, 256, 0, stream>>>(ip);
+    prof_end(stream);
+    prof_begin("inv_scan", stream);
+    inv_scan_kernel<<<1, 1024, 0, stream>>>(ip);
+    prof_end(stream);
+    prof_begin("inv_scatter", stream);
+    inv_index_kernel<true><<<blocks, 256, 0, stream>>>(ip);
+    prof_end(stream);
+
+    P1Params pp;
+    pp.q0 = q0;
+    pp.H_q = a.H_q;
+    pp.H_kv = a.H_kv;
+    pp.B_k = a.B_k;
+    pp.kk = a.kk;
+    pp.G = G;
+    pp.R = R;
+    pp.Tq = Tq;
+    pp.nkeys = nkeys;
+    pp.scale = a.scale;
+    pp.scale_log2 = a.scale * 1.4426950408889634f;
+    pp.c = c;
+    pp.status = a.status;
+    prof_begin("attn_phase1", stream);
+    attn_phase1_kernel<D_H, B_K><<<sms, kThreads, smem, stream>>>(tq, tk, tv, pp);
+    prof_end(stream);
+
+    MergeParams mp;
+    mp.idx = a.idx;
+    mp.o = static_cast<__nv_bfloat16*>(a.o);
+    mp.lse = a.lse;
+    mp.q0 = q0;
+    mp.nq = nq;
+    mp.H_q = a.H_q;
+    mp.H_kv = a.H_kv;
+    mp.kk = a.kk;
+    mp.G = G;
+    mp.B_k = a.B_k;
+    mp.c = c;
+    const int64_t rows = nq * a.H_q;
+    prof_begin("attn_merge", stream);
+    attn_merge_kernel<D_H><<<static_cast<unsigned>((rows * 32 + 255) / 256), 256, 0, stream>>>(mp);
+    prof_end(stream);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace
+
+size_t attn_workspace_bytes(int64_t N, int H_q, int H_kv, int d_h, int B_k, int kk) {
+  const int64_t B = (N + B_k - 1) / B_k;
+  size_t total = 0;
+  carve(nullptr, chunk_len(N, B_k), H_q, H_kv, d_h, kk, H_kv * B, &total);
+  return total;
+}
+
+cudaError_t launch_sparse_attn(const AttnLaunch& a, cudaStream_t s) {
+  if (a.d_h == 128 && a.B_k == 128) return launch_typed<128, 128>(a, s);
+  if (a.d_h == 128 && a.B_k == 64) return launch_typed<128, 64>(a, s);
+  if (a.d_h == 64 && a.B_k == 128) return launch_typed<64, 128>(a, s);
+  if (a.d_h == 64 && a.B_k == 64) return launch_typed<64, 64>(a, s);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace msa

@@ -1,0 +1,172 @@
+/*
+ * msa.h -- C ABI of the B200 (sm_100a) MiniMax Sparse Attention forward path.
+ *
+ * The method (arXiv:2606.13392, "MiniMax Sparse Attention"; equations as
+ * numbered in the xllm-io paper review, section "核心公式"):
+ *   Index Branch  Eq. 6  S[i,r,j] = <Q_idx[i,r], K_idx[j]> / sqrt(d_idx), j <= i
+ *                        M[i,r,b] = max over the visible tokens j of block b
+ *                 Eq. 7  I[i,r]   = Top-k blocks of M[i,r,:], the local block
+ *                                   b_i = i / B_k always kept (one of the k slots;
+ *                                   chlience notes 5.1.1)
+ *   Main Branch   Eq. 8  O[i,h]   = softmax(Q[i,h] K_r[I]^T / sqrt(d_h)) V_r[I],
+ *                                   r = h / (H_q / H_kv), causal j <= i (Eq. 1)
+ *
+ * Conventions for every entry point:
+ *   - Tensors are dense, row-major, in the axis order written beside each
+ *     argument; "bf16" arguments hold IEEE bfloat16 values.  All tensor
+ *     pointers are DEVICE pointers, 16-byte aligned, owned by the caller; the
+ *     library never allocates or frees memory and keeps no pointer after the
+ *     call returns.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t, NULL = the
+ *     legacy default stream).  Arguments are validated on the host first; on
+ *     a validation error nothing is launched and the outputs are untouched.
+ *   - `workspace` is caller-allocated device memory of at least the size the
+ *     matching *_workspace() query returns; its first 16 bytes hold the
+ *     device status word (see msa_get_device_status).  One workspace must not
+ *     be used by two calls that overlap on the GPU.
+ *   - Block indices are 0-based; selection rows are ascending, padded with -1.
+ */
+#ifndef MSA_B200_H
+#define MSA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MSA_API __attribute__((visibility("default")))
+#else
+#define MSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MSA_OK = 0,
+  MSA_ERR_INVALID_ARG = 1,         /* null/misaligned pointer, inconsistent sizes */
+  MSA_ERR_UNSUPPORTED = 2,         /* legal sizes this build has no kernel for */
+  MSA_ERR_WORKSPACE_TOO_SMALL = 3, /* ws_bytes below the *_workspace() size */
+  MSA_ERR_CUDA = 4,                /* a CUDA runtime call or launch failed */
+  MSA_ERR_DEVICE = 5               /* the device status word reports an error */
+} msa_status;
+
+/* Problem sizes of one prefill sequence (batch 1).
+ *   N      tokens;                  H_q, H_kv  query / KV heads, H_q % H_kv == 0
+ *   d_h    head dim (64 or 128);    d_idx      index head dim (32, 64 or 128)
+ *   B_k    block size (64 or 128);  k          selected blocks, 1 <= k <= 32
+ *   attn_scale  softmax scale of Eq. 8 (0 selects 1/sqrt(d_h))
+ *   idx_scale   scale of Eq. 6 (0 selects 1/sqrt(d_idx)); a positive scale does
+ *               not change the selection, only a negative one would (rejected). */
+typedef struct {
+  int64_t N;
+  int32_t H_q, H_kv, d_h, d_idx, B_k, k;
+  float attn_scale;
+  float idx_scale;
+} msa_dims;
+
+/* Decode batch: S independent sequences with caches of capacity L_max. */
+typedef struct {
+  int32_t S;
+  int64_t L_max;
+  int32_t H_q, H_kv, d_h, d_idx, B_k, k;
+  float attn_scale;
+  float idx_scale;
+} msa_decode_dims;
+
+/* ---------------------------------------------------------------------------
+ * Index Branch, Eq. 6-7 (xllm-io review "核心公式"; chlience notes 5.1.1):
+ * for every query i and group r, score all causal keys against the shared
+ * index key head, max-pool per block, keep the local block plus the k-1 best
+ * earlier blocks (ties -> lower block index).  The N x B score matrix is never
+ * written to memory.
+ *   q_idx    [N, H_kv, d_idx] bf16
+ *   k_idx    [N, d_idx]       bf16
+ *   idx_out  [N, H_kv, k]     int32, written: ascending, -1 padded
+ * Supported: H_kv in {1,2,4,8} with 128/H_kv <= B_k.
+ * ------------------------------------------------------------------------- */
+MSA_API size_t msa_index_topk_workspace(const msa_dims* dims);
+MSA_API msa_status msa_index_topk(const msa_dims* dims, const void* q_idx, const void* k_idx,
+                          int32_t* idx_out, void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Main Branch, Eq. 8 with the causal rule of Eq. 1 (xllm-io review "核心公式";
+ * chlience notes 5.1): exact softmax attention of every query head over the
+ * tokens of its group's selected blocks.
+ *   q    [N, H_q, d_h]  bf16      k, v  [N, H_kv, d_h] bf16
+ *   idx  [N, H_kv, k]   int32     entries in [-1, B); -1 = empty slot; an entry
+ *                                 must appear at most once per row; blocks after
+ *                                 the query's own block contribute nothing
+ *   o    [N, H_q, d_h]  bf16, written (round to nearest even from fp32)
+ *   lse  [N, H_q]       fp32 natural-log LSE of the scaled logits, or NULL
+ * A row whose selection is empty gets o = 0 and lse = -inf.
+ * Supported: d_h in {64,128}, B_k in {64,128}, 128 % (H_q/H_kv) == 0, and
+ * H_q % 8 == 0 when H_q/H_kv < 8.
+ * ------------------------------------------------------------------------- */
+MSA_API size_t msa_sparse_attn_fwd_workspace(const msa_dims* dims);
+MSA_API msa_status msa_sparse_attn_fwd(const msa_dims* dims, const void* q, const void* k,
+                               const void* v, const int32_t* idx, void* o, float* lse,
+                               void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * One decode step for S sequences (Eq. 1's i <= t: the new token attends to
+ * itself).  For each sequence s with L = seq_len[s] (read on the device):
+ * append k_new/v_new/k_idx_new at row L, then run Eq. 6-8 for the single query
+ * i = L over rows 0..L, then seq_len[s] = L + 1.
+ *   q         [S, H_q, d_h] bf16        q_idx      [S, H_kv, d_idx] bf16
+ *   k_new     [S, H_kv, d_h] bf16       v_new      [S, H_kv, d_h] bf16
+ *   k_idx_new [S, d_idx] bf16
+ *   k_cache, v_cache  [S, L_max, H_kv, d_h] bf16 (read and appended to)
+ *   k_idx_cache       [S, L_max, d_idx] bf16     (read and appended to)
+ *   seq_len   [S] int32, device, incremented
+ *   o         [S, H_q, d_h] bf16, written
+ *   idx_out   [S, H_kv, k] int32 or NULL: the selection used
+ * A sequence with seq_len >= L_max is skipped and MSA_DEV_CACHE_FULL recorded.
+ * Supported: d_h in {64,128}, d_idx in {32,64,128}, B_k in {64,128},
+ * H_q/H_kv <= 16, H_kv <= 8, 1 <= k <= 32.
+ * ------------------------------------------------------------------------- */
+MSA_API size_t msa_sparse_decode_workspace(const msa_decode_dims* dims);
+MSA_API msa_status msa_sparse_decode(const msa_decode_dims* dims, const void* q, const void* q_idx,
+                             const void* k_new, const void* v_new, const void* k_idx_new,
+                             void* k_cache, void* v_cache, void* k_idx_cache, int32_t* seq_len,
+                             void* o, int32_t* idx_out, void* workspace, size_t ws_bytes,
+                             void* stream);
+
+/* Device status codes written into the workspace's status word. */
+#define MSA_DEV_OK 0
+#define MSA_DEV_TIMEOUT 1    /* a bounded on-device wait gave up; outputs invalid */
+#define MSA_DEV_BAD_INDEX 2  /* idx held a block outside [-1, B); entry ignored */
+#define MSA_DEV_CACHE_FULL 3 /* decode: a sequence had no room left; skipped */
+#define MSA_DEV_CAPACITY 4   /* an internal list overflowed its reservation */
+
+/* Synchronises `stream`, then copies the status word of `workspace` (written
+ * by the last call that used it) into *code (and *where, if not NULL).
+ * Returns MSA_ERR_DEVICE if *code != 0, MSA_OK otherwise. */
+MSA_API msa_status msa_get_device_status(const void* workspace, void* stream, int32_t* code,
+                                 int32_t* where);
+
+/* Per-kernel timing for measurement tools.  msa_profile_enable(1) clears the
+ * record and starts recording a CUDA event pair around every kernel that the
+ * entry points above launch (on the caller's stream); msa_profile_enable(0)
+ * stops.  msa_profile_read waits for the recorded events, aggregates them by
+ * kernel name into out[0 .. max_entries-1] and returns the number of distinct
+ * kernels (-1 on a CUDA error).  Recording costs two event records per launch;
+ * it is off by default. */
+typedef struct {
+  char name[48];
+  int32_t launches;
+  double total_ms;
+} msa_kernel_time;
+MSA_API msa_status msa_profile_enable(int32_t on);
+MSA_API int32_t msa_profile_read(msa_kernel_time* out, int32_t max_entries);
+
+/* Static description of a status value. */
+MSA_API const char* msa_status_string(msa_status s);
+
+/* Library version string and the compute capability it was built for. */
+MSA_API const char* msa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MSA_B200_H */

@@ -1,0 +1,23 @@
+"""Helpers for the GPU tests: numpy bf16 bit arrays <-> torch CUDA tensors."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+
+def to_dev(bits: np.ndarray, device="cuda") -> torch.Tensor:
+    """uint16 bf16 bit patterns -> bf16 CUDA tensor (same shape)."""
+    t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16))
+    return t.view(torch.bfloat16).to(device)
+
+
+def to_host_bits(t: torch.Tensor) -> np.ndarray:
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def bf16_to_f64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def dev_inputs(inp: dict, device="cuda") -> dict:
+    return {k: to_dev(v, device) for k, v in inp.items()}
