@@ -22,6 +22,8 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <type_traits>
+
 #include "msa_internal.h"
 
 namespace msa {
@@ -274,46 +276,61 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int n_tiles = p.c.n_tiles[0];
-  const int nctas = gridDim.x;
+  // contiguous tile range of this CTA (tiles are equal-sized units of work)
+  const int t_beg = static_cast<int>(static_cast<int64_t>(n_tiles) * blockIdx.x / gridDim.x);
+  const int t_end = static_cast<int>(static_cast<int64_t>(n_tiles) * (blockIdx.x + 1) / gridDim.x);
+  const int my_tiles = t_end - t_beg;
 
   if (warp == 0) {
     // ------------------------------------------------------- TMA producer --
+    // The whole warp walks this CTA's contiguous tile range: one binary search
+    // for the first tile, then the (group, block) key only moves forward.
+    // Lane q fetches the slot of the tile's q-th query and issues its TMA box.
     if (lane == 0) {
       prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
-      int n = 0;
-      for (int t = blockIdx.x; t < n_tiles; t += nctas, ++n) {
-        const int st = n & 1;
-        if (!mbar_wait(&empty[st], ((n >> 1) & 1) ^ 1, abort_flag, p.status, 50)) break;
-        const int key = find_key(p.c.tile_off, p.nkeys, t);
-        const int lt = t - p.c.tile_off[key];
-        const int cnt = p.c.offsets[key + 1] - p.c.offsets[key];
-        const int len = min(p.Tq, cnt - lt * p.Tq);
-        const int r = key / static_cast<int>(p.nkeys / p.H_kv);
-        const int b = key - r * static_cast<int>(p.nkeys / p.H_kv);
-        TileInfo& ti = info[st];
+    }
+    const int nb = static_cast<int>(p.nkeys / p.H_kv);
+    const int per_q = p.H_kv * p.kk;
+    int key = t_beg < t_end ? find_key(p.c.tile_off, p.nkeys, t_beg) : 0;
+    for (int t = t_beg, n = 0; t < t_end; ++t, ++n) {
+      const int st = n & 1;
+      if (!mbar_wait(&empty[st], ((n >> 1) & 1) ^ 1, abort_flag, p.status, 50)) break;
+      while (p.c.tile_off[key + 1] <= t) ++key;
+      const int lt = t - p.c.tile_off[key];
+      const int off = p.c.offsets[key];
+      const int cnt = p.c.offsets[key + 1] - off;
+      const int len = min(p.Tq, cnt - lt * p.Tq);
+      const int r = key / nb;
+      const int b = key - r * nb;
+      uint32_t myslot = 0;
+      if (lane < len) myslot = p.c.entries[off + lt * p.Tq + lane];
+      TileInfo& ti = info[st];
+      if (lane < len) ti.slot[lane] = myslot;
+      if (lane == 0) {
         ti.r = r;
         ti.b = b;
         ti.len = len;
-        const uint32_t* ent = p.c.entries + p.c.offsets[key] + lt * p.Tq;
-        for (int q = 0; q < len; ++q) ti.slot[q] = ent[q];
-        uint8_t* sQ = smem + st * SH::STAGE_BYTES;
-        uint8_t* sK = sQ + SH::QP_BYTES;
-        uint8_t* sV = sK + SH::K_BYTES;
+      }
+      __syncwarp();
+      uint8_t* sQ = smem + st * SH::STAGE_BYTES;
+      uint8_t* sK = sQ + SH::QP_BYTES;
+      uint8_t* sV = sK + SH::K_BYTES;
+      if (lane == 0)
         mbar_arrive_expect_tx(&full[st], SH::K_BYTES + SH::V_BYTES + len * p.R * D_H * 2);
-        const int h0 = p.G >= 8 ? r * p.G : (r * p.G / 8) * 8;
-        for (int c = 0; c < SH::DCH; ++c) {
-          tma_load_3d(sK + c * B_K * 128, &tm_k, &full[st], c * 64, r, b * B_K);
-          tma_load_3d(sV + c * B_K * 128, &tm_v, &full[st], c * 64, r, b * B_K);
-        }
-        const int per_q = p.H_kv * p.kk;
-        for (int q = 0; q < len; ++q) {
-          const int i = static_cast<int>(p.q0 + ti.slot[q] / per_q);
-          for (int c = 0; c < SH::DCH; ++c)
-            tma_load_3d(sQ + c * kRowsPerTile * 128 + q * p.R * 128, &tm_q, &full[st], c * 64,
-                        h0, i);
-        }
+      __syncwarp();
+      const int h0 = p.G >= 8 ? r * p.G : (r * p.G / 8) * 8;
+      if (lane < SH::DCH) {
+        tma_load_3d(sK + lane * B_K * 128, &tm_k, &full[st], lane * 64, r, b * B_K);
+        tma_load_3d(sV + lane * B_K * 128, &tm_v, &full[st], lane * 64, r, b * B_K);
+      }
+      if (lane < len) {
+        const int i = static_cast<int>(p.q0 + myslot / per_q);
+#pragma unroll
+        for (int c = 0; c < SH::DCH; ++c)
+          tma_load_3d(sQ + c * kRowsPerTile * 128 + lane * p.R * 128, &tm_q, &full[st], c * 64,
+                      h0, i);
       }
     }
   } else if (warp == 1) {
@@ -342,7 +359,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         umma_commit(&s_full[st]);
         return true;
       };
-      const int my_tiles = blockIdx.x < n_tiles ? (n_tiles - 1 - blockIdx.x) / nctas + 1 : 0;
       bool ok = my_tiles == 0 || issue_s(0);
       for (int n = 0; ok && n < my_tiles; ++n) {
         const int st = n & 1;
@@ -380,8 +396,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q_local = row / p.R;
     const int hrow = row - q_local * p.R;
     const int per_q = p.H_kv * p.kk;
-    int n = grp;
-    for (int t = blockIdx.x + grp * nctas; t < n_tiles; t += 2 * nctas, n += 2) {
+    for (int n = grp; n < my_tiles; n += 2) {
       const int st = grp;
       const uint32_t ph = (n >> 1) & 1;
       uint8_t* sP = smem + st * SH::STAGE_BYTES;
@@ -398,13 +413,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t i = p.q0 + slot / per_q;
       // ---- softmax over the block's keys (exp2 with the scale folded in)
       float sv[B_K];
+      {
+        uint32_t r32[B_K / 32][32];
 #pragma unroll
-      for (int c = 0; c < B_K / 32; ++c) {
-        uint32_t r32[32];
-        tmem_ld32(tS + c * 32, r32);
+        for (int c = 0; c < B_K / 32; ++c) tmem_ld32(tS + c * 32, r32[c]);
         tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 32; ++j) sv[c * 32 + j] = __uint_as_float(r32[j]);
+        for (int c = 0; c < B_K / 32; ++c)
+#pragma unroll
+          for (int j = 0; j < 32; ++j) sv[c * 32 + j] = __uint_as_float(r32[c][j]);
       }
       const int64_t j0 = static_cast<int64_t>(ti_b) * B_K;
       if (j0 + B_K - 1 > i) {  // the query's own block: causal rule j <= i
@@ -452,30 +469,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int g = hrow - goff;
       __half* dst = p.c.part_o + (static_cast<int64_t>(slot) * p.G + g) * D_H;
       const float inv_l = 1.0f / l;
+      uint32_t ro[D_H / 32][32];
 #pragma unroll
-      for (int c = 0; c < D_H / 32; ++c) {
-        uint32_t r32[32];
-        tmem_ld32(tO + c * 32, r32);
-        tmem_wait_ld();
-        if (useful) {
+      for (int c = 0; c < D_H / 32; ++c) tmem_ld32(tO + c * 32, ro[c]);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&o_empty[st]);
+      if (useful) {
+#pragma unroll
+        for (int c = 0; c < D_H / 32; ++c)
 #pragma unroll
           for (int j = 0; j < 32; j += 8) {
             uint4 w;
-            __half2 a0 = __floats2half2_rn(__uint_as_float(r32[j + 0]) * inv_l, __uint_as_float(r32[j + 1]) * inv_l);
-            __half2 a1 = __floats2half2_rn(__uint_as_float(r32[j + 2]) * inv_l, __uint_as_float(r32[j + 3]) * inv_l);
-            __half2 a2 = __floats2half2_rn(__uint_as_float(r32[j + 4]) * inv_l, __uint_as_float(r32[j + 5]) * inv_l);
-            __half2 a3 = __floats2half2_rn(__uint_as_float(r32[j + 6]) * inv_l, __uint_as_float(r32[j + 7]) * inv_l);
+            __half2 a0 = __floats2half2_rn(__uint_as_float(ro[c][j + 0]) * inv_l, __uint_as_float(ro[c][j + 1]) * inv_l);
+            __half2 a1 = __floats2half2_rn(__uint_as_float(ro[c][j + 2]) * inv_l, __uint_as_float(ro[c][j + 3]) * inv_l);
+            __half2 a2 = __floats2half2_rn(__uint_as_float(ro[c][j + 4]) * inv_l, __uint_as_float(ro[c][j + 5]) * inv_l);
+            __half2 a3 = __floats2half2_rn(__uint_as_float(ro[c][j + 6]) * inv_l, __uint_as_float(ro[c][j + 7]) * inv_l);
             w.x = *reinterpret_cast<uint32_t*>(&a0);
             w.y = *reinterpret_cast<uint32_t*>(&a1);
             w.z = *reinterpret_cast<uint32_t*>(&a2);
             w.w = *reinterpret_cast<uint32_t*>(&a3);
             *reinterpret_cast<uint4*>(dst + c * 32 + j) = w;
           }
-        }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&o_empty[st]);
       if (useful) p.c.part_lse[static_cast<int64_t>(slot) * p.G + g] = mx * p.scale + logf(l);
     }
   }
@@ -498,10 +515,13 @@ struct MergeParams {
   ChunkBufs c;
 };
 
-// One warp per (query, head): LSE-weighted merge of the row's partials.
+// One warp per (query, head): LSE-weighted merge of the row's partials.  Lane
+// s reads slot s's LSE, the weights come from warp reductions, and the
+// partial rows are then fetched eight at a time so their loads overlap.
 template <int D_H>
 __global__ void __launch_bounds__(256) attn_merge_kernel(const MergeParams p) {
   constexpr int PER = D_H / 32;  // elements per lane
+  using Vec = typename std::conditional<PER == 4, uint2, uint32_t>::type;
   const int lane = threadIdx.x & 31;
   const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   if (row >= p.nq * p.H_q) return;
@@ -510,34 +530,46 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(const MergeParams p) {
   const int r = h / p.G, g = h - r * p.G;
   const int64_t i = p.q0 + il;
   const int64_t b_i = i / p.B_k;
+  const int64_t slot0 = (il * p.H_kv + r) * p.kk;
   int32_t myb = -1;
   if (lane < p.kk) myb = p.idx[(i * p.H_kv + r) * p.kk + lane];
-  const unsigned use = __ballot_sync(0xFFFFFFFFu, lane < p.kk && myb >= 0 && myb <= b_i);
-  float m = -INFINITY, wsum = 0.0f;
+  const bool valid = lane < p.kk && myb >= 0 && myb <= b_i;
+  const float ls = valid ? p.c.part_lse[(slot0 + lane) * p.G + g] : -INFINITY;
+  float m = ls;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+  const float w = valid ? __expf(ls - m) : 0.0f;
+  float wsum = w;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xFFFFFFFFu, wsum, o);
+  const unsigned use = __ballot_sync(0xFFFFFFFFu, valid);
   float acc[PER];
 #pragma unroll
   for (int e = 0; e < PER; ++e) acc[e] = 0.0f;
-  unsigned rest = use;
-  while (rest) {
-    const int s = __ffs(rest) - 1;
-    rest &= rest - 1;
-    const int64_t slot = (il * p.H_kv + r) * p.kk + s;
-    const float ls = p.c.part_lse[slot * p.G + g];
-    const __half* src = p.c.part_o + (slot * p.G + g) * D_H + lane * PER;
-    float x[PER];
+  const __half* base = p.c.part_o + (slot0 * p.G + g) * D_H + lane * PER;
+  const int64_t stride = static_cast<int64_t>(p.G) * D_H;  // between slots
+  for (int s0 = 0; s0 < p.kk; s0 += 8) {
+    Vec x[8];
+    float wj[8];
 #pragma unroll
-    for (int e = 0; e < PER; e += 2) {
-      const float2 a = __half22float2(*reinterpret_cast<const __half2*>(src + e));
-      x[e] = a.x;
-      x[e + 1] = a.y;
+    for (int j = 0; j < 8; ++j) {
+      const int s = s0 + j;
+      wj[j] = __shfl_sync(0xFFFFFFFFu, w, s & 31);
+      const bool on = s < p.kk && ((use >> (s & 31)) & 1u);
+      if (on) x[j] = *reinterpret_cast<const Vec*>(base + s * stride);
+      else x[j] = Vec{};
+      if (!on) wj[j] = 0.0f;
     }
-    const float mn = fmaxf(m, ls);
-    const float a_old = __expf(m - mn);
-    const float a_new = __expf(ls - mn);
 #pragma unroll
-    for (int e = 0; e < PER; ++e) acc[e] = acc[e] * a_old + x[e] * a_new;
-    wsum = wsum * a_old + a_new;
-    m = mn;
+    for (int j = 0; j < 8; ++j) {
+      const __half2* hv = reinterpret_cast<const __half2*>(&x[j]);
+#pragma unroll
+      for (int e = 0; e < PER; e += 2) {
+        const float2 f = __half22float2(hv[e / 2]);
+        acc[e] = fmaf(wj[j], f.x, acc[e]);
+        acc[e + 1] = fmaf(wj[j], f.y, acc[e + 1]);
+      }
+    }
   }
   __nv_bfloat16* dst = p.o + (i * p.H_q + h) * static_cast<int64_t>(D_H) + lane * PER;
   const float inv = wsum > 0.0f ? 1.0f / wsum : 0.0f;

@@ -21,3 +21,18 @@ def bf16_to_f64(t: torch.Tensor) -> np.ndarray:
 
 def dev_inputs(inp: dict, device="cuda") -> dict:
     return {k: to_dev(v, device) for k, v in inp.items()}
+
+
+_CACHE = {}
+
+
+def prefill_inputs_cached(cfg, seed=None):
+    """inputs.prefill_inputs, memoised per (config, seed) for the test session."""
+    from block_sparse_gqa_idx_b200 import inputs
+
+    key = (cfg, seed)
+    if key not in _CACHE:
+        if len(_CACHE) > 4:
+            _CACHE.clear()
+        _CACHE[key] = inputs.prefill_inputs(cfg, seed)
+    return _CACHE[key]

@@ -13,7 +13,7 @@ import torch
 import oracle
 from block_sparse_gqa_idx_b200 import inputs
 from tests import compare
-from tests.gpu_util import bf16_to_f64, dev_inputs, to_dev
+from tests.gpu_util import bf16_to_f64, dev_inputs, prefill_inputs_cached, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -34,7 +34,7 @@ def _cfg(name, **kw):
 
 
 def _check_index(msa, cfg, rows=None, seed=None):
-    inp = inputs.prefill_inputs(cfg, seed)
+    inp = prefill_inputs_cached(cfg, seed)
     dev = dev_inputs(inp)
     idx = msa.index_topk(dev["q_idx"], dev["k_idx"], cfg.B_k, cfg.k)
     torch.cuda.synchronize()
@@ -96,7 +96,7 @@ def _check_attn(msa, inp, dev, idx_dev, cfg, rows, what):
 
 def test_attention_tiny_all_rows(msa):
     cfg = inputs.CONFIGS["tiny"]
-    inp = inputs.prefill_inputs(cfg)
+    inp = prefill_inputs_cached(cfg)
     dev = dev_inputs(inp)
     idx = msa.index_topk(dev["q_idx"], dev["k_idx"], cfg.B_k, cfg.k)
     _check_attn(msa, inp, dev, idx, cfg, np.arange(cfg.N), "tiny")
@@ -104,7 +104,7 @@ def test_attention_tiny_all_rows(msa):
 
 def test_attention_32k_shape_truncated(msa):
     cfg = _cfg("32k", N=8192)
-    inp = inputs.prefill_inputs(cfg)
+    inp = prefill_inputs_cached(cfg)
     dev = dev_inputs(inp)
     idx = msa.index_topk(dev["q_idx"], dev["k_idx"], cfg.B_k, cfg.k)
     rng = np.random.default_rng(1)
@@ -122,7 +122,7 @@ def test_attention_32k_shape_truncated(msa):
 def test_attention_edge_shapes(msa, N, H_q, H_kv, d_h, B_k, k):
     cfg = inputs.MSAConfig("edge", N=N, H_q=H_q, H_kv=H_kv, d_h=d_h, d_idx=64, B_k=B_k, k=k,
                            structure="iid", seed_index=23)
-    inp = inputs.prefill_inputs(cfg)
+    inp = prefill_inputs_cached(cfg)
     dev = dev_inputs(inp)
     idx = msa.index_topk(dev["q_idx"], dev["k_idx"], cfg.B_k, cfg.k)
     _check_attn(msa, inp, dev, idx, cfg, np.arange(N), f"edge {N},{H_q},{H_kv},{d_h},{B_k},{k}")
@@ -133,7 +133,7 @@ def test_attention_dense_equivalence(msa):
     N, H_q, H_kv, d_h, B_k = 640, 16, 2, 128, 128
     cfg = inputs.MSAConfig("dense", N=N, H_q=H_q, H_kv=H_kv, d_h=d_h, d_idx=64, B_k=B_k, k=5,
                            seed_index=29)
-    inp = inputs.prefill_inputs(cfg)
+    inp = prefill_inputs_cached(cfg)
     dev = dev_inputs(inp)
     idx = msa.index_topk(dev["q_idx"], dev["k_idx"], B_k, 5)
     o, lse = msa.sparse_attn_fwd(dev["q"], dev["k"], dev["v"], idx, B_k)
@@ -146,7 +146,7 @@ def test_attention_synthetic_sink_zipf_selection(msa):
     """Sink-skewed selections (block 0 in ~90% of rows, Zipf(1.1) by recency):
     hot-block splitting and tiles mixing local and non-local rows."""
     cfg = _cfg("32k", N=6144)
-    inp = inputs.prefill_inputs(cfg)
+    inp = prefill_inputs_cached(cfg)
     dev = dev_inputs(inp)
     sel = inputs.zipf_indices(cfg.N, cfg.H_kv, cfg.B_k, cfg.k)
     idx = torch.from_numpy(sel).cuda()
@@ -160,7 +160,7 @@ def test_attention_empty_and_future_entries(msa):
     (causal rule); an all-empty row gives o = 0, lse = -inf."""
     cfg = inputs.MSAConfig("odd", N=512, H_q=16, H_kv=2, d_h=64, d_idx=64, B_k=64, k=4,
                            seed_index=31)
-    inp = inputs.prefill_inputs(cfg)
+    inp = prefill_inputs_cached(cfg)
     dev = dev_inputs(inp)
     idx = np.full((cfg.N, cfg.H_kv, cfg.k), -1, dtype=np.int32)
     B = cfg.B
@@ -181,7 +181,7 @@ def test_attention_empty_and_future_entries(msa):
 
 def test_attention_128k_sampled(msa):
     cfg = inputs.CONFIGS["128k"]
-    inp = inputs.prefill_inputs(cfg)
+    inp = prefill_inputs_cached(cfg)
     dev = dev_inputs(inp)
     idx = msa.index_topk(dev["q_idx"], dev["k_idx"], cfg.B_k, cfg.k)
     rng = np.random.default_rng(3)
@@ -192,7 +192,7 @@ def test_attention_128k_sampled(msa):
 def test_device_status_reports_bad_index(msa):
     cfg = inputs.MSAConfig("bad", N=256, H_q=16, H_kv=2, d_h=64, d_idx=64, B_k=64, k=2,
                            seed_index=37)
-    inp = inputs.prefill_inputs(cfg)
+    inp = prefill_inputs_cached(cfg)
     dev = dev_inputs(inp)
     idx = np.zeros((cfg.N, cfg.H_kv, cfg.k), dtype=np.int32)
     idx[:, :, 1] = -1
