@@ -48,7 +48,7 @@ class msa_kernel_time(ctypes.Structure):
 EXPORTS = ("msa_index_topk_workspace", "msa_index_topk", "msa_sparse_attn_fwd_workspace",
            "msa_sparse_attn_fwd", "msa_sparse_decode_workspace", "msa_sparse_decode",
            "msa_get_device_status", "msa_profile_enable", "msa_profile_read",
-           "msa_status_string", "msa_version")
+           "msa_status_string", "msa_version", "msa_sparse_decode_noalloc")
 
 
 def _load() -> ctypes.CDLL:
@@ -71,6 +71,8 @@ def _load() -> ctypes.CDLL:
     lib.msa_sparse_decode_workspace.restype = Z
     lib.msa_sparse_decode.argtypes = [DD] + [P] * 12 + [Z, P]
     lib.msa_sparse_decode.restype = I32
+    lib.msa_sparse_decode_noalloc.argtypes = [DD] + [P] * 11 + [P]
+    lib.msa_sparse_decode_noalloc.restype = I32
     lib.msa_get_device_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_int32),
                                           ctypes.POINTER(ctypes.c_int32)]
     lib.msa_get_device_status.restype = I32
@@ -252,6 +254,39 @@ def profile_read() -> dict:
         raise MSAError("msa_profile_read", 4, "CUDA error")
     return {buf[j].name.decode(): (int(buf[j].launches), float(buf[j].total_ms))
             for j in range(min(n, 64))}
+
+
+def sparse_decode_noalloc(q, q_idx, k_new, v_new, k_idx_new, k_cache, v_cache, k_idx_cache,
+                          seq_len, B_k: int, kk: int, attn_scale: float = 0.0,
+                          o: Optional[torch.Tensor] = None,
+                          idx_out: Optional[torch.Tensor] = None, stream=None):
+    """sparse_decode without a workspace: the library's fixed scratch array is
+    used (for callers that cannot allocate device memory while serving).  Pass
+    ``o`` to avoid the one output allocation this binding would otherwise make."""
+    S, H_q, d_h = q.shape
+    H_kv, d_idx = q_idx.shape[1], q_idx.shape[2]
+    L_max = k_cache.shape[1]
+    _want(q, "q", torch.bfloat16, (S, H_q, d_h))
+    _want(q_idx, "q_idx", torch.bfloat16, (S, H_kv, d_idx))
+    _want(k_new, "k_new", torch.bfloat16, (S, H_kv, d_h))
+    _want(v_new, "v_new", torch.bfloat16, (S, H_kv, d_h))
+    _want(k_idx_new, "k_idx_new", torch.bfloat16, (S, d_idx))
+    _want(k_cache, "k_cache", torch.bfloat16, (S, L_max, H_kv, d_h))
+    _want(v_cache, "v_cache", torch.bfloat16, (S, L_max, H_kv, d_h))
+    _want(k_idx_cache, "k_idx_cache", torch.bfloat16, (S, L_max, d_idx))
+    _want(seq_len, "seq_len", torch.int32, (S,))
+    if o is None:
+        o = torch.empty((S, H_q, d_h), dtype=torch.bfloat16, device=q.device)
+    _want(o, "o", torch.bfloat16, (S, H_q, d_h))
+    if idx_out is not None:
+        _want(idx_out, "idx_out", torch.int32, (S, H_kv, kk))
+    d = decode_dims(S, L_max, H_q, H_kv, d_h, d_idx, B_k, kk, attn_scale)
+    _raise("msa_sparse_decode_noalloc",
+           LIB.msa_sparse_decode_noalloc(ctypes.byref(d), _ptr(q), _ptr(q_idx), _ptr(k_new),
+                                         _ptr(v_new), _ptr(k_idx_new), _ptr(k_cache),
+                                         _ptr(v_cache), _ptr(k_idx_cache), _ptr(seq_len),
+                                         _ptr(o), _ptr(idx_out), _stream(stream)))
+    return o, idx_out
 
 
 def device_status(workspace: torch.Tensor, stream=None) -> Tuple[int, int]:

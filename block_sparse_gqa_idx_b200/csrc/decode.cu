@@ -607,3 +607,62 @@ cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t stream) {
 }
 
 }  // namespace msa
+
+// ------------------------------------------------------------------------
+// Decode without a caller workspace (msa_sparse_decode_noalloc in msa.h).
+// Callers that cannot allocate device memory while serving get the step's
+// scratch from this fixed array instead; every GPU that runs the library's
+// kernels holds it until the process exits.
+// ------------------------------------------------------------------------
+#include <mutex>
+
+#include "../../include/msa.h"
+
+static __device__ __align__(256) uint8_t g_decode_scratch[MSA_DECODE_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of g_decode_scratch on the current device, looked up once
+// per device with that device current.  (In host code the array's name is
+// only a host-side stand-in, never a usable device pointer.)
+void* decode_scratch(msa_status* st) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    *st = MSA_ERR_CUDA;
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lk(g_scratch_mu);
+  if (g_scratch_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || p == nullptr) {
+      *st = MSA_ERR_CUDA;
+      return nullptr;
+    }
+    g_scratch_ptr[dev] = p;
+  }
+  *st = MSA_OK;
+  return g_scratch_ptr[dev];
+}
+}  // namespace
+
+extern "C" msa_status msa_sparse_decode_noalloc(const msa_decode_dims* d, const void* q,
+                                                const void* q_idx, const void* k_new,
+                                                const void* v_new, const void* k_idx_new,
+                                                void* k_cache, void* v_cache, void* k_idx_cache,
+                                                int32_t* seq_len, void* o, int32_t* idx_out,
+                                                void* stream) {
+  if (d == nullptr) return MSA_ERR_INVALID_ARG;
+  const size_t need = msa_sparse_decode_workspace(d);
+  if (need == 0) return MSA_ERR_INVALID_ARG;
+  if (need > MSA_DECODE_NOALLOC_SCRATCH_BYTES) return MSA_ERR_WORKSPACE_TOO_SMALL;
+  msa_status st = MSA_OK;
+  void* ws = decode_scratch(&st);
+  if (ws == nullptr) return st;
+  // The regular entry point validates every argument, clears the status word
+  // at the head of the scratch and launches the same kernels.
+  return msa_sparse_decode(d, q, q_idx, k_new, v_new, k_idx_new, k_cache, v_cache, k_idx_cache,
+                           seq_len, o, idx_out, ws, MSA_DECODE_NOALLOC_SCRATCH_BYTES, stream);
+}

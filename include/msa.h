@@ -132,6 +132,39 @@ MSA_API msa_status msa_sparse_decode(const msa_decode_dims* dims, const void* q,
                              void* o, int32_t* idx_out, void* workspace, size_t ws_bytes,
                              void* stream);
 
+/* ---------------------------------------------------------------------------
+ * msa_sparse_decode_noalloc: the decode step above without a caller workspace.
+ * (Not part of the method: the paper has no counterpart; this is a deployment
+ * convenience.)
+ * Some callers cannot hand the library a device workspace: a host program in
+ * plain C that has no device allocator of its own, or a serving loop whose
+ * device memory is entirely reserved up front (model weights plus a fixed KV
+ * cache pool) and which must not allocate, or grow a caching allocator,
+ * while it is answering requests.  This entry point takes its scratch (block
+ * maxima, selections, per-slot partial outputs and the status word) from one
+ * fixed array inside the library, MSA_DECODE_NOALLOC_SCRATCH_BYTES large,
+ * which every GPU that runs the library's kernels holds until the process
+ * exits.  The caller still passes all inputs and outputs.
+ *   - Same arguments, layouts and results as msa_sparse_decode, minus the
+ *     workspace.  Returns MSA_ERR_WORKSPACE_TOO_SMALL, launching nothing, if
+ *     msa_sparse_decode_workspace(dims) exceeds the fixed size.
+ *   - The first call on a device looks up the array's device address (once per
+ *     device, with that device current); make that first call before any
+ *     stream capture.  The call allocates no memory.
+ *   - All calls share the one array and it keeps the last call's contents:
+ *     two calls that overlap on the GPU (other streams, other host threads)
+ *     race and corrupt each other's results.  Each call clears the status
+ *     word it needs; the word itself is not readable from the host, so a
+ *     sequence skipped for a full cache shows only as seq_len not advancing.
+ * ------------------------------------------------------------------------- */
+#define MSA_DECODE_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+MSA_API msa_status msa_sparse_decode_noalloc(const msa_decode_dims* dims, const void* q,
+                                             const void* q_idx, const void* k_new,
+                                             const void* v_new, const void* k_idx_new,
+                                             void* k_cache, void* v_cache, void* k_idx_cache,
+                                             int32_t* seq_len, void* o, int32_t* idx_out,
+                                             void* stream);
+
 /* Device status codes written into the workspace's status word. */
 #define MSA_DEV_OK 0
 #define MSA_DEV_TIMEOUT 1    /* a bounded on-device wait gave up; outputs invalid */
