@@ -212,19 +212,20 @@ struct P1Params {
 
 template <int D_H, int B_K>
 struct P1Shape {
+  static constexpr int QS = 4;                                                  // Q/P ring depth
   static constexpr int QP_BYTES = kRowsPerTile * (D_H > B_K ? D_H : B_K) * 2;  // Q, later P
   static constexpr int K_BYTES = B_K * D_H * 2;
   static constexpr int V_BYTES = B_K * D_H * 2;
-  static constexpr int STAGE_BYTES = QP_BYTES + K_BYTES + V_BYTES;
   static constexpr int DCH = D_H / 64;  // 128-byte chunks along d
   static constexpr int PCH = B_K / 64;  // 128-byte chunks along keys (P)
-  static constexpr uint32_t TM_S = 0, TM_O = 128;  // column offsets inside a stage
+  static constexpr uint32_t TM_S = 0, TM_O = 128;  // column offsets inside a TMEM stage
 };
 
+constexpr int kMaxTq = 16;  // queries per tile (128 rows / at least 8 rows per query)
+
 struct TileInfo {
-  int r, b, len;
-  int pad;
-  uint32_t slot[128];
+  int r, b, len, gen;  // group, block, queries in the tile, K/V generation
+  uint32_t slot[kMaxTq];
 };
 
 __device__ __forceinline__ int find_key(const int32_t* tile_off, int64_t nkeys, int t) {
@@ -237,31 +238,49 @@ __device__ __forceinline__ int find_key(const int32_t* tile_off, int64_t nkeys, 
   return static_cast<int>(lo);
 }
 
+// Phase 1.  Each CTA owns a contiguous range of tiles; tiles of one (group,
+// block) key come in long runs there, so the K/V block sits in one shared
+// slot for the whole run (reloaded only when the key changes) while the
+// gathered query rows stream through a 4-deep ring.  TMEM holds two tiles
+// (S and O, 128 + 128 columns each); two softmax/epilogue groups of four
+// warps take alternate tiles.
+//   warp 0      producer (all lanes: lane q issues query q's TMA box)
+//   warp 1      MMA issuer (lane 0) and TMEM owner
+//   warps 2..9  softmax + epilogue, group (w-2)/4
 template <int D_H, int B_K>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_phase1_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const P1Params p) {
   using SH = P1Shape<D_H, B_K>;
+  constexpr int QS = SH::QS;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  TileInfo* info = reinterpret_cast<TileInfo*>(smem + 2 * SH::STAGE_BYTES);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(info + 2);
-  uint64_t* full = bars;          // [2] TMA landed
-  uint64_t* empty = bars + 2;     // [2] stage smem free (O MMA done)
-  uint64_t* s_full = bars + 4;    // [2] S in TMEM
-  uint64_t* p_full = bars + 6;    // [2] P in smem (S read)
-  uint64_t* o_full = bars + 8;    // [2] O in TMEM
-  uint64_t* o_empty = bars + 10;  // [2] O read
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
+  uint8_t* sK = smem + QS * SH::QP_BYTES;
+  uint8_t* sV = sK + SH::K_BYTES;
+  TileInfo* info = reinterpret_cast<TileInfo*>(sV + SH::V_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(info + QS);
+  uint64_t* q_full = bars;             // [QS] gathered Q landed
+  uint64_t* q_empty = q_full + QS;     // [QS] O MMA of the stage's tile done
+  uint64_t* kv_full = q_empty + QS;    // K/V block landed
+  uint64_t* kv_empty = kv_full + 1;    // last tile of a K/V run finished its O MMA
+  uint64_t* s_full = kv_empty + 1;     // [2] S in TMEM
+  uint64_t* p_full = s_full + 2;       // [2] P in smem (S read)
+  uint64_t* o_full = p_full + 2;       // [2] O in TMEM
+  uint64_t* o_empty = o_full + 2;      // [2] O read
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_empty + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
+    for (int s = 0; s < QS; ++s) {
+      mbar_init(&q_full[s], 1);
+      mbar_init(&q_empty[s], 1);
+    }
+    mbar_init(kv_full, 1);
+    mbar_init(kv_empty, 1);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
       mbar_init(&s_full[s], 1);
       mbar_init(&p_full[s], 4);
       mbar_init(&o_full[s], 1);
@@ -283,9 +302,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------- TMA producer --
-    // The whole warp walks this CTA's contiguous tile range: one binary search
-    // for the first tile, then the (group, block) key only moves forward.
-    // Lane q fetches the slot of the tile's q-th query and issues its TMA box.
     if (lane == 0) {
       prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_k);
@@ -293,60 +309,104 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     const int nb = static_cast<int>(p.nkeys / p.H_kv);
     const int per_q = p.H_kv * p.kk;
-    int key = t_beg < t_end ? find_key(p.c.tile_off, p.nkeys, t_beg) : 0;
-    for (int t = t_beg, n = 0; t < t_end; ++t, ++n) {
-      const int st = n & 1;
-      if (!mbar_wait(&empty[st], ((n >> 1) & 1) ^ 1, abort_flag, p.status, 50)) break;
-      while (p.c.tile_off[key + 1] <= t) ++key;
-      const int lt = t - p.c.tile_off[key];
-      const int off = p.c.offsets[key];
-      const int cnt = p.c.offsets[key + 1] - off;
-      const int len = min(p.Tq, cnt - lt * p.Tq);
-      const int r = key / nb;
-      const int b = key - r * nb;
-      uint32_t myslot = 0;
-      if (lane < len) myslot = p.c.entries[off + lt * p.Tq + lane];
-      TileInfo& ti = info[st];
+    // tile cursor: key, its first tile, its entry range
+    int key = 0, kt0 = 0, kend = 0, koff = 0, kcnt = 0;
+    auto seek = [&](int t) {
+      while (kend <= t) {
+        ++key;
+        kt0 = p.c.tile_off[key];
+        kend = p.c.tile_off[key + 1];
+      }
+      koff = p.c.offsets[key];
+      kcnt = p.c.offsets[key + 1] - koff;
+    };
+    uint32_t next_slot = 0;
+    int next_len = 0;
+    if (my_tiles > 0) {
+      key = find_key(p.c.tile_off, p.nkeys, t_beg);
+      kt0 = p.c.tile_off[key];
+      kend = p.c.tile_off[key + 1];
+      koff = p.c.offsets[key];
+      kcnt = p.c.offsets[key + 1] - koff;
+      const int lt = t_beg - kt0;
+      next_len = min(p.Tq, kcnt - lt * p.Tq);
+      if (lane < next_len) next_slot = p.c.entries[koff + lt * p.Tq + lane];
+    }
+    int kv_key = -1, kvgen = 0;
+    for (int n = 0; n < my_tiles; ++n) {
+      const int t = t_beg + n;
+      const int cur_key = key, len = next_len;
+      const uint32_t myslot = next_slot;
+      const int r = cur_key / nb, b = cur_key - r * nb;
+      // fetch the next tile's slots now; their latency hides behind the waits
+      if (n + 1 < my_tiles) {
+        if (t + 1 >= kend) seek(t + 1);
+        const int lt = t + 1 - kt0;
+        next_len = min(p.Tq, kcnt - lt * p.Tq);
+        next_slot = lane < next_len ? p.c.entries[koff + lt * p.Tq + lane] : 0u;
+      }
+      const bool new_kv = cur_key != kv_key;
+      const int gen = new_kv ? kvgen : kvgen - 1;
+      // Q of this tile first (the MMA warp needs it to see a K/V switch)
+      const int qs = n % QS;
+      if (!mbar_wait(&q_empty[qs], ((n / QS) & 1) ^ 1, abort_flag, p.status, 50)) break;
+      TileInfo& ti = info[qs];
       if (lane < len) ti.slot[lane] = myslot;
       if (lane == 0) {
         ti.r = r;
         ti.b = b;
         ti.len = len;
+        ti.gen = gen;
+        mbar_arrive_expect_tx(&q_full[qs], len * p.R * D_H * 2);
       }
-      __syncwarp();
-      uint8_t* sQ = smem + st * SH::STAGE_BYTES;
-      uint8_t* sK = sQ + SH::QP_BYTES;
-      uint8_t* sV = sK + SH::K_BYTES;
-      if (lane == 0)
-        mbar_arrive_expect_tx(&full[st], SH::K_BYTES + SH::V_BYTES + len * p.R * D_H * 2);
       __syncwarp();
       const int h0 = p.G >= 8 ? r * p.G : (r * p.G / 8) * 8;
-      if (lane < SH::DCH) {
-        tma_load_3d(sK + lane * B_K * 128, &tm_k, &full[st], lane * 64, r, b * B_K);
-        tma_load_3d(sV + lane * B_K * 128, &tm_v, &full[st], lane * 64, r, b * B_K);
-      }
       if (lane < len) {
         const int i = static_cast<int>(p.q0 + myslot / per_q);
+        uint8_t* sQ = smem + qs * SH::QP_BYTES;
 #pragma unroll
         for (int c = 0; c < SH::DCH; ++c)
-          tma_load_3d(sQ + c * kRowsPerTile * 128 + lane * p.R * 128, &tm_q, &full[st], c * 64,
+          tma_load_3d(sQ + c * kRowsPerTile * 128 + lane * p.R * 128, &tm_q, &q_full[qs], c * 64,
                       h0, i);
+      }
+      if (new_kv) {
+        // the slot is free once every tile of the previous run finished O = P V
+        if (kvgen > 0 &&
+            !mbar_wait(kv_empty, (kvgen - 1) & 1, abort_flag, p.status, 51))
+          break;
+        if (lane == 0) mbar_arrive_expect_tx(kv_full, SH::K_BYTES + SH::V_BYTES);
+        __syncwarp();
+        if (lane < SH::DCH) {
+          tma_load_3d(sK + lane * B_K * 128, &tm_k, kv_full, lane * 64, r, b * B_K);
+          tma_load_3d(sV + lane * B_K * 128, &tm_v, kv_full, lane * 64, r, b * B_K);
+        }
+        kv_key = cur_key;
+        ++kvgen;
       }
     }
   } else if (warp == 1) {
     // -------------------------------------------------------- MMA issuer --
-    // Software-pipelined: S of tile n+1 is issued before waiting for the
-    // softmax of tile n, so the tensor core works while P is being built.
+    // S of tile n+1 is issued before waiting for the softmax of tile n, so the
+    // tensor core works while P is built; at a K/V switch O(n) goes first and
+    // releases the slot.
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, B_K, 0, 0);
       constexpr uint32_t idesc_o = idesc_bf16_f32(128, D_H, 0, 1);
-      auto issue_s = [&](int n) -> bool {
-        const int st = n & 1;
-        if (!mbar_wait(&full[st], (n >> 1) & 1, abort_flag, p.status, 60)) return false;
+      int gen_have = -1;
+      auto wait_q = [&](int n, int* gen) -> bool {
+        const int qs = n % QS;
+        if (!mbar_wait(&q_full[qs], (n / QS) & 1, abort_flag, p.status, 60)) return false;
+        *gen = info[qs].gen;
+        return true;
+      };
+      auto issue_s = [&](int n, int gen) -> bool {
+        if (gen != gen_have) {
+          if (!mbar_wait(kv_full, gen & 1, abort_flag, p.status, 63)) return false;
+          gen_have = gen;
+        }
         tc_fence_after();
-        uint8_t* sQ = smem + st * SH::STAGE_BYTES;
-        const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sQ + SH::QP_BYTES);
-        const uint32_t tS = tmem_base + st * 256 + SH::TM_S;
+        const uint32_t q_base = smem_u32(smem + (n % QS) * SH::QP_BYTES), k_base = smem_u32(sK);
+        const uint32_t tS = tmem_base + (n & 1) * 256 + SH::TM_S;
 #pragma unroll
         for (int c = 0; c < SH::DCH; ++c)
 #pragma unroll
@@ -356,22 +416,26 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t bd = umma_desc(k_base + c * B_K * 128 + s * 32, 16, 1024, SW_128B);
             umma_bf16(tS, ad, bd, idesc_s, (c | s) != 0);
           }
-        umma_commit(&s_full[st]);
+        umma_commit(&s_full[n & 1]);
         return true;
       };
-      bool ok = my_tiles == 0 || issue_s(0);
+      int gcur = 0;
+      bool ok = my_tiles == 0 || (wait_q(0, &gcur) && issue_s(0, gcur));
       for (int n = 0; ok && n < my_tiles; ++n) {
         const int st = n & 1;
         const uint32_t ph = (n >> 1) & 1;
-        // the S accumulator of stage (n+1)&1 was last read by the softmax of
-        // tile n-1, whose p_full was waited for in the previous iteration
-        if (n + 1 < my_tiles && !issue_s(n + 1)) break;
+        const bool has_next = n + 1 < my_tiles;
+        int gnext = gcur;
+        if (has_next && !wait_q(n + 1, &gnext)) break;
+        const bool change = has_next && gnext != gcur;
+        // S of tile n+1 reuses the TMEM stage of tile n-1, whose P was waited
+        // for in the previous iteration
+        if (has_next && !change && !issue_s(n + 1, gnext)) break;
         if (!mbar_wait(&p_full[st], ph, abort_flag, p.status, 61)) break;
         if (!mbar_wait(&o_empty[st], ph ^ 1, abort_flag, p.status, 62)) break;
         tc_fence_after();
-        uint8_t* sQ = smem + st * SH::STAGE_BYTES;
-        const uint32_t q_base = smem_u32(sQ);
-        const uint32_t v_base = smem_u32(sQ + SH::QP_BYTES + SH::K_BYTES);
+        const uint32_t q_base = smem_u32(smem + (n % QS) * SH::QP_BYTES);
+        const uint32_t v_base = smem_u32(sV);
         const uint32_t tO = tmem_base + st * 256 + SH::TM_O;
 #pragma unroll
         for (int c = 0; c < SH::PCH; ++c)
@@ -385,12 +449,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             umma_bf16(tO, ad, bd, idesc_o, (c | s) != 0);
           }
         umma_commit(&o_full[st]);
-        umma_commit(&empty[st]);
+        umma_commit(&q_empty[n % QS]);
+        if (change) {
+          umma_commit(kv_empty);
+          if (!issue_s(n + 1, gnext)) break;
+        }
+        gcur = gnext;
       }
     }
   } else {
     // ------------------------------------------ softmax + epilogue groups --
-    const int grp = (warp - 2) >> 2;  // handles local tiles n with n % 2 == grp
+    const int grp = (warp - 2) >> 2;  // handles tiles n with n % 2 == grp
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const int q_local = row / p.R;
@@ -399,17 +468,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int n = grp; n < my_tiles; n += 2) {
       const int st = grp;
       const uint32_t ph = (n >> 1) & 1;
-      uint8_t* sP = smem + st * SH::STAGE_BYTES;
+      const int qs = n % QS;
+      uint8_t* sP = smem + qs * SH::QP_BYTES;
       const uint32_t tS = tmem_base + st * 256 + SH::TM_S + (static_cast<uint32_t>(quarter * 32) << 16);
       const uint32_t tO = tmem_base + st * 256 + SH::TM_O + (static_cast<uint32_t>(quarter * 32) << 16);
       if (!mbar_wait(&s_full[st], ph, abort_flag, p.status, 70)) break;
-      // full[st] cannot advance before this group's p_full, so this wait
-      // returns at once; it orders the producer's TileInfo writes before reads
-      if (!mbar_wait(&full[st], ph, abort_flag, p.status, 72)) break;
+      // q_full[qs] cannot advance before this tile's O MMA, so this returns at
+      // once; it orders the producer's TileInfo writes before the reads below
+      if (!mbar_wait(&q_full[qs], (n / QS) & 1, abort_flag, p.status, 72)) break;
       tc_fence_after();
-      const int ti_r = info[st].r, ti_b = info[st].b, ti_len = info[st].len;
+      const int ti_r = info[qs].r, ti_b = info[qs].b, ti_len = info[qs].len;
       const bool live = q_local < ti_len;
-      const uint32_t slot = live ? info[st].slot[q_local] : 0u;
+      const uint32_t slot = live ? info[qs].slot[q_local] : 0u;
       const int64_t i = p.q0 + slot / per_q;
       // ---- softmax over the block's keys (exp2 with the scale folded in)
       float sv[B_K];
@@ -441,7 +511,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         sv[j] = e;
         l += e;
       }
-      // P (bf16) into the stage's Q buffer, K-major 128B-swizzled rows
+      // P (bf16) over the stage's Q rows (consumed by S), K-major 128B-swizzled
 #pragma unroll
       for (int c = 0; c < B_K / 8; ++c) {
         uint4 w;
@@ -492,8 +562,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             w.w = *reinterpret_cast<uint32_t*>(&a3);
             *reinterpret_cast<uint4*>(dst + c * 32 + j) = w;
           }
+        p.c.part_lse[static_cast<int64_t>(slot) * p.G + g] = mx * p.scale + logf(l);
       }
-      if (useful) p.c.part_lse[static_cast<int64_t>(slot) * p.G + g] = mx * p.scale + logf(l);
     }
   }
 
@@ -515,74 +585,99 @@ struct MergeParams {
   ChunkBufs c;
 };
 
-// One warp per (query, head): LSE-weighted merge of the row's partials.  Lane
-// s reads slot s's LSE, the weights come from warp reductions, and the
-// partial rows are then fetched eight at a time so their loads overlap.
-template <int D_H>
+// LSE-weighted merge of each row's partials (split-K softmax normalisation).
+// W warps per (query, group); a lane owns E = min(32, G*D_H/(32*W)) consecutive
+// outputs of one head.  Per slot a lane needs its head's LSE (4 B) and E fp16
+// partial values: all of a row's LSEs are fetched at once, then the partial
+// rows four slots at a time, so each warp keeps several KB of loads in flight.
+// A warp writes its G x D_H output block as contiguous 16-byte pieces.
+template <int D_H, int E>
 __global__ void __launch_bounds__(256) attn_merge_kernel(const MergeParams p) {
-  constexpr int PER = D_H / 32;  // elements per lane
-  using Vec = typename std::conditional<PER == 4, uint2, uint32_t>::type;
+  static_assert(E % 8 == 0 && D_H % E == 0, "lane slice must be whole 16-byte pieces of one head");
+  constexpr int V16 = E / 8;  // 16-byte loads per slot
   const int lane = threadIdx.x & 31;
-  const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  if (row >= p.nq * p.H_q) return;
-  const int64_t il = row / p.H_q;
-  const int h = static_cast<int>(row - il * p.H_q);
-  const int r = h / p.G, g = h - r * p.G;
+  const int W = (p.G * D_H) / (32 * E);  // warps per (query, group)
+  const int64_t gw = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t unit = gw / W;
+  if (unit >= p.nq * p.H_kv) return;
+  const int wq = static_cast<int>(gw - unit * W);
+  const int64_t il = unit / p.H_kv;
+  const int r = static_cast<int>(unit - il * p.H_kv);
+  const int e0 = (wq * 32 + lane) * E;  // element offset inside the [G, D_H] block
+  const int g = e0 / D_H, d0 = e0 - g * D_H;
   const int64_t i = p.q0 + il;
   const int64_t b_i = i / p.B_k;
   const int64_t slot0 = (il * p.H_kv + r) * p.kk;
   int32_t myb = -1;
   if (lane < p.kk) myb = p.idx[(i * p.H_kv + r) * p.kk + lane];
-  const bool valid = lane < p.kk && myb >= 0 && myb <= b_i;
-  const float ls = valid ? p.c.part_lse[(slot0 + lane) * p.G + g] : -INFINITY;
-  float m = ls;
+  const unsigned use = __ballot_sync(0xFFFFFFFFu, lane < p.kk && myb >= 0 && myb <= b_i);
+  // this lane's head: LSE of every used slot
+  float ls[32];
+  float m = -INFINITY;
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-  const float w = valid ? __expf(ls - m) : 0.0f;
-  float wsum = w;
+  for (int s = 0; s < 32; ++s) {
+    ls[s] = -INFINITY;
+    if (s < p.kk && ((use >> s) & 1u)) ls[s] = p.c.part_lse[(slot0 + s) * p.G + g];
+  }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xFFFFFFFFu, wsum, o);
-  const unsigned use = __ballot_sync(0xFFFFFFFFu, valid);
-  float acc[PER];
+  for (int s = 0; s < 32; ++s) m = fmaxf(m, ls[s]);
+  float acc[E];
 #pragma unroll
-  for (int e = 0; e < PER; ++e) acc[e] = 0.0f;
-  const __half* base = p.c.part_o + (slot0 * p.G + g) * D_H + lane * PER;
+  for (int e = 0; e < E; ++e) acc[e] = 0.0f;
+  float wsum = 0.0f;
+  const __half* base = p.c.part_o + (slot0 * p.G + g) * D_H + d0;
   const int64_t stride = static_cast<int64_t>(p.G) * D_H;  // between slots
-  for (int s0 = 0; s0 < p.kk; s0 += 8) {
-    Vec x[8];
-    float wj[8];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
+  for (int s0 = 0; s0 < 32; s0 += 4) {  // fully unrolled: ls[] stays in registers
+    if (s0 >= p.kk) break;
+    uint4 x[4][V16];
+    float w[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
       const int s = s0 + j;
-      wj[j] = __shfl_sync(0xFFFFFFFFu, w, s & 31);
-      const bool on = s < p.kk && ((use >> (s & 31)) & 1u);
-      if (on) x[j] = *reinterpret_cast<const Vec*>(base + s * stride);
-      else x[j] = Vec{};
-      if (!on) wj[j] = 0.0f;
+      const bool on = s < p.kk && ((use >> s) & 1u);
+      w[j] = on ? __expf(ls[s] - m) : 0.0f;
+#pragma unroll
+      for (int u = 0; u < V16; ++u)
+        x[j][u] = on ? *reinterpret_cast<const uint4*>(base + s * stride + u * 8) : make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const __half2* hv = reinterpret_cast<const __half2*>(&x[j]);
+    for (int j = 0; j < 4; ++j) {
+      wsum += w[j];
 #pragma unroll
-      for (int e = 0; e < PER; e += 2) {
-        const float2 f = __half22float2(hv[e / 2]);
-        acc[e] = fmaf(wj[j], f.x, acc[e]);
-        acc[e + 1] = fmaf(wj[j], f.y, acc[e + 1]);
+      for (int u = 0; u < V16; ++u) {
+        const __half2* hv = reinterpret_cast<const __half2*>(&x[j][u]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __half22float2(hv[e]);
+          acc[u * 8 + 2 * e] = fmaf(w[j], f.x, acc[u * 8 + 2 * e]);
+          acc[u * 8 + 2 * e + 1] = fmaf(w[j], f.y, acc[u * 8 + 2 * e + 1]);
+        }
       }
     }
   }
-  __nv_bfloat16* dst = p.o + (i * p.H_q + h) * static_cast<int64_t>(D_H) + lane * PER;
+  const int h = r * p.G + g;
+  __nv_bfloat16* dst = p.o + (i * p.H_q + h) * static_cast<int64_t>(D_H) + d0;
   const float inv = wsum > 0.0f ? 1.0f / wsum : 0.0f;
 #pragma unroll
-  for (int e = 0; e < PER; e += 2)
-    *reinterpret_cast<__nv_bfloat162*>(dst + e) = __floats2bfloat162_rn(acc[e] * inv, acc[e + 1] * inv);
-  if (p.lse != nullptr && lane == 0) p.lse[i * p.H_q + h] = use ? m + logf(wsum) : -INFINITY;
+  for (int u = 0; u < V16; ++u) {
+    uint4 o4;
+    uint32_t* ow = reinterpret_cast<uint32_t*>(&o4);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      __nv_bfloat162 t = __floats2bfloat162_rn(acc[u * 8 + 2 * e] * inv, acc[u * 8 + 2 * e + 1] * inv);
+      ow[e] = *reinterpret_cast<uint32_t*>(&t);
+    }
+    *reinterpret_cast<uint4*>(dst + u * 8) = o4;
+  }
+  if (p.lse != nullptr && d0 == 0) p.lse[i * p.H_q + h] = use ? m + logf(wsum) : -INFINITY;
 }
 
 template <int D_H, int B_K>
 size_t p1_smem_bytes() {
   using SH = P1Shape<D_H, B_K>;
-  return 1024 + 2 * SH::STAGE_BYTES + 2 * sizeof(TileInfo) + 12 * 8 + 16;
+  return 1024 + SH::QS * SH::QP_BYTES + SH::K_BYTES + SH::V_BYTES + SH::QS * sizeof(TileInfo) +
+         (2 * SH::QS + 2 + 8) * 8 + 16;
 }
 
 template <int D_H, int B_K>
@@ -680,9 +775,17 @@ cudaError_t launch_typed(const AttnLaunch& a, cudaStream_t stream) {
     mp.G = G;
     mp.B_k = a.B_k;
     mp.c = c;
-    const int64_t rows = nq * a.H_q;
     prof_begin("attn_merge", stream);
-    attn_merge_kernel<D_H><<<static_cast<unsigned>((rows * 32 + 255) / 256), 256, 0, stream>>>(mp);
+    {
+      const int per_unit = G * D_H / 32;           // outputs per lane with one warp
+      const int E = per_unit >= 32 ? 32 : (per_unit >= 16 ? 16 : 8);
+      const int W = G * D_H / (32 * E);
+      const int64_t warps = nq * a.H_kv * W;
+      const unsigned blocks = static_cast<unsigned>((warps * 32 + 255) / 256);
+      if (E == 32) attn_merge_kernel<D_H, 32><<<blocks, 256, 0, stream>>>(mp);
+      else if (E == 16) attn_merge_kernel<D_H, 16><<<blocks, 256, 0, stream>>>(mp);
+      else attn_merge_kernel<D_H, 8><<<blocks, 256, 0, stream>>>(mp);
+    }
     prof_end(stream);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
