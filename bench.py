@@ -312,6 +312,105 @@ def run_msa(args, cfg, rank, world, local):
     return 0
 
 
+# -------------------------------------------------------------- decode arm --
+def run_decode(args, cfg, rank, world, local):
+    """Decode workload: S sequences, one new token each per step (append +
+    index scan + Top-k + gathered attention).  Reports us per step and per
+    token, and the HBM roofline of the step from its algorithmic bytes."""
+    import torch
+
+    import block_sparse_gqa_idx_b200 as msa
+    from block_sparse_gqa_idx_b200 import inputs
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    t0 = time.time()
+    st = inputs.decode_state(cfg, seed=cfg.seed + 1000 * rank)
+    gen_s = time.time() - t0
+
+    def dv(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    caches = {k: dv(st[k]) for k in ("k_cache", "v_cache", "k_idx_cache")}
+    seq_len = torch.from_numpy(st["seq_len"]).to(dev)
+    n_steps = args.warmup + args.steps
+    assert n_steps <= cfg.steps, "more steps than the cache has room for"
+    steps_in = [{k: dv(v) for k, v in inputs.decode_step_inputs(cfg, j, st["sink"]).items()}
+                for j in range(n_steps)]
+    S, H_q, H_kv, d_h, d_idx, B_k, kk = cfg.S, cfg.H_q, cfg.H_kv, cfg.d_h, cfg.d_idx, cfg.B_k, cfg.k
+    o = torch.empty((S, H_q, d_h), dtype=torch.bfloat16, device=dev)
+    idx = torch.empty((S, H_kv, kk), dtype=torch.int32, device=dev)
+    dd = msa.decode_dims(S, cfg.L_max, H_q, H_kv, d_h, d_idx, B_k, kk)
+    ws = torch.empty(msa.sparse_decode_workspace_size(dd), dtype=torch.uint8, device=dev)
+
+    def step(j):
+        x = steps_in[j]
+        msa.sparse_decode(x["q"], x["q_idx"], x["k_new"], x["v_new"], x["k_idx_new"],
+                          caches["k_cache"], caches["v_cache"], caches["k_idx_cache"], seq_len,
+                          B_k, kk, o=o, idx_out=idx, workspace=ws, stream=stream)
+
+    for j in range(args.warmup):
+        step(j)
+    torch.cuda.synchronize()
+    L_before = seq_len.clone()
+    clocks = Clocks(local)
+    clocks.start()
+    msa.profile_enable(True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for j in range(args.warmup, n_steps):
+        step(j)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    msa.profile_enable(False)
+    clk = clocks.stop()
+    prof = msa.profile_read()
+    ms = e0.elapsed_time(e1) / args.steps
+    code, where = msa.device_status(ws)
+    if code != 0:
+        raise RuntimeError(f"device status {code} at {where}")
+    # algorithmic bytes per step: the K_idx scan of every cached token, the
+    # selected K and V rows (causal part of each block), the new rows and q/o
+    L = L_before.double().mean().item() + (args.steps - 1) / 2.0
+    sel_rows = 0.0
+    sel = idx.cpu().numpy()
+    Lend = seq_len.cpu().numpy()
+    for s_ in range(S):
+        Li = int(Lend[s_])  # length after the last timed step (query at Li-1)
+        for r in range(H_kv):
+            for b in sel[s_, r]:
+                if b >= 0:
+                    sel_rows += min(B_k, Li - int(b) * B_k)
+    bytes_step = (S * L * d_idx * 2 + sel_rows * d_h * 2 * 2
+                  + S * (H_q * d_h * 2 * 2 + H_kv * d_idx * 2 + H_kv * d_h * 2 * 2 * 2 + d_idx * 2 * 2))
+    pk, pk_kind = peaks()
+    gbs = bytes_step / (ms * 1e-3) / 1e9
+    total_ms = sum(v[1] for v in prof.values())
+    kernels = {n: {"launches": v[0], "ms_per_step": v[1] / args.steps,
+                   "share": v[1] / total_ms if total_ms else None} for n, v in prof.items()}
+    scan_ms = prof.get("dec_scan", (1, 0.0))[1] / args.steps
+    scan_bytes = S * L * d_idx * 2
+    line = {
+        "metric": "MSA decode us/token @128K x64 sequences", "value": 1e3 * ms / S,
+        "unit": "us/token", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms, "us_per_step": 1e3 * ms, "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": cfg.name, "S": S, "L": L, "H_q": H_q, "H_kv": H_kv, "d_h": d_h,
+                   "d_idx": d_idx, "B_k": B_k, "k": kk,
+                   "l2": "caches 9.7 GB, larger than L2; no flush"},
+        "roofline": {"kernel": "decode step", "bound": "hbm", "achieved": gbs,
+                     "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": gbs / pk["hbm_gbs"],
+                     "traffic": None, "bytes_per_step": bytes_step, "peak_kind": pk_kind,
+                     "scan_kernel_gbs": scan_bytes / (scan_ms * 1e-3) / 1e9 if scan_ms else None},
+        "gpu_launches": sum(v[0] for v in prof.values()), "kernels": kernels, "clocks": clk,
+        "input_generation_s": gen_s,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -325,6 +424,11 @@ def main():
     args = ap.parse_args()
     world, rank, local = dist_init()
     cfg = workload(args.workload)
+    if args.workload == "decode":
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable": "decode reference arm not provided"}))
+            return 0
+        return run_decode(args, cfg, rank, world, local)
     if args.impl == "reference":
         return run_reference(args, cfg, rank, world)
     if world > 1:

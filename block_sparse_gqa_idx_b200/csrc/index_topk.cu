@@ -91,8 +91,11 @@ __device__ __forceinline__ float unorder_key(uint64_t key) {
   return __uint_as_float((o & 0x80000000u) ? (o & 0x7FFFFFFFu) : ~o);
 }
 
-template <int D_IDX>
-__global__ void __launch_bounds__(kThreads, 1)
+// REG: keep the running Top-(k-1) of each row in registers (k <= 16, a
+// branch-free sorted-insertion network); otherwise in a shared-memory min-heap.
+// 320 threads x 200 registers fit the 64K register file; one CTA per SM.
+template <int D_IDX, bool REG>
+__global__ void __maxnreg__(200)
     index_topk_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k, const IndexParams p) {
   using S = IndexShape<D_IDX>;
@@ -103,7 +106,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sB = sA + 2 * S::A_BYTES;                    // STAGES x B_BYTES
   uint64_t* heap = reinterpret_cast<uint64_t*>(sB + S::STAGES * S::B_BYTES);
   const int HS = p.k - 1;                               // heap size per row
-  uint64_t* bars = heap + static_cast<size_t>(kEpiThreads) * (HS > 0 ? HS : 1);
+  uint64_t* bars = heap + static_cast<size_t>(kEpiThreads) * ((!REG && HS > 0) ? HS : 1);
   uint64_t* a_full = bars;
   uint64_t* a_empty = bars + 1;
   uint64_t* b_full = bars + 2;
@@ -250,7 +253,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int nt = nt0 > nt1 ? nt0 : nt1;
       const int my_nt = mt == 0 ? nt0 : nt1;
       const int my_c = mt == 0 ? c0 : c1;
-      for (int s = 0; s < HS; ++s) heap[s * kEpiThreads + hrow] = 0ull;
+      // running Top-(k-1): register list (descending; slots before RL-HS hold
+      // +inf sentinels that never move) or shared-memory heap
+      constexpr int RL = 15;
+      float lv[RL];
+      int li[RL];
+      if constexpr (REG) {
+#pragma unroll
+        for (int s = 0; s < RL; ++s) {
+          lv[s] = s < RL - HS ? INFINITY : -INFINITY;
+          li[s] = -1;
+        }
+      } else {
+        for (int s = 0; s < HS; ++s) heap[s * kEpiThreads + hrow] = 0ull;
+      }
       float root = HS > 0 ? -INFINITY : INFINITY;
       bool ok = true;
       for (int t = 0; t < nt; ++t, ++acnt) {
@@ -300,29 +316,46 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int h = 0; h < per_tile; ++h) {
           const int b = t * per_tile + h;
-          if (b >= my_c || !(m[h] > root)) continue;
-          // replace the root (worst kept) and sift down; ties -> lower block
-          const uint64_t key = (static_cast<uint64_t>(order_bits(m[h])) << 32) |
-                               static_cast<uint64_t>(0xFFFFFFFFu - static_cast<uint32_t>(b));
-          int pos = 0;
-          while (true) {
-            const int c1i = 2 * pos + 1;
-            if (c1i >= HS) break;
-            uint64_t km = heap[c1i * kEpiThreads + hrow];
-            int cm = c1i;
-            if (c1i + 1 < HS) {
-              const uint64_t k2 = heap[(c1i + 1) * kEpiThreads + hrow];
-              if (k2 < km) {
-                km = k2;
-                cm = c1i + 1;
-              }
+          if constexpr (REG) {
+            // a candidate enters only above the last kept score (strict: an
+            // equal score belongs to a lower, earlier block, which stays)
+            const float x = b < my_c ? m[h] : -INFINITY;
+            if (!__any_sync(0xFFFFFFFFu, x > lv[RL - 1])) continue;
+            bool c[RL];
+#pragma unroll
+            for (int s2 = 0; s2 < RL; ++s2) c[s2] = x > lv[s2];
+#pragma unroll
+            for (int s2 = RL - 1; s2 > 0; --s2) {
+              lv[s2] = c[s2 - 1] ? lv[s2 - 1] : (c[s2] ? x : lv[s2]);
+              li[s2] = c[s2 - 1] ? li[s2 - 1] : (c[s2] ? b : li[s2]);
             }
-            if (km >= key) break;
-            heap[pos * kEpiThreads + hrow] = km;
-            pos = cm;
+            lv[0] = c[0] ? x : lv[0];
+            li[0] = c[0] ? b : li[0];
+          } else {
+            if (b >= my_c || !(m[h] > root)) continue;
+            // replace the root (worst kept) and sift down; ties -> lower block
+            const uint64_t key = (static_cast<uint64_t>(order_bits(m[h])) << 32) |
+                                 static_cast<uint64_t>(0xFFFFFFFFu - static_cast<uint32_t>(b));
+            int pos = 0;
+            while (true) {
+              const int c1i = 2 * pos + 1;
+              if (c1i >= HS) break;
+              uint64_t km = heap[c1i * kEpiThreads + hrow];
+              int cm = c1i;
+              if (c1i + 1 < HS) {
+                const uint64_t k2 = heap[(c1i + 1) * kEpiThreads + hrow];
+                if (k2 < km) {
+                  km = k2;
+                  cm = c1i + 1;
+                }
+              }
+              if (km >= key) break;
+              heap[pos * kEpiThreads + hrow] = km;
+              pos = cm;
+            }
+            heap[pos * kEpiThreads + hrow] = key;
+            root = unorder_key(heap[hrow]);
           }
-          heap[pos * kEpiThreads + hrow] = key;
-          root = unorder_key(heap[hrow]);
         }
       }
       if (!ok) break;
@@ -333,9 +366,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         int sel[32];
         int n = 0;
         sel[n++] = my_c;  // the local block (Eq. 7: always kept)
-        for (int s = 0; s < HS; ++s) {
-          const uint64_t key = heap[s * kEpiThreads + hrow];
-          if (key != 0ull) sel[n++] = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(key));
+        if constexpr (REG) {
+#pragma unroll
+          for (int s = 0; s < RL; ++s)
+            if (li[s] >= 0) sel[n++] = li[s];
+        } else {
+          for (int s = 0; s < HS; ++s) {
+            const uint64_t key = heap[s * kEpiThreads + hrow];
+            if (key != 0ull) sel[n++] = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(key));
+          }
         }
         for (int a = 1; a < n; ++a) {  // ascending
           const int x = sel[a];
@@ -361,9 +400,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 template <int D_IDX>
-size_t index_smem_bytes(int k) {
+size_t index_smem_bytes(int k, bool reg) {
   using S = IndexShape<D_IDX>;
-  const int hs = k - 1 > 0 ? k - 1 : 1;
+  const int hs = (!reg && k - 1 > 0) ? k - 1 : 1;
   return 1024 + 2 * S::A_BYTES + S::STAGES * S::B_BYTES + static_cast<size_t>(kEpiThreads) * hs * 8 +
          (4 + 2 * S::STAGES + 2) * 8 + 16;
 }
@@ -393,16 +432,17 @@ cudaError_t launch_typed(const IndexLaunch& a, cudaStream_t stream) {
   p.n_units = (p.n_mtiles + 1) / 2;
   p.idx_out = a.idx_out;
   p.status = a.status;
-  const size_t smem = index_smem_bytes<D_IDX>(a.k);
-  cudaError_t e = cudaFuncSetAttribute(index_topk_kernel<D_IDX>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+  const bool reg = a.k <= 16;
+  const size_t smem = index_smem_bytes<D_IDX>(a.k, reg);
+  auto kern = reg ? index_topk_kernel<D_IDX, true> : index_topk_kernel<D_IDX, false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   int grid = num_sms();
   if (grid > p.n_units) grid = p.n_units;
   if (grid < 1) grid = 1;
   prof_begin("index_topk", stream);
-  index_topk_kernel<D_IDX><<<grid, kThreads, smem, stream>>>(tq, tk, p);
+  kern<<<grid, kThreads, smem, stream>>>(tq, tk, p);
   prof_end(stream);
   return cudaGetLastError();
 }

@@ -248,7 +248,7 @@ __device__ __forceinline__ int find_key(const int32_t* tile_off, int64_t nkeys, 
 //   warp 1      MMA issuer (lane 0) and TMEM owner
 //   warps 2..9  softmax + epilogue, group (w-2)/4
 template <int D_H, int B_K>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __maxnreg__(200)
     attn_phase1_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const P1Params p) {
