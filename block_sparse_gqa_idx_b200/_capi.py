@@ -48,7 +48,7 @@ class msa_kernel_time(ctypes.Structure):
 EXPORTS = ("msa_index_topk_workspace", "msa_index_topk", "msa_sparse_attn_fwd_workspace",
            "msa_sparse_attn_fwd", "msa_sparse_decode_workspace", "msa_sparse_decode",
            "msa_get_device_status", "msa_profile_enable", "msa_profile_read",
-           "msa_status_string", "msa_version", "msa_sparse_decode_noalloc")
+           "msa_status_string", "msa_version", "msa_sparse_decode_noalloc", "msa_last_error")
 
 
 def _load() -> ctypes.CDLL:
@@ -82,6 +82,8 @@ def _load() -> ctypes.CDLL:
     lib.msa_profile_read.restype = ctypes.c_int32
     lib.msa_status_string.argtypes = [I32]
     lib.msa_status_string.restype = ctypes.c_char_p
+    lib.msa_last_error.argtypes = []
+    lib.msa_last_error.restype = ctypes.c_char_p
     lib.msa_version.argtypes = []
     lib.msa_version.restype = ctypes.c_char_p
     return lib
@@ -96,7 +98,10 @@ def version() -> str:
 
 def _raise(what: str, st: int) -> None:
     if st != 0:
-        raise MSAError(what, st, LIB.msa_status_string(st).decode())
+        text = LIB.msa_status_string(st).decode()
+        if st == 4:
+            text += ": " + LIB.msa_last_error().decode()
+        raise MSAError(what, st, text)
 
 
 def _ptr(t: Optional[torch.Tensor]):

@@ -1,9 +1,9 @@
 // decode.cu -- one MSA decode step for S independent sequences.
 //
 // Per sequence s with L = seq_len[s]:
-//   append   k/v/k_idx of the new token at row L (Eq. 1: the query sees i <= t,
-//            itself included)
-//   scan     Eq. 6 for the single query i = L over the full blocks 0..b_i-1
+//   scan     append k/v/k_idx of the new token at row L (Eq. 1: the query
+//            sees i <= t, itself included), then Eq. 6 for the single query
+//            i = L over the full blocks 0..b_i-1
 //            (b_i = L / B_k; the local block b_i is forced and needs no score):
 //            block maxima of the H_kv index-query dots, streamed from the K_idx
 //            cache.  HBM-bound: 2*d_idx bytes per cached token.
@@ -75,33 +75,6 @@ struct DecParams {
   DevStatus* status;
 };
 
-// ------------------------------------------------------------------ append --
-__global__ void dec_append_kernel(const DecParams p) {
-  const int s = blockIdx.x;
-  const int64_t L = p.seq_len[s];
-  if (L < 0 || L >= p.L_max) {
-    if (threadIdx.x == 0) {
-      p.w.Lcur[s] = -1;
-      report(p.status, DEV_ERR_CACHE_FULL, 80, s, static_cast<int>(L));
-    }
-    return;
-  }
-  if (threadIdx.x == 0) p.w.Lcur[s] = static_cast<int32_t>(L);
-  const int kv16 = p.H_kv * p.d_h / 8;  // 16-byte pieces per K (or V) row
-  const int ki16 = p.d_idx / 8;
-  const uint4* kn = reinterpret_cast<const uint4*>(p.k_new + static_cast<int64_t>(s) * p.H_kv * p.d_h);
-  const uint4* vn = reinterpret_cast<const uint4*>(p.v_new + static_cast<int64_t>(s) * p.H_kv * p.d_h);
-  const uint4* kin = reinterpret_cast<const uint4*>(p.k_idx_new + static_cast<int64_t>(s) * p.d_idx);
-  uint4* kc = reinterpret_cast<uint4*>(p.k_cache + (s * p.L_max + L) * p.H_kv * p.d_h);
-  uint4* vc = reinterpret_cast<uint4*>(p.v_cache + (s * p.L_max + L) * p.H_kv * p.d_h);
-  uint4* kic = reinterpret_cast<uint4*>(p.k_idx_cache + (s * p.L_max + L) * p.d_idx);
-  for (int t = threadIdx.x; t < kv16; t += blockDim.x) {
-    kc[t] = kn[t];
-    vc[t] = vn[t];
-  }
-  for (int t = threadIdx.x; t < ki16; t += blockDim.x) kic[t] = kin[t];
-}
-
 // -------------------------------------------------------------------- scan --
 __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
                                                uint32_t b1) {
@@ -124,8 +97,31 @@ __global__ void __launch_bounds__(256) dec_scan_kernel(const DecParams p, int ns
   constexpr int NMMA = D_IDX / 16;    // MMAs per 16-key tile
   constexpr int NV = DT / 8;          // 16-byte loads per key row
   const int s = blockIdx.y;
-  const int64_t L = p.w.Lcur[s];
-  if (L < 0) return;
+  const int64_t L = p.seq_len[s];  // written back (L + 1) only by the merge kernel
+  if (L < 0 || L >= p.L_max) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+      p.w.Lcur[s] = -1;
+      report(p.status, DEV_ERR_CACHE_FULL, 80, s, static_cast<int>(L));
+    }
+    return;
+  }
+  if (blockIdx.x == 0) {
+    // append the new token's rows at position L (the scan below never reads
+    // them: they lie in the local block, which is forced, not scored)
+    const int kv16 = p.H_kv * p.d_h / 8;  // 16-byte pieces per K (or V) row
+    const uint4* kn = reinterpret_cast<const uint4*>(p.k_new + static_cast<int64_t>(s) * p.H_kv * p.d_h);
+    const uint4* vn = reinterpret_cast<const uint4*>(p.v_new + static_cast<int64_t>(s) * p.H_kv * p.d_h);
+    const uint4* kin = reinterpret_cast<const uint4*>(p.k_idx_new + static_cast<int64_t>(s) * D_IDX);
+    uint4* kc = reinterpret_cast<uint4*>(p.k_cache + (s * p.L_max + L) * p.H_kv * p.d_h);
+    uint4* vc = reinterpret_cast<uint4*>(p.v_cache + (s * p.L_max + L) * p.H_kv * p.d_h);
+    uint4* kic = reinterpret_cast<uint4*>(p.k_idx_cache + (s * p.L_max + L) * D_IDX);
+    for (int t = threadIdx.x; t < kv16; t += blockDim.x) {
+      kc[t] = kn[t];
+      vc[t] = vn[t];
+    }
+    for (int t = threadIdx.x; t < D_IDX / 8; t += blockDim.x) kic[t] = kin[t];
+    if (threadIdx.x == 0) p.w.Lcur[s] = static_cast<int32_t>(L);
+  }
   const int64_t b_i = L / p.B_k;  // candidate blocks 0 .. b_i-1
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
@@ -189,24 +185,30 @@ __device__ __forceinline__ uint64_t pack_key(float v, int b) {
   return (static_cast<uint64_t>(u) << 32) | (0xFFFFFFFFu - static_cast<uint32_t>(b));
 }
 
+// One CTA (8 warps) per (sequence, group).  Warp w scans blocks w*32+lane,
+// +256, ... keeping per-lane sorted lists in shared memory, and reduces them
+// to its best k-1 in k-1 rounds of warp argmax.  Warp 0 then ranks the 8
+// warps' winners against each other (count of larger keys), keeps the k-1
+// best, adds the local block and writes the set in ascending block order.
 __global__ void __launch_bounds__(256) dec_topk_kernel(const DecParams p) {
-  extern __shared__ uint64_t lists[];  // [8 warps][k-1 slots][32 lanes]
+  extern __shared__ uint64_t lists[];  // [8 warps][k-1][32 lanes] + winners [8][k-1]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int pair = blockIdx.x * 8 + warp;
-  if (pair >= p.S * p.H_kv) return;
+  const int pair = blockIdx.x;
   const int s = pair / p.H_kv, r = pair - s * p.H_kv;
   const int64_t L = p.w.Lcur[s];
   if (L < 0) return;
   const int b_i = static_cast<int>(L / p.B_k);
   const int HS = p.kk - 1;
-  uint64_t* my = lists + static_cast<size_t>(warp) * (HS > 0 ? HS : 1) * 32;
+  const int hs1 = HS > 0 ? HS : 1;
+  uint64_t* my = lists + static_cast<size_t>(warp) * hs1 * 32;
+  uint64_t* win = lists + static_cast<size_t>(8) * hs1 * 32;  // [8][hs1]
+  __shared__ int32_t chosen[33];
   const float* Mrow = p.w.M + (static_cast<int64_t>(s) * p.H_kv + r) * p.Bmax;
   int cnt = 0;
   uint64_t worst = 0;  // smallest kept key once the list is full
-  for (int b = lane; b < b_i && HS > 0; b += 32) {
+  for (int b = warp * 32 + lane; b < b_i && HS > 0; b += 256) {
     const uint64_t key = pack_key(Mrow[b], b);
     if (cnt == HS && key <= worst) continue;
-    // insert into the lane's descending list
     int pos = cnt < HS ? cnt : HS - 1;
     while (pos > 0 && my[(pos - 1) * 32 + lane] < key) {
       my[pos * 32 + lane] = my[(pos - 1) * 32 + lane];
@@ -216,11 +218,9 @@ __global__ void __launch_bounds__(256) dec_topk_kernel(const DecParams p) {
     if (cnt < HS) ++cnt;
     worst = my[(cnt - 1) * 32 + lane];
   }
-  // k-1 rounds of warp argmax over the lanes' list heads
+  // this warp's best HS keys (0 = none), by rounds of warp argmax
   int head = 0;
-  int32_t mine = -1;  // lane j keeps the j-th winner
-  const int rounds = HS < b_i ? HS : b_i;
-  for (int round = 0; round < rounds; ++round) {
+  for (int round = 0; round < HS; ++round) {
     const uint64_t cand = head < cnt ? my[head * 32 + lane] : 0ull;
     uint64_t best = cand;
 #pragma unroll
@@ -229,23 +229,38 @@ __global__ void __launch_bounds__(256) dec_topk_kernel(const DecParams p) {
       best = other > best ? other : best;
     }
     if (cand == best && cand != 0ull) ++head;
-    if (lane == round) mine = static_cast<int32_t>(0xFFFFFFFFu - static_cast<uint32_t>(best));
+    if (lane == 0) win[warp * hs1 + round] = best;
   }
-  if (lane == rounds) mine = b_i;  // the local block (Eq. 7: always kept)
-  // ascending order: rank of each lane's block among the valid ones
-  const int nsel = rounds + 1;
-  int rank = 0;
-  for (int j = 0; j < nsel; ++j) {
-    const int32_t x = __shfl_sync(0xFFFFFFFFu, mine, j);
-    if (lane < nsel && x < mine) ++rank;
+  __syncthreads();
+  if (warp != 0) return;
+  // rank the 8 warps' winners: a key is kept if fewer than HS keys beat it
+  const int T = 8 * HS;
+  int nkept = 0;
+  for (int base = 0; base < T; base += 32) {
+    const int j = base + lane;
+    const uint64_t mine = j < T ? win[j] : 0ull;
+    int rank = 0;
+    if (mine != 0ull)
+      for (int m = 0; m < T; ++m) rank += win[m] > mine ? 1 : 0;
+    const bool keep = mine != 0ull && rank < HS;
+    if (keep) chosen[rank] = static_cast<int32_t>(0xFFFFFFFFu - static_cast<uint32_t>(mine));
+    nkept += __popc(__ballot_sync(0xFFFFFFFFu, keep));
   }
+  __syncwarp();
+  if (lane == 0) chosen[nkept] = b_i;  // the local block (Eq. 7: always kept)
+  __syncwarp();
+  const int nsel = nkept + 1;
+  const int32_t v = lane < nsel ? chosen[lane] : -1;
+  int pos = 0;
+  for (int m = 0; m < nsel; ++m) pos += chosen[m] < v ? 1 : 0;
   int32_t* dst = p.w.sel + (static_cast<int64_t>(s) * p.H_kv + r) * p.kk;
-  if (lane < nsel) dst[rank] = mine;
-  else if (lane < p.kk) dst[lane] = -1;
-  if (p.idx_out != nullptr) {
-    int32_t* d2 = p.idx_out + (static_cast<int64_t>(s) * p.H_kv + r) * p.kk;
-    if (lane < nsel) d2[rank] = mine;
-    else if (lane < p.kk) d2[lane] = -1;
+  int32_t* dst2 = p.idx_out != nullptr ? p.idx_out + (static_cast<int64_t>(s) * p.H_kv + r) * p.kk : nullptr;
+  if (lane < nsel) {
+    dst[pos] = v;
+    if (dst2) dst2[pos] = v;
+  } else if (lane < p.kk) {
+    dst[lane] = -1;
+    if (dst2) dst2[lane] = -1;
   }
 }
 
@@ -292,8 +307,8 @@ __global__ void __launch_bounds__(128) dec_attend_kernel(const __grid_constant__
   uint8_t* sK = smem;
   uint8_t* sV = smem + BK * D_H * 2;
   float* red = reinterpret_cast<float*>(sV + BK * D_H * 2);  // [4][16] m, [4][16] l
-  float* obuf = red + 128;                                    // [4][16][D_H]
-  uint64_t* bar = reinterpret_cast<uint64_t*>(obuf + 4 * 16 * D_H);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(red + 128);    // [0] K landed, [1] V landed
+  float* obuf = reinterpret_cast<float*>(smem);  // [4][16][D_H], over K/V once both are used
 
   const int item = blockIdx.x;  // (s, r, slot)
   const int slot = item % p.kk;
@@ -308,17 +323,17 @@ __global__ void __launch_bounds__(128) dec_attend_kernel(const __grid_constant__
   const int g = lane >> 2, t = lane & 3;
 
   if (threadIdx.x == 0) {
-    mbar_init(bar, 1);
+    mbar_init(&bar[0], 1);
+    mbar_init(&bar[1], 1);
     fence_mbar_init();
   }
   __syncthreads();
   if (threadIdx.x == 0) {
-    mbar_arrive_expect_tx(bar, 2 * BK * D_H * 2);
     const int row0 = static_cast<int>(s * p.L_max + static_cast<int64_t>(b) * BK);
-    for (int c = 0; c < D_H / 64; ++c) {
-      tma_load_3d(sK + c * BK * 128, &tm_k, bar, c * 64, r, row0);
-      tma_load_3d(sV + c * BK * 128, &tm_v, bar, c * 64, r, row0);
-    }
+    mbar_arrive_expect_tx(&bar[0], BK * D_H * 2);
+    for (int c = 0; c < D_H / 64; ++c) tma_load_3d(sK + c * BK * 128, &tm_k, &bar[0], c * 64, r, row0);
+    mbar_arrive_expect_tx(&bar[1], BK * D_H * 2);
+    for (int c = 0; c < D_H / 64; ++c) tma_load_3d(sV + c * BK * 128, &tm_v, &bar[1], c * 64, r, row0);
   }
   // Q fragments (rows = heads, zero beyond G) while the tiles land.
   uint32_t qa[D_H / 16][4];
@@ -333,7 +348,7 @@ __global__ void __launch_bounds__(128) dec_attend_kernel(const __grid_constant__
       qa[ks][3] = g + 8 < p.G ? *reinterpret_cast<const uint32_t*>(qb + (g + 8) * D_H + d + 8) : 0u;
     }
   }
-  bool ok = mbar_wait(bar, 0, nullptr, p.status, 90);
+  bool ok = mbar_wait(&bar[0], 0, nullptr, p.status, 90);
   const int kw0 = warp * KW;  // first key (within the block) of this warp
   float sacc[NT][4];
 #pragma unroll
@@ -397,6 +412,7 @@ __global__ void __launch_bounds__(128) dec_attend_kernel(const __grid_constant__
   float oacc[DT][4];
 #pragma unroll
   for (int n = 0; n < DT; ++n) oacc[n][0] = oacc[n][1] = oacc[n][2] = oacc[n][3] = 0.f;
+  ok = ok && mbar_wait(&bar[1], 0, nullptr, p.status, 91);
   if (ok) {
     const uint32_t vb = smem_u32(sV);
 #pragma unroll
@@ -414,7 +430,9 @@ __global__ void __launch_bounds__(128) dec_attend_kernel(const __grid_constant__
       }
     }
   }
-  // merge the four warps' (m, l, O) through shared memory (log2 domain)
+  // merge the four warps' (m, l, O) through shared memory (log2 domain);
+  // obuf overlays the K/V tiles, so every warp must be done with them first
+  __syncthreads();
   if (t == 0) {
     red[warp * 16 + g] = m_lo;
     red[warp * 16 + g + 8] = m_hi;
@@ -457,6 +475,9 @@ __global__ void __launch_bounds__(128) dec_attend_kernel(const __grid_constant__
 }
 
 // ------------------------------------------------------------------- merge --
+// One warp per (sequence, head): lane s reads slot s's selection and LSE, the
+// weights come from warp reductions, then every slot's partial row (lane:
+// D_H/32 consecutive floats) is fetched with all loads in flight.
 template <int D_H>
 __global__ void __launch_bounds__(256) dec_merge_kernel(const DecParams p) {
   constexpr int PER = D_H / 32;
@@ -467,38 +488,60 @@ __global__ void __launch_bounds__(256) dec_merge_kernel(const DecParams p) {
   const int r = h / p.G, g = h - r * p.G;
   const int64_t L = p.w.Lcur[s];
   if (L < 0) return;
-  const int32_t* sel = p.w.sel + (static_cast<int64_t>(s) * p.H_kv + r) * p.kk;
-  const unsigned use = __ballot_sync(0xFFFFFFFFu, lane < p.kk && sel[lane < p.kk ? lane : 0] >= 0);
-  float m = -INFINITY, wsum = 0.f, acc[PER];
+  const int64_t base_slot = (static_cast<int64_t>(s) * p.H_kv + r) * p.kk;
+  const bool valid = lane < p.kk && p.w.sel[base_slot + (lane < p.kk ? lane : 0)] >= 0;
+  float ls = valid ? p.w.part_lse[(base_slot + lane) * p.G + g] : -INFINITY;
+  float m = ls;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+  const float w = (valid && ls != -INFINITY) ? __expf(ls - m) : 0.f;
+  float wsum = w;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xFFFFFFFFu, wsum, o);
+  const unsigned use = __ballot_sync(0xFFFFFFFFu, w > 0.f);
+  float acc[PER];
 #pragma unroll
   for (int e = 0; e < PER; ++e) acc[e] = 0.f;
-  unsigned rest = use;
-  while (rest) {
-    const int sl = __ffs(rest) - 1;
-    rest &= rest - 1;
-    const int64_t pslot = ((static_cast<int64_t>(s) * p.H_kv + r) * p.kk + sl) * p.G + g;
-    const float ls = p.w.part_lse[pslot];
-    if (ls == -INFINITY) continue;
-    const float* src = p.w.part_o + pslot * D_H + lane * PER;
-    const float mn = fmaxf(m, ls);
-    const float a_old = __expf(m - mn), a_new = __expf(ls - mn);
+  const float* src = p.w.part_o + (base_slot * p.G + g) * D_H + lane * PER;
+  const int64_t stride = static_cast<int64_t>(p.G) * D_H;
 #pragma unroll
-    for (int e = 0; e < PER; ++e) acc[e] = acc[e] * a_old + src[e] * a_new;
-    wsum = wsum * a_old + a_new;
-    m = mn;
+  for (int s0 = 0; s0 < 32; s0 += 8) {
+    if (s0 >= p.kk) break;
+    float x[8][PER];
+    float wj[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int sl = s0 + j;
+      wj[j] = __shfl_sync(0xFFFFFFFFu, w, sl);
+      const bool on = (use >> sl) & 1u;
+#pragma unroll
+      for (int e = 0; e < PER; e += 4) {
+        const float4 f = on ? *reinterpret_cast<const float4*>(src + sl * stride + e)
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+        x[j][e] = f.x;
+        x[j][e + 1] = f.y;
+        x[j][e + 2] = f.z;
+        x[j][e + 3] = f.w;
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+#pragma unroll
+      for (int e = 0; e < PER; ++e) acc[e] = fmaf(wj[j], x[j][e], acc[e]);
   }
   const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
   __nv_bfloat16* dst = p.o + (static_cast<int64_t>(s) * p.H_q + h) * D_H + lane * PER;
 #pragma unroll
   for (int e = 0; e < PER; e += 2)
     *reinterpret_cast<__nv_bfloat162*>(dst + e) = __floats2bfloat162_rn(acc[e] * inv, acc[e + 1] * inv);
-  // seq_len is read only by the append kernel; the rest of the step uses Lcur
+  // seq_len is read only by the scan kernel; the rest of the step uses Lcur
   if (h == 0 && lane == 0) p.seq_len[s] = static_cast<int32_t>(L + 1);
 }
 
 template <int D_H, int BK>
 size_t attend_smem() {
-  return 1024 + 2 * BK * D_H * 2 + 128 * 4 + 4 * 16 * D_H * 4 + 16;
+  static_assert(4 * 16 * D_H * 4 <= 2 * BK * D_H * 2, "warp-merge buffer must fit over K/V");
+  return 1024 + 2 * BK * D_H * 2 + 128 * 4 + 16;
 }
 
 template <int D_H, int BK>
@@ -571,11 +614,7 @@ cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t stream) {
   if (need > a.ws_bytes) return cudaErrorInvalidValue;
   p.status = a.status;
 
-  prof_begin("dec_append", stream);
-  dec_append_kernel<<<a.S, 128, 0, stream>>>(p);
-  prof_end(stream);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  cudaError_t e = cudaSuccess;
   switch (a.d_idx) {
     case 32: e = launch_scan<32>(p, stream); break;
     case 64: e = launch_scan<64>(p, stream); break;
@@ -584,12 +623,12 @@ cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t stream) {
   }
   if (e != cudaSuccess) return e;
   const int hs = a.kk - 1 > 0 ? a.kk - 1 : 1;
-  const size_t topk_smem = 8 * hs * 32 * sizeof(uint64_t);
+  const size_t topk_smem = (8 * hs * 32 + 8 * hs) * sizeof(uint64_t);
   e = cudaFuncSetAttribute(dec_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(topk_smem));
   if (e != cudaSuccess) return e;
   prof_begin("dec_topk", stream);
-  dec_topk_kernel<<<(a.S * a.H_kv + 7) / 8, 256, topk_smem, stream>>>(p);
+  dec_topk_kernel<<<a.S * a.H_kv, 256, topk_smem, stream>>>(p);
   prof_end(stream);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;

@@ -93,9 +93,10 @@ __device__ __forceinline__ float unorder_key(uint64_t key) {
 
 // REG: keep the running Top-(k-1) of each row in registers (k <= 16, a
 // branch-free sorted-insertion network); otherwise in a shared-memory min-heap.
-// 320 threads x 200 registers fit the 64K register file; one CTA per SM.
+// 10 warps: three of them share one SM sub-partition's 16K registers, so the
+// kernel lives within 168 registers per thread; one CTA per SM.
 template <int D_IDX, bool REG>
-__global__ void __maxnreg__(200)
+__global__ void __launch_bounds__(kThreads, 1)
     index_topk_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k, const IndexParams p) {
   using S = IndexShape<D_IDX>;
@@ -276,43 +277,51 @@ __global__ void __maxnreg__(200)
           break;
         }
         tc_fence_after();
-        uint32_t r0[32], r1[32], r2[32], r3[32];
+        // the row's 128 scores in two halves of 64 columns: the first half is
+        // reduced before the second is loaded, which keeps the peak register
+        // use low enough for the running Top-k list
         const bool active = t < my_nt;
+        const uint32_t ta = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                            acc * 256 + mt * 128;
+        float x0 = -INFINITY, x1 = -INFINITY, x2 = -INFINITY, x3 = -INFINITY;
         if (active) {
-          const uint32_t ta = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
-                              acc * 256 + mt * 128;
-          tmem_ld32(ta + 0, r0);
-          tmem_ld32(ta + 32, r1);
-          tmem_ld32(ta + 64, r2);
-          tmem_ld32(ta + 96, r3);
+          uint32_t ra[32], rb[32];
+          tmem_ld32(ta + 0, ra);
+          tmem_ld32(ta + 32, rb);
           tmem_wait_ld();
+          x0 = __uint_as_float(ra[0]);
+          x1 = __uint_as_float(rb[0]);
+#pragma unroll
+          for (int j = 1; j < 31; j += 2) {
+            x0 = fmax3(x0, __uint_as_float(ra[j]), __uint_as_float(ra[j + 1]));
+            x1 = fmax3(x1, __uint_as_float(rb[j]), __uint_as_float(rb[j + 1]));
+          }
+          x0 = fmaxf(x0, __uint_as_float(ra[31]));
+          x1 = fmaxf(x1, __uint_as_float(rb[31]));
+          tmem_ld32(ta + 64, ra);
+          tmem_ld32(ta + 96, rb);
+          tmem_wait_ld();
+          x2 = __uint_as_float(ra[0]);
+          x3 = __uint_as_float(rb[0]);
+#pragma unroll
+          for (int j = 1; j < 31; j += 2) {
+            x2 = fmax3(x2, __uint_as_float(ra[j]), __uint_as_float(ra[j + 1]));
+            x3 = fmax3(x3, __uint_as_float(rb[j]), __uint_as_float(rb[j + 1]));
+          }
+          x2 = fmaxf(x2, __uint_as_float(ra[31]));
+          x3 = fmaxf(x3, __uint_as_float(rb[31]));
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[acc]);
         if (!active) continue;
         float m[2];
-        {
-          float x0 = __uint_as_float(r0[0]), x1 = __uint_as_float(r1[0]);
-          float x2 = __uint_as_float(r2[0]), x3 = __uint_as_float(r3[0]);
-#pragma unroll
-          for (int j = 1; j < 31; j += 2) {
-            x0 = fmax3(x0, __uint_as_float(r0[j]), __uint_as_float(r0[j + 1]));
-            x1 = fmax3(x1, __uint_as_float(r1[j]), __uint_as_float(r1[j + 1]));
-            x2 = fmax3(x2, __uint_as_float(r2[j]), __uint_as_float(r2[j + 1]));
-            x3 = fmax3(x3, __uint_as_float(r3[j]), __uint_as_float(r3[j + 1]));
-          }
-          x0 = fmaxf(x0, __uint_as_float(r0[31]));
-          x1 = fmaxf(x1, __uint_as_float(r1[31]));
-          x2 = fmaxf(x2, __uint_as_float(r2[31]));
-          x3 = fmaxf(x3, __uint_as_float(r3[31]));
-          if (per_tile == 1) {
-            m[0] = fmax3(x0, x1, fmaxf(x2, x3));
-            m[1] = -INFINITY;
-          } else {
-            m[0] = fmaxf(x0, x1);
-            m[1] = fmaxf(x2, x3);
-          }
+        if (per_tile == 1) {
+          m[0] = fmax3(x0, x1, fmaxf(x2, x3));
+          m[1] = -INFINITY;
+        } else {
+          m[0] = fmaxf(x0, x1);
+          m[1] = fmaxf(x2, x3);
         }
         for (int h = 0; h < per_tile; ++h) {
           const int b = t * per_tile + h;

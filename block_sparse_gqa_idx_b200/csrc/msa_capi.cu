@@ -121,7 +121,13 @@ msa_status check_common(int64_t N, int H_q, int H_kv, int d_h, int d_idx, int B_
   return MSA_OK;
 }
 
-msa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? MSA_OK : MSA_ERR_CUDA; }
+thread_local cudaError_t g_last_cuda_error = cudaSuccess;
+
+msa_status from_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return MSA_OK;
+  g_last_cuda_error = e;
+  return MSA_ERR_CUDA;
+}
 
 msa::DevStatus* status_of(void* ws) { return reinterpret_cast<msa::DevStatus*>(ws); }
 
@@ -143,6 +149,10 @@ const char* msa_status_string(msa_status s) {
 
 const char* msa_version(void) { return "msa-b200 0.1 (sm_100a)"; }
 
+const char* msa_last_error(void) {
+  return g_last_cuda_error == cudaSuccess ? "no CUDA error" : cudaGetErrorString(g_last_cuda_error);
+}
+
 // ------------------------------------------------------------ Index Branch --
 size_t msa_index_topk_workspace(const msa_dims* d) {
   (void)d;
@@ -162,7 +172,7 @@ msa_status msa_index_topk(const msa_dims* d, const void* q_idx, const void* k_id
   if (d->N * d->H_kv >= (int64_t(1) << 31) - 256) return MSA_ERR_UNSUPPORTED;
   if (ws_bytes < msa_index_topk_workspace(d)) return MSA_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(ws, 0, sizeof(msa::DevStatus), s) != cudaSuccess) return MSA_ERR_CUDA;
+  if (from_cuda(cudaMemsetAsync(ws, 0, sizeof(msa::DevStatus), s)) != MSA_OK) return MSA_ERR_CUDA;
   msa::IndexLaunch a;
   a.q_idx = q_idx;
   a.k_idx = k_idx;
@@ -201,7 +211,7 @@ msa_status msa_sparse_attn_fwd(const msa_dims* d, const void* q, const void* k, 
     return MSA_ERR_UNSUPPORTED;
   if (ws_bytes < msa_sparse_attn_fwd_workspace(d)) return MSA_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(ws, 0, sizeof(msa::DevStatus), s) != cudaSuccess) return MSA_ERR_CUDA;
+  if (from_cuda(cudaMemsetAsync(ws, 0, sizeof(msa::DevStatus), s)) != MSA_OK) return MSA_ERR_CUDA;
   msa::AttnLaunch a;
   a.q = q;
   a.k = k;
@@ -251,7 +261,7 @@ msa_status msa_sparse_decode(const msa_decode_dims* d, const void* q, const void
   if (d->L_max >= (int64_t(1) << 31)) return MSA_ERR_UNSUPPORTED;
   if (ws_bytes < msa_sparse_decode_workspace(d)) return MSA_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(ws, 0, sizeof(msa::DevStatus), s) != cudaSuccess) return MSA_ERR_CUDA;
+  if (from_cuda(cudaMemsetAsync(ws, 0, sizeof(msa::DevStatus), s)) != MSA_OK) return MSA_ERR_CUDA;
   msa::DecodeLaunch a;
   a.q = q;
   a.q_idx = q_idx;

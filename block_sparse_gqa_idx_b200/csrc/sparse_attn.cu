@@ -46,7 +46,7 @@ struct ChunkBufs {
   int32_t* cursor;    // [nkeys]
   int32_t* n_tiles;   // [1]
   uint32_t* entries;  // [Nc * H_kv * k]
-  __half* part_o;     // [Nc * H_kv * k, G, d_h]
+  __half* part_o;     // [Nc * H_kv * k, d_h / 8, G, 8]: per slot, 16-byte d-chunks head-minor
   float* part_lse;    // [Nc * H_kv * k, G]
 };
 
@@ -202,6 +202,7 @@ __global__ void __launch_bounds__(1024) inv_scan_kernel(const InvParams p) {
 // ------------------------------------------------------------------ step 2 --
 struct P1Params {
   int64_t q0;
+  int q4d;  // 1: one 4-D TMA box per gathered query ([d-chunk][head] rows, 8 heads)
   int H_q, H_kv, B_k, kk, G, R, Tq;
   int64_t nkeys;
   float scale_log2;  // softmax scale * log2(e)
@@ -248,7 +249,7 @@ __device__ __forceinline__ int find_key(const int32_t* tile_off, int64_t nkeys, 
 //   warp 1      MMA issuer (lane 0) and TMEM owner
 //   warps 2..9  softmax + epilogue, group (w-2)/4
 template <int D_H, int B_K>
-__global__ void __maxnreg__(200)
+__global__ void __launch_bounds__(kThreads, 1)
     attn_phase1_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const P1Params p) {
@@ -364,10 +365,16 @@ __global__ void __maxnreg__(200)
       if (lane < len) {
         const int i = static_cast<int>(p.q0 + myslot / per_q);
         uint8_t* sQ = smem + qs * SH::QP_BYTES;
+        if (p.q4d) {
+          // query-major: [query][d-chunk][8 heads x 128 B]
+          tma_load_4d(sQ + lane * 8 * D_H * 2, &tm_q, &q_full[qs], 0, h0, 0, i);
+        } else {
+          // chunk-major: [d-chunk][query rows x 128 B]
 #pragma unroll
-        for (int c = 0; c < SH::DCH; ++c)
-          tma_load_3d(sQ + c * kRowsPerTile * 128 + lane * p.R * 128, &tm_q, &q_full[qs], c * 64,
-                      h0, i);
+          for (int c = 0; c < SH::DCH; ++c)
+            tma_load_3d(sQ + c * kRowsPerTile * 128 + lane * p.R * 128, &tm_q, &q_full[qs],
+                        c * 64, h0, i);
+        }
       }
       if (new_kv) {
         // the slot is free once every tile of the previous run finished O = P V
@@ -407,12 +414,14 @@ __global__ void __maxnreg__(200)
         tc_fence_after();
         const uint32_t q_base = smem_u32(smem + (n % QS) * SH::QP_BYTES), k_base = smem_u32(sK);
         const uint32_t tS = tmem_base + (n & 1) * 256 + SH::TM_S;
+        // 8-row groups: consecutive queries (query-major) or consecutive rows
+        const uint32_t q_sbo = p.q4d ? 8 * D_H * 2 : 1024;
+        const uint32_t q_cstep = p.q4d ? 8 * 128 : kRowsPerTile * 128;
 #pragma unroll
         for (int c = 0; c < SH::DCH; ++c)
 #pragma unroll
           for (int s = 0; s < 4; ++s) {
-            const uint64_t ad =
-                umma_desc(q_base + c * kRowsPerTile * 128 + s * 32, 16, 1024, SW_128B);
+            const uint64_t ad = umma_desc(q_base + c * q_cstep + s * 32, 16, q_sbo, SW_128B);
             const uint64_t bd = umma_desc(k_base + c * B_K * 128 + s * 32, 16, 1024, SW_128B);
             umma_bf16(tS, ad, bd, idesc_s, (c | s) != 0);
           }
@@ -537,7 +546,10 @@ __global__ void __maxnreg__(200)
       const int goff = p.G >= 8 ? 0 : (ti_r * p.G) % 8;  // group's first head in the box
       const bool useful = live && hrow >= goff && hrow < goff + p.G;
       const int g = hrow - goff;
-      __half* dst = p.c.part_o + (static_cast<int64_t>(slot) * p.G + g) * D_H;
+      // partial layout [slot][d/8][g][8]: at each store the G lanes of one
+      // query write G consecutive 16-byte pieces (whole 128-byte lines for G=8)
+      __half* dst = p.c.part_o + static_cast<int64_t>(slot) * p.G * D_H + g * 8;
+      const int cstride = p.G * 8;  // elements between consecutive d-chunks
       const float inv_l = 1.0f / l;
       uint32_t ro[D_H / 32][32];
 #pragma unroll
@@ -560,7 +572,7 @@ __global__ void __maxnreg__(200)
             w.y = *reinterpret_cast<uint32_t*>(&a1);
             w.z = *reinterpret_cast<uint32_t*>(&a2);
             w.w = *reinterpret_cast<uint32_t*>(&a3);
-            *reinterpret_cast<uint4*>(dst + c * 32 + j) = w;
+            *reinterpret_cast<uint4*>(dst + ((c * 32 + j) >> 3) * cstride) = w;
           }
         p.c.part_lse[static_cast<int64_t>(slot) * p.G + g] = mx * p.scale + logf(l);
       }
@@ -625,8 +637,10 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(const MergeParams p) {
 #pragma unroll
   for (int e = 0; e < E; ++e) acc[e] = 0.0f;
   float wsum = 0.0f;
-  const __half* base = p.c.part_o + (slot0 * p.G + g) * D_H + d0;
+  // partial layout [slot][d/8][g][8]
+  const __half* base = p.c.part_o + slot0 * p.G * D_H + (d0 >> 3) * p.G * 8 + g * 8;
   const int64_t stride = static_cast<int64_t>(p.G) * D_H;  // between slots
+  const int cstride = p.G * 8;                              // between d-chunks
 #pragma unroll
   for (int s0 = 0; s0 < 32; s0 += 4) {  // fully unrolled: ls[] stays in registers
     if (s0 >= p.kk) break;
@@ -639,7 +653,8 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(const MergeParams p) {
       w[j] = on ? __expf(ls[s] - m) : 0.0f;
 #pragma unroll
       for (int u = 0; u < V16; ++u)
-        x[j][u] = on ? *reinterpret_cast<const uint4*>(base + s * stride + u * 8) : make_uint4(0, 0, 0, 0);
+        x[j][u] = on ? *reinterpret_cast<const uint4*>(base + s * stride + u * cstride)
+                     : make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -693,7 +708,18 @@ cudaError_t launch_typed(const AttnLaunch& a, cudaStream_t stream) {
   if (need > a.ws_bytes) return cudaErrorInvalidValue;
 
   CUtensorMap tq, tk, tv;
-  {
+  int q4d = 0;
+  if (R == 8) {
+    // (64 d, heads, d-chunk, query): one box = 8 heads x all of d, landing as
+    // [d-chunk][head] 128-byte rows
+    const uint64_t dims[4] = {64, static_cast<uint64_t>(a.H_q), static_cast<uint64_t>(D_H / 64),
+                              static_cast<uint64_t>(a.N)};
+    const uint64_t strides[3] = {static_cast<uint64_t>(D_H) * 2, 128,
+                                 static_cast<uint64_t>(a.H_q) * D_H * 2};
+    const uint32_t box[4] = {64, 8, static_cast<uint32_t>(D_H / 64), 1};
+    q4d = make_tmap_bf16(&tq, a.q, 4, dims, strides, box, 128) ? 1 : 0;
+  }
+  if (!q4d) {
     const uint64_t dims[3] = {static_cast<uint64_t>(D_H), static_cast<uint64_t>(a.H_q),
                               static_cast<uint64_t>(a.N)};
     const uint64_t strides[2] = {static_cast<uint64_t>(D_H) * 2,
@@ -747,6 +773,7 @@ cudaError_t launch_typed(const AttnLaunch& a, cudaStream_t stream) {
 
     P1Params pp;
     pp.q0 = q0;
+    pp.q4d = q4d;
     pp.H_q = a.H_q;
     pp.H_kv = a.H_kv;
     pp.B_k = a.B_k;

@@ -196,6 +196,10 @@ MSA_API int32_t msa_profile_read(msa_kernel_time* out, int32_t max_entries);
 /* Static description of a status value. */
 MSA_API const char* msa_status_string(msa_status s);
 
+/* Text of the last CUDA runtime error behind an MSA_ERR_CUDA returned to the
+ * calling thread ("no CUDA error" if there was none).  Static storage. */
+MSA_API const char* msa_last_error(void);
+
 /* Library version string and the compute capability it was built for. */
 MSA_API const char* msa_version(void);
 
