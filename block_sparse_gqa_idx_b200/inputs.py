@@ -152,22 +152,33 @@ def _unit(rng: np.random.Generator, d: int) -> np.ndarray:
 
 def prefill_inputs(cfg: MSAConfig, seed: Optional[int] = None) -> Dict[str, np.ndarray]:
     """q [N,H_q,d_h], k/v [N,H_kv,d_h], q_idx [N,H_kv,d_idx], k_idx [N,d_idx] (bf16 bits)."""
+    from concurrent.futures import ThreadPoolExecutor
+
     ss = np.random.SeedSequence(cfg.seed if seed is None else seed)
     r_q, r_k, r_v, r_qi, r_ki, r_s = (np.random.default_rng(s) for s in ss.spawn(6))
     N, H_q, H_kv, d_h, d_idx = cfg.N, cfg.H_q, cfg.H_kv, cfg.d_h, cfg.d_idx
-    out = {
-        "q": _normal_bf16(r_q, (N, H_q, d_h)),
-        "k": _normal_bf16(r_k, (N, H_kv, d_h)),
-        "v": _normal_bf16(r_v, (N, H_kv, d_h)),
-    }
-    if cfg.structure == "iid":
-        out["q_idx"] = _normal_bf16(r_qi, (N, H_kv, d_idx))
-        out["k_idx"] = _normal_bf16(r_ki, (N, d_idx))
-        return out
-    if cfg.structure not in ("sink_ar1", "sink_ar1_retrieval"):
+    if cfg.structure not in ("iid", "sink_ar1", "sink_ar1_retrieval"):
         raise ValueError(f"unknown structure {cfg.structure!r}")
-    qi = _ar1(r_qi, N, H_kv * d_idx, 0.9).reshape(N, H_kv, d_idx)
-    ki = _ar1(r_ki, N, d_idx, 0.9)
+    iid = cfg.structure == "iid"
+    # the tensors draw from independent streams: generate them concurrently
+    jobs = {
+        "q": lambda: _normal_bf16(r_q, (N, H_q, d_h)),
+        "k": lambda: _normal_bf16(r_k, (N, H_kv, d_h)),
+        "v": lambda: _normal_bf16(r_v, (N, H_kv, d_h)),
+        "qi": (lambda: _normal_bf16(r_qi, (N, H_kv, d_idx))) if iid
+        else (lambda: _ar1(r_qi, N, H_kv * d_idx, 0.9).reshape(N, H_kv, d_idx)),
+        "ki": (lambda: _normal_bf16(r_ki, (N, d_idx))) if iid
+        else (lambda: _ar1(r_ki, N, d_idx, 0.9)),
+    }
+    with ThreadPoolExecutor(max_workers=len(jobs)) as ex:
+        futs = {name: ex.submit(fn) for name, fn in jobs.items()}
+        res = {name: f.result() for name, f in futs.items()}
+    out = {"q": res["q"], "k": res["k"], "v": res["v"]}
+    if iid:
+        out["q_idx"] = res["qi"]
+        out["k_idx"] = res["ki"]
+        return out
+    qi, ki = res["qi"], res["ki"]
     u = _unit(r_s, d_idx)
     qi += u[None, None, :]
     ki[: min(N, cfg.B_k)] += (2.0 * math.sqrt(d_idx) * cfg.sink_strength) * u[None, :]
@@ -195,9 +206,14 @@ def decode_state(cfg: DecodeConfig, seed: Optional[int] = None) -> Dict[str, np.
     k_cache/v_cache [S, L_max, H_kv, d_h], k_idx_cache [S, L_max, d_idx] with the
     first L0 rows filled (i.i.d. N(0,1), sink on block 0 of every sequence) and
     the rest zero; seq_len [S] int32 = L0; sink [S, d_idx] float32 (u per sequence).
+    Every sequence has its own seeded streams, so sequences are generated in
+    parallel threads.
     """
+    from concurrent.futures import ThreadPoolExecutor
+
     ss = np.random.SeedSequence(cfg.seed if seed is None else seed)
-    r_k, r_v, r_ki, r_s = (np.random.default_rng(s) for s in ss.spawn(4))
+    r_s = np.random.default_rng(ss.spawn(1)[0])
+    per_seq = ss.spawn(1 + cfg.S)[1:]
     S, L0, Lm, H_kv, d_h, d_idx = cfg.S, cfg.L0, cfg.L_max, cfg.H_kv, cfg.d_h, cfg.d_idx
     k_cache = np.zeros((S, Lm, H_kv, d_h), dtype=np.uint16)
     v_cache = np.zeros((S, Lm, H_kv, d_h), dtype=np.uint16)
@@ -205,12 +221,19 @@ def decode_state(cfg: DecodeConfig, seed: Optional[int] = None) -> Dict[str, np.
     sink = np.stack([_unit(r_s, d_idx) for _ in range(S)])
     nb = min(L0, cfg.B_k)
     shift = 2.0 * math.sqrt(d_idx) * cfg.sink_strength
-    for s in range(S):
+
+    def fill(s):
+        r_k, r_v, r_ki = (np.random.default_rng(x) for x in per_seq[s].spawn(3))
         k_cache[s, :L0] = _normal_bf16(r_k, (L0, H_kv, d_h))
         v_cache[s, :L0] = _normal_bf16(r_v, (L0, H_kv, d_h))
         ki = r_ki.standard_normal((L0, d_idx), dtype=np.float32)
         ki[:nb] += shift * sink[s][None, :]
         k_idx_cache[s, :L0] = bf16_bits(ki)
+
+    import os
+
+    with ThreadPoolExecutor(max_workers=min(S, os.cpu_count() or 1)) as ex:
+        list(ex.map(fill, range(S)))
     return {"k_cache": k_cache, "v_cache": v_cache, "k_idx_cache": k_idx_cache,
             "seq_len": np.full(S, L0, dtype=np.int32), "sink": sink}
 
