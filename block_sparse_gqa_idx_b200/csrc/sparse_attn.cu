@@ -31,7 +31,12 @@ namespace {
 
 constexpr int kThreads = 320;
 constexpr int kRowsPerTile = 128;
-constexpr int kMaxChunk = 1 << 17;  // queries per chunk (bounds the partial buffer)
+// Queries per chunk.  A chunk's gathered Q rows (8192 x H_q x d_h x 2 B = 64 MB
+// at the pages' heads) stay resident in L2 while all their k blocks are
+// processed, so each query is read from HBM about once instead of k times;
+// the price is re-reading K/V blocks once per chunk.  It also bounds the
+// partial-output workspace.
+constexpr int kMaxChunk = 1 << 13;
 
 // Rows per query inside an MMA tile: the group's G heads, or 8 heads (one
 // 128-byte swizzle atom) when G < 8 (the extra heads are computed and dropped).
@@ -213,7 +218,8 @@ struct P1Params {
 
 template <int D_H, int B_K>
 struct P1Shape {
-  static constexpr int QS = 4;                                                  // Q/P ring depth
+  static constexpr int QS = 3;                                                  // Q/P ring depth
+  static constexpr int NKV = 2;                                                 // K/V slots
   static constexpr int QP_BYTES = kRowsPerTile * (D_H > B_K ? D_H : B_K) * 2;  // Q, later P
   static constexpr int K_BYTES = B_K * D_H * 2;
   static constexpr int V_BYTES = B_K * D_H * 2;
@@ -258,15 +264,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint8_t* sK = smem + QS * SH::QP_BYTES;
-  uint8_t* sV = sK + SH::K_BYTES;
-  TileInfo* info = reinterpret_cast<TileInfo*>(sV + SH::V_BYTES);
+  // K/V slot j: K at sKV + j * (K_BYTES + V_BYTES), V right after it
+  uint8_t* sKV = smem + QS * SH::QP_BYTES;
+  TileInfo* info = reinterpret_cast<TileInfo*>(sKV + SH::NKV * (SH::K_BYTES + SH::V_BYTES));
   uint64_t* bars = reinterpret_cast<uint64_t*>(info + QS);
   uint64_t* q_full = bars;             // [QS] gathered Q landed
   uint64_t* q_empty = q_full + QS;     // [QS] O MMA of the stage's tile done
-  uint64_t* kv_full = q_empty + QS;    // K/V block landed
-  uint64_t* kv_empty = kv_full + 1;    // last tile of a K/V run finished its O MMA
-  uint64_t* s_full = kv_empty + 1;     // [2] S in TMEM
+  uint64_t* kv_full = q_empty + QS;    // [NKV] K/V block landed
+  uint64_t* kv_empty = kv_full + SH::NKV;  // [NKV] last tile of a K/V run finished O = P V
+  uint64_t* s_full = kv_empty + SH::NKV;   // [2] S in TMEM
   uint64_t* p_full = s_full + 2;       // [2] P in smem (S read)
   uint64_t* o_full = p_full + 2;       // [2] O in TMEM
   uint64_t* o_empty = o_full + 2;      // [2] O read
@@ -279,8 +285,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&q_full[s], 1);
       mbar_init(&q_empty[s], 1);
     }
-    mbar_init(kv_full, 1);
-    mbar_init(kv_empty, 1);
+    for (int j = 0; j < SH::NKV; ++j) {
+      mbar_init(&kv_full[j], 1);
+      mbar_init(&kv_empty[j], 1);
+    }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&s_full[s], 1);
       mbar_init(&p_full[s], 4);
@@ -377,15 +385,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (new_kv) {
-        // the slot is free once every tile of the previous run finished O = P V
-        if (kvgen > 0 &&
-            !mbar_wait(kv_empty, (kvgen - 1) & 1, abort_flag, p.status, 51))
+        // generation g lives in slot g % NKV; the slot is free once every tile
+        // of generation g - NKV finished O = P V
+        const int slot = kvgen % SH::NKV;
+        if (kvgen >= SH::NKV &&
+            !mbar_wait(&kv_empty[slot], ((kvgen / SH::NKV) - 1) & 1, abort_flag, p.status, 51))
           break;
-        if (lane == 0) mbar_arrive_expect_tx(kv_full, SH::K_BYTES + SH::V_BYTES);
+        uint8_t* sK = sKV + slot * (SH::K_BYTES + SH::V_BYTES);
+        uint8_t* sV = sK + SH::K_BYTES;
+        if (lane == 0) mbar_arrive_expect_tx(&kv_full[slot], SH::K_BYTES + SH::V_BYTES);
         __syncwarp();
         if (lane < SH::DCH) {
-          tma_load_3d(sK + lane * B_K * 128, &tm_k, kv_full, lane * 64, r, b * B_K);
-          tma_load_3d(sV + lane * B_K * 128, &tm_v, kv_full, lane * 64, r, b * B_K);
+          tma_load_3d(sK + lane * B_K * 128, &tm_k, &kv_full[slot], lane * 64, r, b * B_K);
+          tma_load_3d(sV + lane * B_K * 128, &tm_v, &kv_full[slot], lane * 64, r, b * B_K);
         }
         kv_key = cur_key;
         ++kvgen;
@@ -394,8 +406,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // -------------------------------------------------------- MMA issuer --
     // S of tile n+1 is issued before waiting for the softmax of tile n, so the
-    // tensor core works while P is built; at a K/V switch O(n) goes first and
-    // releases the slot.
+    // tensor core works while P is built.  A new K/V run lives in the other
+    // slot, so a switch costs nothing here; after O(n) of a run's last tile the
+    // run's slot is released.
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, B_K, 0, 0);
       constexpr uint32_t idesc_o = idesc_bf16_f32(128, D_H, 0, 1);
@@ -408,11 +421,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       auto issue_s = [&](int n, int gen) -> bool {
         if (gen != gen_have) {
-          if (!mbar_wait(kv_full, gen & 1, abort_flag, p.status, 63)) return false;
+          if (!mbar_wait(&kv_full[gen % SH::NKV], (gen / SH::NKV) & 1, abort_flag, p.status, 63))
+            return false;
           gen_have = gen;
         }
         tc_fence_after();
-        const uint32_t q_base = smem_u32(smem + (n % QS) * SH::QP_BYTES), k_base = smem_u32(sK);
+        const uint32_t q_base = smem_u32(smem + (n % QS) * SH::QP_BYTES);
+        const uint32_t k_base = smem_u32(sKV + (gen % SH::NKV) * (SH::K_BYTES + SH::V_BYTES));
         const uint32_t tS = tmem_base + (n & 1) * 256 + SH::TM_S;
         // 8-row groups: consecutive queries (query-major) or consecutive rows
         const uint32_t q_sbo = p.q4d ? 8 * D_H * 2 : 1024;
@@ -439,12 +454,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool change = has_next && gnext != gcur;
         // S of tile n+1 reuses the TMEM stage of tile n-1, whose P was waited
         // for in the previous iteration
-        if (has_next && !change && !issue_s(n + 1, gnext)) break;
+        if (has_next && !issue_s(n + 1, gnext)) break;
         if (!mbar_wait(&p_full[st], ph, abort_flag, p.status, 61)) break;
         if (!mbar_wait(&o_empty[st], ph ^ 1, abort_flag, p.status, 62)) break;
         tc_fence_after();
         const uint32_t q_base = smem_u32(smem + (n % QS) * SH::QP_BYTES);
-        const uint32_t v_base = smem_u32(sV);
+        const uint32_t v_base =
+            smem_u32(sKV + (gcur % SH::NKV) * (SH::K_BYTES + SH::V_BYTES) + SH::K_BYTES);
         const uint32_t tO = tmem_base + st * 256 + SH::TM_O;
 #pragma unroll
         for (int c = 0; c < SH::PCH; ++c)
@@ -459,10 +475,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         umma_commit(&o_full[st]);
         umma_commit(&q_empty[n % QS]);
-        if (change) {
-          umma_commit(kv_empty);
-          if (!issue_s(n + 1, gnext)) break;
-        }
+        if (change) umma_commit(&kv_empty[gcur % SH::NKV]);
         gcur = gnext;
       }
     }
@@ -691,8 +704,8 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(const MergeParams p) {
 template <int D_H, int B_K>
 size_t p1_smem_bytes() {
   using SH = P1Shape<D_H, B_K>;
-  return 1024 + SH::QS * SH::QP_BYTES + SH::K_BYTES + SH::V_BYTES + SH::QS * sizeof(TileInfo) +
-         (2 * SH::QS + 2 + 8) * 8 + 16;
+  return 1024 + SH::QS * SH::QP_BYTES + SH::NKV * (SH::K_BYTES + SH::V_BYTES) +
+         SH::QS * sizeof(TileInfo) + (2 * SH::QS + 2 * SH::NKV + 8) * 8 + 16;
 }
 
 template <int D_H, int B_K>

@@ -288,3 +288,29 @@ def test_decode_full_size_sampled(msa):
     """The 64 x 131072-token decode workload, two steps; four sequences checked."""
     cfg = inputs.CONFIGS["decode"]
     _decode_run(msa, cfg, 2, [0, 17, 42, 63])
+
+
+def test_forward_1m_sampled(msa):
+    """The 1M-token sink-skewed workload through the whole forward (index +
+    attention, 128 query chunks); sampled rows checked against the oracle."""
+    cfg = inputs.CONFIGS["1m"]
+    inp = prefill_inputs_cached(cfg)
+    dev = dev_inputs(inp)
+    o, lse, idx = msa.forward(dev["q"], dev["k"], dev["v"], dev["q_idx"], dev["k_idx"], cfg.B_k,
+                              cfg.k)
+    torch.cuda.synchronize()
+    del dev
+    rng = np.random.default_rng(5)
+    rows = np.unique(np.concatenate([rng.integers(0, cfg.N, 20),
+                                     [0, 129, 8191, 8192, cfg.N // 2, cfg.N - 1]]))
+    gidx = idx.cpu().numpy()[rows]
+    ref, cut, nxt = oracle.index_topk(inp["q_idx"], inp["k_idx"], cfg.B_k, cfg.k, rows=rows)
+    exact, band, fails = compare.check_topk(gidx, ref, cut, nxt, rows, cfg.B_k, cfg.k,
+                                            q_idx_rows=inp["q_idx"][rows], k_idx=inp["k_idx"])
+    assert not fails, fails
+    # the workload's defining property: block 0 chosen by >= 90% of (row, group)
+    late = rows >= cfg.B_k
+    assert (ref[late] == 0).any(axis=2).mean() >= 0.9
+    ro, rlse = oracle.sparse_attn(inp["q"][rows], inp["k"], inp["v"], gidx, cfg.B_k, rows,
+                                  N=cfg.N)
+    compare.assert_attn_close(bf16_to_f64(o)[rows], ro, lse.cpu().numpy()[rows], rlse, what="1m")
