@@ -13,9 +13,10 @@ notes, 5.1) at the sizes listed in ``CONFIGS``.  The planted structure is:
 * ``sink_ar1``: Q, K, V i.i.d. N(0, 1).  Q_idx (each group) and K_idx follow
   an AR(1) process along the sequence, x_0 = e_0, x_i = rho x_{i-1} +
   sqrt(1 - rho^2) e_i (rho = 0.9, N(0,1) marginals), for locality.  A seeded
-  unit vector u is added to every index query and 2*sqrt(d_idx)*u*strength to
-  every index key of block 0, so block-0 scores gain about +2*strength on
-  average: an attention sink.
+  unit vector u is added, times ``sink_strength``, to every index query, and
+  2*sqrt(d_idx)*u to every index key of block 0: block-0 scores gain
+  +2*strength on average, against a spread of 2 from the queries' own
+  component along u, so the strength sets how many rows pick the sink.
 * ``sink_ar1_retrieval``: ``sink_ar1`` plus, per group, 8 "retrieval" blocks
   drawn from [1, B-2]; each gets a unit vector v, one random token of the
   block gets K_idx += 2*sqrt(d_idx)*v, and a random 1/8 of the later queries
@@ -180,8 +181,8 @@ def prefill_inputs(cfg: MSAConfig, seed: Optional[int] = None) -> Dict[str, np.n
         return out
     qi, ki = res["qi"], res["ki"]
     u = _unit(r_s, d_idx)
-    qi += u[None, None, :]
-    ki[: min(N, cfg.B_k)] += (2.0 * math.sqrt(d_idx) * cfg.sink_strength) * u[None, :]
+    qi += cfg.sink_strength * u[None, None, :]
+    ki[: min(N, cfg.B_k)] += (2.0 * math.sqrt(d_idx)) * u[None, :]
     if cfg.structure == "sink_ar1_retrieval":
         B = cfg.B
         if B >= 4:
