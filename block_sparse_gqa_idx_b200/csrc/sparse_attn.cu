@@ -31,12 +31,11 @@ namespace {
 
 constexpr int kThreads = 320;
 constexpr int kRowsPerTile = 128;
-// Queries per chunk.  A chunk's gathered Q rows (8192 x H_q x d_h x 2 B = 64 MB
-// at the pages' heads) stay resident in L2 while all their k blocks are
-// processed, so each query is read from HBM about once instead of k times;
-// the price is re-reading K/V blocks once per chunk.  It also bounds the
-// partial-output workspace.
-constexpr int kMaxChunk = 1 << 13;
+// Queries per chunk: bounds the partial-output workspace.  Chunks are kept
+// large so that every (group, block) list holds many queries per chunk: K/V
+// blocks are then reused over long runs of tiles (small chunks would keep the
+// gathered Q in L2 but re-read K/V for nearly every tile at 1M tokens).
+constexpr int kMaxChunk = 1 << 17;
 
 // Rows per query inside an MMA tile: the group's G heads, or 8 heads (one
 // 128-byte swizzle atom) when G < 8 (the extra heads are computed and dropped).
@@ -218,8 +217,8 @@ struct P1Params {
 
 template <int D_H, int B_K>
 struct P1Shape {
-  static constexpr int QS = 3;                                                  // Q/P ring depth
-  static constexpr int NKV = 2;                                                 // K/V slots
+  static constexpr int QS = 4;   // Q/P ring depth
+  static constexpr int NKV = 1;  // K/V slots (the ring and two slots do not both fit)
   static constexpr int QP_BYTES = kRowsPerTile * (D_H > B_K ? D_H : B_K) * 2;  // Q, later P
   static constexpr int K_BYTES = B_K * D_H * 2;
   static constexpr int V_BYTES = B_K * D_H * 2;
@@ -406,9 +405,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // -------------------------------------------------------- MMA issuer --
     // S of tile n+1 is issued before waiting for the softmax of tile n, so the
-    // tensor core works while P is built.  A new K/V run lives in the other
-    // slot, so a switch costs nothing here; after O(n) of a run's last tile the
-    // run's slot is released.
+    // tensor core works while P is built.  After O(n) of a run's last tile the
+    // run's K/V slot is released; with a single slot the next run's K/V can
+    // only land after that, so at a switch O(n) goes first.
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, B_K, 0, 0);
       constexpr uint32_t idesc_o = idesc_bf16_f32(128, D_H, 0, 1);
@@ -454,7 +453,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool change = has_next && gnext != gcur;
         // S of tile n+1 reuses the TMEM stage of tile n-1, whose P was waited
         // for in the previous iteration
-        if (has_next && !issue_s(n + 1, gnext)) break;
+        const bool s_first = has_next && (SH::NKV > 1 || !change);
+        if (s_first && !issue_s(n + 1, gnext)) break;
         if (!mbar_wait(&p_full[st], ph, abort_flag, p.status, 61)) break;
         if (!mbar_wait(&o_empty[st], ph ^ 1, abort_flag, p.status, 62)) break;
         tc_fence_after();
@@ -475,7 +475,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         umma_commit(&o_full[st]);
         umma_commit(&q_empty[n % QS]);
-        if (change) umma_commit(&kv_empty[gcur % SH::NKV]);
+        if (change) {
+          umma_commit(&kv_empty[gcur % SH::NKV]);
+          if (!s_first && !issue_s(n + 1, gnext)) break;
+        }
         gcur = gnext;
       }
     }

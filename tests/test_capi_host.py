@@ -41,10 +41,10 @@ def test_workspace_sizes(capi):
     d = capi.dims(131072, 32, 4, 128, 64, 128, 16)
     assert capi.index_topk_workspace_size(d) >= 16
     ws = capi.sparse_attn_fwd_workspace_size(d)
-    # fp16 partials of every (query, group, slot) and head of one 8192-query
-    # chunk: 8192*H_q*k*d_h*2 bytes, plus the inverse index
-    assert ws >= 8192 * 32 * 16 * 128 * 2
-    assert ws < 8192 * 32 * 16 * 128 * 2 * 1.2
+    # fp16 partials of every (query, group, slot) and head of one 131072-query
+    # chunk: 131072*H_q*k*d_h*2 bytes, plus the inverse index
+    assert ws >= 131072 * 32 * 16 * 128 * 2
+    assert ws < 131072 * 32 * 16 * 128 * 2 * 1.2
     d1m = capi.dims(1 << 20, 32, 4, 128, 64, 128, 16)
     # the prefill works in query chunks: 1M needs about the same workspace
     assert capi.sparse_attn_fwd_workspace_size(d1m) < ws * 1.1
