@@ -217,7 +217,7 @@ struct P1Params {
 
 template <int D_H, int B_K>
 struct P1Shape {
-  static constexpr int QS = 4;   // Q/P ring depth
+  static constexpr int QS = 5;   // Q/P ring depth
   static constexpr int NKV = 1;  // K/V slots (the ring and two slots do not both fit)
   static constexpr int QP_BYTES = kRowsPerTile * (D_H > B_K ? D_H : B_K) * 2;  // Q, later P
   static constexpr int K_BYTES = B_K * D_H * 2;
