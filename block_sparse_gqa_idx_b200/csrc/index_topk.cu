@@ -285,35 +285,31 @@ __global__ void __launch_bounds__(kThreads, 1)
                             acc * 256 + mt * 128;
         float x0 = -INFINITY, x1 = -INFINITY, x2 = -INFINITY, x3 = -INFINITY;
         if (active) {
-          // max of 64 columns as four independent 3-input-max chains of depth 8
-          auto pool64 = [](const uint32_t (&a)[32], const uint32_t (&b)[32], float& lo, float& hi) {
-            float c[4];
-#pragma unroll
-            for (int q = 0; q < 2; ++q) {
-              const uint32_t* u = a + 16 * q;
-              const uint32_t* v = b + 16 * q;
-              float y = fmax3(__uint_as_float(u[0]), __uint_as_float(u[1]), __uint_as_float(u[2]));
-              float z = fmax3(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2]));
-#pragma unroll
-              for (int j = 3; j < 15; j += 2) {
-                y = fmax3(y, __uint_as_float(u[j]), __uint_as_float(u[j + 1]));
-                z = fmax3(z, __uint_as_float(v[j]), __uint_as_float(v[j + 1]));
-              }
-              c[q] = fmaxf(y, __uint_as_float(u[15]));
-              c[2 + q] = fmaxf(z, __uint_as_float(v[15]));
-            }
-            lo = fmaxf(c[0], c[1]);
-            hi = fmaxf(c[2], c[3]);
-          };
           uint32_t ra[32], rb[32];
           tmem_ld32(ta + 0, ra);
           tmem_ld32(ta + 32, rb);
           tmem_wait_ld();
-          pool64(ra, rb, x0, x1);
+          x0 = __uint_as_float(ra[0]);
+          x1 = __uint_as_float(rb[0]);
+#pragma unroll
+          for (int j = 1; j < 31; j += 2) {
+            x0 = fmax3(x0, __uint_as_float(ra[j]), __uint_as_float(ra[j + 1]));
+            x1 = fmax3(x1, __uint_as_float(rb[j]), __uint_as_float(rb[j + 1]));
+          }
+          x0 = fmaxf(x0, __uint_as_float(ra[31]));
+          x1 = fmaxf(x1, __uint_as_float(rb[31]));
           tmem_ld32(ta + 64, ra);
           tmem_ld32(ta + 96, rb);
           tmem_wait_ld();
-          pool64(ra, rb, x2, x3);
+          x2 = __uint_as_float(ra[0]);
+          x3 = __uint_as_float(rb[0]);
+#pragma unroll
+          for (int j = 1; j < 31; j += 2) {
+            x2 = fmax3(x2, __uint_as_float(ra[j]), __uint_as_float(ra[j + 1]));
+            x3 = fmax3(x3, __uint_as_float(rb[j]), __uint_as_float(rb[j + 1]));
+          }
+          x2 = fmaxf(x2, __uint_as_float(ra[31]));
+          x3 = fmaxf(x3, __uint_as_float(rb[31]));
         }
         tc_fence_before();
         __syncwarp();
