@@ -448,13 +448,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int st = n & 1;
         const uint32_t ph = (n >> 1) & 1;
         const bool has_next = n + 1 < my_tiles;
+        // S of tile n+1 goes before O(n) only if its gathered rows have
+        // already landed: O(n) must never wait behind the next gather.  (S of
+        // tile n+1 reuses the TMEM stage of tile n-1, whose P was waited for in
+        // the previous iteration.)
         int gnext = gcur;
-        if (has_next && !wait_q(n + 1, &gnext)) break;
-        const bool change = has_next && gnext != gcur;
-        // S of tile n+1 reuses the TMEM stage of tile n-1, whose P was waited
-        // for in the previous iteration
-        const bool s_first = has_next && (SH::NKV > 1 || !change);
-        if (s_first && !issue_s(n + 1, gnext)) break;
+        bool s_done = false;
+        if (has_next && mbar_try_wait(&q_full[(n + 1) % QS], ((n + 1) / QS) & 1)) {
+          gnext = info[(n + 1) % QS].gen;
+          if (SH::NKV > 1 || gnext == gcur) {
+            if (!issue_s(n + 1, gnext)) break;
+            s_done = true;
+          }
+        }
         if (!mbar_wait(&p_full[st], ph, abort_flag, p.status, 61)) break;
         if (!mbar_wait(&o_empty[st], ph ^ 1, abort_flag, p.status, 62)) break;
         tc_fence_after();
@@ -475,9 +481,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         umma_commit(&o_full[st]);
         umma_commit(&q_empty[n % QS]);
-        if (change) {
+        if (has_next && !s_done) {
+          if (!wait_q(n + 1, &gnext)) break;
+          // a run's last tile releases its K/V slot once O(n) has finished
+          if (gnext != gcur) umma_commit(&kv_empty[gcur % SH::NKV]);
+          if (!issue_s(n + 1, gnext)) break;
+        } else if (has_next && gnext != gcur) {
           umma_commit(&kv_empty[gcur % SH::NKV]);
-          if (!s_first && !issue_s(n + 1, gnext)) break;
         }
         gcur = gnext;
       }
