@@ -205,7 +205,7 @@ msa_status msa_sparse_attn_fwd(const msa_dims* d, const void* q, const void* k, 
       !aligned16(ws) || (lse != nullptr && !aligned16(lse)))
     return MSA_ERR_INVALID_ARG;
   const int G = d->H_q / d->H_kv;
-  if (G > 128 || 128 % G != 0) return MSA_ERR_UNSUPPORTED;
+  if (G > 32 || 32 % G != 0) return MSA_ERR_UNSUPPORTED;     // a query's rows in one warp
   if (G < 8 && d->H_q % 8 != 0) return MSA_ERR_UNSUPPORTED;  // 8-head TMA boxes
   if (d->N * d->H_q >= (int64_t(1) << 31) - 256 || d->N * d->H_kv * d->k >= (int64_t(1) << 31))
     return MSA_ERR_UNSUPPORTED;

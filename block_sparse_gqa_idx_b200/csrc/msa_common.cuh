@@ -121,6 +121,16 @@ MSA_DEVI void tma_load_4d(void* dst, const CUtensorMap* map, uint64_t* bar, int 
 MSA_DEVI void prefetch_tmap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
+// Bulk (non-tensor) copy shared -> global, tracked by the issuing thread's
+// bulk groups; addresses 16-byte aligned, size a multiple of 16.
+MSA_DEVI void bulk_store(void* gdst, const void* ssrc, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst),
+               "r"(smem_u32(ssrc)), "r"(bytes)
+               : "memory");
+}
+MSA_DEVI void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until the source shared memory of every committed bulk copy was read.
+MSA_DEVI void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 // Make generic-proxy smem writes visible to the async proxy (UMMA/TMA reads).
 MSA_DEVI void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 

@@ -268,7 +268,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   TileInfo* info = reinterpret_cast<TileInfo*>(sKV + SH::NKV * (SH::K_BYTES + SH::V_BYTES));
   uint64_t* bars = reinterpret_cast<uint64_t*>(info + QS);
   uint64_t* q_full = bars;             // [QS] gathered Q landed
-  uint64_t* q_empty = q_full + QS;     // [QS] O MMA of the stage's tile done
+  uint64_t* q_empty = q_full + QS;     // [QS] stage free: partials of its tile copied out
   uint64_t* kv_full = q_empty + QS;    // [NKV] K/V block landed
   uint64_t* kv_empty = kv_full + SH::NKV;  // [NKV] last tile of a K/V run finished O = P V
   uint64_t* s_full = kv_empty + SH::NKV;   // [2] S in TMEM
@@ -282,7 +282,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < QS; ++s) {
       mbar_init(&q_full[s], 1);
-      mbar_init(&q_empty[s], 1);
+      mbar_init(&q_empty[s], 4);  // the tile's 4 epilogue warps, after their bulk stores
     }
     for (int j = 0; j < SH::NKV; ++j) {
       mbar_init(&kv_full[j], 1);
@@ -480,7 +480,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             umma_bf16(tO, ad, bd, idesc_o, (c | s) != 0);
           }
         umma_commit(&o_full[st]);
-        umma_commit(&q_empty[n % QS]);
         if (has_next && !s_done) {
           if (!wait_q(n + 1, &gnext)) break;
           // a run's last tile releases its K/V slot once O(n) has finished
@@ -572,10 +571,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int goff = p.G >= 8 ? 0 : (ti_r * p.G) % 8;  // group's first head in the box
       const bool useful = live && hrow >= goff && hrow < goff + p.G;
       const int g = hrow - goff;
-      // partial layout [slot][d/8][g][8]: at each store the G lanes of one
-      // query write G consecutive 16-byte pieces (whole 128-byte lines for G=8)
-      __half* dst = p.c.part_o + static_cast<int64_t>(slot) * p.G * D_H + g * 8;
-      const int cstride = p.G * 8;  // elements between consecutive d-chunks
+      // partial layout [slot][d/8][g][8].  The tile's partials are staged in its
+      // Q/P buffer (P is dead once O = P V completed) in exactly that layout,
+      // so each query's G x d_h block is one contiguous bulk copy to HBM.
+      const int qbytes = p.G * D_H * 2;  // one query's partial block
+      uint8_t* stage = sP + q_local * qbytes;
       const float inv_l = 1.0f / l;
       uint32_t ro[D_H / 32][32];
 #pragma unroll
@@ -598,8 +598,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             w.y = *reinterpret_cast<uint32_t*>(&a1);
             w.z = *reinterpret_cast<uint32_t*>(&a2);
             w.w = *reinterpret_cast<uint32_t*>(&a3);
-            *reinterpret_cast<uint4*>(dst + ((c * 32 + j) >> 3) * cstride) = w;
+            *reinterpret_cast<uint4*>(stage + (((c * 32 + j) >> 3) * p.G + g) * 16) = w;
           }
+      }
+      fence_async_smem();
+      __syncwarp();
+      // one lane per query (its first useful head) copies the query's block
+      if (useful && g == 0) {
+        bulk_store(p.c.part_o + static_cast<int64_t>(slot) * p.G * D_H, stage, qbytes);
+        bulk_commit();
+        bulk_wait_read_all();
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&q_empty[qs]);
+      if (useful) {
         p.c.part_lse[static_cast<int64_t>(slot) * p.G + g] = mx * p.scale + logf(l);
       }
     }

@@ -100,8 +100,8 @@ MSA_API msa_status msa_index_topk(const msa_dims* dims, const void* q_idx, const
  *   o    [N, H_q, d_h]  bf16, written (round to nearest even from fp32)
  *   lse  [N, H_q]       fp32 natural-log LSE of the scaled logits, or NULL
  * A row whose selection is empty gets o = 0 and lse = -inf.
- * Supported: d_h in {64,128}, B_k in {64,128}, 128 % (H_q/H_kv) == 0, and
- * H_q % 8 == 0 when H_q/H_kv < 8.
+ * Supported: d_h in {64,128}, B_k in {64,128}, H_q/H_kv in {1,2,4,8,16,32},
+ * and H_q % 8 == 0 when H_q/H_kv < 8.
  * ------------------------------------------------------------------------- */
 MSA_API size_t msa_sparse_attn_fwd_workspace(const msa_dims* dims);
 MSA_API msa_status msa_sparse_attn_fwd(const msa_dims* dims, const void* q, const void* k,
