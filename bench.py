@@ -99,6 +99,26 @@ class Clocks:
                 "samples": len(rows)}
 
 
+def max_over_ranks(value: float, device, world: int) -> float:
+    """The step time every rank saw, reduced with MAX (timing is the slowest
+    replica's).  device: where the collective's tensor lives (cuda for NCCL,
+    cpu for gloo)."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_tokens_per_s(world: int, tokens_per_rank: int, ms_max: float) -> float:
+    """Whole-job throughput of independent replicas: all ranks' tokens over the
+    slowest rank's time."""
+    return world * tokens_per_rank / (ms_max * 1e-3)
+
+
 def workload(name: str):
     from block_sparse_gqa_idx_b200 import inputs
 
@@ -208,12 +228,8 @@ def run_msa(args, cfg, rank, world, local):
     msa.profile_enable(False)
     clk = clocks.stop()
     prof = msa.profile_read()
-    ms = e0.elapsed_time(e1) / args.steps
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    value = world * N / (ms * 1e-3)
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dev, world)
+    value = aggregate_tokens_per_s(world, N, ms)
 
     # ---- end to end: pinned host inputs -> device -> forward -> host result.
     # Every step uploads its inputs from pinned host memory and downloads its
@@ -270,11 +286,7 @@ def run_msa(args, cfg, rank, world, local):
     e2e_run(e2e_steps)
     f1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = f0.elapsed_time(f1) / e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(f0.elapsed_time(f1) / e2e_steps, dev, world)
     barrier()
 
     if rank != 0:
@@ -333,7 +345,7 @@ def run_msa(args, cfg, rank, world, local):
         "tc_frac_eq12": (f_idx + f_main) / (ms * 1e-3) / 1e12 / pk["bf16_tflops"],
         "roofline": roofline,
         "cpu_baseline": cpu,
-        "e2e": {"value": world * N / (e2e_ms * 1e-3), "unit": "tokens/s",
+        "e2e": {"value": aggregate_tokens_per_s(world, N, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                 "steps": e2e_steps,
                 "note": "pinned host -> device -> forward -> host every step; copies of "
