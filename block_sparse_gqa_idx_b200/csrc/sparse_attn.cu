@@ -499,7 +499,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q_local = row / p.R;
     const int hrow = row - q_local * p.R;
     const int per_q = p.H_kv * p.kk;
-    int pending_qs = -1;  // stage whose partials were copied out but not yet released
     for (int n = grp; n < my_tiles; n += 2) {
       const int st = grp;
       const uint32_t ph = (n >> 1) & 1;
@@ -534,30 +533,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; j < B_K; ++j)
           if (j0 + j > i) sv[j] = -INFINITY;
       }
-      // row max and sum as 8 independent chains (the softmax sits on the
-      // critical path between the two MMAs of a tile)
-      constexpr int CH8 = B_K / 8;
-      float mc[8];
+      float mx = sv[0];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        float y = fmaxf(sv[q * CH8], sv[q * CH8 + 1]);
-#pragma unroll
-        for (int j = 2; j + 1 < CH8; j += 2) y = fmax3(y, sv[q * CH8 + j], sv[q * CH8 + j + 1]);
-        if (CH8 % 2 == 1) y = fmaxf(y, sv[q * CH8 + CH8 - 1]);
-        mc[q] = y;
-      }
-      const float mx = fmaxf(fmax3(mc[0], mc[1], mc[2]), fmax3(fmax3(mc[3], mc[4], mc[5]), mc[6], mc[7]));
+      for (int j = 1; j + 1 < B_K; j += 2) mx = fmax3(mx, sv[j], sv[j + 1]);
+      mx = fmaxf(mx, sv[B_K - 1]);
       const float mscaled = mx * p.scale_log2;
-      float lc[8];
-#pragma unroll
-      for (int q = 0; q < 8; ++q) lc[q] = 0.0f;
+      float l = 0.0f;
 #pragma unroll
       for (int j = 0; j < B_K; ++j) {
         const float e = exp2f(fmaf(sv[j], p.scale_log2, -mscaled));
         sv[j] = e;
-        lc[j & 7] += e;
+        l += e;
       }
-      const float l = ((lc[0] + lc[1]) + (lc[2] + lc[3])) + ((lc[4] + lc[5]) + (lc[6] + lc[7]));
       // P (bf16) over the stage's Q rows (consumed by S), K-major 128B-swizzled
 #pragma unroll
       for (int c = 0; c < B_K / 8; ++c) {
@@ -616,23 +603,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       fence_async_smem();
       __syncwarp();
-      // release the previous tile's stage (its copies were issued a whole
-      // tile ago), then one lane per query copies this tile's block out
-      bulk_wait_read_all();
-      __syncwarp();
-      if (lane == 0 && pending_qs >= 0) mbar_arrive(&q_empty[pending_qs]);
+      // one lane per query (its first useful head) copies the query's block
       if (useful && g == 0) {
         bulk_store(p.c.part_o + static_cast<int64_t>(slot) * p.G * D_H, stage, qbytes);
         bulk_commit();
+        bulk_wait_read_all();
       }
-      pending_qs = qs;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&q_empty[qs]);
       if (useful) {
         p.c.part_lse[static_cast<int64_t>(slot) * p.G + g] = mx * p.scale + logf(l);
       }
     }
-    bulk_wait_read_all();
-    __syncwarp();
-    if (lane == 0 && pending_qs >= 0) mbar_arrive(&q_empty[pending_qs]);
   }
 
   tc_fence_before();
