@@ -268,7 +268,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   TileInfo* info = reinterpret_cast<TileInfo*>(sKV + SH::NKV * (SH::K_BYTES + SH::V_BYTES));
   uint64_t* bars = reinterpret_cast<uint64_t*>(info + QS);
   uint64_t* q_full = bars;             // [QS] gathered Q landed
-  uint64_t* q_empty = q_full + QS;     // [QS] stage free: O = P V of its tile done
+  uint64_t* q_empty = q_full + QS;     // [QS] stage free: partials of its tile copied out
   uint64_t* kv_full = q_empty + QS;    // [NKV] K/V block landed
   uint64_t* kv_empty = kv_full + SH::NKV;  // [NKV] last tile of a K/V run finished O = P V
   uint64_t* s_full = kv_empty + SH::NKV;   // [2] S in TMEM
@@ -282,7 +282,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < QS; ++s) {
       mbar_init(&q_full[s], 1);
-      mbar_init(&q_empty[s], 1);  // committed after the tile's O = P V
+      mbar_init(&q_empty[s], 4);  // the tile's 4 epilogue warps, after their bulk stores
     }
     for (int j = 0; j < SH::NKV; ++j) {
       mbar_init(&kv_full[j], 1);
@@ -480,7 +480,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             umma_bf16(tO, ad, bd, idesc_o, (c | s) != 0);
           }
         umma_commit(&o_full[st]);
-        umma_commit(&q_empty[n % QS]);
         if (has_next && !s_done) {
           if (!wait_q(n + 1, &gnext)) break;
           // a run's last tile releases its K/V slot once O(n) has finished
@@ -494,41 +493,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------ softmax + epilogue groups --
-    // Group grp handles tiles n = grp, grp+2, ... and is software-pipelined:
-    // the softmax of tile n+2 runs while O(n) = P V is on the tensor core,
-    // then the epilogue of tile n.  (S(n+2) can exist by then: the MMA issues
-    // it once P(n) was published, and O(n+2) waits for this epilogue.)
-    const int grp = (warp - 2) >> 2;
+    const int grp = (warp - 2) >> 2;  // handles tiles n with n % 2 == grp
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const int q_local = row / p.R;
     const int hrow = row - q_local * p.R;
     const int per_q = p.H_kv * p.kk;
-    const int st = grp;
-    const uint32_t tS = tmem_base + st * 256 + SH::TM_S + (static_cast<uint32_t>(quarter * 32) << 16);
-    const uint32_t tO = tmem_base + st * 256 + SH::TM_O + (static_cast<uint32_t>(quarter * 32) << 16);
-    struct RowState {
-      uint32_t slot;
-      bool useful;
-      int g;
-      float mx, l;
-    };
-    // softmax of tile n: S -> P (bf16, over the stage's consumed Q rows)
-    auto softmax = [&](int n, RowState& rs) -> bool {
+    for (int n = grp; n < my_tiles; n += 2) {
+      const int st = grp;
       const uint32_t ph = (n >> 1) & 1;
       const int qs = n % QS;
-      if (!mbar_wait(&s_full[st], ph, abort_flag, p.status, 70)) return false;
+      uint8_t* sP = smem + qs * SH::QP_BYTES;
+      const uint32_t tS = tmem_base + st * 256 + SH::TM_S + (static_cast<uint32_t>(quarter * 32) << 16);
+      const uint32_t tO = tmem_base + st * 256 + SH::TM_O + (static_cast<uint32_t>(quarter * 32) << 16);
+      if (!mbar_wait(&s_full[st], ph, abort_flag, p.status, 70)) break;
       // q_full[qs] cannot advance before this tile's O MMA, so this returns at
       // once; it orders the producer's TileInfo writes before the reads below
-      if (!mbar_wait(&q_full[qs], (n / QS) & 1, abort_flag, p.status, 72)) return false;
+      if (!mbar_wait(&q_full[qs], (n / QS) & 1, abort_flag, p.status, 72)) break;
       tc_fence_after();
       const int ti_r = info[qs].r, ti_b = info[qs].b, ti_len = info[qs].len;
       const bool live = q_local < ti_len;
-      rs.slot = live ? info[qs].slot[q_local] : 0u;
-      const int goff = p.G >= 8 ? 0 : (ti_r * p.G) % 8;  // group's first head in the box
-      rs.useful = live && hrow >= goff && hrow < goff + p.G;
-      rs.g = hrow - goff;
-      const int64_t i = p.q0 + rs.slot / per_q;
+      const uint32_t slot = live ? info[qs].slot[q_local] : 0u;
+      const int64_t i = p.q0 + slot / per_q;
+      // ---- softmax over the block's keys (exp2 with the scale folded in)
       float sv[B_K];
       {
         uint32_t r32[B_K / 32][32];
@@ -546,28 +533,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; j < B_K; ++j)
           if (j0 + j > i) sv[j] = -INFINITY;
       }
-      // max and sum as 8 independent chains
-      constexpr int C8 = B_K / 8;
-      float mc[8];
+      float mx = sv[0];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        float y = sv[q * C8];
-#pragma unroll
-        for (int j = 1; j + 1 < C8; j += 2) y = fmax3(y, sv[q * C8 + j], sv[q * C8 + j + 1]);
-        mc[q] = fmaxf(y, sv[q * C8 + C8 - 1]);
-      }
-      const float mx = fmaxf(fmax3(mc[0], mc[1], mc[2]), fmax3(fmax3(mc[3], mc[4], mc[5]), mc[6], mc[7]));
+      for (int j = 1; j + 1 < B_K; j += 2) mx = fmax3(mx, sv[j], sv[j + 1]);
+      mx = fmaxf(mx, sv[B_K - 1]);
       const float mscaled = mx * p.scale_log2;
-      float lc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      float l = 0.0f;
 #pragma unroll
       for (int j = 0; j < B_K; ++j) {
         const float e = exp2f(fmaf(sv[j], p.scale_log2, -mscaled));
         sv[j] = e;
-        lc[j & 7] += e;
+        l += e;
       }
-      rs.mx = mx;
-      rs.l = ((lc[0] + lc[1]) + (lc[2] + lc[3])) + ((lc[4] + lc[5]) + (lc[6] + lc[7]));
-      uint8_t* sP = smem + qs * SH::QP_BYTES;
+      // P (bf16) over the stage's Q rows (consumed by S), K-major 128B-swizzled
 #pragma unroll
       for (int c = 0; c < B_K / 8; ++c) {
         uint4 w;
@@ -587,12 +565,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[st]);
-      return true;
-    };
-    // epilogue of tile n: O / l as an fp16 partial and its LSE into the slot
-    auto epilogue = [&](int n, const RowState& rs) -> bool {
-      if (!mbar_wait(&o_full[st], (n >> 1) & 1, abort_flag, p.status, 71)) return false;
+      // ---- O = P V; write O / l as an fp16 partial and lse into the slot
+      if (!mbar_wait(&o_full[st], ph, abort_flag, p.status, 71)) break;
       tc_fence_after();
+      const int goff = p.G >= 8 ? 0 : (ti_r * p.G) % 8;  // group's first head in the box
+      const bool useful = live && hrow >= goff && hrow < goff + p.G;
+      const int g = hrow - goff;
+      // partial layout [slot][d/8][g][8].  The tile's partials are staged in its
+      // Q/P buffer (P is dead once O = P V completed) in exactly that layout,
+      // so each query's G x d_h block is one contiguous bulk copy to HBM.
+      const int qbytes = p.G * D_H * 2;  // one query's partial block
+      uint8_t* stage = sP + q_local * qbytes;
+      const float inv_l = 1.0f / l;
       uint32_t ro[D_H / 32][32];
 #pragma unroll
       for (int c = 0; c < D_H / 32; ++c) tmem_ld32(tO + c * 32, ro[c]);
@@ -600,12 +584,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&o_empty[st]);
-      if (rs.useful) {
-        // partial layout [slot][d/8][g][8]: at each store the G lanes of one
-        // query write G consecutive 16-byte pieces (whole 128-byte lines for G=8)
-        __half* dst = p.c.part_o + static_cast<int64_t>(rs.slot) * p.G * D_H + rs.g * 8;
-        const int cstride = p.G * 8;
-        const float inv_l = 1.0f / rs.l;
+      if (useful) {
 #pragma unroll
         for (int c = 0; c < D_H / 32; ++c)
 #pragma unroll
@@ -619,18 +598,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             w.y = *reinterpret_cast<uint32_t*>(&a1);
             w.z = *reinterpret_cast<uint32_t*>(&a2);
             w.w = *reinterpret_cast<uint32_t*>(&a3);
-            *reinterpret_cast<uint4*>(dst + ((c * 32 + j) >> 3) * cstride) = w;
+            *reinterpret_cast<uint4*>(stage + (((c * 32 + j) >> 3) * p.G + g) * 16) = w;
           }
-        p.c.part_lse[static_cast<int64_t>(rs.slot) * p.G + rs.g] = rs.mx * p.scale + logf(rs.l);
       }
-      return true;
-    };
-    RowState cur, nxt;
-    bool ok = grp >= my_tiles || softmax(grp, cur);
-    for (int n = grp; ok && n < my_tiles; n += 2) {
-      if (n + 2 < my_tiles && !softmax(n + 2, nxt)) break;
-      if (!epilogue(n, cur)) break;
-      cur = nxt;
+      fence_async_smem();
+      __syncwarp();
+      // one lane per query (its first useful head) copies the query's block
+      if (useful && g == 0) {
+        bulk_store(p.c.part_o + static_cast<int64_t>(slot) * p.G * D_H, stage, qbytes);
+        bulk_commit();
+        bulk_wait_read_all();
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&q_empty[qs]);
+      if (useful) {
+        p.c.part_lse[static_cast<int64_t>(slot) * p.G + g] = mx * p.scale + logf(l);
+      }
     }
   }
 
