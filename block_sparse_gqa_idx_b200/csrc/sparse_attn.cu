@@ -642,7 +642,7 @@ struct MergeParams {
 // rows four slots at a time, so each warp keeps several KB of loads in flight.
 // A warp writes its G x D_H output block as contiguous 16-byte pieces.
 template <int D_H, int E>
-__global__ void __launch_bounds__(256) attn_merge_kernel(const MergeParams p) {
+__global__ void __launch_bounds__(256, 2) attn_merge_kernel(const MergeParams p) {
   static_assert(E % 8 == 0 && D_H % E == 0, "lane slice must be whole 16-byte pieces of one head");
   constexpr int V16 = E / 8;  // 16-byte loads per slot
   const int lane = threadIdx.x & 31;
@@ -661,16 +661,12 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(const MergeParams p) {
   int32_t myb = -1;
   if (lane < p.kk) myb = p.idx[(i * p.H_kv + r) * p.kk + lane];
   const unsigned use = __ballot_sync(0xFFFFFFFFu, lane < p.kk && myb >= 0 && myb <= b_i);
-  // this lane's head: LSE of every used slot
-  float ls[32];
+  // this lane's head: the largest LSE of its used slots (read again below,
+  // from L1, rather than held in registers)
+  const float* lse_h = p.c.part_lse + slot0 * p.G + g;
   float m = -INFINITY;
-#pragma unroll
-  for (int s = 0; s < 32; ++s) {
-    ls[s] = -INFINITY;
-    if (s < p.kk && ((use >> s) & 1u)) ls[s] = p.c.part_lse[(slot0 + s) * p.G + g];
-  }
-#pragma unroll
-  for (int s = 0; s < 32; ++s) m = fmaxf(m, ls[s]);
+  for (int s = 0; s < p.kk; ++s)
+    if ((use >> s) & 1u) m = fmaxf(m, lse_h[s * p.G]);
   float acc[E];
 #pragma unroll
   for (int e = 0; e < E; ++e) acc[e] = 0.0f;
@@ -680,15 +676,14 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(const MergeParams p) {
   const int64_t stride = static_cast<int64_t>(p.G) * D_H;  // between slots
   const int cstride = p.G * 8;                              // between d-chunks
 #pragma unroll
-  for (int s0 = 0; s0 < 32; s0 += 4) {  // fully unrolled: ls[] stays in registers
-    if (s0 >= p.kk) break;
+  for (int s0 = 0; s0 < p.kk; s0 += 4) {
     uint4 x[4][V16];
     float w[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int s = s0 + j;
       const bool on = s < p.kk && ((use >> s) & 1u);
-      w[j] = on ? __expf(ls[s] - m) : 0.0f;
+      w[j] = on ? __expf(lse_h[s * p.G] - m) : 0.0f;
 #pragma unroll
       for (int u = 0; u < V16; ++u)
         x[j][u] = on ? *reinterpret_cast<const uint4*>(base + s * stride + u * cstride)
