@@ -7,7 +7,7 @@ synthetic inputs with a sink block and retrieval blocks).  Inputs (Q alone is
 1.07 GB) are larger than the 126 MB L2, so no flush is needed between steps.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl msa|reference]
-                    [--workload 128k|32k|1m|decode]
+                    [--workload 128k|32k|1m|decode|decode8]
 
 For N > 1 each rank runs an independent replica (its own sequence): the path
 has no exchange step, so there is no collective on the data path; timing is
@@ -32,6 +32,38 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of a kernel from
+# one ncu capture, per unit of work, with the SHA-256 of the kernel's source
+# file at capture time: the figure is reported only while that file is
+# unchanged.  kernel -> (source, sha256, bytes per unit, unit, capture)
+NCU_TRAFFIC = {
+    "attn_phase1": ("sparse_attn.cu",
+                    "d90594744ff3c8ee58378bea6599c9fea880d987d76ab3c0ad6e1d0054cdb80e",
+                    (3.672019e9 + 4.190698e9) / 32768, "query",
+                    "profiles/prefill_32k_ncu_full.md: 32K capture, scaled by queries"),
+    "attn_merge": ("sparse_attn.cu",
+                   "d90594744ff3c8ee58378bea6599c9fea880d987d76ab3c0ad6e1d0054cdb80e",
+                   (4.243662e9 + 0.269400e9) / 32768, "query",
+                   "profiles/prefill_32k_ncu_full.md: 32K capture, scaled by queries"),
+}
+
+
+def ncu_traffic(kernel: str, units: float):
+    """Bytes per launch from NCU_TRAFFIC, or None (no capture, or the kernel
+    source changed since it was taken)."""
+    import hashlib
+
+    ent = NCU_TRAFFIC.get(kernel)
+    if ent is None:
+        return None, None
+    src, sha, per_unit, _, where = ent
+    path = os.path.join(ROOT, "block_sparse_gqa_idx_b200", "csrc", src)
+    with open(path, "rb") as f:
+        if hashlib.sha256(f.read()).hexdigest() != sha:
+            return None, None
+    return per_unit * units, where
 
 
 def peaks():
@@ -312,9 +344,10 @@ def run_msa(args, cfg, rank, world, local):
     else:
         unit, bound = "GB/s", "hbm"
         achieved, peak = None, pk["hbm_gbs"]
+    traffic, traffic_src = ncu_traffic(dom, N / (launches / args.steps))
     roofline = {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
-                "frac": (achieved / peak) if achieved else None, "traffic": None,
-                "peak_kind": f"{pk_kind} burst",
+                "frac": (achieved / peak) if achieved else None, "traffic": traffic,
+                "traffic_source": traffic_src, "peak_kind": f"{pk_kind} burst",
                 "share": dom_ms / total_ms if total_ms else None}
 
     # ---- CPU oracle on a bounded sample (rank 0, N=1 only)
@@ -432,6 +465,7 @@ def run_decode(args, cfg, rank, world, local):
                   + S * (H_q * d_h * 2 * 2 + H_kv * d_idx * 2 + H_kv * d_h * 2 * 2 * 2 + d_idx * 2 * 2))
     pk, pk_kind = peaks()
     gbs = bytes_step / (ms * 1e-3) / 1e9
+    cache_gb = S * cfg.L_max * (2 * H_kv * d_h + d_idx) * 2 / 1e9
     total_ms = sum(v[1] for v in prof.values())
     kernels = {n: {"launches": v[0], "ms_per_step": v[1] / args.steps,
                    "share": v[1] / total_ms if total_ms else None} for n, v in prof.items()}
@@ -444,7 +478,7 @@ def run_decode(args, cfg, rank, world, local):
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": cfg.name, "S": S, "L": L, "H_q": H_q, "H_kv": H_kv, "d_h": d_h,
                    "d_idx": d_idx, "B_k": B_k, "k": kk,
-                   "l2": "caches 9.7 GB, larger than L2; no flush"},
+                   "l2": f"caches {cache_gb:.1f} GB (K, V, K_idx), larger than L2; no flush"},
         "roofline": {"kernel": "decode step", "bound": "hbm", "achieved": gbs,
                      "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": gbs / pk["hbm_gbs"],
                      "traffic": None, "bytes_per_step": bytes_step, "peak_kind": pk_kind,
@@ -472,7 +506,7 @@ def main():
     cfg = workload(args.workload)
     if args.cpu_rows == 0:
         args.cpu_rows = 32 if getattr(cfg, "N", 0) >= (1 << 20) else 256
-    if args.workload == "decode":
+    if args.workload.startswith("decode"):
         if args.impl == "reference":
             print(json.dumps({"impl": "reference", "unavailable": "decode reference arm not provided"}))
             return 0

@@ -105,6 +105,10 @@ CONFIGS: Dict[str, object] = {
     # decode: 64 sequences of 131072 cached tokens, 256 appended steps
     "decode": DecodeConfig("decode", S=64, L0=131072, steps=256, H_q=32, H_kv=4, d_h=128,
                            d_idx=64, B_k=128, k=16, seed_index=3),
+    # the decode step at 8 sequences (2.3 GB of caches): a case small enough
+    # for counter captures of the decode kernels
+    "decode8": DecodeConfig("decode8", S=8, L0=131072, steps=256, H_q=32, H_kv=4, d_h=128,
+                            d_idx=64, B_k=128, k=16, seed_index=5),
     # 1M-token prefill with a strong sink (block 0 picked by >= 90% of rows)
     "1m": MSAConfig("1m", N=1048576, H_q=32, H_kv=4, d_h=128, d_idx=64, B_k=128, k=16,
                     structure="sink_ar1", sink_strength=3.0, seed_index=4),
