@@ -38,16 +38,17 @@ namespace msa {
 namespace {
 
 constexpr int kThreads = 320;
-constexpr int kRows = 128;         // rows per M-tile (UMMA M)
-constexpr int kKeys = 128;         // keys per K_idx tile (UMMA N)
-constexpr int kEpiThreads = 256;   // 2 M-tiles x 128 rows
-constexpr uint32_t kTmemCols = 512;
+constexpr int kRows = 128;           // rows per M-tile (UMMA M)
+constexpr int kKeys = 256;           // keys per K_idx tile (UMMA N)
+constexpr int kHalf = 128;           // key columns of a tile read by one epilogue group
+constexpr int kEpiThreads = 256;     // 2 groups x 128 rows
+constexpr uint32_t kTmemCols = 512;  // 2 accumulator stages x 256 columns
+constexpr int kMaxHeap = 31;         // k - 1 for the largest supported k
 
 struct IndexParams {
   int64_t N;
   int H_kv, B_k, k;
   int n_mtiles;
-  int n_units;
   int32_t* idx_out;
   DevStatus* status;
 };
@@ -62,14 +63,20 @@ struct IndexShape {
   static constexpr int SBO = 8 * SWB;                              // 8-row atom
   static constexpr int A_BYTES = kRows * D_IDX * 2;                // one M-tile
   static constexpr int B_BYTES = kKeys * D_IDX * 2;                // one key tile
-  static constexpr int STAGES = (D_IDX == 128) ? 3 : 6;
+  // key tiles in flight: what shared memory holds beside A and the per-row
+  // Top-k keys (sized for the largest k)
+  static constexpr int FIXED = 1024 + A_BYTES + kEpiThreads * kMaxHeap * 8 + 512;
+  static constexpr int FIT = (227 * 1024 - FIXED) / B_BYTES;
+  static constexpr int STAGES = FIT > 6 ? 6 : FIT;
+  static_assert(STAGES >= 2, "two key tiles must fit");
 };
 
 __device__ __forceinline__ int unit_of(int round, int cta, int nctas) {
   return round * nctas + ((round & 1) ? (nctas - 1 - cta) : cta);
 }
 
-// Number of 128-key tiles holding blocks 0..c-1 of an M-tile (0 if absent).
+// The block c of an M-tile's queries and the number of 256-key tiles holding
+// its candidate blocks 0..c-1 (0 if the M-tile does not exist or c = 0).
 __device__ __forceinline__ int mtile_ntiles(const IndexParams& p, int m, int* c_out) {
   if (m >= p.n_mtiles) {
     *c_out = 0;
@@ -81,9 +88,19 @@ __device__ __forceinline__ int mtile_ntiles(const IndexParams& p, int m, int* c_
   return static_cast<int>((static_cast<int64_t>(c) * p.B_k + kKeys - 1) / kKeys);
 }
 
+// Top-k keys: the score's order-preserving bits above the inverted block
+// index, so a larger key is a higher score or, at equal scores, a lower
+// block (Eq. 7 with ties to the lower index).  0 is an empty slot.
 __device__ __forceinline__ uint32_t order_bits(float f) {
   const uint32_t u = __float_as_uint(f);
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ uint64_t pack_key(float score, int b) {
+  return (static_cast<uint64_t>(order_bits(score)) << 32) |
+         static_cast<uint64_t>(0xFFFFFFFFu - static_cast<uint32_t>(b));
+}
+__device__ __forceinline__ int key_block(uint64_t key) {
+  return static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(key));
 }
 __device__ __forceinline__ float unorder_key(uint64_t key) {
   if (key == 0) return -INFINITY;  // empty slot
@@ -91,8 +108,15 @@ __device__ __forceinline__ float unorder_key(uint64_t key) {
   return __uint_as_float((o & 0x80000000u) ? (o & 0x7FFFFFFFu) : ~o);
 }
 
-// REG: keep the running Top-(k-1) of each row in registers (k <= 16, a
-// branch-free sorted-insertion network); otherwise in a shared-memory min-heap.
+// A work unit is one M-tile of 128 rows against 256-key K_idx tiles: one
+// 128x256xd_idx UMMA per tile (the wide N halves the shared-memory operand
+// bytes per FLOP against two 128-wide MMAs).  Epilogue group g reads the
+// tile's columns [128g, 128g+128) -- at B_k = 128 the even or the odd blocks
+// -- and keeps its own running Top-(k-1) of them; at the end of the unit
+// group 1 hands its list to group 0 through shared memory and group 0 merges
+// the two and writes the row.
+// REG: the running list lives in registers (k <= 16, a branch-free sorted
+// insertion network); otherwise in a shared-memory min-heap.
 // 10 warps: three of them share one SM sub-partition's 16K registers, so the
 // kernel lives within 168 registers per thread; one CTA per SM.
 template <int D_IDX, bool REG>
@@ -103,18 +127,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint8_t* sA = smem;                                   // 2 x A_BYTES
-  uint8_t* sB = sA + 2 * S::A_BYTES;                    // STAGES x B_BYTES
-  uint64_t* heap = reinterpret_cast<uint64_t*>(sB + S::STAGES * S::B_BYTES);
-  const int HS = p.k - 1;                               // heap size per row
-  uint64_t* bars = heap + static_cast<size_t>(kEpiThreads) * ((!REG && HS > 0) ? HS : 1);
+  uint8_t* sA = smem;                                   // A_BYTES
+  uint8_t* sB = sA + S::A_BYTES;                        // STAGES x B_BYTES
+  // [HS][kEpiThreads] Top-k keys per (slot, group column): the running heap
+  // (shared-memory path) and the hand-over to group 0 (both paths)
+  uint64_t* keys = reinterpret_cast<uint64_t*>(sB + S::STAGES * S::B_BYTES);
+  const int HS = p.k - 1;                               // non-local slots per row
+  uint64_t* bars = keys + static_cast<size_t>(kEpiThreads) * (HS > 0 ? HS : 1);
   uint64_t* a_full = bars;
   uint64_t* a_empty = bars + 1;
   uint64_t* b_full = bars + 2;
   uint64_t* b_empty = b_full + S::STAGES;
   uint64_t* acc_full = b_empty + S::STAGES;
   uint64_t* acc_empty = acc_full + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  uint64_t* xch_full = acc_empty + 2;   // group 1's list is in shared memory
+  uint64_t* xch_empty = xch_full + 1;   // group 0 has read it
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(xch_empty + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -131,6 +159,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&acc_full[s], 1);
       mbar_init(&acc_empty[s], 8);
     }
+    mbar_init(xch_full, 4);
+    mbar_init(xch_empty, 4);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -152,19 +182,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t g = 0, ua = 0;
       for (int round = 0;; ++round) {
         const int u = unit_of(round, cta, nctas);
-        if (u >= p.n_units || *abort_flag) break;
-        const int v = p.n_units - 1 - u;  // longest first
-        int c0, c1;
-        const int nt0 = mtile_ntiles(p, 2 * v, &c0);
-        const int nt1 = mtile_ntiles(p, 2 * v + 1, &c1);
-        const int nt = nt0 > nt1 ? nt0 : nt1;
+        if (u >= p.n_mtiles || *abort_flag) break;
+        const int m = p.n_mtiles - 1 - u;  // longest first
+        int c;
+        const int nt = mtile_ntiles(p, m, &c);
         if (nt == 0) continue;
         if (!mbar_wait(a_empty, (ua & 1) ^ 1, abort_flag, p.status, 10)) break;
-        mbar_arrive_expect_tx(a_full, 2 * S::A_BYTES);
-        for (int mt = 0; mt < 2; ++mt)
-          for (int c = 0; c < S::CH; ++c)
-            tma_load_2d(sA + mt * S::A_BYTES + c * kRows * S::SWB, &tm_q, a_full, c * S::CHE,
-                        (2 * v + mt) * kRows);
+        mbar_arrive_expect_tx(a_full, S::A_BYTES);
+        for (int ch = 0; ch < S::CH; ++ch)
+          tma_load_2d(sA + ch * kRows * S::SWB, &tm_q, a_full, ch * S::CHE, m * kRows);
         ++ua;
         bool ok = true;
         for (int t = 0; t < nt; ++t, ++g) {
@@ -174,9 +200,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           mbar_arrive_expect_tx(&b_full[st], S::B_BYTES);
-          for (int c = 0; c < S::CH; ++c)
-            tma_load_2d(sB + st * S::B_BYTES + c * kKeys * S::SWB, &tm_k, &b_full[st],
-                        c * S::CHE, t * kKeys);
+          for (int ch = 0; ch < S::CH; ++ch)
+            tma_load_2d(sB + st * S::B_BYTES + ch * kKeys * S::SWB, &tm_k, &b_full[st],
+                        ch * S::CHE, t * kKeys);
         }
         if (!ok) break;
       }
@@ -188,12 +214,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t g = 0, acnt = 0, ua = 0;
       for (int round = 0;; ++round) {
         const int u = unit_of(round, cta, nctas);
-        if (u >= p.n_units || *abort_flag) break;
-        const int v = p.n_units - 1 - u;
-        int c0, c1;
-        const int nt0 = mtile_ntiles(p, 2 * v, &c0);
-        const int nt1 = mtile_ntiles(p, 2 * v + 1, &c1);
-        const int nt = nt0 > nt1 ? nt0 : nt1;
+        if (u >= p.n_mtiles || *abort_flag) break;
+        const int m = p.n_mtiles - 1 - u;
+        int c;
+        const int nt = mtile_ntiles(p, m, &c);
         if (nt == 0) continue;
         if (!mbar_wait(a_full, ua & 1, abort_flag, p.status, 20)) break;
         tc_fence_after();
@@ -210,21 +234,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc_fence_after();
-          for (int mt = 0; mt < 2; ++mt) {
-            if (t >= (mt == 0 ? nt0 : nt1)) continue;
-            const uint32_t d_tmem = tmem_base + acc * 256 + mt * 128;
-            const uint32_t a_base = smem_u32(sA + mt * S::A_BYTES);
-            const uint32_t b_base = smem_u32(sB + st * S::B_BYTES);
+          const uint32_t d_tmem = tmem_base + acc * kKeys;
+          const uint32_t a_base = smem_u32(sA);
+          const uint32_t b_base = smem_u32(sB + st * S::B_BYTES);
 #pragma unroll
-            for (int c = 0; c < S::CH; ++c) {
+          for (int ch = 0; ch < S::CH; ++ch) {
 #pragma unroll
-              for (int s = 0; s < S::KSTEPS; ++s) {
-                const uint64_t ad =
-                    umma_desc(a_base + c * kRows * S::SWB + s * 32, 16, S::SBO, S::SWZ);
-                const uint64_t bd =
-                    umma_desc(b_base + c * kKeys * S::SWB + s * 32, 16, S::SBO, S::SWZ);
-                umma_bf16(d_tmem, ad, bd, idesc, (c | s) != 0);
-              }
+            for (int s = 0; s < S::KSTEPS; ++s) {
+              const uint64_t ad =
+                  umma_desc(a_base + ch * kRows * S::SWB + s * 32, 16, S::SBO, S::SWZ);
+              const uint64_t bd =
+                  umma_desc(b_base + ch * kKeys * S::SWB + s * 32, 16, S::SBO, S::SWZ);
+              umma_bf16(d_tmem, ad, bd, idesc, (ch | s) != 0);
             }
           }
           umma_commit(&b_empty[st]);
@@ -237,23 +258,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ---------------------------------------------------------- epilogue --
-    const int e = warp - 2;
-    const int mt = e >> 2;
+    const int grp = (warp - 2) >> 2;          // column half of every key tile
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;      // TMEM lane = row of the M-tile
-    const int hrow = mt * kRows + row;        // heap column
-    const int per_tile = kKeys / p.B_k;       // blocks per key tile (1 or 2)
-    uint32_t acnt = 0;
-    for (int round = 0;; ++round) {
+    const int hcol = grp * kRows + row;       // this thread's column of keys[]
+    const int per_half = kHalf / p.B_k;       // blocks per half tile (1 or 2)
+    uint32_t acnt = 0, ucnt = 0;
+    for (int round = 0;; ++round, ++ucnt) {
       const int u = unit_of(round, cta, nctas);
-      if (u >= p.n_units || *abort_flag) break;
-      const int v = p.n_units - 1 - u;
-      int c0, c1;
-      const int nt0 = mtile_ntiles(p, 2 * v, &c0);
-      const int nt1 = mtile_ntiles(p, 2 * v + 1, &c1);
-      const int nt = nt0 > nt1 ? nt0 : nt1;
-      const int my_nt = mt == 0 ? nt0 : nt1;
-      const int my_c = mt == 0 ? c0 : c1;
+      if (u >= p.n_mtiles || *abort_flag) break;
+      const int m = p.n_mtiles - 1 - u;
+      int c;
+      const int nt = mtile_ntiles(p, m, &c);
+      // group 1 reuses its keys[] column once group 0 has merged the last unit
+      if (grp == 1 && ucnt > 0 &&
+          !mbar_wait(xch_empty, (ucnt - 1) & 1, abort_flag, p.status, 31))
+        break;
       // running Top-(k-1): register list (descending; slots before RL-HS hold
       // +inf sentinels that never move) or shared-memory heap
       constexpr int RL = 15;
@@ -266,7 +286,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           li[s] = -1;
         }
       } else {
-        for (int s = 0; s < HS; ++s) heap[s * kEpiThreads + hrow] = 0ull;
+        for (int s = 0; s < HS; ++s) keys[s * kEpiThreads + hcol] = 0ull;
       }
       float root = HS > 0 ? -INFINITY : INFINITY;
       bool ok = true;
@@ -277,14 +297,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after();
-        // the row's 128 scores in two halves of 64 columns: the first half is
-        // reduced before the second is loaded, which keeps the peak register
-        // use low enough for the running Top-k list
-        const bool active = t < my_nt;
+        // the row's 128 scores of this half in two steps of 64 columns: the
+        // first is reduced before the second is loaded, which keeps the peak
+        // register use low enough for the running Top-k list
         const uint32_t ta = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
-                            acc * 256 + mt * 128;
-        float x0 = -INFINITY, x1 = -INFINITY, x2 = -INFINITY, x3 = -INFINITY;
-        if (active) {
+                            acc * kKeys + grp * kHalf;
+        float x0, x1, x2, x3;
+        {
           uint32_t ra[32], rb[32];
           tmem_ld32(ta + 0, ra);
           tmem_ld32(ta + 32, rb);
@@ -314,77 +333,105 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[acc]);
-        if (!active) continue;
-        float m[2];
-        if (per_tile == 1) {
-          m[0] = fmax3(x0, x1, fmaxf(x2, x3));
-          m[1] = -INFINITY;
+        float mx[2];
+        if (per_half == 1) {
+          mx[0] = fmax3(x0, x1, fmaxf(x2, x3));
+          mx[1] = -INFINITY;
         } else {
-          m[0] = fmaxf(x0, x1);
-          m[1] = fmaxf(x2, x3);
+          mx[0] = fmaxf(x0, x1);
+          mx[1] = fmaxf(x2, x3);
         }
-        for (int h = 0; h < per_tile; ++h) {
-          const int b = t * per_tile + h;
+        for (int h = 0; h < per_half; ++h) {
+          const int b = (2 * t + grp) * per_half + h;
           if constexpr (REG) {
             // a candidate enters only above the last kept score (strict: an
             // equal score belongs to a lower, earlier block, which stays)
-            const float x = b < my_c ? m[h] : -INFINITY;
+            const float x = b < c ? mx[h] : -INFINITY;
             if (!__any_sync(0xFFFFFFFFu, x > lv[RL - 1])) continue;
-            bool c[RL];
+            bool cmp[RL];
 #pragma unroll
-            for (int s2 = 0; s2 < RL; ++s2) c[s2] = x > lv[s2];
+            for (int s2 = 0; s2 < RL; ++s2) cmp[s2] = x > lv[s2];
 #pragma unroll
             for (int s2 = RL - 1; s2 > 0; --s2) {
-              lv[s2] = c[s2 - 1] ? lv[s2 - 1] : (c[s2] ? x : lv[s2]);
-              li[s2] = c[s2 - 1] ? li[s2 - 1] : (c[s2] ? b : li[s2]);
+              lv[s2] = cmp[s2 - 1] ? lv[s2 - 1] : (cmp[s2] ? x : lv[s2]);
+              li[s2] = cmp[s2 - 1] ? li[s2 - 1] : (cmp[s2] ? b : li[s2]);
             }
-            lv[0] = c[0] ? x : lv[0];
-            li[0] = c[0] ? b : li[0];
+            lv[0] = cmp[0] ? x : lv[0];
+            li[0] = cmp[0] ? b : li[0];
           } else {
-            if (b >= my_c || !(m[h] > root)) continue;
+            if (b >= c || !(mx[h] > root)) continue;
             // replace the root (worst kept) and sift down; ties -> lower block
-            const uint64_t key = (static_cast<uint64_t>(order_bits(m[h])) << 32) |
-                                 static_cast<uint64_t>(0xFFFFFFFFu - static_cast<uint32_t>(b));
+            const uint64_t key = pack_key(mx[h], b);
             int pos = 0;
             while (true) {
               const int c1i = 2 * pos + 1;
               if (c1i >= HS) break;
-              uint64_t km = heap[c1i * kEpiThreads + hrow];
+              uint64_t km = keys[c1i * kEpiThreads + hcol];
               int cm = c1i;
               if (c1i + 1 < HS) {
-                const uint64_t k2 = heap[(c1i + 1) * kEpiThreads + hrow];
+                const uint64_t k2 = keys[(c1i + 1) * kEpiThreads + hcol];
                 if (k2 < km) {
                   km = k2;
                   cm = c1i + 1;
                 }
               }
               if (km >= key) break;
-              heap[pos * kEpiThreads + hrow] = km;
+              keys[pos * kEpiThreads + hcol] = km;
               pos = cm;
             }
-            heap[pos * kEpiThreads + hrow] = key;
-            root = unorder_key(heap[hrow]);
+            keys[pos * kEpiThreads + hcol] = key;
+            root = unorder_key(keys[hcol]);
           }
         }
       }
       if (!ok) break;
-      // -------------------------------------------------- write the row --
-      const int m_glob = 2 * v + mt;
-      const int64_t row_glob = static_cast<int64_t>(m_glob) * kRows + row;
-      if (m_glob < p.n_mtiles && row_glob < p.N * p.H_kv) {
-        int sel[32];
-        int n = 0;
-        sel[n++] = my_c;  // the local block (Eq. 7: always kept)
-        if constexpr (REG) {
+      // ---------------------------------- hand over, merge, write the row --
+      if constexpr (REG) {
+        // the register list as keys, best first
 #pragma unroll
-          for (int s = 0; s < RL; ++s)
-            if (li[s] >= 0) sel[n++] = li[s];
-        } else {
-          for (int s = 0; s < HS; ++s) {
-            const uint64_t key = heap[s * kEpiThreads + hrow];
-            if (key != 0ull) sel[n++] = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(key));
-          }
+        for (int s = 0; s < RL; ++s)
+          if (s >= RL - HS)
+            keys[(s - (RL - HS)) * kEpiThreads + hcol] = li[s] >= 0 ? pack_key(lv[s], li[s]) : 0ull;
+      }
+      if (grp == 1) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(xch_full);
+        continue;
+      }
+      if (!mbar_wait(xch_full, ucnt & 1, abort_flag, p.status, 32)) break;
+      int sel[32];
+      int n = 0;
+      sel[n++] = c;  // the local block (Eq. 7: always kept)
+      if constexpr (REG) {
+        // both lists are sorted best first: a two-way merge
+        int ia = 0, ib = 0;
+        for (int s = 0; s < HS; ++s) {
+          const uint64_t ka = ia < HS ? keys[ia * kEpiThreads + row] : 0ull;
+          const uint64_t kb = ib < HS ? keys[ib * kEpiThreads + kRows + row] : 0ull;
+          const uint64_t kbest = ka >= kb ? ka : kb;
+          if (kbest == 0ull) break;
+          if (ka >= kb) ++ia;
+          else ++ib;
+          sel[n++] = key_block(kbest);
         }
+      } else {
+        // two heaps: take the best remaining key HS times
+        uint64_t taken_below = ~0ull;  // keys are distinct, so "below the last taken"
+        for (int s = 0; s < HS; ++s) {
+          uint64_t best = 0ull;
+          for (int j = 0; j < 2 * HS; ++j) {
+            const uint64_t kj = keys[(j % HS) * kEpiThreads + (j / HS) * kRows + row];
+            if (kj < taken_below && kj > best) best = kj;
+          }
+          if (best == 0ull) break;
+          taken_below = best;
+          sel[n++] = key_block(best);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(xch_empty);
+      const int64_t row_glob = static_cast<int64_t>(m) * kRows + row;
+      if (row_glob < p.N * p.H_kv) {
         for (int a = 1; a < n; ++a) {  // ascending
           const int x = sel[a];
           int b = a - 1;
@@ -409,11 +456,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 template <int D_IDX>
-size_t index_smem_bytes(int k, bool reg) {
+size_t index_smem_bytes(int k) {
   using S = IndexShape<D_IDX>;
-  const int hs = (!reg && k - 1 > 0) ? k - 1 : 1;
-  return 1024 + 2 * S::A_BYTES + S::STAGES * S::B_BYTES + static_cast<size_t>(kEpiThreads) * hs * 8 +
-         (4 + 2 * S::STAGES + 2) * 8 + 16;
+  const int hs = k - 1 > 0 ? k - 1 : 1;
+  return 1024 + S::A_BYTES + S::STAGES * S::B_BYTES + static_cast<size_t>(kEpiThreads) * hs * 8 +
+         (2 + 2 * S::STAGES + 4 + 2) * 8 + 16;
 }
 
 template <int D_IDX>
@@ -438,17 +485,16 @@ cudaError_t launch_typed(const IndexLaunch& a, cudaStream_t stream) {
   p.B_k = a.B_k;
   p.k = a.k;
   p.n_mtiles = static_cast<int>((a.N * a.H_kv + kRows - 1) / kRows);
-  p.n_units = (p.n_mtiles + 1) / 2;
   p.idx_out = a.idx_out;
   p.status = a.status;
   const bool reg = a.k <= 16;
-  const size_t smem = index_smem_bytes<D_IDX>(a.k, reg);
+  const size_t smem = index_smem_bytes<D_IDX>(a.k);
   auto kern = reg ? index_topk_kernel<D_IDX, true> : index_topk_kernel<D_IDX, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   int grid = num_sms();
-  if (grid > p.n_units) grid = p.n_units;
+  if (grid > p.n_mtiles) grid = p.n_mtiles;
   if (grid < 1) grid = 1;
   prof_begin("index_topk", stream);
   kern<<<grid, kThreads, smem, stream>>>(tq, tk, p);
