@@ -331,23 +331,28 @@ def run_msa(args, cfg, rank, world, local):
     dom = max(prof, key=lambda n: prof[n][1])
     launches, dom_ms = prof[dom]
     per_launch_ms = dom_ms / launches
+    # a kernel inside a timed region of about a second or more runs under the
+    # power cap: its denominator is the sustained GEMM rate, else the burst one
+    sustained = ms * args.steps >= 1000.0
+    tc_peak = pk["bf16_tflops_sustained"] if sustained else pk["bf16_tflops"]
+    tc_kind = "sustained" if sustained else "burst"
     if dom == "index_topk":
         work, unit, bound = f_idx, "TFLOP/s", "tensor"
         achieved = work / (per_launch_ms * 1e-3) / 1e12
-        peak = pk["bf16_tflops"]
+        peak = tc_peak
     elif dom == "attn_phase1":
         # one launch per query chunk and step: the Main Branch FLOPs of a chunk
         work = f_main / (launches / args.steps)
         unit, bound = "TFLOP/s", "tensor"
         achieved = work / (per_launch_ms * 1e-3) / 1e12
-        peak = pk["bf16_tflops"]
+        peak = tc_peak
     else:
         unit, bound = "GB/s", "hbm"
         achieved, peak = None, pk["hbm_gbs"]
     traffic, traffic_src = ncu_traffic(dom, N / (launches / args.steps))
     roofline = {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
                 "frac": (achieved / peak) if achieved else None, "traffic": traffic,
-                "traffic_source": traffic_src, "peak_kind": f"{pk_kind} burst",
+                "traffic_source": traffic_src, "peak_kind": f"{pk_kind} {tc_kind}",
                 "share": dom_ms / total_ms if total_ms else None}
 
     # ---- CPU oracle on a bounded sample (rank 0, N=1 only)
