@@ -9,24 +9,29 @@
 //   * Rows of the MMA are (query, group) pairs: Q_idx is [N, H_kv, d_idx], so
 //     128 consecutive rows of the [N*H_kv, d_idx] view are 128/H_kv queries x
 //     all H_kv groups, and they all share the one index key head (Eq. 5).  A
-//     work unit is two such 128-row M-tiles; every 128-key K_idx tile streamed
-//     by TMA feeds two 128x128xd_idx UMMAs (A = Q_idx rows, B = K_idx rows,
-//     both K-major, fp32 accumulators in TMEM).
+//     work unit is one such 128-row M-tile; every 256-key K_idx tile streamed
+//     by TMA feeds one 128x256xd_idx UMMA (A = Q_idx rows, B = K_idx rows,
+//     both K-major, fp32 accumulators in TMEM).  At N = 256 an MMA step reads
+//     96 bytes of shared-memory operands per clock at peak rate, against 128
+//     (all of it) for two N = 128 MMAs, which measured about 20% slower.
 //   * All queries of an M-tile live in one block c (128/H_kv divides B_k), so
 //     the non-local candidates are exactly blocks 0..c-1: every key tile is
 //     fully visible and needs no causal mask.  The local block is forced and
 //     needs no score at all.
-//   * Epilogue: one TMEM lane (= one row) per thread.  tcgen05.ld pulls the
-//     row's 128 scores, a 3-input max tree pools them per block, and a
-//     per-row min-heap of k-1 packed keys (score bits, inverted block index)
-//     in shared memory keeps the running Top-(k-1).  The root's score is
-//     cached in a register, so a block costs one compare unless it enters.
-//     The scale 1/sqrt(d_idx) is positive and is not applied: the order of
-//     the raw dot products is the order of Eq. 6's scores.
+//   * Epilogue: one TMEM lane (= one row) per thread; two groups of four
+//     warps read the two 128-column halves of a tile (at B_k = 128 the even
+//     and the odd blocks).  tcgen05.ld pulls a row's 128 scores of the half,
+//     a 3-input max tree pools them per block, and each group keeps its own
+//     running Top-(k-1) of packed keys (score bits, inverted block index): a
+//     sorted register list for k <= 16, else a min-heap in shared memory
+//     whose root score is cached in a register, so a block costs one compare
+//     unless it enters.  At the end of a unit group 1 hands its list to
+//     group 0 through shared memory and group 0 merges the two and writes the
+//     row.  The scale 1/sqrt(d_idx) is positive and is not applied: the order
+//     of the raw dot products is the order of Eq. 6's scores.
 //   * Warp roles: warp 0 = TMA producer, warp 1 = MMA issuer (and TMEM
-//     owner), warps 2..9 = epilogue (4 per M-tile; warp w reads TMEM lanes
-//     32*(w%4) .. +31).  TMEM holds 2 accumulator stages x 2 M-tiles x 128
-//     columns = 512 columns.
+//     owner), warps 2..9 = epilogue (warp w reads TMEM lanes 32*(w%4) .. +31).
+//     TMEM holds 2 accumulator stages x 256 columns = 512 columns.
 //   * Persistent grid of one CTA per SM; units are visited longest-first in a
 //     snake order over CTAs to balance the causal triangle.
 #include <cuda.h>
