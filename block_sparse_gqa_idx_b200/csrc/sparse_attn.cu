@@ -30,6 +30,8 @@ namespace msa {
 namespace {
 
 constexpr int kThreads = 320;
+// Largest per-CTA key histogram of the inverse index (H_kv * B keys).
+constexpr size_t kMaxHistBytes = 192 * 1024;
 constexpr int kRowsPerTile = 128;
 // Queries per chunk: bounds the partial-output workspace.  Chunks are kept
 // large so that every (group, block) list holds many queries per chunk: K/V
@@ -94,6 +96,64 @@ struct InvParams {
   DevStatus* status;
 };
 
+// The key (group r, block b) of entry e of the chunk, or -1 when the entry
+// selects nothing (-1 padding, or a block after the query's own).  Entry e is
+// (query, group, slot) in the layout of I, so e is also the entry's output
+// slot id and I is read contiguously.
+__device__ __forceinline__ int inv_key(const InvParams& p, int64_t e, bool report_bad) {
+  const int64_t per_q = static_cast<int64_t>(p.H_kv) * p.kk;
+  const int64_t il = e / per_q;
+  const int r = static_cast<int>((e - il * per_q) / p.kk);
+  const int64_t i = p.q0 + il;
+  const int32_t b = p.idx[p.q0 * per_q + e];
+  if (b < -1 || b >= p.B) {
+    if (report_bad) report(p.status, DEV_ERR_BAD_INDEX, 40, static_cast<int>(i), b);
+    return -1;
+  }
+  return (b >= 0 && b <= i / p.B_k) ? r * static_cast<int>(p.B) + b : -1;
+}
+
+// Inverse index with a per-CTA histogram of every key in shared memory.  A
+// CTA owns a contiguous range of entries (a range of queries).  Counting: the
+// CTA counts its entries per key in shared memory and adds each non-zero
+// count to the global one with a single atomic.  Scattering: the CTA counts
+// again, reserves each key's range of the key's list with one atomic on the
+// key's cursor, and places every entry at a shared-memory atomic's position
+// inside that range.
+template <bool SCATTER>
+__global__ void __launch_bounds__(512) inv_index_smem_kernel(const InvParams p) {
+  extern __shared__ int32_t hist[];  // [H_kv * B]
+  const int nkeys = static_cast<int>(p.H_kv * p.B);
+  const int64_t total = p.nq * p.H_kv * p.kk;
+  const int64_t per = (total + gridDim.x - 1) / gridDim.x;
+  const int64_t e0 = static_cast<int64_t>(blockIdx.x) * per;
+  const int64_t e1 = e0 + per < total ? e0 + per : total;
+  for (int j = threadIdx.x; j < nkeys; j += blockDim.x) hist[j] = 0;
+  __syncthreads();
+  for (int64_t e = e0 + threadIdx.x; e < e1; e += blockDim.x) {
+    const int key = inv_key(p, e, !SCATTER);
+    if (key >= 0) atomicAdd(&hist[key], 1);
+  }
+  __syncthreads();
+  if constexpr (!SCATTER) {
+    for (int j = threadIdx.x; j < nkeys; j += blockDim.x) {
+      const int n = hist[j];
+      if (n > 0) atomicAdd(&p.c.counts[j], n);
+    }
+  } else {
+    for (int j = threadIdx.x; j < nkeys; j += blockDim.x) {
+      const int n = hist[j];
+      if (n > 0) hist[j] = atomicAdd(&p.c.cursor[j], n);
+    }
+    __syncthreads();
+    for (int64_t e = e0 + threadIdx.x; e < e1; e += blockDim.x) {
+      const int key = inv_key(p, e, false);
+      if (key >= 0) p.c.entries[atomicAdd(&hist[key], 1)] = static_cast<uint32_t>(e);
+    }
+  }
+}
+
+// Inverse index for key sets too large for a shared-memory histogram.
 // Thread order: slot-major, then group, then query, so lanes of a warp read the
 // same slot of consecutive queries -- hot blocks (a sink, the previous block)
 // collapse into one aggregated atomic per warp.
@@ -775,6 +835,22 @@ cudaError_t launch_typed(const AttnLaunch& a, cudaStream_t stream) {
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const int sms = num_sms();
+  // inverse index: a shared-memory histogram of every key per CTA when it fits
+  const size_t hist_bytes = sizeof(int32_t) * static_cast<size_t>(nkeys);
+  int hist_grid = sms;
+  if (hist_bytes <= kMaxHistBytes) {
+    e = cudaFuncSetAttribute(inv_index_smem_kernel<false>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(hist_bytes));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(inv_index_smem_kernel<true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(hist_bytes));
+    if (e != cudaSuccess) return e;
+    // CTAs that fit beside one another on an SM (at most 4 per SM)
+    const size_t per_sm = 200 * 1024 / (hist_bytes + 1024);
+    hist_grid = sms * static_cast<int>(per_sm < 1 ? 1 : (per_sm > 4 ? 4 : per_sm));
+  }
 
   for (int64_t q0 = 0; q0 < a.N; q0 += Nc) {
     const int64_t nq = (a.N - q0) < Nc ? (a.N - q0) : Nc;
@@ -792,17 +868,29 @@ cudaError_t launch_typed(const AttnLaunch& a, cudaStream_t stream) {
     ip.c = c;
     ip.status = a.status;
     const int64_t total = nq * a.H_kv * a.kk;
-    int blocks = static_cast<int>((total + 255) / 256);
-    if (blocks > sms * 16) blocks = sms * 16;
-    prof_begin("inv_count", stream);
-    inv_index_kernel<false><<<blocks, 256, 0, stream>>>(ip);
-    prof_end(stream);
-    prof_begin("inv_scan", stream);
-    inv_scan_kernel<<<1, 1024, 0, stream>>>(ip);
-    prof_end(stream);
-    prof_begin("inv_scatter", stream);
-    inv_index_kernel<true><<<blocks, 256, 0, stream>>>(ip);
-    prof_end(stream);
+    if (hist_bytes <= kMaxHistBytes) {
+      prof_begin("inv_count", stream);
+      inv_index_smem_kernel<false><<<hist_grid, 512, hist_bytes, stream>>>(ip);
+      prof_end(stream);
+      prof_begin("inv_scan", stream);
+      inv_scan_kernel<<<1, 1024, 0, stream>>>(ip);
+      prof_end(stream);
+      prof_begin("inv_scatter", stream);
+      inv_index_smem_kernel<true><<<hist_grid, 512, hist_bytes, stream>>>(ip);
+      prof_end(stream);
+    } else {
+      int blocks = static_cast<int>((total + 255) / 256);
+      if (blocks > sms * 16) blocks = sms * 16;
+      prof_begin("inv_count", stream);
+      inv_index_kernel<false><<<blocks, 256, 0, stream>>>(ip);
+      prof_end(stream);
+      prof_begin("inv_scan", stream);
+      inv_scan_kernel<<<1, 1024, 0, stream>>>(ip);
+      prof_end(stream);
+      prof_begin("inv_scatter", stream);
+      inv_index_kernel<true><<<blocks, 256, 0, stream>>>(ip);
+      prof_end(stream);
+    }
 
     P1Params pp;
     pp.q0 = q0;
