@@ -189,6 +189,31 @@ def test_attention_128k_sampled(msa):
     _check_attn(msa, inp, dev, idx, cfg, rows, "128k")
 
 
+def test_attention_key_set_beyond_shared_histogram(msa):
+    """H_kv * B = 50000 (group, block) keys: more than a per-CTA shared-memory
+    histogram of the inverse index holds, so the global-atomic inverse index
+    runs.  Selection: the local block and k-1 earlier blocks at a per-row
+    random stride (strictly decreasing, so distinct), ascending, -1 padded."""
+    N, H_kv, d_h, B_k, k = 400000, 8, 64, 64, 8
+    assert H_kv * ((N + B_k - 1) // B_k) * 4 > 192 * 1024
+    rng = np.random.default_rng(41)
+    inp = {t: inputs.bf16_bits(rng.standard_normal((N, H_kv, d_h), dtype=np.float32))
+           for t in ("q", "k", "v")}
+    b_i = (np.arange(N) // B_k)[:, None, None]
+    stride = rng.integers(1, 14, size=(N, H_kv, 1))
+    offset = rng.integers(0, 6, size=(N, H_kv, 1))
+    j = np.arange(k)[None, None, :]
+    blk = np.where(j == 0, b_i, b_i - j * stride - offset)
+    blk = np.where(blk < 0, np.iinfo(np.int32).max, blk)
+    idx = np.sort(blk, axis=2)
+    idx = np.where(idx == np.iinfo(np.int32).max, -1, idx).astype(np.int32)
+    cfg = inputs.MSAConfig("wide", N=N, H_q=H_kv, H_kv=H_kv, d_h=d_h, d_idx=64, B_k=B_k, k=k,
+                           seed_index=41)
+    dev = dev_inputs(inp)
+    rows = np.unique(np.concatenate([rng.integers(0, N, 64), [0, 63, 64, N - 1]]))
+    _check_attn(msa, inp, dev, torch.from_numpy(idx).cuda(), cfg, rows, "wide key set")
+
+
 def test_device_status_reports_bad_index(msa):
     cfg = inputs.MSAConfig("bad", N=256, H_q=16, H_kv=2, d_h=64, d_idx=64, B_k=64, k=2,
                            seed_index=37)
