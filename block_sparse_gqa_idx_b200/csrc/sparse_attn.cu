@@ -781,6 +781,63 @@ __global__ void __launch_bounds__(256, 2) attn_merge_kernel(const MergeParams p)
   if (p.lse != nullptr && d0 == 0) p.lse[i * p.H_q + h] = use ? m + logf(wsum) : -INFINITY;
 }
 
+// Merge for G * D_H < 256 outputs per (query, group), where one warp per
+// (query, group) would have idle lanes: one thread per 8 consecutive outputs
+// of one head; each thread reads its (query, group)'s selection and its
+// head's LSEs itself.
+template <int D_H>
+__global__ void __launch_bounds__(256) attn_merge_small_kernel(const MergeParams p) {
+  const int per_unit = p.G * D_H / 8;  // threads per (query, group)
+  const int64_t gt = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t unit = gt / per_unit;
+  if (unit >= p.nq * p.H_kv) return;
+  const int e0 = static_cast<int>(gt - unit * per_unit) * 8;
+  const int g = e0 / D_H, d0 = e0 - g * D_H;
+  const int64_t il = unit / p.H_kv;
+  const int r = static_cast<int>(unit - il * p.H_kv);
+  const int64_t i = p.q0 + il;
+  const int64_t b_i = i / p.B_k;
+  const int64_t slot0 = (il * p.H_kv + r) * p.kk;
+  const int32_t* sel = p.idx + (i * p.H_kv + r) * p.kk;
+  const float* lse_h = p.c.part_lse + slot0 * p.G + g;
+  float m = -INFINITY;
+  for (int s = 0; s < p.kk; ++s) {
+    const int b = sel[s];
+    if (b >= 0 && b <= b_i) m = fmaxf(m, lse_h[s * p.G]);
+  }
+  float acc[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
+  float wsum = 0.0f;
+  // partial layout [slot][d/8][g][8]
+  const __half* base = p.c.part_o + slot0 * p.G * D_H + (d0 >> 3) * p.G * 8 + g * 8;
+  for (int s = 0; s < p.kk; ++s) {
+    const int b = sel[s];
+    if (b < 0 || b > b_i) continue;
+    const float w = __expf(lse_h[s * p.G] - m);
+    wsum += w;
+    const uint4 x = *reinterpret_cast<const uint4*>(base + static_cast<int64_t>(s) * p.G * D_H);
+    const __half2* hv = reinterpret_cast<const __half2*>(&x);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = __half22float2(hv[e]);
+      acc[2 * e] = fmaf(w, f.x, acc[2 * e]);
+      acc[2 * e + 1] = fmaf(w, f.y, acc[2 * e + 1]);
+    }
+  }
+  const int h = r * p.G + g;
+  const float inv = wsum > 0.0f ? 1.0f / wsum : 0.0f;
+  uint4 o4;
+  uint32_t* ow = reinterpret_cast<uint32_t*>(&o4);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    __nv_bfloat162 t = __floats2bfloat162_rn(acc[2 * e] * inv, acc[2 * e + 1] * inv);
+    ow[e] = *reinterpret_cast<uint32_t*>(&t);
+  }
+  *reinterpret_cast<uint4*>(p.o + (i * p.H_q + h) * static_cast<int64_t>(D_H) + d0) = o4;
+  if (p.lse != nullptr && d0 == 0) p.lse[i * p.H_q + h] = wsum > 0.0f ? m + logf(wsum) : -INFINITY;
+}
+
 template <int D_H, int B_K>
 size_t p1_smem_bytes() {
   using SH = P1Shape<D_H, B_K>;
@@ -924,7 +981,11 @@ cudaError_t launch_typed(const AttnLaunch& a, cudaStream_t stream) {
     mp.B_k = a.B_k;
     mp.c = c;
     prof_begin("attn_merge", stream);
-    {
+    if (G * D_H < 256) {
+      const int64_t threads = nq * a.H_kv * (G * D_H / 8);
+      const unsigned blocks = static_cast<unsigned>((threads + 255) / 256);
+      attn_merge_small_kernel<D_H><<<blocks, 256, 0, stream>>>(mp);
+    } else {
       const int per_unit = G * D_H / 32;           // outputs per lane with one warp
       const int E = per_unit >= 32 ? 32 : (per_unit >= 16 ? 16 : 8);
       const int W = G * D_H / (32 * E);

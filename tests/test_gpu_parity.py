@@ -118,6 +118,9 @@ def test_attention_32k_shape_truncated(msa):
     (700, 8, 2, 128, 128, 3),    # G = 4 (8-head boxes, half used), d_h = 128
     (513, 64, 4, 128, 128, 4),   # G = 16 (pages' 64/4 heads)
     (300, 16, 2, 128, 64, 8),    # k * B_k >= N: every visible block selected
+    (600, 8, 8, 64, 64, 4),      # G = 1, d_h = 64: 64 outputs per (query, group)
+    (600, 8, 4, 64, 64, 4),      # G = 2, d_h = 64: 128 outputs per (query, group)
+    (640, 8, 8, 128, 128, 3),    # G = 1, d_h = 128
 ])
 def test_attention_edge_shapes(msa, N, H_q, H_kv, d_h, B_k, k):
     cfg = inputs.MSAConfig("edge", N=N, H_q=H_q, H_kv=H_kv, d_h=d_h, d_idx=64, B_k=B_k, k=k,
