@@ -40,12 +40,12 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # unchanged.  kernel -> (source, sha256, bytes per unit, unit, capture)
 NCU_TRAFFIC = {
     "attn_phase1": ("sparse_attn.cu",
-                    "d90594744ff3c8ee58378bea6599c9fea880d987d76ab3c0ad6e1d0054cdb80e",
-                    (3.672019e9 + 4.190698e9) / 32768, "query",
+                    "eaa00bcc129b2792ba862d81a9a1705809c41fd75cb86b727054e51247d9eaf2",
+                    (3.666177e9 + 4.195406e9) / 32768, "query",
                     "profiles/prefill_32k_ncu_full.md: 32K capture, scaled by queries"),
     "attn_merge": ("sparse_attn.cu",
-                   "d90594744ff3c8ee58378bea6599c9fea880d987d76ab3c0ad6e1d0054cdb80e",
-                   (4.243662e9 + 0.269400e9) / 32768, "query",
+                   "eaa00bcc129b2792ba862d81a9a1705809c41fd75cb86b727054e51247d9eaf2",
+                   (4.243224e9 + 0.269582e9) / 32768, "query",
                    "profiles/prefill_32k_ncu_full.md: 32K capture, scaled by queries"),
 }
 
