@@ -48,7 +48,8 @@ class msa_kernel_time(ctypes.Structure):
 EXPORTS = ("msa_index_topk_workspace", "msa_index_topk", "msa_sparse_attn_fwd_workspace",
            "msa_sparse_attn_fwd", "msa_sparse_decode_workspace", "msa_sparse_decode",
            "msa_get_device_status", "msa_profile_enable", "msa_profile_read",
-           "msa_status_string", "msa_version", "msa_sparse_decode_noalloc", "msa_last_error")
+           "msa_status_string", "msa_version", "msa_sparse_decode_noalloc", "msa_last_error",
+           "msa_selftest_bounded_wait")
 
 
 def _load() -> ctypes.CDLL:
@@ -76,6 +77,8 @@ def _load() -> ctypes.CDLL:
     lib.msa_get_device_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_int32),
                                           ctypes.POINTER(ctypes.c_int32)]
     lib.msa_get_device_status.restype = I32
+    lib.msa_selftest_bounded_wait.argtypes = [P, P]
+    lib.msa_selftest_bounded_wait.restype = I32
     lib.msa_profile_enable.argtypes = [ctypes.c_int32]
     lib.msa_profile_enable.restype = I32
     lib.msa_profile_read.argtypes = [ctypes.POINTER(msa_kernel_time), ctypes.c_int32]
@@ -292,6 +295,13 @@ def sparse_decode_noalloc(q, q_idx, k_new, v_new, k_idx_new, k_cache, v_cache, k
                                          _ptr(v_cache), _ptr(k_idx_cache), _ptr(seq_len),
                                          _ptr(o), _ptr(idx_out), _stream(stream)))
     return o, idx_out
+
+
+def selftest_bounded_wait(workspace: torch.Tensor, stream=None) -> None:
+    """Launch the library's bounded-wait self-test (times out after about 2 s
+    and records MSA_DEV_TIMEOUT, where 99, in the workspace's status word)."""
+    _raise("msa_selftest_bounded_wait",
+           LIB.msa_selftest_bounded_wait(_ptr(workspace), _stream(stream)))
 
 
 def device_status(workspace: torch.Tensor, stream=None) -> Tuple[int, int]:

@@ -131,6 +131,22 @@ msa_status from_cuda(cudaError_t e) {
 
 msa::DevStatus* status_of(void* ws) { return reinterpret_cast<msa::DevStatus*>(ws); }
 
+// Failure-detection self-test: one thread waits, through the bounded wait of
+// every kernel here, on an mbarrier that nothing completes.  The wait gives up
+// after its limit, records the timeout and the kernel returns.
+constexpr int kSelftestWhere = 99;
+__global__ void selftest_wait_kernel(msa::DevStatus* st) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    msa::mbar_init(&bar, 1);
+    abort_flag = 0;
+    msa::fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) msa::mbar_wait(&bar, 0, &abort_flag, st, kSelftestWhere);
+}
+
 }  // namespace
 
 extern "C" {
@@ -324,6 +340,14 @@ int32_t msa_profile_read(msa_kernel_time* out, int32_t max_entries) {
   const int32_t n = static_cast<int32_t>(acc.size());
   for (int32_t j = 0; j < n && j < max_entries && out != nullptr; ++j) out[j] = acc[j];
   return n;
+}
+
+msa_status msa_selftest_bounded_wait(void* ws, void* stream) {
+  if (ws == nullptr || !aligned16(ws)) return MSA_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (from_cuda(cudaMemsetAsync(ws, 0, sizeof(msa::DevStatus), s)) != MSA_OK) return MSA_ERR_CUDA;
+  selftest_wait_kernel<<<1, 32, 0, s>>>(status_of(ws));
+  return from_cuda(cudaGetLastError());
 }
 
 msa_status msa_get_device_status(const void* ws, void* stream, int32_t* code, int32_t* where) {

@@ -178,6 +178,17 @@ MSA_API msa_status msa_sparse_decode_noalloc(const msa_decode_dims* dims, const 
 MSA_API msa_status msa_get_device_status(const void* workspace, void* stream, int32_t* code,
                                  int32_t* where);
 
+/* Failure-detection self-test (no counterpart on the pages).  Every on-device
+ * wait in this library is bounded: on timeout the kernel records
+ * MSA_DEV_TIMEOUT in the workspace's status word and returns, with no trap,
+ * so the context stays usable.  This call exercises exactly that path: it
+ * launches one thread that waits, through the same bounded wait, on a barrier
+ * that nothing completes; after the limit (about 2 s) the status word reads
+ * MSA_DEV_TIMEOUT with where = 99.  `workspace`: at least 256 bytes of device
+ * memory, 16-byte aligned, owned by the caller.  Asynchronous on `stream`;
+ * read the outcome with msa_get_device_status. */
+MSA_API msa_status msa_selftest_bounded_wait(void* workspace, void* stream);
+
 /* Per-kernel timing for measurement tools.  msa_profile_enable(1) clears the
  * record and starts recording a CUDA event pair around every kernel that the
  * entry points above launch (on the caller's stream); msa_profile_enable(0)

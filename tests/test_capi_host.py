@@ -94,6 +94,11 @@ def test_decode_rejects_on_host(capi):
     assert capi.LIB.msa_sparse_decode(ctypes.byref(dd), *args, 1 << 30, None) == 2
 
 
+def test_selftest_rejects_bad_workspace_on_host(capi):
+    assert capi.LIB.msa_selftest_bounded_wait(None, None) == 1
+    assert capi.LIB.msa_selftest_bounded_wait(ctypes.c_void_p((1 << 20) + 4), None) == 1
+
+
 def test_status_strings(capi):
     texts = {capi.LIB.msa_status_string(i).decode() for i in range(6)}
     assert len(texts) == 6

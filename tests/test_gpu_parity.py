@@ -217,6 +217,23 @@ def test_attention_key_set_beyond_shared_histogram(msa):
     _check_attn(msa, inp, dev, torch.from_numpy(idx).cuda(), cfg, rows, "wide key set")
 
 
+def test_bounded_wait_times_out_reports_and_context_survives(msa):
+    """Failure detection without a fault: a wait that nothing completes gives
+    up after its limit, the status word says so, and the next call works."""
+    import time
+
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    torch.cuda.synchronize()
+    t0 = time.time()
+    msa.selftest_bounded_wait(ws)
+    code, where = msa.device_status(ws)
+    elapsed = time.time() - t0
+    assert (code, where) == (1, 99)
+    assert 1.0 < elapsed < 20.0
+    cfg = inputs.CONFIGS["tiny"]
+    _check_index(msa, cfg, rows=np.arange(0, cfg.N, 97))
+
+
 def test_device_status_reports_bad_index(msa):
     cfg = inputs.MSAConfig("bad", N=256, H_q=16, H_kv=2, d_h=64, d_idx=64, B_k=64, k=2,
                            seed_index=37)
