@@ -19,6 +19,7 @@ from __future__ import annotations
 
 import argparse
 import json
+import re
 import os
 import statistics
 import subprocess
@@ -35,16 +36,17 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of a kernel from
-# one ncu capture, per unit of work, with the SHA-256 of the kernel's source
-# file at capture time: the figure is reported only while that file is
-# unchanged.  kernel -> (source, sha256, bytes per unit, unit, capture)
+# one ncu capture, per unit of work, with the SHA-256 of the kernel source's
+# code (comments and blank lines removed) at capture time: the figure is
+# reported only while that code is unchanged.
+# kernel -> (source, sha256, bytes per unit, unit, capture)
 NCU_TRAFFIC = {
     "attn_phase1": ("sparse_attn.cu",
-                    "eaa00bcc129b2792ba862d81a9a1705809c41fd75cb86b727054e51247d9eaf2",
+                    "fcfe89b57dee736d3a21ffded527321b445b10613e32e5dc48938365bead0a81",
                     (3.666177e9 + 4.195406e9) / 32768, "query",
                     "profiles/prefill_32k_ncu_full.md: 32K capture, scaled by queries"),
     "attn_merge": ("sparse_attn.cu",
-                   "eaa00bcc129b2792ba862d81a9a1705809c41fd75cb86b727054e51247d9eaf2",
+                   "fcfe89b57dee736d3a21ffded527321b445b10613e32e5dc48938365bead0a81",
                    (4.243224e9 + 0.269582e9) / 32768, "query",
                    "profiles/prefill_32k_ncu_full.md: 32K capture, scaled by queries"),
 }
@@ -60,9 +62,11 @@ def ncu_traffic(kernel: str, units: float):
         return None, None
     src, sha, per_unit, _, where = ent
     path = os.path.join(ROOT, "block_sparse_gqa_idx_b200", "csrc", src)
-    with open(path, "rb") as f:
-        if hashlib.sha256(f.read()).hexdigest() != sha:
-            return None, None
+    with open(path, encoding="utf-8") as f:
+        code = re.sub(r"//[^\n]*", "", f.read())
+    code = "\n".join(line.rstrip() for line in code.splitlines() if line.strip())
+    if hashlib.sha256(code.encode()).hexdigest() != sha:
+        return None, None
     return per_unit * units, where
 
 

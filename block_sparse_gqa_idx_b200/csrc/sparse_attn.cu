@@ -307,7 +307,7 @@ __device__ __forceinline__ int find_key(const int32_t* tile_off, int64_t nkeys, 
 // Phase 1.  Each CTA owns a contiguous range of tiles; tiles of one (group,
 // block) key come in long runs there, so the K/V block sits in one shared
 // slot for the whole run (reloaded only when the key changes) while the
-// gathered query rows stream through a 4-deep ring.  TMEM holds two tiles
+// gathered query rows stream through a 5-deep ring.  TMEM holds two tiles
 // (S and O, 128 + 128 columns each); two softmax/epilogue groups of four
 // warps take alternate tiles.
 //   warp 0      producer (all lanes: lane q issues query q's TMA box)
