@@ -59,9 +59,10 @@ def _load():
             lib.oracle_sparse_attn.argtypes = [P, P, P, P, I64, I32, I32, I32, I32, I32, D, P, I64,
                                                P, P, I32]
             lib.oracle_dense_attn.argtypes = [P, P, P, I64, I32, I32, I32, D, P, I64, P, P, I32]
+            lib.oracle_index_lse.argtypes = [P, P, P, I64, I32, I32, I32, I32, D, P, I64, P, I32]
             lib.oracle_flops.argtypes = [D] * 7 + [P, P, P]
             for f in ("oracle_block_scores", "oracle_index_topk", "oracle_sparse_attn",
-                      "oracle_dense_attn"):
+                      "oracle_dense_attn", "oracle_index_lse"):
                 getattr(lib, f).restype = I32
             lib.oracle_flops.restype = None
             _lib = lib
@@ -156,6 +157,26 @@ def sparse_attn(q_rows: np.ndarray, k: np.ndarray, v: np.ndarray, idx_rows: np.n
                                       ir.shape[2], float(scale), _p(rows), n, _p(o), _p(lse),
                                       threads), "sparse_attn")
     return o, lse
+
+
+def index_lse(q_idx_rows: np.ndarray, k_idx: np.ndarray, idx_rows: np.ndarray, B_k: int,
+              rows: np.ndarray, N: Optional[int] = None, scale: Optional[float] = None,
+              threads: int = 0) -> np.ndarray:
+    """Eq. 9's Index Branch normaliser (the LSE_idx of the KL loss fusion) for
+    the listed rows: log of the sum of exp(S^idx) over the selected tokens
+    j <= i.  q_idx_rows [n,H_kv,d_idx], k_idx [>=N,d_idx], idx_rows [n,H_kv,kk].
+    Returns [n,H_kv] float64 (-inf for an empty token set)."""
+    qr = _c(q_idx_rows, np.uint16)
+    kr = _c(k_idx, np.uint16)
+    ir = _c(idx_rows, np.int32)
+    rows = _c(rows, np.int64)
+    n, H_kv, d_idx = qr.shape
+    N = kr.shape[0] if N is None else N
+    scale = 1.0 / np.sqrt(d_idx) if scale is None else scale
+    out = np.empty((n, H_kv), dtype=np.float64)
+    _check(_load().oracle_index_lse(_p(qr), _p(kr), _p(ir), N, H_kv, d_idx, B_k, ir.shape[2],
+                                    float(scale), _p(rows), n, _p(out), threads), "index_lse")
+    return out
 
 
 def dense_attn(q_rows: np.ndarray, k: np.ndarray, v: np.ndarray, rows: np.ndarray,

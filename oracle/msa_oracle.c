@@ -301,6 +301,84 @@ int oracle_sparse_attn(const uint16_t *q_rows, const uint16_t *K, const uint16_t
 }
 
 /*
+ * Normaliser of the Index Branch distribution of the KL alignment loss,
+ * Eq. 9 [xllm] ("KL Alignment Loss") with the fusion of [xllm] "4.3 Sparse
+ * KL Loss Fusion" and [chl] 5.4 (each selected block's LSE, reduced over the
+ * Top-k blocks):
+ *   I_tok   = { j in a selected block of (i, r) : j <= i }
+ *   S[j]    = <q_idx[i, r], K_idx[j]> * scale              (Eq. 6; scale = 1/sqrt(d_idx))
+ *   LSE_idx = log sum_{j in I_tok} exp(S[j])
+ * so that P^idx[i, r, j] = exp(S[j] - LSE_idx).  Written as the definition:
+ * the token set first, then a two-pass log-sum-exp (max, then the sum of
+ * exp(S - max)) in double.  An empty token set gives -inf.
+ * q_idx_rows: [n_rows, H_kv, d_idx]; k_idx: [N, d_idx];
+ * idx: [n_rows, H_kv, k]; lse_out: [n_rows, H_kv].
+ */
+int oracle_index_lse(const uint16_t *q_idx_rows, const uint16_t *k_idx, const int32_t *idx,
+                     int64_t N, int H_kv, int d_idx, int B_k, int k, double scale,
+                     const int64_t *rows, int64_t n_rows, double *lse_out, int n_threads)
+{
+    if (!q_idx_rows || !k_idx || !idx || !rows || !lse_out || N <= 0 || H_kv <= 0 ||
+        d_idx <= 0 || B_k <= 0 || k <= 0 || n_rows < 0)
+        return -1;
+    const int64_t B = (N + B_k - 1) / B_k;
+    for (int64_t t = 0; t < n_rows; ++t) {
+        if (rows[t] < 0 || rows[t] >= N) return -2;
+        for (int r = 0; r < H_kv; ++r)
+            for (int sl = 0; sl < k; ++sl) {
+                const int32_t b = idx[(t * H_kv + r) * k + sl];
+                if (b >= B || b < -1) return -4;
+            }
+    }
+    set_threads(n_threads);
+    int err = 0;
+#pragma omp parallel
+    {
+        const int64_t cap = (int64_t)k * B_k;
+        double *s = (double *)malloc(sizeof(double) * (size_t)cap);
+        if (!s) {
+#pragma omp atomic write
+            err = -3;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int64_t p = 0; p < n_rows * H_kv; ++p) {
+                const int64_t t = p / H_kv;
+                const int r = (int)(p % H_kv);
+                const int64_t i = rows[t];
+                const uint16_t *q = q_idx_rows + p * (int64_t)d_idx;
+                /* the scores of the selected token set */
+                int64_t n = 0;
+                for (int sl = 0; sl < k; ++sl) {
+                    const int32_t b = idx[(t * H_kv + r) * k + sl];
+                    if (b < 0) continue;
+                    const int64_t j0 = (int64_t)b * B_k;
+                    int64_t j1 = j0 + B_k;
+                    if (j1 > N) j1 = N;
+                    for (int64_t j = j0; j < j1 && j <= i; ++j) {
+                        const uint16_t *kr = k_idx + j * (int64_t)d_idx;
+                        double dot = 0.0;
+                        for (int d = 0; d < d_idx; ++d) dot += bf(q[d]) * bf(kr[d]);
+                        s[n++] = dot * scale;
+                    }
+                }
+                if (n == 0) {
+                    lse_out[p] = -INFINITY;
+                    continue;
+                }
+                double m = s[0];
+                for (int64_t u = 1; u < n; ++u)
+                    if (s[u] > m) m = s[u];
+                double sum = 0.0;
+                for (int64_t u = 0; u < n; ++u) sum += exp(s[u] - m);
+                lse_out[p] = m + log(sum);
+            }
+        }
+        free(s);
+    }
+    return err;
+}
+
+/*
  * Eq. 1 [xllm]: dense causal GQA attention, every token j <= i.  Written
  * separately from the sparse path so the special case "every visible block
  * selected" can be checked against it.

@@ -37,6 +37,14 @@ int oracle_sparse_attn(const uint16_t *q_rows, const uint16_t *K, const uint16_t
                        int B_k, int k, double scale, const int64_t *rows,
                        int64_t n_rows, double *o_out, double *lse_out, int n_threads);
 
+/* Eq. 9's Index Branch normaliser over the selected token set of each listed
+ * row: lse_out[t, r] = log sum_{j in selected blocks, j <= rows[t]} exp(S^idx).
+ * q_idx_rows: [n_rows, H_kv, d_idx]; k_idx: [N, d_idx]; idx: [n_rows, H_kv, k];
+ * lse_out: [n_rows, H_kv] (-inf for an empty set). */
+int oracle_index_lse(const uint16_t *q_idx_rows, const uint16_t *k_idx, const int32_t *idx,
+                     int64_t N, int H_kv, int d_idx, int B_k, int k, double scale,
+                     const int64_t *rows, int64_t n_rows, double *lse_out, int n_threads);
+
 /* Eq. 1 dense causal GQA for the listed rows (same layouts, no idx). */
 int oracle_dense_attn(const uint16_t *q_rows, const uint16_t *K, const uint16_t *V,
                       int64_t N, int H_q, int H_kv, int d_h, double scale,

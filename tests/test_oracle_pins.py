@@ -340,3 +340,82 @@ def test_decode_equals_last_prefill_row():
         ref = oracle.forward(full, cfg.B_k, cfg.k, rows=np.array([L]))
         assert dec["idx"][s].tolist() == ref["idx"][0].tolist()
         np.testing.assert_allclose(dec["o"][s], ref["o"][0], atol=0)
+
+
+# ------------------------------------------ KL-loss fusion: LSE_idx (Eq. 9) --
+
+def test_index_lse_worked_example():
+    """Hand-worked Eq. 9 normaliser: q = (1, 0), keys (0,0), (1,0), (2,0),
+    (5,0) in one block of 4, query at i = 2, scale 1: the causal set is
+    tokens 0..2 with scores 0, 1, 2, so LSE_idx = log(1 + e + e^2); token 3
+    (score 5) must not count."""
+    q = inputs.bf16_bits(np.array([[[1, 0]]], dtype=np.float32))
+    k = inputs.bf16_bits(np.array([[0, 0], [1, 0], [2, 0], [5, 0]], dtype=np.float32))
+    got = oracle.index_lse(q, k, np.array([[[0]]], np.int32), B_k=4, rows=np.array([2]),
+                           scale=1.0)
+    assert got[0, 0] == pytest.approx(math.log(1 + math.e + math.e ** 2), rel=1e-15)
+
+
+def test_index_lse_equal_keys_closed_form():
+    """Every selected key equal to one vector c: each token scores s = <q, c> *
+    scale, so LSE_idx = s + log(number of selected tokens j <= i), with -1
+    slots skipped, the query's own block cut at j = i and a ragged last block."""
+    rng = np.random.default_rng(5)
+    N, H_kv, d_idx, B_k, k = 300, 2, 8, 64, 3  # blocks 0..4, the last holds 44 tokens
+    c = rng.standard_normal(d_idx).astype(np.float32)
+    k_idx = np.tile(inputs.bf16_bits(c), (N, 1))
+    q = inputs.bf16_bits(rng.standard_normal((4, H_kv, d_idx)).astype(np.float32))
+    rows = np.array([5, 130, 299, 263])
+    idx = np.array([[[0, -1, -1], [0, -1, -1]],
+                    [[0, 2, -1], [1, 2, -1]],
+                    [[0, 3, 4], [4, -1, -1]],
+                    [[1, 4, -1], [2, 3, 4]]], np.int32)
+    got = oracle.index_lse(q, k_idx, idx, B_k, rows, N=N)
+    cw = k_idx[0].astype(np.uint32) << 16
+    cf = cw.view(np.float32).astype(np.float64)
+    for t, i in enumerate(rows):
+        for r in range(H_kv):
+            qf = (q[t, r].astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+            s = float(qf @ cf) / math.sqrt(d_idx)
+            n = 0
+            for b in idx[t, r]:
+                if b >= 0:
+                    n += max(0, min(b * B_k + B_k, N, i + 1) - b * B_k)
+            assert got[t, r] == pytest.approx(s + math.log(n), abs=1e-12)
+
+
+def test_index_lse_empty_set_and_bounds():
+    """No selected token gives -inf; otherwise max S <= LSE_idx <= max S + log n."""
+    cfg = inputs.CONFIGS["tiny"]
+    inp = inputs.prefill_inputs(cfg)
+    rows = np.array([0, 63, 64, 700, 2047])
+    sel = oracle.index_topk(inp["q_idx"], inp["k_idx"], cfg.B_k, cfg.k, rows=rows)[0]
+    got = oracle.index_lse(inp["q_idx"][rows], inp["k_idx"], sel, cfg.B_k, rows)
+    empty = np.full_like(sel, -1)
+    assert np.isneginf(oracle.index_lse(inp["q_idx"][rows], inp["k_idx"], empty, cfg.B_k,
+                                        rows)).all()
+    qf = (inp["q_idx"][rows].astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    kf = (inp["k_idx"].astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    for t, i in enumerate(rows):
+        for r in range(cfg.H_kv):
+            toks = [j for b in sel[t, r] if b >= 0
+                    for j in range(b * cfg.B_k, min(b * cfg.B_k + cfg.B_k, cfg.N)) if j <= i]
+            s = kf[toks] @ qf[t, r] / math.sqrt(cfg.d_idx)
+            assert s.max() - 1e-12 <= got[t, r] <= s.max() + math.log(len(toks)) + 1e-12
+
+
+def test_index_lse_is_a_one_head_attention_lse():
+    """Eq. 9's index distribution is an attention over the selected tokens with
+    Q = q_idx and K = K_idx, so its normaliser equals the LSE the (separately
+    written) Eq. 8 routine returns for one head of dimension d_idx."""
+    cfg = inputs.CONFIGS["tiny"]
+    inp = inputs.prefill_inputs(cfg)
+    rows = np.array([1, 100, 600, 1500, 2047])
+    sel = oracle.index_topk(inp["q_idx"], inp["k_idx"], cfg.B_k, cfg.k, rows=rows)[0]
+    got = oracle.index_lse(inp["q_idx"][rows], inp["k_idx"], sel, cfg.B_k, rows)
+    kv = inp["k_idx"][:, None, :]
+    for r in range(cfg.H_kv):
+        _, lse = oracle.sparse_attn(inp["q_idx"][rows][:, r:r + 1, :], kv, kv,
+                                    sel[:, r:r + 1, :], cfg.B_k, rows,
+                                    scale=1.0 / math.sqrt(cfg.d_idx))
+        np.testing.assert_allclose(got[:, r], lse[:, 0], rtol=0, atol=1e-12)
