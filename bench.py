@@ -36,37 +36,53 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of a kernel from
-# one ncu capture, per unit of work, with the SHA-256 of the kernel source's
-# code (comments and blank lines removed) at capture time: the figure is
+# one ncu capture, per unit of work, with the SHA-256 of the kernel's
+# definition (comments and blank lines removed) at capture time: the figure is
 # reported only while that code is unchanged.
-# kernel -> (source, sha256, bytes per unit, unit, capture)
+# kernel -> (source, kernel function, sha256, bytes per unit, unit, capture)
 NCU_TRAFFIC = {
-    "attn_phase1": ("sparse_attn.cu",
-                    "fcfe89b57dee736d3a21ffded527321b445b10613e32e5dc48938365bead0a81",
+    "attn_phase1": ("sparse_attn.cu", "attn_phase1_kernel",
+                    "55c33176c70b7f95ebd43f63fb70a4db15fda57ea6de67f1a473fe749360a80f",
                     (3.666177e9 + 4.195406e9) / 32768, "query",
                     "profiles/prefill_32k_ncu_full.md: 32K capture, scaled by queries"),
-    "attn_merge": ("sparse_attn.cu",
-                   "fcfe89b57dee736d3a21ffded527321b445b10613e32e5dc48938365bead0a81",
+    "attn_merge": ("sparse_attn.cu", "attn_merge_kernel",
+                   "beaa021d56c8173edcff10bc3f30370f75c95031da3075c63dc4e1054a981835",
                    (4.243224e9 + 0.269582e9) / 32768, "query",
                    "profiles/prefill_32k_ncu_full.md: 32K capture, scaled by queries"),
 }
 
 
-def ncu_traffic(kernel: str, units: float):
-    """Bytes per launch from NCU_TRAFFIC, or None (no capture, or the kernel
-    source changed since it was taken)."""
+def kernel_code_hash(text: str, name: str) -> str:
+    """SHA-256 of a kernel's definition in a CUDA source: from its name to the
+    brace that closes its body, comments and blank lines removed."""
     import hashlib
 
+    code = re.sub(r"//[^\n]*", "", text)
+    i = code.index(name + "(")
+    j = code.index("{", i)
+    depth, k = 0, j
+    for k in range(j, len(code)):
+        if code[k] == "{":
+            depth += 1
+        elif code[k] == "}":
+            depth -= 1
+            if depth == 0:
+                break
+    body = "\n".join(line.rstrip() for line in code[i:k + 1].splitlines() if line.strip())
+    return hashlib.sha256(body.encode()).hexdigest()
+
+
+def ncu_traffic(kernel: str, units: float):
+    """Bytes per launch from NCU_TRAFFIC, or None (no capture, or the kernel
+    changed since it was taken)."""
     ent = NCU_TRAFFIC.get(kernel)
     if ent is None:
         return None, None
-    src, sha, per_unit, _, where = ent
+    src, fn, sha, per_unit, _, where = ent
     path = os.path.join(ROOT, "block_sparse_gqa_idx_b200", "csrc", src)
     with open(path, encoding="utf-8") as f:
-        code = re.sub(r"//[^\n]*", "", f.read())
-    code = "\n".join(line.rstrip() for line in code.splitlines() if line.strip())
-    if hashlib.sha256(code.encode()).hexdigest() != sha:
-        return None, None
+        if kernel_code_hash(f.read(), fn) != sha:
+            return None, None
     return per_unit * units, where
 
 
@@ -230,13 +246,18 @@ def run_msa(args, cfg, rank, world, local):
     lse = torch.empty((N, H_q), dtype=torch.float32, device=dev)
     dims = msa.dims(N, H_q, H_kv, d_h, d_idx, B_k, kk)
     ws = torch.empty(max(msa.sparse_attn_fwd_workspace_size(dims),
-                         msa.index_topk_workspace_size(dims)), dtype=torch.uint8, device=dev)
+                         msa.index_topk_workspace_size(dims),
+                         msa.index_lse_workspace_size(dims)), dtype=torch.uint8, device=dev)
+    lse_idx = torch.empty((N, H_kv), dtype=torch.float32, device=dev) if args.kl_lse else None
 
     def step(src):
         msa.index_topk(src["q_idx"], src["k_idx"], B_k, kk, idx_out=idx, workspace=ws,
                        stream=stream)
         msa.sparse_attn_fwd(src["q"], src["k"], src["v"], idx, B_k, o=o, lse=lse, workspace=ws,
                             stream=stream)
+        if args.kl_lse:  # the KL-loss fusion's Index Branch normaliser (training forward)
+            msa.index_lse(src["q_idx"], src["k_idx"], idx, B_k, lse_idx=lse_idx, workspace=ws,
+                          stream=stream)
 
     def barrier():
         if world > 1:
@@ -304,6 +325,9 @@ def run_msa(args, cfg, rank, world, local):
                            stream=stream)
             msa.sparse_attn_fwd(bufs[b]["q"], bufs[b]["k"], bufs[b]["v"], ib, B_k, o=ob, lse=lb,
                                 workspace=ws, stream=stream)
+            if args.kl_lse:
+                msa.index_lse(bufs[b]["q_idx"], bufs[b]["k_idx"], ib, B_k, lse_idx=lse_idx,
+                              workspace=ws, stream=stream)
             ev_used[b].record(stream)
             ev_out[b].record(stream)
             with torch.cuda.stream(down):
@@ -383,7 +407,8 @@ def run_msa(args, cfg, rank, world, local):
         "data": "synthetic",
         "config": {"workload": cfg.name, "N": N, "H_q": H_q, "H_kv": H_kv, "d_h": d_h,
                    "d_idx": d_idx, "B_k": B_k, "k": kk, "parallelism": f"replicas x{world}",
-                   "l2": "inputs larger than L2 (Q alone 1.07 GB); no flush"},
+                   "l2": "inputs larger than L2 (Q alone 1.07 GB); no flush",
+                   "kl_lse": bool(args.kl_lse)},
         "tc_frac_eq12": (f_idx + f_main) / (ms * 1e-3) / 1e12 / pk["bf16_tflops"],
         "roofline": roofline,
         "cpu_baseline": cpu,
@@ -510,6 +535,8 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=0, help="0: 256, or 32 at 1M tokens")
     ap.add_argument("--ref-rows", type=int, default=32)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kl-lse", action="store_true",
+                    help="add the KL-loss fusion's LSE_idx to every step (a training forward)")
     args = ap.parse_args()
     world, rank, local = dist_init()
     cfg = workload(args.workload)

@@ -15,7 +15,8 @@ has not been built (``python -m block_sparse_gqa_idx_b200.build``).
 _CAPI = ("index_topk", "sparse_attn_fwd", "forward", "sparse_decode", "device_status",
          "version", "MSAError", "dims", "decode_dims", "index_topk_workspace_size",
          "sparse_attn_fwd_workspace_size", "sparse_decode_workspace_size", "EXPORTS", "LIB_PATH",
-         "profile_enable", "profile_read", "sparse_decode_noalloc", "selftest_bounded_wait")
+         "profile_enable", "profile_read", "sparse_decode_noalloc", "selftest_bounded_wait",
+         "index_lse", "index_lse_workspace_size")
 
 __all__ = list(_CAPI) + ["inputs"]
 

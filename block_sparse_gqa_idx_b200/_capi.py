@@ -49,7 +49,7 @@ EXPORTS = ("msa_index_topk_workspace", "msa_index_topk", "msa_sparse_attn_fwd_wo
            "msa_sparse_attn_fwd", "msa_sparse_decode_workspace", "msa_sparse_decode",
            "msa_get_device_status", "msa_profile_enable", "msa_profile_read",
            "msa_status_string", "msa_version", "msa_sparse_decode_noalloc", "msa_last_error",
-           "msa_selftest_bounded_wait")
+           "msa_selftest_bounded_wait", "msa_index_lse_workspace", "msa_index_lse")
 
 
 def _load() -> ctypes.CDLL:
@@ -77,6 +77,10 @@ def _load() -> ctypes.CDLL:
     lib.msa_get_device_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_int32),
                                           ctypes.POINTER(ctypes.c_int32)]
     lib.msa_get_device_status.restype = I32
+    lib.msa_index_lse_workspace.argtypes = [D]
+    lib.msa_index_lse_workspace.restype = Z
+    lib.msa_index_lse.argtypes = [D, P, P, P, P, P, Z, P]
+    lib.msa_index_lse.restype = I32
     lib.msa_selftest_bounded_wait.argtypes = [P, P]
     lib.msa_selftest_bounded_wait.restype = I32
     lib.msa_profile_enable.argtypes = [ctypes.c_int32]
@@ -177,6 +181,32 @@ def index_topk(q_idx: torch.Tensor, k_idx: torch.Tensor, B_k: int, k: int,
                                                 _ptr(idx_out), _ptr(ws), ws.numel(),
                                                 _stream(stream)))
     return idx_out
+
+
+def index_lse_workspace_size(d: msa_dims) -> int:
+    return int(LIB.msa_index_lse_workspace(ctypes.byref(d)))
+
+
+def index_lse(q_idx: torch.Tensor, k_idx: torch.Tensor, idx: torch.Tensor, B_k: int,
+              lse_idx: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+              stream=None) -> torch.Tensor:
+    """KL-loss fusion: LSE_idx [N,H_kv] fp32 = log of the sum of exp(S^idx)
+    over each row's selected tokens j <= i (Eq. 9's Index Branch normaliser).
+    q_idx [N,H_kv,d_idx] bf16, k_idx [N,d_idx] bf16, idx [N,H_kv,k] int32."""
+    N, H_kv, d_idx = q_idx.shape
+    k = idx.shape[2]
+    _want(q_idx, "q_idx", torch.bfloat16, (N, H_kv, d_idx))
+    _want(k_idx, "k_idx", torch.bfloat16, (N, d_idx))
+    _want(idx, "idx", torch.int32, (N, H_kv, k))
+    if lse_idx is None:
+        lse_idx = torch.empty((N, H_kv), dtype=torch.float32, device=q_idx.device)
+    _want(lse_idx, "lse_idx", torch.float32, (N, H_kv))
+    d = dims(N, H_kv, H_kv, 64, d_idx, B_k, k)
+    ws = _workspace(index_lse_workspace_size(d), q_idx.device, workspace)
+    _raise("msa_index_lse", LIB.msa_index_lse(ctypes.byref(d), _ptr(q_idx), _ptr(k_idx),
+                                              _ptr(idx), _ptr(lse_idx), _ptr(ws), ws.numel(),
+                                              _stream(stream)))
+    return lse_idx
 
 
 def sparse_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, idx: torch.Tensor,

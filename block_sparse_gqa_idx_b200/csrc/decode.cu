@@ -76,15 +76,6 @@ struct DecParams {
 };
 
 // -------------------------------------------------------------------- scan --
-__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
-                                               uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-      "{%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
 // One warp scores one 128-key block at a time (B_k = 128: 8 row tiles of 16
 // keys; B_k = 64: 4).  MMA rows = keys, columns = index-query heads (padded
 // to 8), reduction over d_idx.  The d axis is consumed in a per-thread order

@@ -202,6 +202,45 @@ msa_status msa_index_topk(const msa_dims* d, const void* q_idx, const void* k_id
   return from_cuda(msa::launch_index_topk(a, s));
 }
 
+// ----------------------------------------------- KL-loss fusion: LSE_idx --
+size_t msa_index_lse_workspace(const msa_dims* d) {
+  if (d == nullptr || d->N < 1 || d->H_kv < 1 || d->B_k < 1 || d->k < 1) return 0;
+  return kStatusBytes + msa::idx_lse_workspace_bytes(d->N, d->H_kv, d->B_k, d->k);
+}
+
+msa_status msa_index_lse(const msa_dims* d, const void* q_idx, const void* k_idx,
+                         const int32_t* idx, float* lse_idx, void* ws, size_t ws_bytes,
+                         void* stream) {
+  if (d == nullptr || q_idx == nullptr || k_idx == nullptr || idx == nullptr ||
+      lse_idx == nullptr || ws == nullptr)
+    return MSA_ERR_INVALID_ARG;
+  msa_status st = check_common(d->N, d->H_q, d->H_kv, 64, d->d_idx, d->B_k, d->k, d->attn_scale,
+                               d->idx_scale, false, true);
+  if (st != MSA_OK) return st;
+  if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(idx) || !aligned16(lse_idx) ||
+      !aligned16(ws))
+    return MSA_ERR_INVALID_ARG;
+  if (d->N * d->H_kv * d->k >= (int64_t(1) << 31)) return MSA_ERR_UNSUPPORTED;
+  if (ws_bytes < msa_index_lse_workspace(d)) return MSA_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (from_cuda(cudaMemsetAsync(ws, 0, sizeof(msa::DevStatus), s)) != MSA_OK) return MSA_ERR_CUDA;
+  msa::IdxLseLaunch a;
+  a.q_idx = q_idx;
+  a.k_idx = k_idx;
+  a.idx = idx;
+  a.lse_idx = lse_idx;
+  a.N = d->N;
+  a.H_kv = d->H_kv;
+  a.d_idx = d->d_idx;
+  a.B_k = d->B_k;
+  a.kk = d->k;
+  a.scale = d->idx_scale > 0.0f ? d->idx_scale : 1.0f / sqrtf(static_cast<float>(d->d_idx));
+  a.ws = static_cast<uint8_t*>(ws) + kStatusBytes;
+  a.ws_bytes = ws_bytes - kStatusBytes;
+  a.status = status_of(ws);
+  return from_cuda(msa::launch_idx_lse(a, s));
+}
+
 // ------------------------------------------------------------- Main Branch --
 size_t msa_sparse_attn_fwd_workspace(const msa_dims* d) {
   if (d == nullptr || d->N < 1 || d->H_kv < 1 || d->H_q < 1 || d->B_k < 1 || d->k < 1) return 0;

@@ -95,6 +95,18 @@ MSA_DEVI bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, Dev
   }
 }
 
+// -------------------------------------------------------------- mma.sync --
+// D (16x8, f32) += A (16x16, bf16, row) * B (16x8, bf16, col).  Thread
+// (g = lane/4, t = lane%4) holds A rows g and g+8 at k = 2t, 2t+1 (+8), B
+// column g at k = 2t, 2t+1 (+8), and D rows g, g+8 at columns 2t, 2t+1.
+MSA_DEVI void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
 // ------------------------------------------------------------------- TMA --
 MSA_DEVI void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {
   asm volatile(

@@ -46,6 +46,21 @@ struct AttnLaunch {
 size_t attn_workspace_bytes(int64_t N, int H_q, int H_kv, int d_h, int B_k, int kk);
 cudaError_t launch_sparse_attn(const AttnLaunch& a, cudaStream_t s);
 
+struct IdxLseLaunch {
+  const void* q_idx;
+  const void* k_idx;
+  const int32_t* idx;
+  float* lse_idx;
+  int64_t N;
+  int H_kv, d_idx, B_k, kk;
+  float scale;
+  void* ws;  // device workspace after the status word
+  size_t ws_bytes;
+  DevStatus* status;
+};
+size_t idx_lse_workspace_bytes(int64_t N, int H_kv, int B_k, int kk);
+cudaError_t launch_idx_lse(const IdxLseLaunch& a, cudaStream_t s);
+
 struct DecodeLaunch {
   const void* q;
   const void* q_idx;

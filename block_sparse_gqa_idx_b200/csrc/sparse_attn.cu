@@ -263,6 +263,54 @@ __global__ void __launch_bounds__(1024) inv_scan_kernel(const InvParams p) {
   }
 }
 
+// The inverse index's launch shape: a shared-memory histogram of every key per
+// CTA when it fits (up to 4 CTAs per SM), else the global-atomic kernels.
+cudaError_t inv_setup(int64_t nkeys, int sms, size_t* hist_bytes, int* hist_grid) {
+  *hist_bytes = sizeof(int32_t) * static_cast<size_t>(nkeys);
+  *hist_grid = sms;
+  if (*hist_bytes > kMaxHistBytes) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(inv_index_smem_kernel<false>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(*hist_bytes));
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(inv_index_smem_kernel<true>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(*hist_bytes));
+  if (e != cudaSuccess) return e;
+  const size_t per_sm = 200 * 1024 / (*hist_bytes + 1024);
+  *hist_grid = sms * static_cast<int>(per_sm < 1 ? 1 : (per_sm > 4 ? 4 : per_sm));
+  return cudaSuccess;
+}
+
+// Count -> scan -> scatter of one chunk's inverse index (counts zeroed before).
+void launch_inv_index(const InvParams& ip, size_t hist_bytes, int hist_grid, int sms,
+                      cudaStream_t stream) {
+  const int64_t total = ip.nq * ip.H_kv * ip.kk;
+  if (hist_bytes <= kMaxHistBytes) {
+    prof_begin("inv_count", stream);
+    inv_index_smem_kernel<false><<<hist_grid, 512, hist_bytes, stream>>>(ip);
+    prof_end(stream);
+    prof_begin("inv_scan", stream);
+    inv_scan_kernel<<<1, 1024, 0, stream>>>(ip);
+    prof_end(stream);
+    prof_begin("inv_scatter", stream);
+    inv_index_smem_kernel<true><<<hist_grid, 512, hist_bytes, stream>>>(ip);
+    prof_end(stream);
+  } else {
+    int blocks = static_cast<int>((total + 255) / 256);
+    if (blocks > sms * 16) blocks = sms * 16;
+    prof_begin("inv_count", stream);
+    inv_index_kernel<false><<<blocks, 256, 0, stream>>>(ip);
+    prof_end(stream);
+    prof_begin("inv_scan", stream);
+    inv_scan_kernel<<<1, 1024, 0, stream>>>(ip);
+    prof_end(stream);
+    prof_begin("inv_scatter", stream);
+    inv_index_kernel<true><<<blocks, 256, 0, stream>>>(ip);
+    prof_end(stream);
+  }
+}
+
 // ------------------------------------------------------------------ step 2 --
 struct P1Params {
   int64_t q0;
@@ -892,22 +940,10 @@ cudaError_t launch_typed(const AttnLaunch& a, cudaStream_t stream) {
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const int sms = num_sms();
-  // inverse index: a shared-memory histogram of every key per CTA when it fits
-  const size_t hist_bytes = sizeof(int32_t) * static_cast<size_t>(nkeys);
-  int hist_grid = sms;
-  if (hist_bytes <= kMaxHistBytes) {
-    e = cudaFuncSetAttribute(inv_index_smem_kernel<false>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(hist_bytes));
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(inv_index_smem_kernel<true>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(hist_bytes));
-    if (e != cudaSuccess) return e;
-    // CTAs that fit beside one another on an SM (at most 4 per SM)
-    const size_t per_sm = 200 * 1024 / (hist_bytes + 1024);
-    hist_grid = sms * static_cast<int>(per_sm < 1 ? 1 : (per_sm > 4 ? 4 : per_sm));
-  }
+  size_t hist_bytes = 0;
+  int hist_grid = 0;
+  e = inv_setup(nkeys, sms, &hist_bytes, &hist_grid);
+  if (e != cudaSuccess) return e;
 
   for (int64_t q0 = 0; q0 < a.N; q0 += Nc) {
     const int64_t nq = (a.N - q0) < Nc ? (a.N - q0) : Nc;
@@ -924,30 +960,7 @@ cudaError_t launch_typed(const AttnLaunch& a, cudaStream_t stream) {
     ip.Tq = Tq;
     ip.c = c;
     ip.status = a.status;
-    const int64_t total = nq * a.H_kv * a.kk;
-    if (hist_bytes <= kMaxHistBytes) {
-      prof_begin("inv_count", stream);
-      inv_index_smem_kernel<false><<<hist_grid, 512, hist_bytes, stream>>>(ip);
-      prof_end(stream);
-      prof_begin("inv_scan", stream);
-      inv_scan_kernel<<<1, 1024, 0, stream>>>(ip);
-      prof_end(stream);
-      prof_begin("inv_scatter", stream);
-      inv_index_smem_kernel<true><<<hist_grid, 512, hist_bytes, stream>>>(ip);
-      prof_end(stream);
-    } else {
-      int blocks = static_cast<int>((total + 255) / 256);
-      if (blocks > sms * 16) blocks = sms * 16;
-      prof_begin("inv_count", stream);
-      inv_index_kernel<false><<<blocks, 256, 0, stream>>>(ip);
-      prof_end(stream);
-      prof_begin("inv_scan", stream);
-      inv_scan_kernel<<<1, 1024, 0, stream>>>(ip);
-      prof_end(stream);
-      prof_begin("inv_scatter", stream);
-      inv_index_kernel<true><<<blocks, 256, 0, stream>>>(ip);
-      prof_end(stream);
-    }
+    launch_inv_index(ip, hist_bytes, hist_grid, sms, stream);
 
     P1Params pp;
     pp.q0 = q0;
@@ -1002,7 +1015,213 @@ cudaError_t launch_typed(const AttnLaunch& a, cudaStream_t stream) {
   return cudaSuccess;
 }
 
+// ------------------------------------------ KL-loss fusion: LSE_idx (Eq. 9) --
+// The normaliser of the Index Branch distribution over the selected token
+// set, LSE_idx[i, r] = log sum_{j in selected blocks, j <= i} exp(S^idx), as
+// each selected block's LSE reduced over the Top-k blocks (review, "4.3 Sparse
+// KL Loss Fusion"; notes 5.4).  KV-outer like phase 1: the inverse index lists,
+// per (group, block), the selection slots that chose it; a warp takes 16 of
+// them (one 16-row mma.sync tile: the slots' index queries against the
+// block's K_idx rows, both read straight from L2) and writes each slot's
+// block LSE; a second kernel reduces a row's slots.
+struct IdxLseParams {
+  const __nv_bfloat16* q_idx;  // [N, H_kv, d_idx]
+  const __nv_bfloat16* k_idx;  // [N, d_idx]
+  int64_t q0, N, nkeys;
+  int H_kv, kk, B_k;
+  float scale_log2;
+  ChunkBufs c;
+};
+
+constexpr int kLseTile = 16;  // slots per warp tile (mma.sync M)
+
+template <int D_IDX, int B_K>
+__global__ void __launch_bounds__(256) idx_lse_kernel(const IdxLseParams p) {
+  constexpr int KS = D_IDX / 16;  // k-steps
+  constexpr int NT = B_K / 8;     // 8-key n-tiles of a block
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  const int n_tiles = p.c.n_tiles[0];
+  const int64_t warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  const int64_t w = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  // a contiguous range of tiles per warp: keys are walked forward
+  const int t_beg = static_cast<int>(n_tiles * w / warps);
+  const int t_end = static_cast<int>(n_tiles * (w + 1) / warps);
+  if (t_beg >= t_end) return;
+  const int nb = static_cast<int>(p.nkeys / p.H_kv);
+  const int per_q = p.H_kv * p.kk;
+  int key = find_key(p.c.tile_off, p.nkeys, t_beg);
+  int kend = p.c.tile_off[key + 1];
+  for (int tile = t_beg; tile < t_end; ++tile) {
+    while (kend <= tile) kend = p.c.tile_off[++key + 1];
+    const int r = key / nb, b = key - r * nb;
+    const int koff = p.c.offsets[key];
+    const int first = koff + (tile - p.c.tile_off[key]) * kLseTile;
+    const int len = min(kLseTile, p.c.offsets[key + 1] - first);
+    const bool v_lo = g < len, v_hi = g + 8 < len;
+    const uint32_t s_lo = v_lo ? p.c.entries[first + g] : 0u;
+    const uint32_t s_hi = v_hi ? p.c.entries[first + g + 8] : 0u;
+    const int64_t i_lo = p.q0 + s_lo / per_q, i_hi = p.q0 + s_hi / per_q;
+    // A: the index queries of rows g and g+8 (zero for rows past the tile)
+    const __nv_bfloat16* q_lo = p.q_idx + (i_lo * p.H_kv + r) * D_IDX + 2 * t;
+    const __nv_bfloat16* q_hi = p.q_idx + (i_hi * p.H_kv + r) * D_IDX + 2 * t;
+    uint32_t qa[KS][4];
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+      qa[ks][0] = v_lo ? __ldg(reinterpret_cast<const unsigned int*>(q_lo + ks * 16)) : 0u;
+      qa[ks][1] = v_hi ? __ldg(reinterpret_cast<const unsigned int*>(q_hi + ks * 16)) : 0u;
+      qa[ks][2] = v_lo ? __ldg(reinterpret_cast<const unsigned int*>(q_lo + ks * 16 + 8)) : 0u;
+      qa[ks][3] = v_hi ? __ldg(reinterpret_cast<const unsigned int*>(q_hi + ks * 16 + 8)) : 0u;
+    }
+    // S = Q_idx K_idx^T over the block's keys (keys past N read as zero)
+    const int64_t j0 = static_cast<int64_t>(b) * B_K;
+    float acc[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.0f;
+      const int64_t j = j0 + nt * 8 + g;  // this thread's B column (key)
+      const __nv_bfloat16* kr = p.k_idx + j * D_IDX + 2 * t;
+      const bool in = j < p.N;
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {
+        const uint32_t b0 = in ? __ldg(reinterpret_cast<const unsigned int*>(kr + ks * 16)) : 0u;
+        const uint32_t b1 = in ? __ldg(reinterpret_cast<const unsigned int*>(kr + ks * 16 + 8)) : 0u;
+        mma_bf16_16816(acc[nt], qa[ks], b0, b1);
+      }
+    }
+    // the block's LSE for each row, log2 domain: causal rule j <= i
+    float m_lo = -INFINITY, m_hi = -INFINITY;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int64_t j = j0 + nt * 8 + 2 * t + (e & 1);
+        const bool lo = e < 2;
+        float x = acc[nt][e] * p.scale_log2;
+        if (j > (lo ? i_lo : i_hi)) x = -INFINITY;
+        acc[nt][e] = x;
+        if (lo) m_lo = fmaxf(m_lo, x);
+        else m_hi = fmaxf(m_hi, x);
+      }
+#pragma unroll
+    for (int o = 1; o < 4; o <<= 1) {
+      m_lo = fmaxf(m_lo, __shfl_xor_sync(0xFFFFFFFFu, m_lo, o));
+      m_hi = fmaxf(m_hi, __shfl_xor_sync(0xFFFFFFFFu, m_hi, o));
+    }
+    float l_lo = 0.0f, l_hi = 0.0f;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      l_lo += exp2f(acc[nt][0] - m_lo) + exp2f(acc[nt][1] - m_lo);
+      l_hi += exp2f(acc[nt][2] - m_hi) + exp2f(acc[nt][3] - m_hi);
+    }
+#pragma unroll
+    for (int o = 1; o < 4; o <<= 1) {
+      l_lo += __shfl_xor_sync(0xFFFFFFFFu, l_lo, o);
+      l_hi += __shfl_xor_sync(0xFFFFFFFFu, l_hi, o);
+    }
+    // natural-log LSE of the slot's block (every slot here holds j = i or an
+    // earlier block, so m is finite)
+    constexpr float kLn2 = 0.6931471805599453f;
+    if (t == 0 && v_lo) p.c.part_lse[s_lo] = (m_lo + log2f(l_lo)) * kLn2;
+    if (t == 0 && v_hi) p.c.part_lse[s_hi] = (m_hi + log2f(l_hi)) * kLn2;
+  }
+}
+
+// LSE_idx[i, r]: log-sum-exp of the row's block LSEs over its valid slots.
+__global__ void __launch_bounds__(256) idx_lse_combine_kernel(const int32_t* idx, float* lse_idx,
+                                                              const IdxLseParams p, int64_t nq) {
+  const int64_t u = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (u >= nq * p.H_kv) return;
+  const int64_t il = u / p.H_kv;
+  const int r = static_cast<int>(u - il * p.H_kv);
+  const int64_t i = p.q0 + il;
+  const int64_t b_i = i / p.B_k;
+  const int32_t* sel = idx + (i * p.H_kv + r) * p.kk;
+  const float* part = p.c.part_lse + (il * p.H_kv + r) * p.kk;
+  float m = -INFINITY;
+  for (int s = 0; s < p.kk; ++s) {
+    const int b = sel[s];
+    if (b >= 0 && b <= b_i) m = fmaxf(m, part[s]);
+  }
+  float sum = 0.0f;
+  for (int s = 0; s < p.kk; ++s) {
+    const int b = sel[s];
+    if (b >= 0 && b <= b_i) sum += __expf(part[s] - m);
+  }
+  lse_idx[i * p.H_kv + r] = sum > 0.0f ? m + logf(sum) : -INFINITY;
+}
+
+template <int D_IDX, int B_K>
+cudaError_t launch_idx_lse_typed(const IdxLseLaunch& a, cudaStream_t stream) {
+  const int64_t B = (a.N + B_K - 1) / B_K;
+  const int64_t nkeys = a.H_kv * B;
+  const int64_t Nc = chunk_len(a.N, B_K);
+  size_t need = 0;
+  // the inverse index and one fp32 LSE per slot (a chunk's buffers with G = 1, no partial O)
+  ChunkBufs c = carve(a.ws, Nc, a.H_kv, a.H_kv, 0, a.kk, nkeys, &need);
+  if (need > a.ws_bytes) return cudaErrorInvalidValue;
+  const int sms = num_sms();
+  size_t hist_bytes = 0;
+  int hist_grid = 0;
+  cudaError_t e = inv_setup(nkeys, sms, &hist_bytes, &hist_grid);
+  if (e != cudaSuccess) return e;
+  for (int64_t q0 = 0; q0 < a.N; q0 += Nc) {
+    const int64_t nq = (a.N - q0) < Nc ? (a.N - q0) : Nc;
+    e = cudaMemsetAsync(c.counts, 0, sizeof(int32_t) * nkeys, stream);
+    if (e != cudaSuccess) return e;
+    InvParams ip;
+    ip.idx = a.idx;
+    ip.q0 = q0;
+    ip.nq = nq;
+    ip.H_kv = a.H_kv;
+    ip.B_k = B_K;
+    ip.kk = a.kk;
+    ip.B = B;
+    ip.Tq = kLseTile;
+    ip.c = c;
+    ip.status = a.status;
+    launch_inv_index(ip, hist_bytes, hist_grid, sms, stream);
+    IdxLseParams lp;
+    lp.q_idx = static_cast<const __nv_bfloat16*>(a.q_idx);
+    lp.k_idx = static_cast<const __nv_bfloat16*>(a.k_idx);
+    lp.q0 = q0;
+    lp.N = a.N;
+    lp.nkeys = nkeys;
+    lp.H_kv = a.H_kv;
+    lp.kk = a.kk;
+    lp.B_k = B_K;
+    lp.scale_log2 = a.scale * 1.4426950408889634f;
+    lp.c = c;
+    prof_begin("idx_lse", stream);
+    idx_lse_kernel<D_IDX, B_K><<<sms * 8, 256, 0, stream>>>(lp);
+    prof_end(stream);
+    prof_begin("idx_lse_combine", stream);
+    idx_lse_combine_kernel<<<static_cast<unsigned>((nq * a.H_kv + 255) / 256), 256, 0, stream>>>(
+        a.idx, a.lse_idx, lp, nq);
+    prof_end(stream);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
 }  // namespace
+
+size_t idx_lse_workspace_bytes(int64_t N, int H_kv, int B_k, int kk) {
+  const int64_t B = (N + B_k - 1) / B_k;
+  size_t total = 0;
+  carve(nullptr, chunk_len(N, B_k), H_kv, H_kv, 0, kk, H_kv * B, &total);
+  return total;
+}
+
+cudaError_t launch_idx_lse(const IdxLseLaunch& a, cudaStream_t s) {
+  if (a.d_idx == 64 && a.B_k == 128) return launch_idx_lse_typed<64, 128>(a, s);
+  if (a.d_idx == 64 && a.B_k == 64) return launch_idx_lse_typed<64, 64>(a, s);
+  if (a.d_idx == 128 && a.B_k == 128) return launch_idx_lse_typed<128, 128>(a, s);
+  if (a.d_idx == 128 && a.B_k == 64) return launch_idx_lse_typed<128, 64>(a, s);
+  if (a.d_idx == 32 && a.B_k == 128) return launch_idx_lse_typed<32, 128>(a, s);
+  if (a.d_idx == 32 && a.B_k == 64) return launch_idx_lse_typed<32, 64>(a, s);
+  return cudaErrorInvalidValue;
+}
 
 size_t attn_workspace_bytes(int64_t N, int H_q, int H_kv, int d_h, int B_k, int kk) {
   const int64_t B = (N + B_k - 1) / B_k;

@@ -165,6 +165,35 @@ MSA_API msa_status msa_sparse_decode_noalloc(const msa_decode_dims* dims, const 
                                              int32_t* seq_len, void* o, int32_t* idx_out,
                                              void* stream);
 
+/* ---------------------------------------------------------------------------
+ * KL-loss fusion: the Index Branch normaliser (training forward).
+ * Source: xllm-io review "MiniMax Sparse Attention (MSA)", section 三 "KL
+ * Alignment Loss" (Eq. 9-10) and section 五 "4.3 Sparse KL Loss Fusion";
+ * Chlience notes 5.4.  The KL loss compares the Main Branch distribution
+ * (its normalisers are the per-head LSE msa_sparse_attn_fwd writes) with
+ * the Index Branch distribution over the same selected token set,
+ *   P^idx[i,r,j] = exp(S^idx[i,r,j] - LSE_idx[i,r]),
+ *   LSE_idx[i,r] = log sum_{j in selected blocks of (i,r), j <= i} exp(S^idx[i,r,j]),
+ * S^idx as in msa_index_topk (Eq. 6, scale idx_scale, 0 -> 1/sqrt(d_idx)).
+ * Each selected block's LSE is computed and reduced over the row's Top-k
+ * blocks; no score matrix is written.
+ *   q_idx   [N, H_kv, d_idx] bf16      k_idx [N, d_idx] bf16
+ *   idx     [N, H_kv, k] int32         the selection (e.g. msa_index_topk's);
+ *                                      -1 and blocks after the query's own
+ *                                      are skipped
+ *   lse_idx [N, H_kv] fp32, natural log; -inf for a row with no token.
+ * Uses dims->N, H_q, H_kv, d_idx, B_k, k, idx_scale.  All pointers 16-byte
+ * aligned device memory owned by the caller; workspace of at least
+ * msa_index_lse_workspace(dims) bytes.  Errors: as msa_index_topk
+ * (MSA_ERR_UNSUPPORTED for d_idx outside {32,64,128}, B_k outside {64,128},
+ * k > 32); a block index outside [-1, B) records MSA_DEV_BAD_INDEX.
+ * Asynchronous on `stream`.
+ * ------------------------------------------------------------------------- */
+MSA_API size_t msa_index_lse_workspace(const msa_dims* dims);
+MSA_API msa_status msa_index_lse(const msa_dims* dims, const void* q_idx, const void* k_idx,
+                                 const int32_t* idx, float* lse_idx, void* workspace,
+                                 size_t workspace_bytes, void* stream);
+
 /* Device status codes written into the workspace's status word. */
 #define MSA_DEV_OK 0
 #define MSA_DEV_TIMEOUT 1    /* a bounded on-device wait gave up; outputs invalid */

@@ -102,3 +102,13 @@ def test_selftest_rejects_bad_workspace_on_host(capi):
 def test_status_strings(capi):
     texts = {capi.LIB.msa_status_string(i).decode() for i in range(6)}
     assert len(texts) == 6
+
+
+def test_index_lse_rejects_on_host(capi):
+    d = capi.dims(4096, 8, 4, 128, 64, 128, 16)
+    ws_ok = capi.LIB.msa_index_lse_workspace(ctypes.byref(d))
+    assert ws_ok > 4096 * 4 * 16 * 4  # one fp32 LSE per (query, group, slot)
+    assert capi.LIB.msa_index_lse(ctypes.byref(d), None, FAKE, FAKE, FAKE, FAKE, ws_ok, None) == 1
+    assert capi.LIB.msa_index_lse(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, 8, None) == 3
+    d.d_idx = 48
+    assert capi.LIB.msa_index_lse(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 40, None) == 2

@@ -234,6 +234,55 @@ def test_bounded_wait_times_out_reports_and_context_survives(msa):
     _check_index(msa, cfg, rows=np.arange(0, cfg.N, 97))
 
 
+def _check_index_lse(msa, cfg, dev, inp, idx_dev, rows, what):
+    """LSE_idx (Eq. 9's Index Branch normaliser) on the GPU against the oracle
+    for the listed rows, from the same selection."""
+    lse_idx = msa.index_lse(dev["q_idx"], dev["k_idx"], idx_dev, cfg.B_k)
+    torch.cuda.synchronize()
+    rows = np.asarray(rows)
+    sel = idx_dev.cpu().numpy()[rows]
+    ref = oracle.index_lse(inp["q_idx"][rows], inp["k_idx"], sel, cfg.B_k, rows, N=cfg.N)
+    got = lse_idx.cpu().numpy().astype(np.float64)[rows]
+    assert (np.isneginf(got) == np.isneginf(ref)).all(), what
+    fin = np.isfinite(ref)
+    np.testing.assert_allclose(got[fin], ref[fin], rtol=1e-5, atol=1e-4, err_msg=what)
+
+
+def test_index_lse_tiny_all_rows(msa):
+    cfg = inputs.CONFIGS["tiny"]
+    inp = prefill_inputs_cached(cfg)
+    dev = dev_inputs(inp)
+    idx = msa.index_topk(dev["q_idx"], dev["k_idx"], cfg.B_k, cfg.k)
+    _check_index_lse(msa, cfg, dev, inp, idx, np.arange(cfg.N), "tiny")
+
+
+def test_index_lse_32k_recipe_and_128k_sampled(msa):
+    for cfg, n_rand in ((_cfg("32k", N=8192), 200), (inputs.CONFIGS["128k"], 96)):
+        inp = prefill_inputs_cached(cfg)
+        dev = dev_inputs(inp)
+        idx = msa.index_topk(dev["q_idx"], dev["k_idx"], cfg.B_k, cfg.k)
+        rng = np.random.default_rng(7)
+        rows = np.unique(np.concatenate([rng.integers(0, cfg.N, n_rand),
+                                         [0, 1, 127, 128, cfg.N - 1]]))
+        _check_index_lse(msa, cfg, dev, inp, idx, rows, cfg.name)
+
+
+@pytest.mark.parametrize("N,H_kv,d_idx,B_k,k", [
+    (1000, 2, 32, 64, 5),     # ragged tail, B_k = 64
+    (3001, 4, 128, 128, 32),  # largest k, d_idx = 128
+    (300, 4, 64, 128, 8),     # k above the visible blocks: -1 padding everywhere
+])
+def test_index_lse_edge_shapes_and_empty_rows(msa, N, H_kv, d_idx, B_k, k):
+    cfg = inputs.MSAConfig("lse", N=N, H_q=H_kv * 2, H_kv=H_kv, d_h=64, d_idx=d_idx, B_k=B_k,
+                           k=k, structure="iid", seed_index=43)
+    inp = prefill_inputs_cached(cfg)
+    dev = dev_inputs(inp)
+    idx = msa.index_topk(dev["q_idx"], dev["k_idx"], cfg.B_k, cfg.k)
+    idx[5, 0, :] = -1       # a row with no token: -inf
+    idx[N - 1, H_kv - 1, 1:] = -1
+    _check_index_lse(msa, cfg, dev, inp, idx, np.arange(N), "edge")
+
+
 def test_device_status_reports_bad_index(msa):
     cfg = inputs.MSAConfig("bad", N=256, H_q=16, H_kv=2, d_h=64, d_idx=64, B_k=64, k=2,
                            seed_index=37)
