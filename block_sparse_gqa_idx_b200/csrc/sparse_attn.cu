@@ -1035,11 +1035,30 @@ struct IdxLseParams {
 
 constexpr int kLseTile = 16;  // slots per warp tile (mma.sync M)
 
+// Shared-memory row of one K_idx key in idx_lse_kernel: d_idx bf16 plus 16
+// bytes, so the 8 rows an ldmatrix reads fall in distinct bank groups.
+template <int D_IDX>
+__host__ __device__ constexpr int lse_row_bytes() { return D_IDX * 2 + 16; }
+constexpr int kLseWarps = 4;  // warps per CTA of idx_lse_kernel
+
+__device__ __forceinline__ void ldsm4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                      uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
 template <int D_IDX, int B_K>
-__global__ void __launch_bounds__(256) idx_lse_kernel(const IdxLseParams p) {
+__global__ void __launch_bounds__(32 * kLseWarps) idx_lse_kernel(const IdxLseParams p) {
   constexpr int KS = D_IDX / 16;  // k-steps
   constexpr int NT = B_K / 8;     // 8-key n-tiles of a block
+  constexpr int ROW = lse_row_bytes<D_IDX>();
+  extern __shared__ uint8_t lse_smem[];
   const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  // this warp's copy of the current block's K_idx rows (one key's run of tiles)
+  uint8_t* sk = lse_smem + (threadIdx.x >> 5) * B_K * ROW;
+  const uint32_t sk_u32 = smem_u32(sk);
+  int staged = -1;
   const int n_tiles = p.c.n_tiles[0];
   const int64_t warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
   const int64_t w = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
@@ -1054,6 +1073,21 @@ __global__ void __launch_bounds__(256) idx_lse_kernel(const IdxLseParams p) {
   for (int tile = t_beg; tile < t_end; ++tile) {
     while (kend <= tile) kend = p.c.tile_off[++key + 1];
     const int r = key / nb, b = key - r * nb;
+    if (b != staged) {
+      // the block's K_idx rows into shared memory, 16 bytes per lane and
+      // step (rows past N as zeros)
+      constexpr int CPR = D_IDX / 8;  // 16-byte pieces per row
+      __syncwarp();
+      for (int c = lane; c < B_K * CPR; c += 32) {
+        const int row = c / CPR, col = c - row * CPR;
+        const int64_t j = static_cast<int64_t>(b) * B_K + row;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (j < p.N) v = __ldg(reinterpret_cast<const uint4*>(p.k_idx + j * D_IDX) + col);
+        *reinterpret_cast<uint4*>(sk + row * ROW + col * 16) = v;
+      }
+      __syncwarp();
+      staged = b;
+    }
     const int koff = p.c.offsets[key];
     const int first = koff + (tile - p.c.tile_off[key]) * kLseTile;
     const int len = min(kLseTile, p.c.offsets[key + 1] - first);
@@ -1072,21 +1106,26 @@ __global__ void __launch_bounds__(256) idx_lse_kernel(const IdxLseParams p) {
       qa[ks][2] = v_lo ? __ldg(reinterpret_cast<const unsigned int*>(q_lo + ks * 16 + 8)) : 0u;
       qa[ks][3] = v_hi ? __ldg(reinterpret_cast<const unsigned int*>(q_hi + ks * 16 + 8)) : 0u;
     }
-    // S = Q_idx K_idx^T over the block's keys (keys past N read as zero)
+    // S = Q_idx K_idx^T over the block's keys, B fragments by ldmatrix: the
+    // four 8x8 matrices are (keys n, d lo), (keys n, d hi), (keys n+8, d lo),
+    // (keys n+8, d hi)
     const int64_t j0 = static_cast<int64_t>(b) * B_K;
     float acc[NT][4];
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.0f;
-      const int64_t j = j0 + nt * 8 + g;  // this thread's B column (key)
-      const __nv_bfloat16* kr = p.k_idx + j * D_IDX + 2 * t;
-      const bool in = j < p.N;
+    for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.0f;
+    {
+      const int mi = lane >> 3, rr = lane & 7;
 #pragma unroll
-      for (int ks = 0; ks < KS; ++ks) {
-        const uint32_t b0 = in ? __ldg(reinterpret_cast<const unsigned int*>(kr + ks * 16)) : 0u;
-        const uint32_t b1 = in ? __ldg(reinterpret_cast<const unsigned int*>(kr + ks * 16 + 8)) : 0u;
-        mma_bf16_16816(acc[nt], qa[ks], b0, b1);
-      }
+      for (int n2 = 0; n2 < NT / 2; ++n2)
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+          const int key_row = n2 * 16 + (mi >> 1) * 8 + rr;
+          const int d = ks * 16 + (mi & 1) * 8;
+          uint32_t b0, b1, b2, b3;
+          ldsm4(sk_u32 + key_row * ROW + d * 2, b0, b1, b2, b3);
+          mma_bf16_16816(acc[2 * n2], qa[ks], b0, b1);
+          mma_bf16_16816(acc[2 * n2 + 1], qa[ks], b2, b3);
+        }
     }
     // the block's LSE for each row, log2 domain: causal rule j <= i
     float m_lo = -INFINITY, m_hi = -INFINITY;
@@ -1164,6 +1203,11 @@ cudaError_t launch_idx_lse_typed(const IdxLseLaunch& a, cudaStream_t stream) {
   int hist_grid = 0;
   cudaError_t e = inv_setup(nkeys, sms, &hist_bytes, &hist_grid);
   if (e != cudaSuccess) return e;
+  const size_t lse_smem = static_cast<size_t>(kLseWarps) * B_K * lse_row_bytes<D_IDX>();
+  e = cudaFuncSetAttribute(idx_lse_kernel<D_IDX, B_K>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(lse_smem));
+  if (e != cudaSuccess) return e;
+  const int lse_ctas = static_cast<int>(200 * 1024 / (lse_smem + 1024));  // CTAs per SM
   for (int64_t q0 = 0; q0 < a.N; q0 += Nc) {
     const int64_t nq = (a.N - q0) < Nc ? (a.N - q0) : Nc;
     e = cudaMemsetAsync(c.counts, 0, sizeof(int32_t) * nkeys, stream);
@@ -1192,7 +1236,7 @@ cudaError_t launch_idx_lse_typed(const IdxLseLaunch& a, cudaStream_t stream) {
     lp.scale_log2 = a.scale * 1.4426950408889634f;
     lp.c = c;
     prof_begin("idx_lse", stream);
-    idx_lse_kernel<D_IDX, B_K><<<sms * 8, 256, 0, stream>>>(lp);
+    idx_lse_kernel<D_IDX, B_K><<<sms * lse_ctas, 32 * kLseWarps, lse_smem, stream>>>(lp);
     prof_end(stream);
     prof_begin("idx_lse_combine", stream);
     idx_lse_combine_kernel<<<static_cast<unsigned>((nq * a.H_kv + 255) / 256), 256, 0, stream>>>(
