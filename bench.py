@@ -208,7 +208,9 @@ def run_reference(args, cfg, rank, world):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * statistics.mean(times), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": cfg.name, "N": cfg.N, "rows_per_step": n_rows},
+        "config": {"workload": cfg.name, "N": cfg.N, "H_q": cfg.H_q, "H_kv": cfg.H_kv,
+                   "d_h": cfg.d_h, "d_idx": cfg.d_idx, "B_k": cfg.B_k, "k": cfg.k,
+                   "parallelism": f"replicas x{world}", "rows_per_step": n_rows},
         "cpu_baseline": {"value": tps, "unit": "tokens/s", "cores": oracle.max_threads(),
                          "kind": "oracle",
                          "sample": f"{n_rows} uniformly drawn query rows per step of the {cfg.name} "
