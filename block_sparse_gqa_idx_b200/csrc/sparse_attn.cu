@@ -1207,7 +1207,8 @@ cudaError_t launch_idx_lse_typed(const IdxLseLaunch& a, cudaStream_t stream) {
   e = cudaFuncSetAttribute(idx_lse_kernel<D_IDX, B_K>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(lse_smem));
   if (e != cudaSuccess) return e;
-  const int lse_ctas = static_cast<int>(200 * 1024 / (lse_smem + 1024));  // CTAs per SM
+  // CTAs per SM: the SM's 228 KB of shared memory, 1 KB of it reserved per CTA
+  const int lse_ctas = static_cast<int>(228 * 1024 / (lse_smem + 1024));
   for (int64_t q0 = 0; q0 < a.N; q0 += Nc) {
     const int64_t nq = (a.N - q0) < Nc ? (a.N - q0) : Nc;
     e = cudaMemsetAsync(c.counts, 0, sizeof(int32_t) * nkeys, stream);
