@@ -73,6 +73,28 @@ def test_index_topk_edge_shapes(msa, N, H_kv, d_idx, B_k, k):
     _check_index(msa, cfg)
 
 
+def test_index_topk_exact_ties_go_to_lower_blocks(msa):
+    """Every block's K_idx rows identical: all block maxima tie exactly (the
+    same bf16 products in the same order), so Eq. 7's ties-to-the-lower-index
+    rule fixes each row's selection bit-exactly: its own block and blocks
+    0 .. k-2 (or every visible block when there are fewer)."""
+    N, H_kv, d_idx, B_k, k = 4096, 4, 64, 128, 6
+    rng = np.random.default_rng(11)
+    q_idx = inputs.bf16_bits(rng.standard_normal((N, H_kv, d_idx), dtype=np.float32))
+    block = inputs.bf16_bits(rng.standard_normal((B_k, d_idx), dtype=np.float32))
+    k_idx = np.tile(block, (N // B_k, 1))
+    idx = msa.index_topk(to_dev(q_idx), to_dev(k_idx), B_k, k)
+    torch.cuda.synchronize()
+    got = idx.cpu().numpy()
+    for i in range(N):
+        b_i = i // B_k
+        want = sorted(set(range(min(k - 1, b_i))) | {b_i})
+        want = want + [-1] * (k - len(want))
+        assert (got[i] == np.array(want)[None, :]).all(), (i, got[i].tolist(), want)
+    ref = oracle.index_topk(q_idx, k_idx, B_k, k, rows=np.arange(0, N, 37))[0]
+    assert (ref == got[np.arange(0, N, 37)]).all()
+
+
 def test_index_topk_128k_sampled(msa):
     """Full 128K workload (same launch as the benchmark); sampled rows checked."""
     cfg = inputs.CONFIGS["128k"]
