@@ -465,11 +465,19 @@ def run_decode(args, cfg, rank, world, local):
                           caches["k_cache"], caches["v_cache"], caches["k_idx_cache"], seq_len,
                           B_k, kk, o=o, idx_out=idx, workspace=ws, stream=stream)
 
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.barrier()
+
     for j in range(args.warmup):
         step(j)
     torch.cuda.synchronize()
     L_before = seq_len.clone()
     clocks = Clocks(local)
+    barrier()
+    torch.cuda.synchronize()
     clocks.start()
     msa.profile_enable(True)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -478,10 +486,12 @@ def run_decode(args, cfg, rank, world, local):
         step(j)
     e1.record(stream)
     torch.cuda.synchronize()
+    barrier()
     msa.profile_enable(False)
     clk = clocks.stop()
     prof = msa.profile_read()
-    ms = e0.elapsed_time(e1) / args.steps
+    # the slowest replica's step time; every rank's S sequences got a token
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dev, world)
     code, where = msa.device_status(ws)
     if code != 0:
         raise RuntimeError(f"device status {code} at {where}")
@@ -508,7 +518,7 @@ def run_decode(args, cfg, rank, world, local):
     scan_ms = prof.get("dec_scan", (1, 0.0))[1] / args.steps
     scan_bytes = S * L * d_idx * 2
     line = {
-        "metric": METRIC, "value": 1e3 * ms / S,
+        "metric": METRIC, "value": 1e3 * ms / (S * world),
         "unit": "us/token", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms, "us_per_step": 1e3 * ms, "higher_is_better": False,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
@@ -544,12 +554,12 @@ def main():
     cfg = workload(args.workload)
     if args.cpu_rows == 0:
         args.cpu_rows = 32 if getattr(cfg, "N", 0) >= (1 << 20) else 256
-    if args.workload.startswith("decode"):
-        if args.impl == "reference":
-            print(json.dumps({"impl": "reference", "unavailable": "decode reference arm not provided"}))
-            return 0
-        return run_decode(args, cfg, rank, world, local)
     if args.impl == "reference":
+        if args.workload.startswith("decode"):
+            if rank == 0:
+                print(json.dumps({"impl": "reference",
+                                  "unavailable": "decode reference arm not provided"}))
+            return 0
         return run_reference(args, cfg, rank, world)
     if world > 1:
         import datetime
@@ -560,6 +570,8 @@ def main():
         torch.cuda.set_device(local)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     try:
+        if args.workload.startswith("decode"):
+            return run_decode(args, cfg, rank, world, local)
         return run_msa(args, cfg, rank, world, local)
     finally:
         if world > 1:
