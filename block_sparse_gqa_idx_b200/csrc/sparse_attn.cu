@@ -2,10 +2,11 @@
 // KV-outer block-sparse attention on tcgen05, in three steps per query chunk:
 //
 //   1. inverse index: for every (group r, block b) the list of selection slots
-//      (query i, slot s) that chose b -- count, exclusive scan, scatter.  The
-//      scan also cuts each list into tiles of Tq queries (Tq * rows-per-query
-//      = 128 MMA rows), so hot blocks are split over many CTAs with every
-//      output slot fixed in advance: no atomics on the outputs.
+//      (query i, slot s) that chose b -- count, exclusive scan, scatter, each
+//      CTA counting its range of slots in a shared-memory histogram of the
+//      keys.  The scan also cuts each list into tiles of Tq queries (Tq *
+//      rows-per-query = 128 MMA rows), so hot blocks are split over many CTAs
+//      with every output slot fixed in advance: no atomics on the outputs.
 //   2. phase 1: one tile = one KV block (K_b, V_b by TMA) and the gathered
 //      query rows that selected it (one TMA box per query: its group's heads).
 //      S = Q K_b^T (UMMA, fp32 in TMEM) -> causal mask (only rows whose own
@@ -14,6 +15,11 @@
 //      partial with its natural-log LSE into the row's slot.
 //   3. merge: per (query, head), LSE-weighted sum of its partials (split-K
 //      softmax normalisation), bf16 output + fp32 LSE.
+//
+// The file also holds the KL-loss fusion's Index Branch normaliser LSE_idx
+// (review "4.3 Sparse KL Loss Fusion"): the same inverse index in 16-slot
+// tiles, each selected block's index-score LSE per slot (mma.sync), and a
+// log-sum-exp over a row's slots.
 //
 // Source: xllm-io paper review, "核心公式" Eq. 8 and "4.2 Sparse Attention
 // Kernel" (KV-outer with query gather, two-phase forward: partial outputs
