@@ -644,37 +644,29 @@ cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t stream) {
 // scratch from this fixed array instead; every GPU that runs the library's
 // kernels holds it until the process exits.
 // ------------------------------------------------------------------------
-#include <mutex>
-
 #include "../../include/msa.h"
+
+// Dims-only validation of the decode entry points (msa_capi.cu).
+msa_status msa_check_decode_dims(const msa_decode_dims* d);
 
 static __device__ __align__(256) uint8_t g_decode_scratch[MSA_DECODE_NOALLOC_SCRATCH_BYTES];
 
 namespace {
-constexpr int kMaxDevices = 64;
-std::mutex g_scratch_mu;
-void* g_scratch_ptr[kMaxDevices] = {};
-
-// Device address of g_decode_scratch on the current device, looked up once
-// per device with that device current.  (In host code the array's name is
-// only a host-side stand-in, never a usable device pointer.)
+// Device address of g_decode_scratch in the current device's context.  In
+// host code the array's name is only a host-side stand-in, never a usable
+// device pointer, so the address is looked up with the device current.  It
+// is looked up on every call (cheap once the module is loaded) rather than
+// cached per device ordinal: after a cudaDeviceReset, or under another
+// context on the same ordinal, the module is loaded anew and an address kept
+// from before would point at freed memory.
 void* decode_scratch(msa_status* st) {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || p == nullptr) {
     *st = MSA_ERR_CUDA;
     return nullptr;
   }
-  std::lock_guard<std::mutex> lk(g_scratch_mu);
-  if (g_scratch_ptr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || p == nullptr) {
-      *st = MSA_ERR_CUDA;
-      return nullptr;
-    }
-    g_scratch_ptr[dev] = p;
-  }
   *st = MSA_OK;
-  return g_scratch_ptr[dev];
+  return p;
 }
 }  // namespace
 
@@ -684,7 +676,9 @@ extern "C" msa_status msa_sparse_decode_noalloc(const msa_decode_dims* d, const 
                                                 void* k_cache, void* v_cache, void* k_idx_cache,
                                                 int32_t* seq_len, void* o, int32_t* idx_out,
                                                 void* stream) {
-  if (d == nullptr) return MSA_ERR_INVALID_ARG;
+  // the dims are checked before the scratch size is computed from them
+  const msa_status dims_ok = msa_check_decode_dims(d);
+  if (dims_ok != MSA_OK) return dims_ok;
   const size_t need = msa_sparse_decode_workspace(d);
   if (need == 0) return MSA_ERR_INVALID_ARG;
   if (need > MSA_DECODE_NOALLOC_SCRATCH_BYTES) return MSA_ERR_WORKSPACE_TOO_SMALL;

@@ -121,6 +121,45 @@ msa_status check_common(int64_t N, int H_q, int H_kv, int d_h, int d_idx, int B_
   return MSA_OK;
 }
 
+// Size checks of msa_sparse_attn_fwd that depend on the dims alone.
+msa_status check_attn_dims(const msa_dims* d) {
+  msa_status st = check_common(d->N, d->H_q, d->H_kv, d->d_h, 64, d->B_k, d->k, d->attn_scale,
+                               d->idx_scale, true, false);
+  if (st != MSA_OK) return st;
+  const int G = d->H_q / d->H_kv;
+  if (G > 32 || 32 % G != 0) return MSA_ERR_UNSUPPORTED;     // a query's rows in one warp
+  if (G < 8 && d->H_q % 8 != 0) return MSA_ERR_UNSUPPORTED;  // 8-head TMA boxes
+  if (d->N * d->H_q >= (int64_t(1) << 31) - 256 || d->N * d->H_kv * d->k >= (int64_t(1) << 31))
+    return MSA_ERR_UNSUPPORTED;
+  return MSA_OK;
+}
+
+// Size checks of msa_index_lse that depend on the dims alone.
+msa_status check_index_lse_dims(const msa_dims* d) {
+  msa_status st = check_common(d->N, d->H_q, d->H_kv, 64, d->d_idx, d->B_k, d->k, d->attn_scale,
+                               d->idx_scale, false, true);
+  if (st != MSA_OK) return st;
+  if (d->N * d->H_kv * d->k >= (int64_t(1) << 31)) return MSA_ERR_UNSUPPORTED;
+  return MSA_OK;
+}
+
+}  // namespace
+
+// Size checks of msa_sparse_decode (and of its no-workspace variant in
+// decode.cu) that depend on the dims alone.
+msa_status msa_check_decode_dims(const msa_decode_dims* d) {
+  if (d == nullptr || d->S < 1 || d->L_max < 1) return MSA_ERR_INVALID_ARG;
+  msa_status st = check_common(d->L_max, d->H_q, d->H_kv, d->d_h, d->d_idx, d->B_k, d->k,
+                               d->attn_scale, d->idx_scale, true, true);
+  if (st != MSA_OK) return st;
+  const int G = d->H_q / d->H_kv;
+  if (G > 16 || d->H_kv > 8) return MSA_ERR_UNSUPPORTED;
+  if (d->L_max >= (int64_t(1) << 31)) return MSA_ERR_UNSUPPORTED;
+  return MSA_OK;
+}
+
+namespace {
+
 thread_local cudaError_t g_last_cuda_error = cudaSuccess;
 
 msa_status from_cuda(cudaError_t e) {
@@ -204,7 +243,7 @@ msa_status msa_index_topk(const msa_dims* d, const void* q_idx, const void* k_id
 
 // ----------------------------------------------- KL-loss fusion: LSE_idx --
 size_t msa_index_lse_workspace(const msa_dims* d) {
-  if (d == nullptr || d->N < 1 || d->H_kv < 1 || d->B_k < 1 || d->k < 1) return 0;
+  if (d == nullptr || check_index_lse_dims(d) != MSA_OK) return 0;
   return kStatusBytes + msa::idx_lse_workspace_bytes(d->N, d->H_kv, d->B_k, d->k);
 }
 
@@ -214,13 +253,11 @@ msa_status msa_index_lse(const msa_dims* d, const void* q_idx, const void* k_idx
   if (d == nullptr || q_idx == nullptr || k_idx == nullptr || idx == nullptr ||
       lse_idx == nullptr || ws == nullptr)
     return MSA_ERR_INVALID_ARG;
-  msa_status st = check_common(d->N, d->H_q, d->H_kv, 64, d->d_idx, d->B_k, d->k, d->attn_scale,
-                               d->idx_scale, false, true);
+  msa_status st = check_index_lse_dims(d);
   if (st != MSA_OK) return st;
   if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(idx) || !aligned16(lse_idx) ||
       !aligned16(ws))
     return MSA_ERR_INVALID_ARG;
-  if (d->N * d->H_kv * d->k >= (int64_t(1) << 31)) return MSA_ERR_UNSUPPORTED;
   if (ws_bytes < msa_index_lse_workspace(d)) return MSA_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (from_cuda(cudaMemsetAsync(ws, 0, sizeof(msa::DevStatus), s)) != MSA_OK) return MSA_ERR_CUDA;
@@ -243,7 +280,7 @@ msa_status msa_index_lse(const msa_dims* d, const void* q_idx, const void* k_idx
 
 // ------------------------------------------------------------- Main Branch --
 size_t msa_sparse_attn_fwd_workspace(const msa_dims* d) {
-  if (d == nullptr || d->N < 1 || d->H_kv < 1 || d->H_q < 1 || d->B_k < 1 || d->k < 1) return 0;
+  if (d == nullptr || check_attn_dims(d) != MSA_OK) return 0;
   return kStatusBytes + msa::attn_workspace_bytes(d->N, d->H_q, d->H_kv, d->d_h, d->B_k, d->k);
 }
 
@@ -253,17 +290,11 @@ msa_status msa_sparse_attn_fwd(const msa_dims* d, const void* q, const void* k, 
   if (d == nullptr || q == nullptr || k == nullptr || v == nullptr || idx == nullptr ||
       o == nullptr || ws == nullptr)
     return MSA_ERR_INVALID_ARG;
-  msa_status st = check_common(d->N, d->H_q, d->H_kv, d->d_h, 64, d->B_k, d->k, d->attn_scale,
-                               d->idx_scale, true, false);
+  msa_status st = check_attn_dims(d);
   if (st != MSA_OK) return st;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(idx) || !aligned16(o) ||
       !aligned16(ws) || (lse != nullptr && !aligned16(lse)))
     return MSA_ERR_INVALID_ARG;
-  const int G = d->H_q / d->H_kv;
-  if (G > 32 || 32 % G != 0) return MSA_ERR_UNSUPPORTED;     // a query's rows in one warp
-  if (G < 8 && d->H_q % 8 != 0) return MSA_ERR_UNSUPPORTED;  // 8-head TMA boxes
-  if (d->N * d->H_q >= (int64_t(1) << 31) - 256 || d->N * d->H_kv * d->k >= (int64_t(1) << 31))
-    return MSA_ERR_UNSUPPORTED;
   if (ws_bytes < msa_sparse_attn_fwd_workspace(d)) return MSA_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (from_cuda(cudaMemsetAsync(ws, 0, sizeof(msa::DevStatus), s)) != MSA_OK) return MSA_ERR_CUDA;
@@ -289,7 +320,7 @@ msa_status msa_sparse_attn_fwd(const msa_dims* d, const void* q, const void* k, 
 
 // ------------------------------------------------------------------ Decode --
 size_t msa_sparse_decode_workspace(const msa_decode_dims* d) {
-  if (d == nullptr || d->S < 1 || d->L_max < 1 || d->B_k < 1 || d->k < 1) return 0;
+  if (msa_check_decode_dims(d) != MSA_OK) return 0;
   return kStatusBytes +
          msa::decode_workspace_bytes(d->S, d->L_max, d->H_q, d->H_kv, d->d_h, d->B_k, d->k);
 }
@@ -302,18 +333,13 @@ msa_status msa_sparse_decode(const msa_decode_dims* d, const void* q, const void
       k_idx_new == nullptr || k_cache == nullptr || v_cache == nullptr ||
       k_idx_cache == nullptr || seq_len == nullptr || o == nullptr || ws == nullptr)
     return MSA_ERR_INVALID_ARG;
-  if (d->S < 1 || d->L_max < 1) return MSA_ERR_INVALID_ARG;
-  msa_status st = check_common(d->L_max, d->H_q, d->H_kv, d->d_h, d->d_idx, d->B_k, d->k,
-                               d->attn_scale, d->idx_scale, true, true);
+  msa_status st = msa_check_decode_dims(d);
   if (st != MSA_OK) return st;
   const void* ptrs[] = {q, q_idx, k_new, v_new, k_idx_new, k_cache, v_cache, k_idx_cache,
                         seq_len, o, ws};
   for (const void* p : ptrs)
     if (!aligned16(p)) return MSA_ERR_INVALID_ARG;
   if (idx_out != nullptr && !aligned16(idx_out)) return MSA_ERR_INVALID_ARG;
-  const int G = d->H_q / d->H_kv;
-  if (G > 16 || d->H_kv > 8) return MSA_ERR_UNSUPPORTED;
-  if (d->L_max >= (int64_t(1) << 31)) return MSA_ERR_UNSUPPORTED;
   if (ws_bytes < msa_sparse_decode_workspace(d)) return MSA_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (from_cuda(cudaMemsetAsync(ws, 0, sizeof(msa::DevStatus), s)) != MSA_OK) return MSA_ERR_CUDA;

@@ -23,7 +23,8 @@
  *   - `workspace` is caller-allocated device memory of at least the size the
  *     matching *_workspace() query returns; its first 16 bytes hold the
  *     device status word (see msa_get_device_status).  One workspace must not
- *     be used by two calls that overlap on the GPU.
+ *     be used by two calls that overlap on the GPU.  A *_workspace() query
+ *     returns 0 for dims that the matching call would reject.
  *   - Block indices are 0-based; selection rows are ascending, padded with -1.
  */
 #ifndef MSA_B200_H
@@ -148,9 +149,14 @@ MSA_API msa_status msa_sparse_decode(const msa_decode_dims* dims, const void* q,
  *   - Same arguments, layouts and results as msa_sparse_decode, minus the
  *     workspace.  Returns MSA_ERR_WORKSPACE_TOO_SMALL, launching nothing, if
  *     msa_sparse_decode_workspace(dims) exceeds the fixed size.
- *   - The first call on a device looks up the array's device address (once per
- *     device, with that device current); make that first call before any
- *     stream capture.  The call allocates no memory.
+ *   - Every call looks up the array's device address in the current
+ *     device's context (cudaGetSymbolAddress), so a context that was reset
+ *     and created again is served from its own copy.  The first call on a
+ *     device also loads the library's device code there; make that first
+ *     call before any stream capture.  The call allocates no memory.
+ *   - Dims are validated first, as msa_sparse_decode does (invalid sizes
+ *     return MSA_ERR_INVALID_ARG or MSA_ERR_UNSUPPORTED); only then is the
+ *     scratch size compared with the fixed array.
  *   - All calls share the one array and it keeps the last call's contents:
  *     two calls that overlap on the GPU (other streams, other host threads)
  *     race and corrupt each other's results.  Each call clears the status

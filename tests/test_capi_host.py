@@ -112,3 +112,31 @@ def test_index_lse_rejects_on_host(capi):
     assert capi.LIB.msa_index_lse(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, 8, None) == 3
     d.d_idx = 48
     assert capi.LIB.msa_index_lse(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 40, None) == 2
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("H_kv", 0, 1),      # would divide by zero in the size computation
+    ("H_q", 0, 1),
+    ("d_h", -128, 2),    # negative sizes must not wrap into a huge size_t
+    ("H_q", 30, 1),      # H_q % H_kv != 0
+    ("S", 0, 1),
+])
+def test_decode_workspace_and_noalloc_validate_dims_first(capi, field, value, status):
+    dd = capi.decode_dims(4, 1024, 32, 4, 128, 64, 128, 16)
+    setattr(dd, field, value)
+    # the size query answers 0 for dims the call would reject ...
+    assert capi.LIB.msa_sparse_decode_workspace(ctypes.byref(dd)) == 0
+    # ... and the no-workspace entry point reports the dims error itself,
+    # not a scratch-size error, launching nothing
+    assert capi.LIB.msa_sparse_decode_noalloc(ctypes.byref(dd), *([FAKE] * 11), None) == status
+
+
+def test_prefill_workspace_queries_reject_bad_dims(capi):
+    for field, value in (("H_kv", 0), ("H_q", 6), ("d_h", -64), ("k", 0), ("N", -5)):
+        d = capi.dims(4096, 8, 4, 128, 64, 128, 16)
+        setattr(d, field, value)
+        assert capi.LIB.msa_sparse_attn_fwd_workspace(ctypes.byref(d)) == 0, field
+    for field, value in (("H_kv", 0), ("d_idx", 48), ("B_k", 0)):
+        d = capi.dims(4096, 8, 4, 128, 64, 128, 16)
+        setattr(d, field, value)
+        assert capi.LIB.msa_index_lse_workspace(ctypes.byref(d)) == 0, field
