@@ -39,16 +39,11 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # one ncu capture, per unit of work, with the SHA-256 of the kernel's
 # definition (comments and blank lines removed) at capture time: the figure is
 # reported only while that code is unchanged.
-# kernel -> (source, kernel function, sha256, bytes per unit, unit, capture)
+# kernel -> (source, kernel function, sha256, bytes per unit, unit)
 NCU_TRAFFIC = {
-    "attn_phase1": ("sparse_attn.cu", "attn_phase1_kernel",
-                    "55c33176c70b7f95ebd43f63fb70a4db15fda57ea6de67f1a473fe749360a80f",
-                    (3.666177e9 + 4.195406e9) / 32768, "query",
-                    "profiles/prefill_32k_ncu_full.md: 32K capture, scaled by queries"),
     "attn_merge": ("sparse_attn.cu", "attn_merge_kernel",
                    "beaa021d56c8173edcff10bc3f30370f75c95031da3075c63dc4e1054a981835",
-                   (4.243224e9 + 0.269582e9) / 32768, "query",
-                   "profiles/prefill_32k_ncu_full.md: 32K capture, scaled by queries"),
+                   (4.243224e9 + 0.269582e9) / 32768, "query"),
 }
 
 
@@ -73,17 +68,17 @@ def kernel_code_hash(text: str, name: str) -> str:
 
 
 def ncu_traffic(kernel: str, units: float):
-    """Bytes per launch from NCU_TRAFFIC, or None (no capture, or the kernel
-    changed since it was taken)."""
+    """Bytes per launch from NCU_TRAFFIC and a note on where the figure comes
+    from, or (None, None): no capture, or the kernel changed since."""
     ent = NCU_TRAFFIC.get(kernel)
     if ent is None:
         return None, None
-    src, fn, sha, per_unit, _, where = ent
+    src, fn, sha, per_unit, unit = ent
     path = os.path.join(ROOT, "block_sparse_gqa_idx_b200", "csrc", src)
     with open(path, encoding="utf-8") as f:
         if kernel_code_hash(f.read(), fn) != sha:
             return None, None
-    return per_unit * units, where
+    return per_unit * units, f"one ncu capture of {fn}, scaled by {unit}s"
 
 
 def peaks():

@@ -2,17 +2,19 @@
 // KV-outer block-sparse attention on tcgen05, in three steps per query chunk:
 //
 //   1. inverse index: for every (group r, block b) the list of selection slots
-//      (query i, slot s) that chose b -- count, exclusive scan, scatter, each
-//      CTA counting its range of slots in a shared-memory histogram of the
-//      keys.  The scan also cuts each list into tiles of Tq queries (Tq *
-//      rows-per-query = 128 MMA rows), so hot blocks are split over many CTAs
+//      (query i, slot s) that chose b -- count, exclusive scan (multi-CTA),
+//      scatter, each CTA counting its range of slots in a shared-memory
+//      histogram of the keys.  The scan also cuts each list into tiles of Tq
+//      queries (Tq * rows-per-query = 128 MMA rows) and writes each tile's
+//      (key, first entry, length), so hot blocks are split over many CTAs
 //      with every output slot fixed in advance: no atomics on the outputs.
 //   2. phase 1: one tile = one KV block (K_b, V_b by TMA) and the gathered
 //      query rows that selected it (one TMA box per query: its group's heads).
 //      S = Q K_b^T (UMMA, fp32 in TMEM) -> causal mask (only rows whose own
-//      block is b) -> softmax in registers (one row per thread, exp2) -> P
-//      (bf16) to shared memory -> O = P V_b (UMMA) -> O / l written as an fp16
-//      partial with its natural-log LSE into the row's slot.
+//      block is b) -> softmax by eight warps (two threads per row, exp2) ->
+//      P / l (bf16) back into TMEM -> O = P V_b (UMMA with A in TMEM) -> O
+//      written as an fp16 partial, with its natural-log LSE, into the row's
+//      slot.
 //   3. merge: per (query, head), LSE-weighted sum of its partials (split-K
 //      softmax normalisation), bf16 output + fp32 LSE.
 //
@@ -28,6 +30,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <climits>
 #include <type_traits>
 
 #include "msa_internal.h"
@@ -35,7 +38,6 @@
 namespace msa {
 namespace {
 
-constexpr int kThreads = 320;
 // Largest per-CTA key histogram of the inverse index (H_kv * B keys).
 constexpr size_t kMaxHistBytes = 192 * 1024;
 constexpr int kRowsPerTile = 128;
@@ -44,6 +46,13 @@ constexpr int kRowsPerTile = 128;
 // blocks are then reused over long runs of tiles (small chunks would keep the
 // gathered Q in L2 but re-read K/V for nearly every tile at 1M tokens).
 constexpr int kMaxChunk = 1 << 17;
+// Queries per window of the inverse index's keys.  One window per chunk:
+// keys are (group, block) and a key's list spans the whole chunk, so a K/V
+// block is reused over long runs of tiles.  (Windows of 8192 queries, which
+// keep a window's gathered Q rows in L2, were measured slower: a key's list
+// per window is then only a few tiles long -- one at 1M tokens -- and the
+// K/V reloads cost more than the Q reuse saves.)
+constexpr int kWindow = kMaxChunk;
 
 // Rows per query inside an MMA tile: the group's G heads, or 8 heads (one
 // 128-byte swizzle atom) when G < 8 (the extra heads are computed and dropped).
@@ -56,7 +65,9 @@ struct ChunkBufs {
   int32_t* offsets;   // [nkeys + 1]
   int32_t* tile_off;  // [nkeys + 1]
   int32_t* cursor;    // [nkeys]
-  int32_t* n_tiles;   // [1]
+  int32_t* n_tiles;   // [4]
+  int32_t* block_sums;  // [2 * scan blocks]: per block of keys, (count, tiles), then their offsets
+  int4* tile_meta;       // [tiles]: per tile (key, first entry, queries, the key's end tile)
   uint32_t* entries;  // [Nc * H_kv * k]
   __half* part_o;     // [Nc * H_kv * k, d_h / 8, G, 8]: per slot, 16-byte d-chunks head-minor
   float* part_lse;    // [Nc * H_kv * k, G]
@@ -74,14 +85,18 @@ ChunkBufs carve(void* ws, int64_t Nc, int H_q, int H_kv, int d_h, int kk, int64_
   };
   const int G = H_q / H_kv;
   const int64_t slots = Nc * H_kv * kk;
+  c.part_o = reinterpret_cast<__half*>(take(sizeof(__half) * slots * G * d_h));
+  c.part_lse = reinterpret_cast<float*>(take(sizeof(float) * slots * G));
+  c.entries = reinterpret_cast<uint32_t*>(take(sizeof(uint32_t) * slots));
   c.counts = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * nkeys));
   c.cursor = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * nkeys));
   c.offsets = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * (nkeys + 1)));
   c.tile_off = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * (nkeys + 1)));
   c.n_tiles = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * 4));
-  c.entries = reinterpret_cast<uint32_t*>(take(sizeof(uint32_t) * slots));
-  c.part_lse = reinterpret_cast<float*>(take(sizeof(float) * slots * G));
-  c.part_o = reinterpret_cast<__half*>(take(sizeof(__half) * slots * G * d_h));
+  c.block_sums = reinterpret_cast<int32_t*>(
+      take(sizeof(int32_t) * 2 * ((nkeys + 4095) / 4096 + 1)));
+  // tiles <= entries / (smallest tile of 4 queries) + keys
+  c.tile_meta = reinterpret_cast<int4*>(take(sizeof(int4) * (slots / 4 + nkeys + 1)));
   *total = off;
   return c;
 }
@@ -92,20 +107,36 @@ int64_t chunk_len(int64_t N, int B_k) {
 }
 
 // ------------------------------------------------------------------ step 1 --
+// Keys of the inverse index: (query window w, group r, block b), key =
+// (w * H_kv + r) * B + b, windows of Cw consecutive queries of the chunk.  The
+// lists of one window are contiguous in key order, so a schedule that walks
+// the tiles in key order works through one window of queries at a time and
+// their gathered Q rows stay in L2.
 struct InvParams {
   const int32_t* idx;
   int64_t q0, nq;  // chunk [q0, q0 + nq)
   int H_kv, B_k, kk;
   int64_t B;
   int Tq;
+  int Cw, W;  // queries per window, windows in the chunk
   ChunkBufs c;
   DevStatus* status;
 };
 
-// The key (group r, block b) of entry e of the chunk, or -1 when the entry
-// selects nothing (-1 padding, or a block after the query's own).  Entry e is
-// (query, group, slot) in the layout of I, so e is also the entry's output
-// slot id and I is read contiguously.
+constexpr int kScanThreads = 1024;
+constexpr int kScanPerThread = 4;
+constexpr int kScanBlockKeys = kScanThreads * kScanPerThread;
+static_assert(kScanBlockKeys == 4096, "the workspace carve sizes the block sums for 4096 keys");
+
+inline int64_t inv_nkeys(int64_t nq, int Cw, int H_kv, int64_t B) {
+  return (nq + Cw - 1) / Cw * H_kv * B;
+}
+inline int64_t scan_blocks(int64_t nkeys) { return (nkeys + kScanBlockKeys - 1) / kScanBlockKeys; }
+
+// The window-local key (r * B + b) of entry e of the chunk, or -1 when the
+// entry selects nothing (-1 padding, or a block after the query's own).
+// Entry e is (query, group, slot) in the layout of I, so e is also the
+// entry's output slot id and I is read contiguously.
 __device__ __forceinline__ int inv_key(const InvParams& p, int64_t e, bool report_bad) {
   const int64_t per_q = static_cast<int64_t>(p.H_kv) * p.kk;
   const int64_t il = e / per_q;
@@ -119,22 +150,27 @@ __device__ __forceinline__ int inv_key(const InvParams& p, int64_t e, bool repor
   return (b >= 0 && b <= i / p.B_k) ? r * static_cast<int>(p.B) + b : -1;
 }
 
-// Inverse index with a per-CTA histogram of every key in shared memory.  A
-// CTA owns a contiguous range of entries (a range of queries).  Counting: the
-// CTA counts its entries per key in shared memory and adds each non-zero
-// count to the global one with a single atomic.  Scattering: the CTA counts
-// again, reserves each key's range of the key's list with one atomic on the
-// key's cursor, and places every entry at a shared-memory atomic's position
-// inside that range.
+// Inverse index with a per-CTA histogram of one window's keys in shared
+// memory.  The grid is W x (CTAs per window); a CTA owns a contiguous range
+// of its window's entries.  Counting: the CTA counts its entries per key in
+// shared memory and adds each non-zero count to the global one with a single
+// atomic.  Scattering: the CTA counts again, reserves each key's range of the
+// key's list with one atomic on the key's cursor, and places every entry at a
+// shared-memory atomic's position inside that range.
 template <bool SCATTER>
 __global__ void __launch_bounds__(512) inv_index_smem_kernel(const InvParams p) {
   extern __shared__ int32_t hist[];  // [H_kv * B]
-  const int nkeys = static_cast<int>(p.H_kv * p.B);
-  const int64_t total = p.nq * p.H_kv * p.kk;
-  const int64_t per = (total + gridDim.x - 1) / gridDim.x;
-  const int64_t e0 = static_cast<int64_t>(blockIdx.x) * per;
-  const int64_t e1 = e0 + per < total ? e0 + per : total;
-  for (int j = threadIdx.x; j < nkeys; j += blockDim.x) hist[j] = 0;
+  const int nlocal = static_cast<int>(p.H_kv * p.B);
+  const int cpw = gridDim.x / p.W;
+  const int w = blockIdx.x / cpw, cw = blockIdx.x - w * cpw;
+  const int64_t per_q = static_cast<int64_t>(p.H_kv) * p.kk;
+  const int64_t wq1 = min(static_cast<int64_t>(w + 1) * p.Cw, p.nq);
+  const int64_t we0 = static_cast<int64_t>(w) * p.Cw * per_q, we1 = wq1 * per_q;
+  const int64_t per = (we1 - we0 + cpw - 1) / cpw;
+  const int64_t e0 = we0 + cw * per;
+  const int64_t e1 = e0 + per < we1 ? e0 + per : we1;
+  const int64_t kbase = static_cast<int64_t>(w) * nlocal;
+  for (int j = threadIdx.x; j < nlocal; j += blockDim.x) hist[j] = 0;
   __syncthreads();
   for (int64_t e = e0 + threadIdx.x; e < e1; e += blockDim.x) {
     const int key = inv_key(p, e, !SCATTER);
@@ -142,14 +178,14 @@ __global__ void __launch_bounds__(512) inv_index_smem_kernel(const InvParams p) 
   }
   __syncthreads();
   if constexpr (!SCATTER) {
-    for (int j = threadIdx.x; j < nkeys; j += blockDim.x) {
+    for (int j = threadIdx.x; j < nlocal; j += blockDim.x) {
       const int n = hist[j];
-      if (n > 0) atomicAdd(&p.c.counts[j], n);
+      if (n > 0) atomicAdd(&p.c.counts[kbase + j], n);
     }
   } else {
-    for (int j = threadIdx.x; j < nkeys; j += blockDim.x) {
+    for (int j = threadIdx.x; j < nlocal; j += blockDim.x) {
       const int n = hist[j];
-      if (n > 0) hist[j] = atomicAdd(&p.c.cursor[j], n);
+      if (n > 0) hist[j] = atomicAdd(&p.c.cursor[kbase + j], n);
     }
     __syncthreads();
     for (int64_t e = e0 + threadIdx.x; e < e1; e += blockDim.x) {
@@ -168,7 +204,7 @@ __global__ void inv_index_kernel(const InvParams p) {
   const int64_t total = p.nq * p.H_kv * p.kk;
   for (int64_t t = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; t - threadIdx.x < total;
        t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    int key = -1;
+    int64_t key = -1;
     uint32_t slot = 0;
     if (t < total) {
       const int s = static_cast<int>(t / (p.nq * p.H_kv));
@@ -181,7 +217,7 @@ __global__ void inv_index_kernel(const InvParams p) {
       if (b < -1 || b >= p.B) {
         if (!SCATTER) report(p.status, DEV_ERR_BAD_INDEX, 40, static_cast<int>(i), b);
       } else if (b >= 0 && b <= b_i) {
-        key = r * static_cast<int>(p.B) + b;
+        key = ((il / p.Cw) * p.H_kv + r) * p.B + b;
         slot = static_cast<uint32_t>((il * p.H_kv + r) * p.kk + s);
       }
     }
@@ -203,77 +239,149 @@ __global__ void inv_index_kernel(const InvParams p) {
   }
 }
 
-// Single CTA: exclusive scans of the counts and of the per-key tile counts.
-__global__ void __launch_bounds__(1024) inv_scan_kernel(const InvParams p) {
-  __shared__ int32_t warp_sum[2][32];
-  const int64_t nkeys = p.H_kv * p.B;
-  const int per = static_cast<int>((nkeys + blockDim.x - 1) / blockDim.x);
-  const int64_t beg = static_cast<int64_t>(threadIdx.x) * per;
-  int32_t s_cnt = 0, s_til = 0;
-  for (int j = 0; j < per; ++j) {
-    const int64_t e = beg + j;
-    if (e < nkeys) {
-      const int32_t c = p.c.counts[e];
-      s_cnt += c;
-      s_til += (c + p.Tq - 1) / p.Tq;
-    }
-  }
-  // block-wide exclusive scan of (s_cnt, s_til)
+// Exclusive scan of (count, tiles) pairs over a block of kScanBlockKeys keys:
+// per thread kScanPerThread consecutive keys, warp shuffles, then the warp
+// totals.  Returns the thread's exclusive prefix and the block total.
+__device__ __forceinline__ void block_scan2(int32_t a, int32_t b, int32_t* ex_a, int32_t* ex_b,
+                                            int32_t* tot_a, int32_t* tot_b) {
+  __shared__ int32_t ws[2][32];
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  int32_t a = s_cnt, b = s_til;
+  int32_t x = a, y = b;
+#pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const int32_t ya = __shfl_up_sync(0xFFFFFFFFu, a, o);
-    const int32_t yb = __shfl_up_sync(0xFFFFFFFFu, b, o);
+    const int32_t u = __shfl_up_sync(0xFFFFFFFFu, x, o);
+    const int32_t v = __shfl_up_sync(0xFFFFFFFFu, y, o);
     if (lane >= o) {
-      a += ya;
-      b += yb;
+      x += u;
+      y += v;
     }
   }
   if (lane == 31) {
-    warp_sum[0][w] = a;
-    warp_sum[1][w] = b;
+    ws[0][w] = x;
+    ws[1][w] = y;
   }
   __syncthreads();
   if (w == 0) {
-    int32_t x = lane < static_cast<int>(blockDim.x >> 5) ? warp_sum[0][lane] : 0;
-    int32_t y = lane < static_cast<int>(blockDim.x >> 5) ? warp_sum[1][lane] : 0;
+    const int nw = blockDim.x >> 5;
+    int32_t s = lane < nw ? ws[0][lane] : 0, t = lane < nw ? ws[1][lane] : 0;
+#pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const int32_t yx = __shfl_up_sync(0xFFFFFFFFu, x, o);
-      const int32_t yy = __shfl_up_sync(0xFFFFFFFFu, y, o);
+      const int32_t u = __shfl_up_sync(0xFFFFFFFFu, s, o);
+      const int32_t v = __shfl_up_sync(0xFFFFFFFFu, t, o);
       if (lane >= o) {
-        x += yx;
-        y += yy;
+        s += u;
+        t += v;
       }
     }
-    warp_sum[0][lane] = x;
-    warp_sum[1][lane] = y;
+    ws[0][lane] = s;
+    ws[1][lane] = t;
   }
   __syncthreads();
-  int32_t run_cnt = a - s_cnt + (w > 0 ? warp_sum[0][w - 1] : 0);
-  int32_t run_til = b - s_til + (w > 0 ? warp_sum[1][w - 1] : 0);
-  for (int j = 0; j < per; ++j) {
-    const int64_t e = beg + j;
-    if (e < nkeys) {
-      const int32_t c = p.c.counts[e];
-      p.c.offsets[e] = run_cnt;
-      p.c.cursor[e] = run_cnt;
-      p.c.tile_off[e] = run_til;
-      run_cnt += c;
-      run_til += (c + p.Tq - 1) / p.Tq;
+  *ex_a = x - a + (w > 0 ? ws[0][w - 1] : 0);
+  *ex_b = y - b + (w > 0 ? ws[1][w - 1] : 0);
+  *tot_a = ws[0][31];
+  *tot_b = ws[1][31];
+  __syncthreads();
+}
+
+__device__ __forceinline__ int32_t tiles_of(int32_t count, int Tq) { return (count + Tq - 1) / Tq; }
+
+// Scan, pass 1: per block of keys, the total count and the total tiles.
+__global__ void __launch_bounds__(kScanThreads) inv_scan_reduce_kernel(const InvParams p,
+                                                                        int64_t nkeys) {
+  const int64_t k0 = static_cast<int64_t>(blockIdx.x) * kScanBlockKeys + threadIdx.x * kScanPerThread;
+  int32_t a = 0, b = 0;
+#pragma unroll
+  for (int j = 0; j < kScanPerThread; ++j)
+    if (k0 + j < nkeys) {
+      const int32_t c = p.c.counts[k0 + j];
+      a += c;
+      b += tiles_of(c, p.Tq);
     }
-  }
-  if (threadIdx.x == blockDim.x - 1) {
-    p.c.offsets[nkeys] = run_cnt;
-    p.c.tile_off[nkeys] = run_til;
-    p.c.n_tiles[0] = run_til;
+  int32_t ea, eb, ta, tb;
+  block_scan2(a, b, &ea, &eb, &ta, &tb);
+  if (threadIdx.x == 0) {
+    p.c.block_sums[2 * blockIdx.x] = ta;
+    p.c.block_sums[2 * blockIdx.x + 1] = tb;
   }
 }
 
-// The inverse index's launch shape: a shared-memory histogram of every key per
-// CTA when it fits (up to 4 CTAs per SM), else the global-atomic kernels.
-cudaError_t inv_setup(int64_t nkeys, int sms, size_t* hist_bytes, int* hist_grid) {
-  *hist_bytes = sizeof(int32_t) * static_cast<size_t>(nkeys);
-  *hist_grid = sms;
+// Scan, pass 2 (one block): exclusive scan of the block totals in place, and
+// the grand totals.
+__global__ void __launch_bounds__(kScanThreads) inv_scan_top_kernel(const InvParams p,
+                                                                     int64_t nkeys, int nblocks) {
+  int32_t carry_a = 0, carry_b = 0;
+  for (int base = 0; base < nblocks; base += kScanThreads) {
+    const int g = base + threadIdx.x;
+    const int32_t a = g < nblocks ? p.c.block_sums[2 * g] : 0;
+    const int32_t b = g < nblocks ? p.c.block_sums[2 * g + 1] : 0;
+    int32_t ea, eb, ta, tb;
+    block_scan2(a, b, &ea, &eb, &ta, &tb);
+    if (g < nblocks) {
+      p.c.block_sums[2 * g] = carry_a + ea;
+      p.c.block_sums[2 * g + 1] = carry_b + eb;
+    }
+    carry_a += ta;
+    carry_b += tb;
+  }
+  if (threadIdx.x == 0) {
+    p.c.offsets[nkeys] = carry_a;
+    p.c.tile_off[nkeys] = carry_b;
+    p.c.n_tiles[0] = carry_b;
+  }
+}
+
+// Scan, pass 3: each key's list offset, scatter cursor and first tile.
+__global__ void __launch_bounds__(kScanThreads) inv_scan_apply_kernel(const InvParams p,
+                                                                       int64_t nkeys) {
+  const int64_t k0 = static_cast<int64_t>(blockIdx.x) * kScanBlockKeys + threadIdx.x * kScanPerThread;
+  int32_t cnt[kScanPerThread];
+  int32_t a = 0, b = 0;
+#pragma unroll
+  for (int j = 0; j < kScanPerThread; ++j) {
+    cnt[j] = k0 + j < nkeys ? p.c.counts[k0 + j] : 0;
+    a += cnt[j];
+    b += tiles_of(cnt[j], p.Tq);
+  }
+  int32_t ea, eb, ta, tb;
+  block_scan2(a, b, &ea, &eb, &ta, &tb);
+  int32_t run_a = p.c.block_sums[2 * blockIdx.x] + ea;
+  int32_t run_b = p.c.block_sums[2 * blockIdx.x + 1] + eb;
+#pragma unroll
+  for (int j = 0; j < kScanPerThread; ++j)
+    if (k0 + j < nkeys) {
+      p.c.offsets[k0 + j] = run_a;
+      p.c.cursor[k0 + j] = run_a;
+      p.c.tile_off[k0 + j] = run_b;
+      run_a += cnt[j];
+      run_b += tiles_of(cnt[j], p.Tq);
+    }
+}
+
+// Per tile: (key, first entry, queries, the key's end tile), one thread per
+// tile (a hot key has thousands of tiles).
+__global__ void __launch_bounds__(256) inv_tile_meta_kernel(const InvParams p, int64_t nkeys) {
+  const int n_tiles = p.c.n_tiles[0];
+  for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < n_tiles; t += gridDim.x * blockDim.x) {
+    int64_t lo = 0, hi = nkeys;  // tile_off[lo] <= t < tile_off[hi]
+    while (hi - lo > 1) {
+      const int64_t mid = (lo + hi) >> 1;
+      if (p.c.tile_off[mid] <= t) lo = mid;
+      else hi = mid;
+    }
+    const int32_t t0 = p.c.tile_off[lo], t1 = p.c.tile_off[lo + 1];
+    const int32_t o0 = p.c.offsets[lo], o1 = p.c.offsets[lo + 1];
+    const int32_t first = o0 + (t - t0) * p.Tq;
+    p.c.tile_meta[t] = make_int4(static_cast<int>(lo), first, min(p.Tq, o1 - first), t1);
+  }
+}
+
+// The inverse index's launch shape: a shared-memory histogram of one
+// window's keys per CTA when it fits (up to 4 CTAs per SM), else the
+// global-atomic kernels.
+cudaError_t inv_setup(int64_t nlocal, int sms, size_t* hist_bytes, int* hist_ctas) {
+  *hist_bytes = sizeof(int32_t) * static_cast<size_t>(nlocal);
+  *hist_ctas = sms;
   if (*hist_bytes > kMaxHistBytes) return cudaSuccess;
   cudaError_t e = cudaFuncSetAttribute(inv_index_smem_kernel<false>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -284,37 +392,36 @@ cudaError_t inv_setup(int64_t nkeys, int sms, size_t* hist_bytes, int* hist_grid
                              static_cast<int>(*hist_bytes));
   if (e != cudaSuccess) return e;
   const size_t per_sm = 200 * 1024 / (*hist_bytes + 1024);
-  *hist_grid = sms * static_cast<int>(per_sm < 1 ? 1 : (per_sm > 4 ? 4 : per_sm));
+  *hist_ctas = sms * static_cast<int>(per_sm < 1 ? 1 : (per_sm > 4 ? 4 : per_sm));
   return cudaSuccess;
 }
 
 // Count -> scan -> scatter of one chunk's inverse index (counts zeroed before).
-void launch_inv_index(const InvParams& ip, size_t hist_bytes, int hist_grid, int sms,
+void launch_inv_index(const InvParams& ip, size_t hist_bytes, int hist_ctas, int sms,
                       cudaStream_t stream) {
   const int64_t total = ip.nq * ip.H_kv * ip.kk;
-  if (hist_bytes <= kMaxHistBytes) {
-    prof_begin("inv_count", stream);
-    inv_index_smem_kernel<false><<<hist_grid, 512, hist_bytes, stream>>>(ip);
-    prof_end(stream);
-    prof_begin("inv_scan", stream);
-    inv_scan_kernel<<<1, 1024, 0, stream>>>(ip);
-    prof_end(stream);
-    prof_begin("inv_scatter", stream);
-    inv_index_smem_kernel<true><<<hist_grid, 512, hist_bytes, stream>>>(ip);
-    prof_end(stream);
-  } else {
-    int blocks = static_cast<int>((total + 255) / 256);
-    if (blocks > sms * 16) blocks = sms * 16;
-    prof_begin("inv_count", stream);
-    inv_index_kernel<false><<<blocks, 256, 0, stream>>>(ip);
-    prof_end(stream);
-    prof_begin("inv_scan", stream);
-    inv_scan_kernel<<<1, 1024, 0, stream>>>(ip);
-    prof_end(stream);
-    prof_begin("inv_scatter", stream);
-    inv_index_kernel<true><<<blocks, 256, 0, stream>>>(ip);
-    prof_end(stream);
-  }
+  const int64_t nkeys = static_cast<int64_t>(ip.W) * ip.H_kv * ip.B;
+  const int nblocks = static_cast<int>(scan_blocks(nkeys));
+  const bool smem_path = hist_bytes <= kMaxHistBytes;
+  // the histogram grid: whole windows of CTAs
+  const int cpw = (hist_ctas + ip.W - 1) / ip.W;
+  const int hgrid = cpw * ip.W;
+  int blocks = static_cast<int>((total + 255) / 256);
+  if (blocks > sms * 16) blocks = sms * 16;
+  prof_begin("inv_count", stream);
+  if (smem_path) inv_index_smem_kernel<false><<<hgrid, 512, hist_bytes, stream>>>(ip);
+  else inv_index_kernel<false><<<blocks, 256, 0, stream>>>(ip);
+  prof_end(stream);
+  prof_begin("inv_scan", stream);
+  inv_scan_reduce_kernel<<<nblocks, kScanThreads, 0, stream>>>(ip, nkeys);
+  inv_scan_top_kernel<<<1, kScanThreads, 0, stream>>>(ip, nkeys, nblocks);
+  inv_scan_apply_kernel<<<nblocks, kScanThreads, 0, stream>>>(ip, nkeys);
+  inv_tile_meta_kernel<<<sms * 4, 256, 0, stream>>>(ip, nkeys);
+  prof_end(stream);
+  prof_begin("inv_scatter", stream);
+  if (smem_path) inv_index_smem_kernel<true><<<hgrid, 512, hist_bytes, stream>>>(ip);
+  else inv_index_kernel<true><<<blocks, 256, 0, stream>>>(ip);
+  prof_end(stream);
 }
 
 // ------------------------------------------------------------------ step 2 --
@@ -322,30 +429,45 @@ struct P1Params {
   int64_t q0;
   int q4d;  // 1: one 4-D TMA box per gathered query ([d-chunk][head] rows, 8 heads)
   int H_q, H_kv, B_k, kk, G, R, Tq;
-  int64_t nkeys;
+  int B;          // blocks of the sequence
+  int64_t nkeys;  // (window, group, block) keys
   float scale_log2;  // softmax scale * log2(e)
   float scale;
   ChunkBufs c;
   DevStatus* status;
 };
 
+constexpr int kP1Threads = 512;  // 16 warps, four warpgroups
+constexpr int kIR = 8;           // tile-info ring depth (tiles in flight, producer to epilogue)
+constexpr int kNS = 2;           // S/P and O buffers in TMEM
+// Registers per thread of each warpgroup after the split at kernel start
+// (launched with 128 each: 104 + 56 + 2 x 176 = 4 x 128).
+constexpr int kRegEpi = 104, kRegCtl = 56, kRegSoftmax = 176;
+static_assert(kRegEpi + kRegCtl + 2 * kRegSoftmax <= 4 * 128, "register split above the launch");
+
 template <int D_H, int B_K>
 struct P1Shape {
-  static constexpr int QS = 5;   // Q/P ring depth
-  static constexpr int NKV = 1;  // K/V slots (the ring and two slots do not both fit)
-  static constexpr int QP_BYTES = kRowsPerTile * (D_H > B_K ? D_H : B_K) * 2;  // Q, later P
+  static constexpr int Q_BYTES = kRowsPerTile * D_H * 2;  // one gathered Q tile
   static constexpr int K_BYTES = B_K * D_H * 2;
   static constexpr int V_BYTES = B_K * D_H * 2;
-  static constexpr int DCH = D_H / 64;  // 128-byte chunks along d
-  static constexpr int PCH = B_K / 64;  // 128-byte chunks along keys (P)
-  static constexpr uint32_t TM_S = 0, TM_O = 128;  // column offsets inside a TMEM stage
+  static constexpr int NKV = 2;  // K/V slots: the next block lands while the current one is used
+  // what the Q ring may take of the 227 KB: minus 1 KB of alignment slack and
+  // 2 KB for the tile-info ring and the barriers
+  static constexpr int BUDGET = 227 * 1024 - 1024 - 2048;
+  static constexpr int QS_FIT = (BUDGET - NKV * (K_BYTES + V_BYTES)) / Q_BYTES;
+  static constexpr int QS = QS_FIT > 6 ? 6 : QS_FIT;  // Q ring depth
+  static_assert(QS >= 2, "two Q stages must fit");
+  static constexpr int DCH = D_H / 64;                // 128-byte chunks along d
+  // TMEM columns: S/P buffer b at 128 b, O buffer b at 256 + 128 b
+  static constexpr uint32_t TM_S = 0, TM_O = 256;
 };
 
 constexpr int kMaxTq = 16;  // queries per tile (128 rows / at least 8 rows per query)
 
 struct TileInfo {
   int r, b, len, gen;  // group, block, queries in the tile, K/V generation
-  uint32_t slot[kMaxTq];
+  uint32_t slot[kMaxTq];  // each query's output slot
+  int qi[kMaxTq];         // each query's position i
 };
 
 __device__ __forceinline__ int find_key(const int32_t* tile_off, int64_t nkeys, int t) {
@@ -359,151 +481,126 @@ __device__ __forceinline__ int find_key(const int32_t* tile_off, int64_t nkeys, 
 }
 
 // Phase 1.  Each CTA owns a contiguous range of tiles; tiles of one (group,
-// block) key come in long runs there, so the K/V block sits in one shared
-// slot for the whole run (reloaded only when the key changes) while the
-// gathered query rows stream through a 5-deep ring.  TMEM holds two tiles
-// (S and O, 128 + 128 columns each); two softmax/epilogue groups of four
-// warps take alternate tiles.
-//   warp 0      producer (all lanes: lane q issues query q's TMA box)
-//   warp 1      MMA issuer (lane 0) and TMEM owner
-//   warps 2..9  softmax + epilogue, group (w-2)/4
+// block) key come in long runs there, so a K/V block stays in its shared
+// slot for the whole run; the next run's block loads into the other slot
+// meanwhile.  Gathered Q tiles stream through a ring whose stage frees as
+// soon as S = Q K^T has been computed.
+//   warpgroup 0 (warps 0-3)    epilogue: O (TMEM) -> fp16 partial in HBM
+//   warpgroup 1: warp 4        producer (lane q issues query q's TMA box)
+//                warp 5        MMA issuer (lane 0) and TMEM owner
+//   warpgroups 2, 3            softmax, together on every tile (two warps per
+//                              TMEM lane quarter, 16 lanes each)
+// TMEM: two S/P buffers (columns 0-255) and two O buffers (256-511), so S of
+// the next tile is computed while the softmax works on this one, and the
+// tensor core never writes the columns the epilogue is reading.  The softmax reads S, writes
+// P = exp(S - m) / l as bf16 over the stage's first B_K/2 columns, and
+// O = P V takes P straight from TMEM (tcgen05.mma with A in tensor memory).
+// P is normalised, so O needs no rescaling and the epilogue only converts
+// and stores it; the softmax writes each row's LSE.
 template <int D_H, int B_K>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kP1Threads, 1)
     attn_phase1_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const P1Params p) {
   using SH = P1Shape<D_H, B_K>;
-  constexpr int QS = SH::QS;
+  constexpr int QS = SH::QS, NKV = SH::NKV;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  // K/V slot j: K at sKV + j * (K_BYTES + V_BYTES), V right after it
-  uint8_t* sKV = smem + QS * SH::QP_BYTES;
-  TileInfo* info = reinterpret_cast<TileInfo*>(sKV + SH::NKV * (SH::K_BYTES + SH::V_BYTES));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(info + QS);
-  uint64_t* q_full = bars;             // [QS] gathered Q landed
-  uint64_t* q_empty = q_full + QS;     // [QS] stage free: partials of its tile copied out
-  uint64_t* kv_full = q_empty + QS;    // [NKV] K/V block landed
-  uint64_t* kv_empty = kv_full + SH::NKV;  // [NKV] last tile of a K/V run finished O = P V
-  uint64_t* s_full = kv_empty + SH::NKV;   // [2] S in TMEM
-  uint64_t* p_full = s_full + 2;       // [2] P in smem (S read)
-  uint64_t* o_full = p_full + 2;       // [2] O in TMEM
-  uint64_t* o_empty = o_full + 2;      // [2] O read
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_empty + 2);
+  uint8_t* sQ = smem;                      // [QS] gathered Q tiles
+  uint8_t* sKV = sQ + QS * SH::Q_BYTES;    // [NKV] K block, then V block
+  TileInfo* info = reinterpret_cast<TileInfo*>(sKV + NKV * (SH::K_BYTES + SH::V_BYTES));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(info + kIR);
+  uint64_t* q_full = bars;              // [QS] gathered Q landed
+  uint64_t* q_empty = q_full + QS;      // [QS] S of the stage's tile computed
+  uint64_t* kv_full = q_empty + QS;     // [NKV] K/V block landed
+  uint64_t* kv_empty = kv_full + NKV;   // [NKV] last O = P V of the block's run finished
+  uint64_t* i_full = kv_empty + NKV;    // [kIR] tile info written
+  uint64_t* i_empty = i_full + kIR;     // [kIR] the tile's epilogue is done
+  uint64_t* s_full = i_empty + kIR;     // [kNS] S in TMEM
+  uint64_t* p_full = s_full + kNS;      // [kNS] P in TMEM
+  uint64_t* o_full = p_full + kNS;      // [kNS] O in TMEM
+  uint64_t* o_empty = o_full + kNS;     // [kNS] O read
+  uint64_t* fin = o_empty + kNS;        // every MMA of the CTA finished
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fin + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < QS; ++s) {
       mbar_init(&q_full[s], 1);
-      mbar_init(&q_empty[s], 4);  // the tile's 4 epilogue warps, after their bulk stores
+      mbar_init(&q_empty[s], 1);
     }
-    for (int j = 0; j < SH::NKV; ++j) {
+    for (int j = 0; j < NKV; ++j) {
       mbar_init(&kv_full[j], 1);
       mbar_init(&kv_empty[j], 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&s_full[s], 1);
-      mbar_init(&p_full[s], 4);
-      mbar_init(&o_full[s], 1);
-      mbar_init(&o_empty[s], 4);
+    for (int j = 0; j < kIR; ++j) {
+      mbar_init(&i_full[j], 1);
+      mbar_init(&i_empty[j], 4);  // the four epilogue warps
     }
+    for (int s = 0; s < kNS; ++s) {
+      mbar_init(&s_full[s], 1);
+      mbar_init(&p_full[s], 8);   // the eight softmax warps
+      mbar_init(&o_full[s], 1);
+      mbar_init(&o_empty[s], 4);  // the four epilogue warps
+    }
+    mbar_init(fin, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 1) tmem_alloc(tmem_slot, 512);
+  if (warp == 5) tmem_alloc(tmem_slot, 512);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int n_tiles = p.c.n_tiles[0];
-  // contiguous tile range of this CTA (tiles are equal-sized units of work)
+  // contiguous tile range of this CTA (tiles are equal-sized units of work;
+  // a hot block's list is split over several CTAs)
   const int t_beg = static_cast<int>(static_cast<int64_t>(n_tiles) * blockIdx.x / gridDim.x);
   const int t_end = static_cast<int>(static_cast<int64_t>(n_tiles) * (blockIdx.x + 1) / gridDim.x);
   const int my_tiles = t_end - t_beg;
+  auto tile_of = [&](int n) { return t_beg + n; };
+  const int per_q = p.H_kv * p.kk;
+  const int wg = warp >> 2;
 
-  if (warp == 0) {
-    // ------------------------------------------------------- TMA producer --
-    if (lane == 0) {
-      prefetch_tmap(&tm_q);
-      prefetch_tmap(&tm_k);
-      prefetch_tmap(&tm_v);
-    }
-    const int nb = static_cast<int>(p.nkeys / p.H_kv);
-    const int per_q = p.H_kv * p.kk;
-    // tile cursor: key, its first tile, its entry range
-    int key = 0, kt0 = 0, kend = 0, koff = 0, kcnt = 0;
-    auto seek = [&](int t) {
-      while (kend <= t) {
-        ++key;
-        kt0 = p.c.tile_off[key];
-        kend = p.c.tile_off[key + 1];
-      }
-      koff = p.c.offsets[key];
-      kcnt = p.c.offsets[key + 1] - koff;
-    };
-    uint32_t next_slot = 0;
-    int next_len = 0;
-    if (my_tiles > 0) {
-      key = find_key(p.c.tile_off, p.nkeys, t_beg);
-      kt0 = p.c.tile_off[key];
-      kend = p.c.tile_off[key + 1];
-      koff = p.c.offsets[key];
-      kcnt = p.c.offsets[key + 1] - koff;
-      const int lt = t_beg - kt0;
-      next_len = min(p.Tq, kcnt - lt * p.Tq);
-      if (lane < next_len) next_slot = p.c.entries[koff + lt * p.Tq + lane];
-    }
-    int kv_key = -1, kvgen = 0;
-    for (int n = 0; n < my_tiles; ++n) {
-      const int t = t_beg + n;
-      const int cur_key = key, len = next_len;
-      const uint32_t myslot = next_slot;
-      const int r = cur_key / nb, b = cur_key - r * nb;
-      // fetch the next tile's slots now; their latency hides behind the waits
-      if (n + 1 < my_tiles) {
-        if (t + 1 >= kend) seek(t + 1);
-        const int lt = t + 1 - kt0;
-        next_len = min(p.Tq, kcnt - lt * p.Tq);
-        next_slot = lane < next_len ? p.c.entries[koff + lt * p.Tq + lane] : 0u;
-      }
-      const bool new_kv = cur_key != kv_key;
-      const int gen = new_kv ? kvgen : kvgen - 1;
-      // Q of this tile first (the MMA warp needs it to see a K/V switch)
-      const int qs = n % QS;
-      if (!mbar_wait(&q_empty[qs], ((n / QS) & 1) ^ 1, abort_flag, p.status, 50)) break;
-      TileInfo& ti = info[qs];
-      if (lane < len) ti.slot[lane] = myslot;
+  if (wg == 1) {
+    regs_dec<kRegCtl>();
+    if (warp == 4) {
+      // ----------------------------------------------------- TMA producer --
       if (lane == 0) {
-        ti.r = r;
-        ti.b = b;
-        ti.len = len;
-        ti.gen = gen;
-        mbar_arrive_expect_tx(&q_full[qs], len * p.R * D_H * 2);
+        prefetch_tmap(&tm_q);
+        prefetch_tmap(&tm_k);
+        prefetch_tmap(&tm_v);
       }
-      __syncwarp();
-      const int h0 = p.G >= 8 ? r * p.G : (r * p.G / 8) * 8;
-      if (lane < len) {
-        const int i = static_cast<int>(p.q0 + myslot / per_q);
-        uint8_t* sQ = smem + qs * SH::QP_BYTES;
-        if (p.q4d) {
-          // query-major: [query][d-chunk][8 heads x 128 B]
-          tma_load_4d(sQ + lane * 8 * D_H * 2, &tm_q, &q_full[qs], 0, h0, 0, i);
-        } else {
-          // chunk-major: [d-chunk][query rows x 128 B]
-#pragma unroll
-          for (int c = 0; c < SH::DCH; ++c)
-            tma_load_3d(sQ + c * kRowsPerTile * 128 + lane * p.R * 128, &tm_q, &q_full[qs],
-                        c * 64, h0, i);
+      // per tile: (key, first entry, queries, end tile of the key), loaded two
+      // tiles ahead; the tile's slots one tile ahead
+      auto meta_of = [&](int n) -> int4 {
+        return n < my_tiles ? p.c.tile_meta[tile_of(n)] : make_int4(-1, 0, 0, 0);
+      };
+      int4 meta_next = meta_of(0), meta_next2 = meta_of(1);
+      uint32_t next_slot = 0;
+      if (my_tiles > 0 && lane < meta_next.z) next_slot = p.c.entries[meta_next.y + lane];
+      // K/V generations: a generation is a run of this CTA's tiles with one
+      // key; generation g lives in slot g % NKV.  A second cursor finds where
+      // the next generation starts so its block loads as soon as its slot is
+      // free (one generation ahead), not when its first tile comes up.
+      int la_n = 0, la_key = meta_next.x;  // start and key of generation `loaded`
+      int la_end = meta_next.w;            // end tile of la_key
+      int loaded = 0;                      // generations whose load was issued
+      auto advance_la = [&]() {
+        // the first tile after la_n whose key differs from la_key: the
+        // tile where la_key's list ends
+        la_n += la_end - tile_of(la_n);
+        if (la_n < my_tiles) {
+          const int4 m = meta_of(la_n);
+          la_key = m.x;
+          la_end = m.w;
         }
-      }
-      if (new_kv) {
-        // generation g lives in slot g % NKV; the slot is free once every tile
-        // of generation g - NKV finished O = P V
-        const int slot = kvgen % SH::NKV;
-        if (kvgen >= SH::NKV &&
-            !mbar_wait(&kv_empty[slot], ((kvgen / SH::NKV) - 1) & 1, abort_flag, p.status, 51))
-          break;
+      };
+      auto load_kv = [&](int g, int k) {
+        const int slot = g % NKV;
+        const int r = (k / p.B) % p.H_kv, b = k % p.B;
         uint8_t* sK = sKV + slot * (SH::K_BYTES + SH::V_BYTES);
         uint8_t* sV = sK + SH::K_BYTES;
         if (lane == 0) mbar_arrive_expect_tx(&kv_full[slot], SH::K_BYTES + SH::V_BYTES);
@@ -512,39 +609,113 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_3d(sK + lane * B_K * 128, &tm_k, &kv_full[slot], lane * 64, r, b * B_K);
           tma_load_3d(sV + lane * B_K * 128, &tm_v, &kv_full[slot], lane * 64, r, b * B_K);
         }
-        kv_key = cur_key;
-        ++kvgen;
+      };
+      int kv_key = -1, kvgen = 0;
+      for (int n = 0; n < my_tiles; ++n) {
+        const int cur_key = meta_next.x, len = meta_next.z;
+        const uint32_t myslot = next_slot;
+        const int r = (cur_key / p.B) % p.H_kv, b = cur_key % p.B;
+        // the next tile's slots and the metadata of the one after: their
+        // latency hides behind the waits below
+        meta_next = meta_next2;
+        next_slot = (n + 1 < my_tiles && lane < meta_next.z) ? p.c.entries[meta_next.y + lane] : 0u;
+        meta_next2 = meta_of(n + 2);
+        const bool new_kv = cur_key != kv_key;
+        const int gen = new_kv ? kvgen : kvgen - 1;
+        const int is = n % kIR, qs = n % QS;
+        if (!mbar_wait(&i_empty[is], ((n / kIR) & 1) ^ 1, abort_flag, p.status, 50)) break;
+        TileInfo& ti = info[is];
+        if (lane < len) {
+          ti.slot[lane] = myslot;
+          ti.qi[lane] = static_cast<int>(p.q0 + myslot / per_q);
+        }
+        if (lane == 0) {
+          ti.r = r;
+          ti.b = b;
+          ti.len = len;
+          ti.gen = gen;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&i_full[is]);
+        if (!mbar_wait(&q_empty[qs], ((n / QS) & 1) ^ 1, abort_flag, p.status, 52)) break;
+        if (lane == 0) mbar_arrive_expect_tx(&q_full[qs], len * p.R * D_H * 2);
+        __syncwarp();
+        const int h0 = p.G >= 8 ? r * p.G : (r * p.G / 8) * 8;
+        if (lane < len) {
+          const int i = static_cast<int>(p.q0 + myslot / per_q);
+          uint8_t* dst = sQ + qs * SH::Q_BYTES;
+          if (p.q4d) {
+            // query-major: [query][d-chunk][8 heads x 128 B]
+            tma_load_4d(dst + lane * 8 * D_H * 2, &tm_q, &q_full[qs], 0, h0, 0, i);
+          } else {
+            // chunk-major: [d-chunk][query rows x 128 B]
+#pragma unroll
+            for (int c = 0; c < SH::DCH; ++c)
+              tma_load_3d(dst + c * kRowsPerTile * 128 + lane * p.R * 128, &tm_q, &q_full[qs],
+                          c * 64, h0, i);
+          }
+        }
+        if (new_kv) {
+          kv_key = cur_key;
+          ++kvgen;
+        }
+        // load every generation up to the one after this tile's: a
+        // generation's slot is free once every tile of generation g - NKV
+        // finished O = P V (waited for only when this tile needs it)
+        bool stop = false;
+        while (loaded <= gen + 1 && la_n < my_tiles) {
+          const bool need = loaded <= gen;
+          if (loaded >= NKV) {
+            uint64_t* eb = &kv_empty[loaded % NKV];
+            const uint32_t par = ((loaded / NKV) - 1) & 1;
+            if (need) {
+              if (!mbar_wait(eb, par, abort_flag, p.status, 51)) {
+                stop = true;
+                break;
+              }
+            } else if (!__all_sync(0xFFFFFFFFu, mbar_test_wait(eb, par))) {
+              break;
+            }
+          }
+          load_kv(loaded, la_key);
+          ++loaded;
+          advance_la();
+        }
+        if (stop) break;
       }
-    }
-  } else if (warp == 1) {
-    // -------------------------------------------------------- MMA issuer --
-    // S of tile n+1 is issued before waiting for the softmax of tile n, so the
-    // tensor core works while P is built.  After O(n) of a run's last tile the
-    // run's K/V slot is released; with a single slot the next run's K/V can
-    // only land after that, so at a switch O(n) goes first.
-    if (lane == 0) {
+    } else if (warp == 5 && lane == 0) {
+      // ------------------------------------------------------ MMA issuer --
+      // S(n) goes before O(n-1) when tile n's rows and K block have landed,
+      // so the tensor core works while the softmax of n-1 finishes; else
+      // O(n-1) goes first so it never waits behind a gather (or behind a K/V
+      // block that can only load once O(n-1) frees its slot).  S(n) reuses
+      // the S/P buffer of tile n-2, whose O MMA (reading P there) was issued
+      // before it: tcgen05.mma ops of one thread run in issue order.
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, B_K, 0, 0);
       constexpr uint32_t idesc_o = idesc_bf16_f32(128, D_H, 0, 1);
-      int gen_have = -1;
-      auto wait_q = [&](int n, int* gen) -> bool {
-        const int qs = n % QS;
-        if (!mbar_wait(&q_full[qs], (n / QS) & 1, abort_flag, p.status, 60)) return false;
-        *gen = info[qs].gen;
+      const uint32_t q_sbo = p.q4d ? 8 * D_H * 2 : 1024;  // between 8-row groups
+      const uint32_t q_cstep = p.q4d ? 8 * 128 : kRowsPerTile * 128;  // between d-chunks
+      int kv_ready = -1;  // highest K/V generation known to have landed
+      auto prep = [&](int n, int* gen) -> bool {
+        if (!mbar_wait(&i_full[n % kIR], (n / kIR) & 1, abort_flag, p.status, 60)) return false;
+        *gen = info[n % kIR].gen;
         return true;
       };
+      auto s_ready = [&](int n, int gen) -> bool {
+        return mbar_test_wait(&q_full[n % QS], (n / QS) & 1) &&
+               (gen <= kv_ready || mbar_test_wait(&kv_full[gen % NKV], (gen / NKV) & 1));
+      };
       auto issue_s = [&](int n, int gen) -> bool {
-        if (gen != gen_have) {
-          if (!mbar_wait(&kv_full[gen % SH::NKV], (gen / SH::NKV) & 1, abort_flag, p.status, 63))
+        if (!mbar_wait(&q_full[n % QS], (n / QS) & 1, abort_flag, p.status, 61)) return false;
+        if (gen > kv_ready) {
+          if (!mbar_wait(&kv_full[gen % NKV], (gen / NKV) & 1, abort_flag, p.status, 62))
             return false;
-          gen_have = gen;
+          kv_ready = gen;
         }
         tc_fence_after();
-        const uint32_t q_base = smem_u32(smem + (n % QS) * SH::QP_BYTES);
-        const uint32_t k_base = smem_u32(sKV + (gen % SH::NKV) * (SH::K_BYTES + SH::V_BYTES));
-        const uint32_t tS = tmem_base + (n & 1) * 256 + SH::TM_S;
-        // 8-row groups: consecutive queries (query-major) or consecutive rows
-        const uint32_t q_sbo = p.q4d ? 8 * D_H * 2 : 1024;
-        const uint32_t q_cstep = p.q4d ? 8 * 128 : kRowsPerTile * 128;
+        const uint32_t q_base = smem_u32(sQ + (n % QS) * SH::Q_BYTES);
+        const uint32_t k_base = smem_u32(sKV + (gen % NKV) * (SH::K_BYTES + SH::V_BYTES));
+        const uint32_t tS = tmem_base + (n % kNS) * 128 + SH::TM_S;
 #pragma unroll
         for (int c = 0; c < SH::DCH; ++c)
 #pragma unroll
@@ -553,187 +724,245 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t bd = umma_desc(k_base + c * B_K * 128 + s * 32, 16, 1024, SW_128B);
             umma_bf16(tS, ad, bd, idesc_s, (c | s) != 0);
           }
-        umma_commit(&s_full[n & 1]);
+        umma_commit(&s_full[n % kNS]);
+        umma_commit(&q_empty[n % QS]);
         return true;
       };
-      int gcur = 0;
-      bool ok = my_tiles == 0 || (wait_q(0, &gcur) && issue_s(0, gcur));
-      for (int n = 0; ok && n < my_tiles; ++n) {
-        const int st = n & 1;
-        const uint32_t ph = (n >> 1) & 1;
-        const bool has_next = n + 1 < my_tiles;
-        // S of tile n+1 goes before O(n) only if its gathered rows have
-        // already landed: O(n) must never wait behind the next gather.  (S of
-        // tile n+1 reuses the TMEM stage of tile n-1, whose P was waited for in
-        // the previous iteration.)
-        int gnext = gcur;
-        bool s_done = false;
-        if (has_next && mbar_try_wait(&q_full[(n + 1) % QS], ((n + 1) / QS) & 1)) {
-          gnext = info[(n + 1) % QS].gen;
-          if (SH::NKV > 1 || gnext == gcur) {
-            if (!issue_s(n + 1, gnext)) break;
-            s_done = true;
-          }
-        }
-        if (!mbar_wait(&p_full[st], ph, abort_flag, p.status, 61)) break;
-        if (!mbar_wait(&o_empty[st], ph ^ 1, abort_flag, p.status, 62)) break;
+      auto issue_o = [&](int m, int gen, bool last_of_gen) -> bool {
+        if (!mbar_wait(&p_full[m % kNS], (m / kNS) & 1, abort_flag, p.status, 63)) return false;
+        if (!mbar_wait(&o_empty[m % kNS], ((m / kNS) & 1) ^ 1, abort_flag, p.status, 64))
+          return false;
         tc_fence_after();
-        const uint32_t q_base = smem_u32(smem + (n % QS) * SH::QP_BYTES);
         const uint32_t v_base =
-            smem_u32(sKV + (gcur % SH::NKV) * (SH::K_BYTES + SH::V_BYTES) + SH::K_BYTES);
-        const uint32_t tO = tmem_base + st * 256 + SH::TM_O;
+            smem_u32(sKV + (gen % NKV) * (SH::K_BYTES + SH::V_BYTES) + SH::K_BYTES);
+        const uint32_t tP = tmem_base + (m % kNS) * 128 + SH::TM_S;
+        const uint32_t tO = tmem_base + SH::TM_O + (m % kNS) * 128;
 #pragma unroll
-        for (int c = 0; c < SH::PCH; ++c)
-#pragma unroll
-          for (int s = 0; s < 4; ++s) {
-            // P: K-major (keys contiguous), chunk c = keys [64c, 64c+64)
-            const uint64_t ad =
-                umma_desc(q_base + c * kRowsPerTile * 128 + s * 32, 16, 1024, SW_128B);
-            // V: MN-major (d contiguous); 16 keys = two 8-key groups = 2048 B
-            const uint64_t bd = umma_desc(v_base + (c * 4 + s) * 2048, B_K * 128, 1024, SW_128B);
-            umma_bf16(tO, ad, bd, idesc_o, (c | s) != 0);
-          }
-        umma_commit(&o_full[st]);
-        if (has_next && !s_done) {
-          if (!wait_q(n + 1, &gnext)) break;
-          // a run's last tile releases its K/V slot once O(n) has finished
-          if (gnext != gcur) umma_commit(&kv_empty[gcur % SH::NKV]);
-          if (!issue_s(n + 1, gnext)) break;
-        } else if (has_next && gnext != gcur) {
-          umma_commit(&kv_empty[gcur % SH::NKV]);
+        for (int ks = 0; ks < B_K / 16; ++ks) {
+          // V: MN-major (d contiguous); 16 keys = two 8-key groups = 2048 B
+          const uint64_t bd = umma_desc(v_base + ks * 2048, B_K * 128, 1024, SW_128B);
+          umma_bf16_ts(tO, tP + ks * 8, bd, idesc_o, ks != 0);
         }
-        gcur = gnext;
+        umma_commit(&o_full[m % kNS]);
+        if (last_of_gen) umma_commit(&kv_empty[gen % NKV]);
+        return true;
+      };
+      if (my_tiles > 0) {
+        int gprev = 0;
+        bool ok = prep(0, &gprev) && issue_s(0, gprev);
+        for (int n = 1; ok && n < my_tiles; ++n) {
+          int gn = 0;
+          if (!prep(n, &gn)) break;
+          const bool last = gn != gprev;
+          if (s_ready(n, gn)) ok = issue_s(n, gn) && issue_o(n - 1, gprev, last);
+          else ok = issue_o(n - 1, gprev, last) && issue_s(n, gn);
+          gprev = gn;
+        }
+        if (ok) issue_o(my_tiles - 1, gprev, true);
       }
+      // every MMA of this CTA must be done before TMEM is released
+      umma_commit(fin);
+      mbar_wait(fin, 0, nullptr, p.status, 69);
     }
-  } else {
-    // ------------------------------------------ softmax + epilogue groups --
-    const int grp = (warp - 2) >> 2;  // handles tiles n with n % 2 == grp
-    const int quarter = warp & 3;
-    const int row = quarter * 32 + lane;
+  } else if (wg == 0) {
+    // -------------------------------------------------------- epilogue --
+    regs_dec<kRegEpi>();
+    const int row = warp * 32 + lane;  // warp w reads TMEM lanes 32w .. 32w+31
     const int q_local = row / p.R;
     const int hrow = row - q_local * p.R;
-    const int per_q = p.H_kv * p.kk;
-    for (int n = grp; n < my_tiles; n += 2) {
-      const int st = grp;
-      const uint32_t ph = (n >> 1) & 1;
-      const int qs = n % QS;
-      uint8_t* sP = smem + qs * SH::QP_BYTES;
-      const uint32_t tS = tmem_base + st * 256 + SH::TM_S + (static_cast<uint32_t>(quarter * 32) << 16);
-      const uint32_t tO = tmem_base + st * 256 + SH::TM_O + (static_cast<uint32_t>(quarter * 32) << 16);
-      if (!mbar_wait(&s_full[st], ph, abort_flag, p.status, 70)) break;
-      // q_full[qs] cannot advance before this tile's O MMA, so this returns at
-      // once; it orders the producer's TileInfo writes before the reads below
-      if (!mbar_wait(&q_full[qs], (n / QS) & 1, abort_flag, p.status, 72)) break;
+    for (int n = 0; n < my_tiles; ++n) {
+      const int is = n % kIR;
+      if (!mbar_wait(&i_full[is], (n / kIR) & 1, abort_flag, p.status, 70)) break;
+      if (!mbar_wait(&o_full[n % kNS], (n / kNS) & 1, abort_flag, p.status, 71)) break;
       tc_fence_after();
-      const int ti_r = info[qs].r, ti_b = info[qs].b, ti_len = info[qs].len;
-      const bool live = q_local < ti_len;
-      const uint32_t slot = live ? info[qs].slot[q_local] : 0u;
-      const int64_t i = p.q0 + slot / per_q;
-      // ---- softmax over the block's keys (exp2 with the scale folded in)
-      float sv[B_K];
-      {
-        uint32_t r32[B_K / 32][32];
-#pragma unroll
-        for (int c = 0; c < B_K / 32; ++c) tmem_ld32(tS + c * 32, r32[c]);
-        tmem_wait_ld();
-#pragma unroll
-        for (int c = 0; c < B_K / 32; ++c)
-#pragma unroll
-          for (int j = 0; j < 32; ++j) sv[c * 32 + j] = __uint_as_float(r32[c][j]);
-      }
-      const int64_t j0 = static_cast<int64_t>(ti_b) * B_K;
-      if (j0 + B_K - 1 > i) {  // the query's own block: causal rule j <= i
-#pragma unroll
-        for (int j = 0; j < B_K; ++j)
-          if (j0 + j > i) sv[j] = -INFINITY;
-      }
-      float mx = sv[0];
-#pragma unroll
-      for (int j = 1; j + 1 < B_K; j += 2) mx = fmax3(mx, sv[j], sv[j + 1]);
-      mx = fmaxf(mx, sv[B_K - 1]);
-      const float mscaled = mx * p.scale_log2;
-      float l = 0.0f;
-#pragma unroll
-      for (int j = 0; j < B_K; ++j) {
-        const float e = exp2f(fmaf(sv[j], p.scale_log2, -mscaled));
-        sv[j] = e;
-        l += e;
-      }
-      // P (bf16) over the stage's Q rows (consumed by S), K-major 128B-swizzled
-#pragma unroll
-      for (int c = 0; c < B_K / 8; ++c) {
-        uint4 w;
-        __nv_bfloat162 h0 = __floats2bfloat162_rn(sv[c * 8 + 0], sv[c * 8 + 1]);
-        __nv_bfloat162 h1 = __floats2bfloat162_rn(sv[c * 8 + 2], sv[c * 8 + 3]);
-        __nv_bfloat162 h2 = __floats2bfloat162_rn(sv[c * 8 + 4], sv[c * 8 + 5]);
-        __nv_bfloat162 h3 = __floats2bfloat162_rn(sv[c * 8 + 6], sv[c * 8 + 7]);
-        w.x = *reinterpret_cast<uint32_t*>(&h0);
-        w.y = *reinterpret_cast<uint32_t*>(&h1);
-        w.z = *reinterpret_cast<uint32_t*>(&h2);
-        w.w = *reinterpret_cast<uint32_t*>(&h3);
-        const int kc = c >> 3, j16 = c & 7;
-        uint8_t* dst = sP + kc * kRowsPerTile * 128 + row * 128 + ((j16 ^ (row & 7)) << 4);
-        *reinterpret_cast<uint4*>(dst) = w;
-      }
-      fence_async_smem();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[st]);
-      // ---- O = P V; write O / l as an fp16 partial and lse into the slot
-      if (!mbar_wait(&o_full[st], ph, abort_flag, p.status, 71)) break;
-      tc_fence_after();
-      const int goff = p.G >= 8 ? 0 : (ti_r * p.G) % 8;  // group's first head in the box
-      const bool useful = live && hrow >= goff && hrow < goff + p.G;
+      const TileInfo& ti = info[is];
+      const int goff = p.G >= 8 ? 0 : (ti.r * p.G) % 8;  // group's first head in the box
+      const bool useful = q_local < ti.len && hrow >= goff && hrow < goff + p.G;
       const int g = hrow - goff;
-      // partial layout [slot][d/8][g][8].  The tile's partials are staged in its
-      // Q/P buffer (P is dead once O = P V completed) in exactly that layout,
-      // so each query's G x d_h block is one contiguous bulk copy to HBM.
-      const int qbytes = p.G * D_H * 2;  // one query's partial block
-      uint8_t* stage = sP + q_local * qbytes;
-      const float inv_l = 1.0f / l;
-      uint32_t ro[D_H / 32][32];
+      const uint32_t slot = useful ? ti.slot[q_local] : 0u;
+      // partial layout [slot][d/8][g][8]: for one d/8 the G heads of a query
+      // are G consecutive 16-byte pieces, so a warp's stores cover whole
+      // 128-byte lines
+      __half* dst = p.c.part_o + static_cast<int64_t>(slot) * p.G * D_H + g * 8;
+      const uint32_t tO =
+          tmem_base + SH::TM_O + (n % kNS) * 128 + (static_cast<uint32_t>(warp * 32) << 16);
 #pragma unroll
-      for (int c = 0; c < D_H / 32; ++c) tmem_ld32(tO + c * 32, ro[c]);
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&o_empty[st]);
-      if (useful) {
+      for (int hc = 0; hc < D_H / 64; ++hc) {
+        uint32_t ra[32], rb[32];
+        tmem_ld32(tO + hc * 64, ra);
+        tmem_ld32(tO + hc * 64 + 32, rb);
+        tmem_wait_ld();
+        if (hc == D_H / 64 - 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&o_empty[n % kNS]);
+        }
+        if (useful) {
 #pragma unroll
-        for (int c = 0; c < D_H / 32; ++c)
-#pragma unroll
-          for (int j = 0; j < 32; j += 8) {
+          for (int j = 0; j < 64; j += 8) {
+            const uint32_t* src = j < 32 ? &ra[j] : &rb[j - 32];
             uint4 w;
-            __half2 a0 = __floats2half2_rn(__uint_as_float(ro[c][j + 0]) * inv_l, __uint_as_float(ro[c][j + 1]) * inv_l);
-            __half2 a1 = __floats2half2_rn(__uint_as_float(ro[c][j + 2]) * inv_l, __uint_as_float(ro[c][j + 3]) * inv_l);
-            __half2 a2 = __floats2half2_rn(__uint_as_float(ro[c][j + 4]) * inv_l, __uint_as_float(ro[c][j + 5]) * inv_l);
-            __half2 a3 = __floats2half2_rn(__uint_as_float(ro[c][j + 6]) * inv_l, __uint_as_float(ro[c][j + 7]) * inv_l);
+            __half2 a0 = __floats2half2_rn(__uint_as_float(src[0]), __uint_as_float(src[1]));
+            __half2 a1 = __floats2half2_rn(__uint_as_float(src[2]), __uint_as_float(src[3]));
+            __half2 a2 = __floats2half2_rn(__uint_as_float(src[4]), __uint_as_float(src[5]));
+            __half2 a3 = __floats2half2_rn(__uint_as_float(src[6]), __uint_as_float(src[7]));
             w.x = *reinterpret_cast<uint32_t*>(&a0);
             w.y = *reinterpret_cast<uint32_t*>(&a1);
             w.z = *reinterpret_cast<uint32_t*>(&a2);
             w.w = *reinterpret_cast<uint32_t*>(&a3);
-            *reinterpret_cast<uint4*>(stage + (((c * 32 + j) >> 3) * p.G + g) * 16) = w;
+            const int d8 = (hc * 64 + j) >> 3;
+            // written once and read once by the merge: stream past L2 so the
+            // gathered Q rows stay cached
+            __stcs(reinterpret_cast<uint4*>(dst + d8 * p.G * 8), w);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&i_empty[is]);
+    }
+  } else {
+    // ---------------------------------------------------------- softmax --
+    regs_inc<kRegSoftmax>();
+    // All eight warps take every tile: warps w and w + 4 share TMEM lane
+    // quarter w % 4, the first taking its lanes 0-15, the second 16-31.  A
+    // thread holds two rows (lanes lo = base + lane/4 and hi = lo + 8) x the
+    // row's keys 8r + 2c, 8r + 2c + 1 (c = lane % 4, r = 0 .. B_K/8 - 1), so
+    // a row's reductions take two shuffles across its four threads, and the
+    // bf16 pair of keys (8r + 2c, 8r + 2c + 1) is exactly P column 4r + c of
+    // the 16x128b store shape.
+    const int half = (warp - 8) >> 2;
+    const int quarter = warp & 3;
+    const int gq = lane >> 2, cq = lane & 3;
+    const int lane0 = quarter * 32 + half * 16;  // first TMEM lane of this warp
+    const int rowA = lane0 + gq, rowB = rowA + 8;
+    const int qA = rowA / p.R, hA = rowA - qA * p.R;
+    const int qB = rowB / p.R, hB = rowB - qB * p.R;
+    // When S of tile n + 1 is already complete, its TMEM load is issued
+    // before P of tile n is stored, so the load latency overlaps the store
+    // and the barrier hand-off.  (It is never waited for there: the MMA
+    // warp may be waiting for this P before it issues S of n + 1.)
+    uint32_t v[B_K / 2];  // v[4r + 0/1]: row A, keys 8r + 2c + 0/1; v[4r + 2/3]: row B
+    auto s_landed = [&](int n) -> bool {
+      const bool mine = mbar_test_wait(&i_full[n % kIR], (n / kIR) & 1) &&
+                        mbar_test_wait(&s_full[n % kNS], (n / kNS) & 1);
+      return __all_sync(0xFFFFFFFFu, mine);  // every lane saw both phases complete
+    };
+    auto load_s = [&](int n, bool landed) -> bool {
+      const int st = n % kNS;
+      if (!landed) {
+        if (!mbar_wait(&i_full[n % kIR], (n / kIR) & 1, abort_flag, p.status, 80)) return false;
+        if (!mbar_wait(&s_full[st], (n / kNS) & 1, abort_flag, p.status, 81)) return false;
+      }
+      tc_fence_after();
+      const uint32_t tS = tmem_base + st * 128 + SH::TM_S + (static_cast<uint32_t>(lane0) << 16);
+#pragma unroll
+      for (int h = 0; h < B_K / 64; ++h) {
+        uint32_t t32[32];
+        tmem_ld_16x256b_x8(tS + h * 64, t32);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[h * 32 + j] = t32[j];
+      }
+      return true;
+    };
+    bool ok = my_tiles > 0 && load_s(0, false);
+    for (int n = 0; ok && n < my_tiles; ++n) {
+      const int st = n % kNS, is = n % kIR;
+      const uint32_t tS = tmem_base + st * 128 + SH::TM_S + (static_cast<uint32_t>(lane0) << 16);
+      const TileInfo& ti = info[is];
+      const int goff = p.G >= 8 ? 0 : (ti.r * p.G) % 8;  // group's first head in the box
+      const bool liveA = qA < ti.len, liveB = qB < ti.len;
+      const uint32_t slotA = liveA ? ti.slot[qA] : 0u;
+      const uint32_t slotB = liveB ? ti.slot[qB] : 0u;
+      // a padding row (past the tile's queries) is never masked
+      const int iA = liveA ? ti.qi[qA] : INT_MAX;
+      const int iB = liveB ? ti.qi[qB] : INT_MAX;
+      const int jb = ti.b * B_K;  // the block's first key
+      tmem_wait_ld();
+      if (jb + B_K - 1 > (iA < iB ? iA : iB)) {  // a query's own block: j <= i
+#pragma unroll
+        for (int r = 0; r < B_K / 8; ++r)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int j = jb + 8 * r + 2 * cq + e;
+            if (j > iA) v[4 * r + e] = __float_as_uint(-INFINITY);
+            if (j > iB) v[4 * r + 2 + e] = __float_as_uint(-INFINITY);
           }
       }
-      fence_async_smem();
-      __syncwarp();
-      // one lane per query (its first useful head) copies the query's block
-      if (useful && g == 0) {
-        bulk_store(p.c.part_o + static_cast<int64_t>(slot) * p.G * D_H, stage, qbytes);
-        bulk_commit();
-        bulk_wait_read_all();
+      float mA = -INFINITY, mB = -INFINITY;
+#pragma unroll
+      for (int r = 0; r < B_K / 8; ++r) {
+        mA = fmax3(mA, __uint_as_float(v[4 * r]), __uint_as_float(v[4 * r + 1]));
+        mB = fmax3(mB, __uint_as_float(v[4 * r + 2]), __uint_as_float(v[4 * r + 3]));
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&q_empty[qs]);
-      if (useful) {
-        p.c.part_lse[static_cast<int64_t>(slot) * p.G + g] = mx * p.scale + logf(l);
+#pragma unroll
+      for (int o = 1; o < 4; o <<= 1) {
+        mA = fmaxf(mA, __shfl_xor_sync(0xFFFFFFFFu, mA, o));
+        mB = fmaxf(mB, __shfl_xor_sync(0xFFFFFFFFu, mB, o));
       }
+      const float msA = mA * p.scale_log2, msB = mB * p.scale_log2;
+      float lA0 = 0.0f, lA1 = 0.0f, lB0 = 0.0f, lB1 = 0.0f;
+#pragma unroll
+      for (int r = 0; r < B_K / 8; ++r) {
+        const float a0 = ex2_ftz(fmaf(__uint_as_float(v[4 * r]), p.scale_log2, -msA));
+        const float a1 = ex2_ftz(fmaf(__uint_as_float(v[4 * r + 1]), p.scale_log2, -msA));
+        const float b0 = ex2_ftz(fmaf(__uint_as_float(v[4 * r + 2]), p.scale_log2, -msB));
+        const float b1 = ex2_ftz(fmaf(__uint_as_float(v[4 * r + 3]), p.scale_log2, -msB));
+        lA0 += a0;
+        lA1 += a1;
+        lB0 += b0;
+        lB1 += b1;
+        v[4 * r] = __float_as_uint(a0);
+        v[4 * r + 1] = __float_as_uint(a1);
+        v[4 * r + 2] = __float_as_uint(b0);
+        v[4 * r + 3] = __float_as_uint(b1);
+      }
+      float lA = lA0 + lA1, lB = lB0 + lB1;
+#pragma unroll
+      for (int o = 1; o < 4; o <<= 1) {
+        lA += __shfl_xor_sync(0xFFFFFFFFu, lA, o);
+        lB += __shfl_xor_sync(0xFFFFFFFFu, lB, o);
+      }
+      const float invA = 1.0f / lA, invB = 1.0f / lB;
+      // P / l as bf16 pairs: the pair of keys (8r + 2c, 8r + 2c + 1) is P
+      // column 4r + c
+      uint32_t pk[B_K / 4];
+#pragma unroll
+      for (int r = 0; r < B_K / 8; ++r) {
+        __nv_bfloat162 xa = __floats2bfloat162_rn(__uint_as_float(v[4 * r]) * invA,
+                                                  __uint_as_float(v[4 * r + 1]) * invA);
+        __nv_bfloat162 xb = __floats2bfloat162_rn(__uint_as_float(v[4 * r + 2]) * invB,
+                                                  __uint_as_float(v[4 * r + 3]) * invB);
+        pk[2 * r] = *reinterpret_cast<uint32_t*>(&xa);
+        pk[2 * r + 1] = *reinterpret_cast<uint32_t*>(&xb);
+      }
+      const bool more = n + 1 < my_tiles;
+      const bool early = more && s_landed(n + 1);
+      if (early) load_s(n + 1, true);  // into v: this tile's values are all in pk now
+      // P over the stage's first B_K / 2 columns (its S was read)
+#pragma unroll
+      for (int h = 0; h < B_K / 64; ++h) {
+        uint32_t q16[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) q16[j] = pk[h * 16 + j];
+        tmem_st_16x128b_x8(tS + h * 32, q16);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[st]);
+      if (cq == 0) {
+        if (liveA && hA >= goff && hA < goff + p.G)
+          p.c.part_lse[static_cast<int64_t>(slotA) * p.G + (hA - goff)] = mA * p.scale + logf(lA);
+        if (liveB && hB >= goff && hB < goff + p.G)
+          p.c.part_lse[static_cast<int64_t>(slotB) * p.G + (hB - goff)] = mB * p.scale + logf(lB);
+      }
+      if (more && !early) ok = load_s(n + 1, false);
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == 5) {
     tc_fence_after();
     tmem_dealloc(tmem_base, 512);
   }
@@ -895,8 +1124,8 @@ __global__ void __launch_bounds__(256) attn_merge_small_kernel(const MergeParams
 template <int D_H, int B_K>
 size_t p1_smem_bytes() {
   using SH = P1Shape<D_H, B_K>;
-  return 1024 + SH::QS * SH::QP_BYTES + SH::NKV * (SH::K_BYTES + SH::V_BYTES) +
-         SH::QS * sizeof(TileInfo) + (2 * SH::QS + 2 * SH::NKV + 8) * 8 + 16;
+  return 1024 + SH::QS * SH::Q_BYTES + SH::NKV * (SH::K_BYTES + SH::V_BYTES) +
+         kIR * sizeof(TileInfo) + (2 * SH::QS + 2 * SH::NKV + 2 * kIR + 4 * kNS + 1) * 8 + 16;
 }
 
 template <int D_H, int B_K>
@@ -905,10 +1134,10 @@ cudaError_t launch_typed(const AttnLaunch& a, cudaStream_t stream) {
   const int R = rows_per_query(G);
   const int Tq = kRowsPerTile / R;
   const int64_t B = (a.N + a.B_k - 1) / a.B_k;
-  const int64_t nkeys = a.H_kv * B;
   const int64_t Nc = chunk_len(a.N, a.B_k);
+  const int64_t nkeys_max = inv_nkeys(Nc, kWindow, a.H_kv, B);  // per chunk, at most
   size_t need = 0;
-  ChunkBufs c = carve(a.ws, Nc, a.H_q, a.H_kv, a.d_h, a.kk, nkeys, &need);
+  ChunkBufs c = carve(a.ws, Nc, a.H_q, a.H_kv, a.d_h, a.kk, nkeys_max, &need);
   if (need > a.ws_bytes) return cudaErrorInvalidValue;
 
   CUtensorMap tq, tk, tv;
@@ -948,11 +1177,12 @@ cudaError_t launch_typed(const AttnLaunch& a, cudaStream_t stream) {
   const int sms = num_sms();
   size_t hist_bytes = 0;
   int hist_grid = 0;
-  e = inv_setup(nkeys, sms, &hist_bytes, &hist_grid);
+  e = inv_setup(a.H_kv * B, sms, &hist_bytes, &hist_grid);
   if (e != cudaSuccess) return e;
 
   for (int64_t q0 = 0; q0 < a.N; q0 += Nc) {
     const int64_t nq = (a.N - q0) < Nc ? (a.N - q0) : Nc;
+    const int64_t nkeys = inv_nkeys(nq, kWindow, a.H_kv, B);
     e = cudaMemsetAsync(c.counts, 0, sizeof(int32_t) * nkeys, stream);
     if (e != cudaSuccess) return e;
     InvParams ip;
@@ -964,6 +1194,8 @@ cudaError_t launch_typed(const AttnLaunch& a, cudaStream_t stream) {
     ip.kk = a.kk;
     ip.B = B;
     ip.Tq = Tq;
+    ip.Cw = kWindow;
+    ip.W = static_cast<int>((nq + kWindow - 1) / kWindow);
     ip.c = c;
     ip.status = a.status;
     launch_inv_index(ip, hist_bytes, hist_grid, sms, stream);
@@ -978,13 +1210,14 @@ cudaError_t launch_typed(const AttnLaunch& a, cudaStream_t stream) {
     pp.G = G;
     pp.R = R;
     pp.Tq = Tq;
+    pp.B = static_cast<int>(B);
     pp.nkeys = nkeys;
     pp.scale = a.scale;
     pp.scale_log2 = a.scale * 1.4426950408889634f;
     pp.c = c;
     pp.status = a.status;
     prof_begin("attn_phase1", stream);
-    attn_phase1_kernel<D_H, B_K><<<sms, kThreads, smem, stream>>>(tq, tk, tv, pp);
+    attn_phase1_kernel<D_H, B_K><<<sms, kP1Threads, smem, stream>>>(tq, tk, tv, pp);
     prof_end(stream);
 
     MergeParams mp;
@@ -1228,6 +1461,8 @@ cudaError_t launch_idx_lse_typed(const IdxLseLaunch& a, cudaStream_t stream) {
     ip.kk = a.kk;
     ip.B = B;
     ip.Tq = kLseTile;
+    ip.Cw = static_cast<int>(Nc);  // one window: keys (group, block)
+    ip.W = 1;
     ip.c = c;
     ip.status = a.status;
     launch_inv_index(ip, hist_bytes, hist_grid, sms, stream);
@@ -1277,7 +1512,8 @@ cudaError_t launch_idx_lse(const IdxLseLaunch& a, cudaStream_t s) {
 size_t attn_workspace_bytes(int64_t N, int H_q, int H_kv, int d_h, int B_k, int kk) {
   const int64_t B = (N + B_k - 1) / B_k;
   size_t total = 0;
-  carve(nullptr, chunk_len(N, B_k), H_q, H_kv, d_h, kk, H_kv * B, &total);
+  const int64_t Nc = chunk_len(N, B_k);
+  carve(nullptr, Nc, H_q, H_kv, d_h, kk, inv_nkeys(Nc, kWindow, H_kv, B), &total);
   return total;
 }
 

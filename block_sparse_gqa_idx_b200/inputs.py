@@ -9,7 +9,9 @@ Workload shapes follow the pages' setting (B_k = 128, k = 16, G = H_q/H_kv
 adjacent query heads per KV head; xllm-io review, "实验设置" table; chlience
 notes, 5.1) at the sizes listed in ``CONFIGS``.  The planted structure is:
 
-* ``iid``: every tensor i.i.d. N(0, 1).
+* ``iid``: every tensor i.i.d. N(0, 1).  Q, K and V are drawn in blocks of
+  2^24 values, each block from its own child stream of the tensor's seed
+  (so they can be drawn in parallel).
 * ``sink_ar1``: Q, K, V i.i.d. N(0, 1).  Q_idx (each group) and K_idx follow
   an AR(1) process along the sequence, x_0 = e_0, x_i = rho x_{i-1} +
   sqrt(1 - rho^2) e_i (rho = 0.9, N(0,1) marginals), for locality.  A seeded
@@ -135,6 +137,28 @@ def _normal_bf16(rng: np.random.Generator, shape) -> np.ndarray:
     return out.reshape(shape)
 
 
+def _normal_bf16_blocks(seq: np.random.SeedSequence, shape) -> np.ndarray:
+    """i.i.d. N(0,1) as bf16 bits, drawn in blocks of _CHUNK elements, block j
+    from its own stream seq.spawn(...)[j], so the blocks are drawn in
+    parallel threads and the values do not depend on the thread count."""
+    import os
+    from concurrent.futures import ThreadPoolExecutor
+
+    n = int(np.prod(shape))
+    out = np.empty(n, dtype=np.uint16)
+    starts = list(range(0, n, _CHUNK))
+    seqs = seq.spawn(len(starts))
+
+    def fill(j):
+        s = starts[j]
+        e = min(n, s + _CHUNK)
+        out[s:e] = bf16_bits(np.random.default_rng(seqs[j]).standard_normal(e - s, dtype=np.float32))
+
+    with ThreadPoolExecutor(max_workers=min(len(starts), os.cpu_count() or 1)) as ex:
+        list(ex.map(fill, range(len(starts))))
+    return out.reshape(shape)
+
+
 def _ar1(rng: np.random.Generator, n: int, c: int, rho: float) -> np.ndarray:
     """AR(1) along axis 0 with N(0,1) marginals: [n, c] float32."""
     from scipy.signal import lfilter
@@ -160,16 +184,18 @@ def prefill_inputs(cfg: MSAConfig, seed: Optional[int] = None) -> Dict[str, np.n
     from concurrent.futures import ThreadPoolExecutor
 
     ss = np.random.SeedSequence(cfg.seed if seed is None else seed)
-    r_q, r_k, r_v, r_qi, r_ki, r_s = (np.random.default_rng(s) for s in ss.spawn(6))
+    s_q, s_k, s_v, s_qi, s_ki, s_s = ss.spawn(6)
+    r_qi, r_ki, r_s = (np.random.default_rng(s) for s in (s_qi, s_ki, s_s))
     N, H_q, H_kv, d_h, d_idx = cfg.N, cfg.H_q, cfg.H_kv, cfg.d_h, cfg.d_idx
     if cfg.structure not in ("iid", "sink_ar1", "sink_ar1_retrieval"):
         raise ValueError(f"unknown structure {cfg.structure!r}")
     iid = cfg.structure == "iid"
     # the tensors draw from independent streams: generate them concurrently
+    # (Q, K and V block by block, each block from its own stream)
     jobs = {
-        "q": lambda: _normal_bf16(r_q, (N, H_q, d_h)),
-        "k": lambda: _normal_bf16(r_k, (N, H_kv, d_h)),
-        "v": lambda: _normal_bf16(r_v, (N, H_kv, d_h)),
+        "q": lambda: _normal_bf16_blocks(s_q, (N, H_q, d_h)),
+        "k": lambda: _normal_bf16_blocks(s_k, (N, H_kv, d_h)),
+        "v": lambda: _normal_bf16_blocks(s_v, (N, H_kv, d_h)),
         "qi": (lambda: _normal_bf16(r_qi, (N, H_kv, d_idx))) if iid
         else (lambda: _ar1(r_qi, N, H_kv * d_idx, 0.9).reshape(N, H_kv, d_idx)),
         "ki": (lambda: _normal_bf16(r_ki, (N, d_idx))) if iid

@@ -16,7 +16,7 @@ SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
 def test_traffic_figures_match_the_current_kernels():
     for name in bench.NCU_TRAFFIC:
         traffic, where = bench.ncu_traffic(name, 131072)
-        assert traffic is not None and traffic > 0 and where.startswith("profiles/"), name
+        assert traffic is not None and traffic > 0 and "ncu capture" in where, name
 
 
 def test_kernel_hash_ignores_comments_and_other_code():
