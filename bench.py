@@ -7,13 +7,17 @@ synthetic inputs with a sink block and retrieval blocks).  Inputs (Q alone is
 1.07 GB) are larger than the 126 MB L2, so no flush is needed between steps.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl msa|reference]
-                    [--workload 128k|32k|1m|decode|decode8]
+                    [--workload 128k|32k|1m|decode|decode8] [--no-also]
 
-For N > 1 each rank runs an independent replica (its own sequence): the path
-has no exchange step, so there is no collective on the data path; timing is
-the max over ranks and ``value`` is the tokens of all ranks per second.
-``--impl reference`` times the CPU oracle on a bounded row sample instead.
-Prints one JSON line on rank 0.
+On one GPU the 128K line also carries, under "also", the other two parts of
+the metric, each measured the same way: the 1M-token prefill ("1m", 3 steps
+after 2 warm-up steps) and the 64-sequence decode workload ("decode", 200
+steps after 10 warm-up steps, us per token).  For N > 1 each rank runs an
+independent replica (its own sequence): the path has no exchange step, so
+there is no collective on the data path; timing is the max over ranks and
+``value`` is the tokens of all ranks per second.  ``--impl reference`` times
+the CPU oracle on a bounded sample instead (query rows of the prefill, or a
+few sequences of the decode workload).  Prints one JSON line on rank 0.
 """
 from __future__ import annotations
 
@@ -104,8 +108,9 @@ class Clocks:
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, device_index: int):
+    def __init__(self, device_index: int, interval_ms: int = 20):
         self.dev = device_index
+        self.interval = interval_ms
         self.proc = None
         self.path = None
 
@@ -115,9 +120,17 @@ class Clocks:
             os.close(fd)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
-                 "-lms", "20"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+                 "-lms", str(self.interval)], stdout=open(self.path, "w"),
+                stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
+            return
+        # wait (up to 3 s) for the first sample, so a short timed region is
+        # not over before the sampler has started
+        t0 = time.time()
+        while time.time() - t0 < 3.0 and os.path.getsize(self.path) == 0:
+            time.sleep(0.01)
+        self.skip = sum(1 for _ in open(self.path))
 
     def stop(self):
         if self.proc is None:
@@ -129,9 +142,9 @@ class Clocks:
             self.proc.kill()
         rows = []
         with open(self.path) as f:
-            for line in f:
+            for n, line in enumerate(f):
                 p = [x.strip() for x in line.split(",")]
-                if len(p) >= 9:
+                if n >= getattr(self, "skip", 0) and len(p) >= 9:
                     rows.append(p)
         os.unlink(self.path)
         if not rows:
@@ -181,6 +194,7 @@ def flops_of(cfg):
 
 # ------------------------------------------------------------ reference arm --
 def run_reference(args, cfg, rank, world):
+    """The CPU oracle on a bounded row sample of the prefill workload."""
     if rank != 0:
         return 0
     import oracle
@@ -217,11 +231,69 @@ def run_reference(args, cfg, rank, world):
     return 0
 
 
-METRIC = "MSA fwd prefill tokens/s @128K & 1M, % bf16 TC peak; decode \u00b5s/token, % HBM BW"
+def decode_oracle_sample(st, cfg, n_seq: int, step: int = 0):
+    """Time the oracle's decode step (append + Eq. 6-8 for the new token) on
+    the first n_seq sequences of a decode state: (us per token, seconds, cores)."""
+    import oracle
+    from block_sparse_gqa_idx_b200 import inputs
+
+    si = inputs.decode_step_inputs(cfg, step, st["sink"])
+    seqs = list(range(min(n_seq, cfg.S)))
+    t0 = time.perf_counter()
+    oracle.decode_reference(st, si, cfg.B_k, cfg.k, seqs=seqs)
+    dt = time.perf_counter() - t0
+    return 1e6 * dt / len(seqs), dt, oracle.max_threads()
+
+
+def run_reference_decode(args, cfg, rank, world):
+    """The CPU oracle's decode step on a few sequences of the decode workload."""
+    if rank != 0:
+        return 0
+    from block_sparse_gqa_idx_b200 import inputs
+
+    st = inputs.decode_state(cfg)
+    n_seq = args.ref_seqs
+    times = []
+    for it in range(args.warmup + args.steps):
+        us, dt, cores = decode_oracle_sample(st, cfg, n_seq, step=it)
+        if it >= args.warmup:
+            times.append(us)
+    us = statistics.mean(times)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": us, "unit": "us/token",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": us * n_seq * 1e-3, "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": cfg.name, "S": cfg.S, "L0": cfg.L0, "H_q": cfg.H_q,
+                   "H_kv": cfg.H_kv, "d_h": cfg.d_h, "d_idx": cfg.d_idx, "B_k": cfg.B_k,
+                   "k": cfg.k, "parallelism": f"replicas x{world}", "seqs_per_step": n_seq},
+        "cpu_baseline": {"value": us, "unit": "us/token", "cores": cores, "kind": "oracle",
+                         "sample": f"{n_seq} of the {cfg.S} sequences per step (one token each, "
+                                   f"full cache scan)"},
+        "e2e": {"value": us, "unit": "us/token", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+METRIC = "MSA fwd prefill tokens/s @128K & 1M, % bf16 TC peak; decode µs/token, % HBM BW"
+
+
+def tensor_roofline(work_flop: float, per_launch_ms: float, pk: dict, pk_kind: str) -> dict:
+    """Achieved TFLOP/s of one launch against the measured burst bf16 peak
+    (the headline fraction) and, as a second figure, the sustained one."""
+    achieved = work_flop / (per_launch_ms * 1e-3) / 1e12
+    return {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"],
+            "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"],
+            "peak_kind": f"{pk_kind} burst",
+            "frac_of_sustained": achieved / pk["bf16_tflops_sustained"]}
 
 
 # ----------------------------------------------------------------- msa arm --
-def run_msa(args, cfg, rank, world, local):
+def run_msa(args, cfg, rank, world, local, steps, warmup, e2e_steps, cpu_rows):
+    """Time `steps` prefill forwards of one sequence per rank; returns the JSON
+    line on rank 0 (None elsewhere)."""
     import torch
     import torch.distributed as dist
 
@@ -233,7 +305,9 @@ def run_msa(args, cfg, rank, world, local):
     stream = torch.cuda.current_stream(dev)
 
     # every replica gets its own seeded sequence
+    t_gen = time.time()
     inp = inputs.prefill_inputs(cfg, seed=cfg.seed + 1000 * rank)
+    gen_s = time.time() - t_gen
     host = {k: torch.from_numpy(np.ascontiguousarray(v).view(np.int16)).view(torch.bfloat16)
             for k, v in inp.items()}
     d = {k: v.to(dev) for k, v in host.items()}
@@ -247,21 +321,21 @@ def run_msa(args, cfg, rank, world, local):
                          msa.index_lse_workspace_size(dims)), dtype=torch.uint8, device=dev)
     lse_idx = torch.empty((N, H_kv), dtype=torch.float32, device=dev) if args.kl_lse else None
 
-    def step(src):
-        msa.index_topk(src["q_idx"], src["k_idx"], B_k, kk, idx_out=idx, workspace=ws,
+    def step(src, o_, idx_, lse_):
+        msa.index_topk(src["q_idx"], src["k_idx"], B_k, kk, idx_out=idx_, workspace=ws,
                        stream=stream)
-        msa.sparse_attn_fwd(src["q"], src["k"], src["v"], idx, B_k, o=o, lse=lse, workspace=ws,
-                            stream=stream)
+        msa.sparse_attn_fwd(src["q"], src["k"], src["v"], idx_, B_k, o=o_, lse=lse_,
+                            workspace=ws, stream=stream)
         if args.kl_lse:  # the KL-loss fusion's Index Branch normaliser (training forward)
-            msa.index_lse(src["q_idx"], src["k_idx"], idx, B_k, lse_idx=lse_idx, workspace=ws,
+            msa.index_lse(src["q_idx"], src["k_idx"], idx_, B_k, lse_idx=lse_idx, workspace=ws,
                           stream=stream)
 
     def barrier():
         if world > 1:
             dist.barrier()
 
-    for _ in range(args.warmup):
-        step(d)
+    for _ in range(warmup):
+        step(d, o, idx, lse)
     torch.cuda.synchronize()
     code, where = msa.device_status(ws)
     if code != 0:
@@ -274,16 +348,19 @@ def run_msa(args, cfg, rank, world, local):
     msa.profile_enable(True)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(args.steps):
-        step(d)
+    for _ in range(steps):
+        step(d, o, idx, lse)
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
     msa.profile_enable(False)
     clk = clocks.stop()
     prof = msa.profile_read()
-    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dev, world)
+    ms = max_over_ranks(e0.elapsed_time(e1) / steps, dev, world)
     value = aggregate_tokens_per_s(world, N, ms)
+    code, where = msa.device_status(ws)
+    if code != 0:
+        raise RuntimeError(f"device status {code} at {where} after the timed steps")
 
     # ---- end to end: pinned host inputs -> device -> forward -> host result.
     # Every step uploads its inputs from pinned host memory and downloads its
@@ -295,7 +372,6 @@ def run_msa(args, cfg, rank, world, local):
     outs = [(o, idx, lse), (torch.empty_like(o), torch.empty_like(idx), torch.empty_like(lse))]
     o_host = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for _ in range(2)]
     idx_host = [torch.empty(idx.shape, dtype=idx.dtype).pin_memory() for _ in range(2)]
-    e2e_steps = max(2, min(args.steps, 6))
     h2d = sum(v.numel() * v.element_size() for v in pinned.values())
     d2h = o.numel() * o.element_size() + idx.numel() * idx.element_size()
     up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
@@ -318,13 +394,7 @@ def run_msa(args, cfg, rank, world, local):
             stream.wait_event(ev_in[b])
             stream.wait_event(ev_read[b])
             ob, ib, lb = outs[b]
-            msa.index_topk(bufs[b]["q_idx"], bufs[b]["k_idx"], B_k, kk, idx_out=ib, workspace=ws,
-                           stream=stream)
-            msa.sparse_attn_fwd(bufs[b]["q"], bufs[b]["k"], bufs[b]["v"], ib, B_k, o=ob, lse=lb,
-                                workspace=ws, stream=stream)
-            if args.kl_lse:
-                msa.index_lse(bufs[b]["q_idx"], bufs[b]["k_idx"], ib, B_k, lse_idx=lse_idx,
-                              workspace=ws, stream=stream)
+            step(bufs[b], ob, ib, lb)
             ev_used[b].record(stream)
             ev_out[b].record(stream)
             with torch.cuda.stream(down):
@@ -345,9 +415,9 @@ def run_msa(args, cfg, rank, world, local):
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(f0.elapsed_time(f1) / e2e_steps, dev, world)
     barrier()
-
+    del pinned, bufs, outs, o_host, idx_host
     if rank != 0:
-        return 0
+        return None
 
     # ---- roofline of the dominant kernel (live CUDA-event durations)
     pk, pk_kind = peaks()
@@ -356,58 +426,56 @@ def run_msa(args, cfg, rank, world, local):
     dom = max(prof, key=lambda n: prof[n][1])
     launches, dom_ms = prof[dom]
     per_launch_ms = dom_ms / launches
-    # a kernel inside a timed region of about a second or more runs under the
-    # power cap: its denominator is the sustained GEMM rate, else the burst one
-    sustained = ms * args.steps >= 1000.0
-    tc_peak = pk["bf16_tflops_sustained"] if sustained else pk["bf16_tflops"]
-    tc_kind = "sustained" if sustained else "burst"
     if dom == "index_topk":
-        work, unit, bound = f_idx, "TFLOP/s", "tensor"
-        achieved = work / (per_launch_ms * 1e-3) / 1e12
-        peak = tc_peak
+        roofline = tensor_roofline(f_idx, per_launch_ms, pk, pk_kind)
     elif dom == "attn_phase1":
         # one launch per query chunk and step: the Main Branch FLOPs of a chunk
-        work = f_main / (launches / args.steps)
-        unit, bound = "TFLOP/s", "tensor"
-        achieved = work / (per_launch_ms * 1e-3) / 1e12
-        peak = tc_peak
+        roofline = tensor_roofline(f_main / (launches / steps), per_launch_ms, pk, pk_kind)
     else:
-        unit, bound = "GB/s", "hbm"
-        achieved, peak = None, pk["hbm_gbs"]
-    traffic, traffic_src = ncu_traffic(dom, N / (launches / args.steps))
-    roofline = {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
-                "frac": (achieved / peak) if achieved else None, "traffic": traffic,
-                "traffic_source": traffic_src, "peak_kind": f"{pk_kind} {tc_kind}",
+        roofline = {"bound": "hbm", "achieved": None, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                    "frac": None, "peak_kind": pk_kind}
+    traffic, traffic_src = ncu_traffic(dom, N / (launches / steps))
+    roofline = {"kernel": dom, **roofline, "traffic": traffic, "traffic_source": traffic_src,
                 "share": dom_ms / total_ms if total_ms else None}
+    # each tensor-bound kernel against the same peak
+    per_kernel = {}
+    for name, work in (("index_topk", f_idx), ("attn_phase1", f_main)):
+        if name in prof:
+            nl, tms = prof[name]
+            per_kernel[name] = tensor_roofline(work / (nl / steps), tms / nl, pk, pk_kind)
 
     # ---- CPU oracle on a bounded sample (rank 0, N=1 only)
     cpu = None
-    if world == 1 and not args.no_cpu_baseline:
+    if world == 1 and cpu_rows > 0:
         import oracle
 
         rng = np.random.default_rng(11)
-        rows = np.sort(rng.choice(N, size=args.cpu_rows, replace=False))
+        rows = np.sort(rng.choice(N, size=cpu_rows, replace=False))
         t0 = time.perf_counter()
         oracle.forward(inp, B_k, kk, rows=rows)
         dt = time.perf_counter() - t0
-        cpu = {"value": args.cpu_rows / dt, "unit": "tokens/s", "cores": oracle.max_threads(),
+        cpu = {"value": cpu_rows / dt, "unit": "tokens/s", "cores": oracle.max_threads(),
                "kind": "oracle",
-               "sample": f"{args.cpu_rows} uniformly drawn query rows of the {cfg.name} workload "
+               "sample": f"{cpu_rows} uniformly drawn query rows of the {cfg.name} workload "
                          f"(index + attention, full causal prefix), {dt:.1f} s"}
 
-    kernels = {n: {"launches": v[0], "ms_per_step": v[1] / args.steps,
+    kernels = {n: {"launches": v[0], "ms_per_step": v[1] / steps,
                    "share": v[1] / total_ms if total_ms else None} for n, v in prof.items()}
-    line = {
+    # time between kernels: the step time minus the kernels' summed event time
+    idle = max(0.0, ms - total_ms / steps)
+    return {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "steps": steps, "warmup": warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
         "config": {"workload": cfg.name, "N": N, "H_q": H_q, "H_kv": H_kv, "d_h": d_h,
                    "d_idx": d_idx, "B_k": B_k, "k": kk, "parallelism": f"replicas x{world}",
-                   "l2": "inputs larger than L2 (Q alone 1.07 GB); no flush",
+                   "l2": "inputs larger than L2 (Q alone %.2f GB); no flush"
+                         % (N * H_q * d_h * 2 / 1e9),
                    "kl_lse": bool(args.kl_lse)},
         "tc_frac_eq12": (f_idx + f_main) / (ms * 1e-3) / 1e12 / pk["bf16_tflops"],
         "roofline": roofline,
+        "roofline_per_kernel": per_kernel,
         "cpu_baseline": cpu,
         "e2e": {"value": aggregate_tokens_per_s(world, N, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
@@ -416,17 +484,18 @@ def run_msa(args, cfg, rank, world, local):
                         "neighbouring steps overlap compute on two copy streams"},
         "gpu_launches": sum(v[0] for v in prof.values()),
         "kernels": kernels,
+        "idle_ms_per_step": idle, "idle_frac": idle / ms if ms else None,
         "clocks": clk,
+        "input_generation_s": gen_s,
     }
-    print(json.dumps(line), flush=True)
-    return 0
 
 
 # -------------------------------------------------------------- decode arm --
-def run_decode(args, cfg, rank, world, local):
+def run_decode(args, cfg, rank, world, local, steps, warmup, e2e_steps, cpu_seqs):
     """Decode workload: S sequences, one new token each per step (append +
-    index scan + Top-k + gathered attention).  Reports us per step and per
-    token, and the HBM roofline of the step from its algorithmic bytes."""
+    index scan + Top-k + gathered attention).  Reports us per token (the step
+    time divided by the sequences of all ranks), us per step, and the HBM
+    roofline of the step from its algorithmic bytes; returns the line on rank 0."""
     import torch
 
     import block_sparse_gqa_idx_b200 as msa
@@ -444,18 +513,17 @@ def run_decode(args, cfg, rank, world, local):
 
     caches = {k: dv(st[k]) for k in ("k_cache", "v_cache", "k_idx_cache")}
     seq_len = torch.from_numpy(st["seq_len"]).to(dev)
-    n_steps = args.warmup + args.steps
+    n_steps = warmup + steps + e2e_steps
     assert n_steps <= cfg.steps, "more steps than the cache has room for"
-    steps_in = [{k: dv(v) for k, v in inputs.decode_step_inputs(cfg, j, st["sink"]).items()}
-                for j in range(n_steps)]
+    host_in = [inputs.decode_step_inputs(cfg, j, st["sink"]) for j in range(n_steps)]
+    steps_in = [{k: dv(v) for k, v in h.items()} for h in host_in[:warmup + steps]]
     S, H_q, H_kv, d_h, d_idx, B_k, kk = cfg.S, cfg.H_q, cfg.H_kv, cfg.d_h, cfg.d_idx, cfg.B_k, cfg.k
     o = torch.empty((S, H_q, d_h), dtype=torch.bfloat16, device=dev)
     idx = torch.empty((S, H_kv, kk), dtype=torch.int32, device=dev)
     dd = msa.decode_dims(S, cfg.L_max, H_q, H_kv, d_h, d_idx, B_k, kk)
     ws = torch.empty(msa.sparse_decode_workspace_size(dd), dtype=torch.uint8, device=dev)
 
-    def step(j):
-        x = steps_in[j]
+    def step(x):
         msa.sparse_decode(x["q"], x["q_idx"], x["k_new"], x["v_new"], x["k_idx_new"],
                           caches["k_cache"], caches["v_cache"], caches["k_idx_cache"], seq_len,
                           B_k, kk, o=o, idx_out=idx, workspace=ws, stream=stream)
@@ -466,19 +534,19 @@ def run_decode(args, cfg, rank, world, local):
 
             dist.barrier()
 
-    for j in range(args.warmup):
-        step(j)
+    for j in range(warmup):
+        step(steps_in[j])
     torch.cuda.synchronize()
     L_before = seq_len.clone()
-    clocks = Clocks(local)
+    clocks = Clocks(local, interval_ms=10)
     barrier()
     torch.cuda.synchronize()
     clocks.start()
     msa.profile_enable(True)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for j in range(args.warmup, n_steps):
-        step(j)
+    for j in range(warmup, warmup + steps):
+        step(steps_in[j])
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
@@ -486,13 +554,13 @@ def run_decode(args, cfg, rank, world, local):
     clk = clocks.stop()
     prof = msa.profile_read()
     # the slowest replica's step time; every rank's S sequences got a token
-    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dev, world)
+    ms = max_over_ranks(e0.elapsed_time(e1) / steps, dev, world)
     code, where = msa.device_status(ws)
     if code != 0:
         raise RuntimeError(f"device status {code} at {where}")
     # algorithmic bytes per step: the K_idx scan of every cached token, the
     # selected K and V rows (causal part of each block), the new rows and q/o
-    L = L_before.double().mean().item() + (args.steps - 1) / 2.0
+    L = L_before.double().mean().item() + (steps - 1) / 2.0
     sel_rows = 0.0
     sel = idx.cpu().numpy()
     Lend = seq_len.cpu().numpy()
@@ -504,17 +572,48 @@ def run_decode(args, cfg, rank, world, local):
                     sel_rows += min(B_k, Li - int(b) * B_k)
     bytes_step = (S * L * d_idx * 2 + sel_rows * d_h * 2 * 2
                   + S * (H_q * d_h * 2 * 2 + H_kv * d_idx * 2 + H_kv * d_h * 2 * 2 * 2 + d_idx * 2 * 2))
+
+    # ---- end to end: each step's new rows from pinned host memory, the
+    # step, and O and the selection back to pinned host memory
+    pinned = [{k: torch.from_numpy(np.ascontiguousarray(v).view(np.int16)).view(torch.bfloat16)
+               .pin_memory() for k, v in h.items()} for h in host_in[warmup + steps:]]
+    dev_in = {k: torch.empty_like(v, device=dev) for k, v in pinned[0].items()}
+    o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    idx_host = torch.empty(idx.shape, dtype=idx.dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in pinned[0].values())
+    d2h = o.numel() * o.element_size() + idx.numel() * idx.element_size()
+    torch.cuda.synchronize()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for x in pinned:
+        for k, v in x.items():
+            dev_in[k].copy_(v, non_blocking=True)
+        step(dev_in)
+        o_host.copy_(o, non_blocking=True)
+        idx_host.copy_(idx, non_blocking=True)
+    f1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(f0.elapsed_time(f1) / max(1, len(pinned)), dev, world)
+    if rank != 0:
+        return None
     pk, pk_kind = peaks()
     gbs = bytes_step / (ms * 1e-3) / 1e9
     cache_gb = S * cfg.L_max * (2 * H_kv * d_h + d_idx) * 2 / 1e9
     total_ms = sum(v[1] for v in prof.values())
-    kernels = {n: {"launches": v[0], "ms_per_step": v[1] / args.steps,
+    kernels = {n: {"launches": v[0], "ms_per_step": v[1] / steps,
                    "share": v[1] / total_ms if total_ms else None} for n, v in prof.items()}
-    scan_ms = prof.get("dec_scan", (1, 0.0))[1] / args.steps
+    scan_ms = prof.get("dec_scan", (1, 0.0))[1] / steps
     scan_bytes = S * L * d_idx * 2
-    line = {
+    cpu = None
+    if world == 1 and cpu_seqs > 0:
+        us_cpu, dt_cpu, cores = decode_oracle_sample(st, cfg, cpu_seqs)
+        cpu = {"value": us_cpu, "unit": "us/token", "cores": cores, "kind": "oracle",
+               "sample": f"{cpu_seqs} of the {S} sequences, one decode step each (append, "
+                         f"full K_idx scan, Top-k, attention), {dt_cpu:.1f} s"}
+    idle = max(0.0, ms - total_ms / steps)
+    return {
         "metric": METRIC, "value": 1e3 * ms / (S * world),
-        "unit": "us/token", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "unit": "us/token", "n_gpus": world, "steps": steps, "warmup": warmup,
         "ms_per_step": ms, "us_per_step": 1e3 * ms, "higher_is_better": False,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": cfg.name, "S": S, "L": L, "H_q": H_q, "H_kv": H_kv, "d_h": d_h,
@@ -524,12 +623,24 @@ def run_decode(args, cfg, rank, world, local):
                      "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": gbs / pk["hbm_gbs"],
                      "traffic": None, "bytes_per_step": bytes_step, "peak_kind": pk_kind,
                      "scan_kernel_gbs": scan_bytes / (scan_ms * 1e-3) / 1e9 if scan_ms else None},
-        "gpu_launches": sum(v[0] for v in prof.values()), "kernels": kernels, "clocks": clk,
-        "input_generation_s": gen_s,
+        "cpu_baseline": cpu,
+        "e2e": {"value": 1e3 * e2e_ms / (S * world), "unit": "us/token",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "us_per_step": 1e3 * e2e_ms, "steps": len(pinned),
+                "note": "each step's new rows from pinned host memory, the step, and O and "
+                        "the selection back to pinned host memory, in stream order"},
+        "gpu_launches": sum(v[0] for v in prof.values()), "kernels": kernels,
+        "idle_ms_per_step": idle, "clocks": clk, "input_generation_s": gen_s,
     }
-    if rank == 0:
-        print(json.dumps(line), flush=True)
-    return 0
+
+
+def free_device_memory():
+    import gc
+
+    import torch
+
+    gc.collect()
+    torch.cuda.empty_cache()
 
 
 def main():
@@ -541,20 +652,25 @@ def main():
     ap.add_argument("--workload", default="128k")
     ap.add_argument("--cpu-rows", type=int, default=0, help="0: 256, or 32 at 1M tokens")
     ap.add_argument("--ref-rows", type=int, default=32)
+    ap.add_argument("--ref-seqs", type=int, default=2,
+                    help="sequences per step of the decode reference arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-also", action="store_true",
+                    help="time only --workload (by default the 128K line also carries the "
+                         "1M prefill and the decode workload)")
     ap.add_argument("--kl-lse", action="store_true",
                     help="add the KL-loss fusion's LSE_idx to every step (a training forward)")
     args = ap.parse_args()
     world, rank, local = dist_init()
     cfg = workload(args.workload)
+    is_decode = args.workload.startswith("decode")
     if args.cpu_rows == 0:
         args.cpu_rows = 32 if getattr(cfg, "N", 0) >= (1 << 20) else 256
+    if args.no_cpu_baseline:
+        args.cpu_rows = 0
     if args.impl == "reference":
-        if args.workload.startswith("decode"):
-            if rank == 0:
-                print(json.dumps({"impl": "reference",
-                                  "unavailable": "decode reference arm not provided"}))
-            return 0
+        if is_decode:
+            return run_reference_decode(args, cfg, rank, world)
         return run_reference(args, cfg, rank, world)
     if world > 1:
         import datetime
@@ -565,9 +681,29 @@ def main():
         torch.cuda.set_device(local)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     try:
-        if args.workload.startswith("decode"):
-            return run_decode(args, cfg, rank, world, local)
-        return run_msa(args, cfg, rank, world, local)
+        if is_decode:
+            line = run_decode(args, cfg, rank, world, local, args.steps, args.warmup, 8,
+                              0 if args.no_cpu_baseline else 4)
+        else:
+            e2e_steps = 2 if cfg.N >= (1 << 20) else max(2, min(args.steps, 6))
+            line = run_msa(args, cfg, rank, world, local, args.steps, args.warmup, e2e_steps,
+                           args.cpu_rows)
+        # the other two parts of the metric, on one GPU: the 1M-token prefill
+        # and the decode workload, each a nested line of its own
+        if world == 1 and args.workload == "128k" and not args.no_also and not args.kl_lse:
+            also = {}
+            free_device_memory()
+            c1m = workload("1m")
+            also["1m"] = run_msa(args, c1m, rank, world, local, steps=3, warmup=2, e2e_steps=2,
+                                 cpu_rows=0 if args.no_cpu_baseline else 32)
+            free_device_memory()
+            cdec = workload("decode")
+            also["decode"] = run_decode(args, cdec, rank, world, local, steps=200, warmup=10,
+                                        e2e_steps=8, cpu_seqs=0 if args.no_cpu_baseline else 4)
+            line["also"] = also
+        if rank == 0 and line is not None:
+            print(json.dumps(line), flush=True)
+        return 0
     finally:
         if world > 1:
             import torch.distributed as dist
