@@ -62,7 +62,7 @@ def _load() -> ctypes.CDLL:
     D, DD = ctypes.POINTER(msa_dims), ctypes.POINTER(msa_decode_dims)
     lib.msa_index_topk_workspace.argtypes = [D]
     lib.msa_index_topk_workspace.restype = Z
-    lib.msa_index_topk.argtypes = [D, P, P, P, P, Z, P]
+    lib.msa_index_topk.argtypes = [D, P, P, P, P, P, Z, P]
     lib.msa_index_topk.restype = I32
     lib.msa_sparse_attn_fwd_workspace.argtypes = [D]
     lib.msa_sparse_attn_fwd_workspace.restype = Z
@@ -167,19 +167,24 @@ def sparse_decode_workspace_size(d: msa_decode_dims) -> int:
 
 def index_topk(q_idx: torch.Tensor, k_idx: torch.Tensor, B_k: int, k: int,
                idx_out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
-               stream=None) -> torch.Tensor:
-    """Eq. 6-7: q_idx [N,H_kv,d_idx] bf16, k_idx [N,d_idx] bf16 -> idx [N,H_kv,k] int32."""
+               stream=None, score_out: Optional[torch.Tensor] = None,
+               idx_scale: float = 0.0) -> torch.Tensor:
+    """Eq. 6-7: q_idx [N,H_kv,d_idx] bf16, k_idx [N,d_idx] bf16 -> idx [N,H_kv,k] int32.
+    If ``score_out`` ([N,H_kv,k] fp32) is given, it receives each selected
+    block's Eq. 6 score (scale ``idx_scale``, 0 -> 1/sqrt(d_idx)), -inf in -1 slots."""
     N, H_kv, d_idx = q_idx.shape
     _want(q_idx, "q_idx", torch.bfloat16, (N, H_kv, d_idx))
     _want(k_idx, "k_idx", torch.bfloat16, (N, d_idx))
     if idx_out is None:
         idx_out = torch.empty((N, H_kv, k), dtype=torch.int32, device=q_idx.device)
     _want(idx_out, "idx_out", torch.int32, (N, H_kv, k))
-    d = dims(N, H_kv, H_kv, 64, d_idx, B_k, k)
+    if score_out is not None:
+        _want(score_out, "score_out", torch.float32, (N, H_kv, k))
+    d = dims(N, H_kv, H_kv, 64, d_idx, B_k, k, idx_scale=idx_scale)
     ws = _workspace(index_topk_workspace_size(d), q_idx.device, workspace)
     _raise("msa_index_topk", LIB.msa_index_topk(ctypes.byref(d), _ptr(q_idx), _ptr(k_idx),
-                                                _ptr(idx_out), _ptr(ws), ws.numel(),
-                                                _stream(stream)))
+                                                _ptr(idx_out), _ptr(score_out), _ptr(ws),
+                                                ws.numel(), _stream(stream)))
     return idx_out
 
 

@@ -55,6 +55,8 @@ struct IndexParams {
   int H_kv, B_k, k;
   int n_mtiles;
   int32_t* idx_out;
+  float* score_out;  // [N, H_kv, k] or null: the selected blocks' Eq. 6 scores
+  float scale;       // Eq. 6 scale applied to score_out
   DevStatus* status;
 };
 
@@ -405,7 +407,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!mbar_wait(xch_full, ucnt & 1, abort_flag, p.status, 32)) break;
       int sel[32];
+      float scr[32];  // raw (unscaled) block scores; the local block's is written elsewhere
       int n = 0;
+      scr[n] = 0.0f;
       sel[n++] = c;  // the local block (Eq. 7: always kept)
       if constexpr (REG) {
         // both lists are sorted best first: a two-way merge
@@ -417,6 +421,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (kbest == 0ull) break;
           if (ka >= kb) ++ia;
           else ++ib;
+          scr[n] = unorder_key(kbest);
           sel[n++] = key_block(kbest);
         }
       } else {
@@ -430,6 +435,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (best == 0ull) break;
           taken_below = best;
+          scr[n] = unorder_key(best);
           sel[n++] = key_block(best);
         }
       }
@@ -439,15 +445,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (row_glob < p.N * p.H_kv) {
         for (int a = 1; a < n; ++a) {  // ascending
           const int x = sel[a];
+          const float xs = scr[a];
           int b = a - 1;
           while (b >= 0 && sel[b] > x) {
             sel[b + 1] = sel[b];
+            scr[b + 1] = scr[b];
             --b;
           }
           sel[b + 1] = x;
+          scr[b + 1] = xs;
         }
         int32_t* out = p.idx_out + row_glob * p.k;
         for (int s = 0; s < p.k; ++s) out[s] = s < n ? sel[s] : -1;
+        if (p.score_out != nullptr) {
+          // the local block (the largest index, so slot n - 1) is scored by
+          // local_block_score_kernel
+          float* so = p.score_out + row_glob * p.k;
+          for (int s = 0; s < p.k; ++s)
+            if (s != n - 1) so[s] = s < n ? scr[s] * p.scale : -INFINITY;
+        }
       }
     }
   }
@@ -457,6 +473,51 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+// score_out of each row's local block (its last valid slot, min(k, b_i + 1)
+// - 1): the Eq. 6 maximum over the block's keys j <= i, one warp per (query,
+// group), lane l scoring keys l, l + 32, ... of the block.
+template <int D_IDX>
+__global__ void __launch_bounds__(256) local_block_score_kernel(const __nv_bfloat16* q_idx,
+                                                                const __nv_bfloat16* k_idx,
+                                                                const IndexParams p) {
+  const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (row >= p.N * p.H_kv) return;
+  const int64_t i = row / p.H_kv;
+  const int64_t b_i = i / p.B_k;
+  float q[D_IDX];
+  const __nv_bfloat16* qr = q_idx + row * D_IDX;
+#pragma unroll
+  for (int d = 0; d < D_IDX; d += 2) {
+    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(qr + d));
+    q[d] = f.x;
+    q[d + 1] = f.y;
+  }
+  float m = -INFINITY;
+  for (int64_t j = b_i * p.B_k + lane; j <= i; j += 32) {
+    const __nv_bfloat16* kr = k_idx + j * D_IDX;
+    float dot = 0.0f;
+#pragma unroll
+    for (int d = 0; d < D_IDX; d += 8) {
+      const uint4 w = *reinterpret_cast<const uint4*>(kr + d);
+      const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(h[e]);
+        dot = fmaf(q[d + 2 * e], f.x, dot);
+        dot = fmaf(q[d + 2 * e + 1], f.y, dot);
+      }
+    }
+    m = fmaxf(m, dot);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+  if (lane == 0) {
+    const int64_t slot = (b_i + 1 < p.k ? b_i + 1 : p.k) - 1;
+    p.score_out[row * p.k + slot] = m * p.scale;
   }
 }
 
@@ -491,6 +552,8 @@ cudaError_t launch_typed(const IndexLaunch& a, cudaStream_t stream) {
   p.k = a.k;
   p.n_mtiles = static_cast<int>((a.N * a.H_kv + kRows - 1) / kRows);
   p.idx_out = a.idx_out;
+  p.score_out = a.score_out;
+  p.scale = a.scale;
   p.status = a.status;
   const bool reg = a.k <= 16;
   const size_t smem = index_smem_bytes<D_IDX>(a.k);
@@ -504,6 +567,13 @@ cudaError_t launch_typed(const IndexLaunch& a, cudaStream_t stream) {
   prof_begin("index_topk", stream);
   kern<<<grid, kThreads, smem, stream>>>(tq, tk, p);
   prof_end(stream);
+  if (a.score_out != nullptr) {
+    const int64_t threads = a.N * a.H_kv * 32;
+    prof_begin("local_block_score", stream);
+    local_block_score_kernel<D_IDX><<<static_cast<unsigned>((threads + 255) / 256), 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(a.q_idx), static_cast<const __nv_bfloat16*>(a.k_idx), p);
+    prof_end(stream);
+  }
   return cudaGetLastError();
 }
 

@@ -215,13 +215,15 @@ size_t msa_index_topk_workspace(const msa_dims* d) {
 }
 
 msa_status msa_index_topk(const msa_dims* d, const void* q_idx, const void* k_idx,
-                          int32_t* idx_out, void* ws, size_t ws_bytes, void* stream) {
+                          int32_t* idx_out, float* score_out, void* ws, size_t ws_bytes,
+                          void* stream) {
   if (d == nullptr || q_idx == nullptr || k_idx == nullptr || idx_out == nullptr || ws == nullptr)
     return MSA_ERR_INVALID_ARG;
   msa_status st = check_common(d->N, d->H_q, d->H_kv, 64, d->d_idx, d->B_k, d->k, d->attn_scale,
                                d->idx_scale, false, true);
   if (st != MSA_OK) return st;
-  if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(idx_out) || !aligned16(ws))
+  if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(idx_out) || !aligned16(ws) ||
+      (score_out != nullptr && !aligned16(score_out)))
     return MSA_ERR_INVALID_ARG;
   if (!pow2_in(d->H_kv, 1, 8) || 128 / d->H_kv > d->B_k) return MSA_ERR_UNSUPPORTED;
   if (d->N * d->H_kv >= (int64_t(1) << 31) - 256) return MSA_ERR_UNSUPPORTED;
@@ -232,6 +234,8 @@ msa_status msa_index_topk(const msa_dims* d, const void* q_idx, const void* k_id
   a.q_idx = q_idx;
   a.k_idx = k_idx;
   a.idx_out = idx_out;
+  a.score_out = score_out;
+  a.scale = d->idx_scale > 0.0f ? d->idx_scale : 1.0f / sqrtf(static_cast<float>(d->d_idx));
   a.N = d->N;
   a.H_kv = d->H_kv;
   a.d_idx = d->d_idx;

@@ -23,6 +23,8 @@ struct IndexLaunch {
   const void* q_idx;
   const void* k_idx;
   int32_t* idx_out;
+  float* score_out;  // or null
+  float scale;       // Eq. 6 scale for score_out
   int64_t N;
   int H_kv, d_idx, B_k, k;
   DevStatus* status;

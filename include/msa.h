@@ -84,11 +84,16 @@ typedef struct {
  *   q_idx    [N, H_kv, d_idx] bf16
  *   k_idx    [N, d_idx]       bf16
  *   idx_out  [N, H_kv, k]     int32, written: ascending, -1 padded
+ *   score_out [N, H_kv, k]    fp32 or NULL: slot s holds the Eq. 6 block score
+ *                             (max over the block's keys j <= i of the scaled
+ *                             dot product, idx_scale applied) of idx_out's
+ *                             block in slot s; -inf where idx_out is -1
  * Supported: H_kv in {1,2,4,8} with 128/H_kv <= B_k.
  * ------------------------------------------------------------------------- */
 MSA_API size_t msa_index_topk_workspace(const msa_dims* dims);
 MSA_API msa_status msa_index_topk(const msa_dims* dims, const void* q_idx, const void* k_idx,
-                          int32_t* idx_out, void* workspace, size_t ws_bytes, void* stream);
+                                  int32_t* idx_out, float* score_out, void* workspace,
+                                  size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
  * Main Branch, Eq. 8 with the causal rule of Eq. 1 (xllm-io review "核心公式";

@@ -66,19 +66,21 @@ FAKE = ctypes.c_void_p(1 << 20)  # aligned, never dereferenced: validation fails
 def test_index_topk_rejects_on_host(capi, field, value, status):
     d = capi.dims(4096, 8, 4, 128, 64, 128, 16)
     setattr(d, field, value)
-    st = capi.LIB.msa_index_topk(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, 1 << 20, None)
+    st = capi.LIB.msa_index_topk(ctypes.byref(d), FAKE, FAKE, FAKE, None, FAKE, 1 << 20, None)
     assert st == status
 
 
 def test_misaligned_and_null_pointers_rejected(capi):
     d = capi.dims(4096, 8, 4, 128, 64, 128, 16)
     bad = ctypes.c_void_p((1 << 20) + 2)
-    assert capi.LIB.msa_index_topk(ctypes.byref(d), bad, FAKE, FAKE, FAKE, 1 << 20, None) == 1
-    assert capi.LIB.msa_index_topk(ctypes.byref(d), None, FAKE, FAKE, FAKE, 1 << 20, None) == 1
+    assert capi.LIB.msa_index_topk(ctypes.byref(d), bad, FAKE, FAKE, None, FAKE, 1 << 20, None) == 1
+    assert capi.LIB.msa_index_topk(ctypes.byref(d), None, FAKE, FAKE, None, FAKE, 1 << 20, None) == 1
+    # a misaligned score_out is rejected too
+    assert capi.LIB.msa_index_topk(ctypes.byref(d), FAKE, FAKE, FAKE, bad, FAKE, 1 << 20, None) == 1
     assert capi.LIB.msa_sparse_attn_fwd(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, None,
                                         None, 0, None) == 1
     # a too-small workspace is reported before anything is launched
-    assert capi.LIB.msa_index_topk(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, 8, None) == 3
+    assert capi.LIB.msa_index_topk(ctypes.byref(d), FAKE, FAKE, FAKE, None, FAKE, 8, None) == 3
     d.d_h = 96
     assert capi.LIB.msa_sparse_attn_fwd(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE,
                                         1 << 40, None) == 2

@@ -33,11 +33,64 @@ def _cfg(name, **kw):
     return dataclasses.replace(inputs.CONFIGS[name], **kw)
 
 
-def _check_index(msa, cfg, rows=None, seed=None):
+# Outputs are poisoned before every call (NaN for O, LSE and block scores, -7
+# for the selection), so a row the kernels never write fails the comparison.
+SENTINEL = -7
+
+
+def _index(msa, dev, cfg, scores=False):
+    N = dev["q_idx"].shape[0]
+    idx = torch.full((N, cfg.H_kv, cfg.k), SENTINEL, dtype=torch.int32, device="cuda")
+    sc = (torch.full((N, cfg.H_kv, cfg.k), float("nan"), dtype=torch.float32, device="cuda")
+          if scores else None)
+    msa.index_topk(dev["q_idx"], dev["k_idx"], cfg.B_k, cfg.k, idx_out=idx, score_out=sc)
+    torch.cuda.synchronize()
+    return (idx, sc) if scores else idx
+
+
+def _attn(msa, dev, idx_dev, B_k):
+    N, H_q, d_h = dev["q"].shape
+    o = torch.full((N, H_q, d_h), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lse = torch.full((N, H_q), float("nan"), dtype=torch.float32, device="cuda")
+    msa.sparse_attn_fwd(dev["q"], dev["k"], dev["v"], idx_dev, B_k, o=o, lse=lse)
+    torch.cuda.synchronize()
+    return o, lse
+
+
+def structured_rows(cfg, gidx=None, extra=(), per_group=16):
+    """Every row of blocks 0, 1, B/2 and B-1, plus (given the selection) the
+    first and the last `per_group` queries of each group that selected block
+    0 -- the hot list that the tile schedule splits the most."""
+    B_k, N, B = cfg.B_k, cfg.N, cfg.B
+    parts = [np.arange(b * B_k, min((b + 1) * B_k, N)) for b in sorted({0, 1, B // 2, B - 1})
+             if b * B_k < N]
+    if gidx is not None:
+        for r in range(cfg.H_kv):
+            hot = np.nonzero((gidx[:, r, :] == 0).any(axis=1))[0]
+            parts += [hot[:per_group], hot[-per_group:]]
+    parts.append(np.asarray(extra, dtype=np.int64))
+    return np.unique(np.concatenate(parts).astype(np.int64))
+
+
+def _check_scores(sc, gidx, inp, cfg, rows):
+    """score_out of the sampled rows against the oracle's block scores, within
+    the tie band's 1e-3 relative tolerance; -inf in the -1 slots."""
+    for i in rows:
+        for r in range(cfg.H_kv):
+            M = oracle.block_scores(inp["q_idx"][i, r], inp["k_idx"], cfg.B_k, int(i))
+            for s_ in range(cfg.k):
+                b = int(gidx[i, r, s_])
+                got = float(sc[i, r, s_])
+                if b < 0:
+                    assert got == -np.inf, (i, r, s_, got)
+                else:
+                    assert abs(got - M[b]) <= compare._band(got, M[b]), (i, r, s_, b, got, M[b])
+
+
+def _check_index(msa, cfg, rows=None, seed=None, score_rows=None):
     inp = prefill_inputs_cached(cfg, seed)
     dev = dev_inputs(inp)
-    idx = msa.index_topk(dev["q_idx"], dev["k_idx"], cfg.B_k, cfg.k)
-    torch.cuda.synchronize()
+    idx, sc = _index(msa, dev, cfg, scores=True)
     gidx = idx.cpu().numpy()
     rows = np.arange(cfg.N) if rows is None else np.asarray(rows)
     ref, cut, nxt = oracle.index_topk(inp["q_idx"], inp["k_idx"], cfg.B_k, cfg.k, rows=rows)
@@ -45,6 +98,7 @@ def _check_index(msa, cfg, rows=None, seed=None):
                                             q_idx_rows=inp["q_idx"][rows], k_idx=inp["k_idx"])
     assert not fails, f"{cfg.name}: {len(fails)} mismatching rows, e.g. {fails[:3]}"
     assert exact + band == rows.size * cfg.H_kv
+    _check_scores(sc.cpu().numpy(), gidx, inp, cfg, rows if score_rows is None else score_rows)
     return inp, dev, gidx, exact, band
 
 
@@ -54,9 +108,15 @@ def test_index_topk_tiny_all_rows(msa):
     assert band <= 2  # i.i.d. N(0,1) scores: ties in fp32 are essentially absent
 
 
-def test_index_topk_32k_shape_truncated(msa):
-    cfg = _cfg("32k", N=8192)
-    _check_index(msa, cfg)
+def test_index_topk_32k_full(msa):
+    """The 32K workload at its full length: every row of blocks 0, 1, B/2,
+    B-1, the ends of each group's block-0 list and random rows."""
+    cfg = inputs.CONFIGS["32k"]
+    inp = prefill_inputs_cached(cfg)
+    gidx = _index(msa, dev_inputs(inp), cfg).cpu().numpy()
+    rng = np.random.default_rng(4)
+    rows = structured_rows(cfg, gidx, extra=rng.integers(0, cfg.N, 64))
+    _check_index(msa, cfg, rows=rows, score_rows=rows[::8])
 
 
 @pytest.mark.parametrize("N,H_kv,d_idx,B_k,k", [
@@ -96,17 +156,19 @@ def test_index_topk_exact_ties_go_to_lower_blocks(msa):
 
 
 def test_index_topk_128k_sampled(msa):
-    """Full 128K workload (same launch as the benchmark); sampled rows checked."""
+    """Full 128K workload (same launch as the benchmark): every row of blocks
+    0, 1, B/2, B-1, the ends of each group's block-0 list and random rows."""
     cfg = inputs.CONFIGS["128k"]
+    inp = prefill_inputs_cached(cfg)
+    gidx = _index(msa, dev_inputs(inp), cfg).cpu().numpy()
     rng = np.random.default_rng(0)
-    rows = np.unique(np.concatenate([
-        rng.integers(0, cfg.N, 48), [0, 127, 128, 4095, cfg.N // 2, cfg.N - 129, cfg.N - 1]]))
-    _check_index(msa, cfg, rows=rows)
+    rows = structured_rows(cfg, gidx, extra=np.concatenate([
+        rng.integers(0, cfg.N, 48), [4095, cfg.N // 2, cfg.N - 129]]))
+    _check_index(msa, cfg, rows=rows, score_rows=rows[::16])
 
 
 def _check_attn(msa, inp, dev, idx_dev, cfg, rows, what):
-    o, lse = msa.sparse_attn_fwd(dev["q"], dev["k"], dev["v"], idx_dev, cfg.B_k)
-    torch.cuda.synchronize()
+    o, lse = _attn(msa, dev, idx_dev, cfg.B_k)
     rows = np.asarray(rows)
     idx_rows = idx_dev.cpu().numpy()[rows]
     ro, rlse = oracle.sparse_attn(inp["q"][rows], inp["k"], inp["v"], idx_rows, cfg.B_k, rows,
@@ -120,19 +182,20 @@ def test_attention_tiny_all_rows(msa):
     cfg = inputs.CONFIGS["tiny"]
     inp = prefill_inputs_cached(cfg)
     dev = dev_inputs(inp)
-    idx = msa.index_topk(dev["q_idx"], dev["k_idx"], cfg.B_k, cfg.k)
+    idx = _index(msa, dev, cfg)
     _check_attn(msa, inp, dev, idx, cfg, np.arange(cfg.N), "tiny")
 
 
-def test_attention_32k_shape_truncated(msa):
-    cfg = _cfg("32k", N=8192)
+def test_attention_32k_full(msa):
+    """The 32K workload at its full length: every row of blocks 0, 1, B/2,
+    B-1, the ends of each group's block-0 list and random rows."""
+    cfg = inputs.CONFIGS["32k"]
     inp = prefill_inputs_cached(cfg)
     dev = dev_inputs(inp)
-    idx = msa.index_topk(dev["q_idx"], dev["k_idx"], cfg.B_k, cfg.k)
+    idx = _index(msa, dev, cfg)
     rng = np.random.default_rng(1)
-    rows = np.unique(np.concatenate([rng.integers(0, cfg.N, 400), np.arange(0, 300),
-                                     np.arange(cfg.N - 130, cfg.N)]))
-    _check_attn(msa, inp, dev, idx, cfg, rows, "32k@8192")
+    rows = structured_rows(cfg, idx.cpu().numpy(), extra=rng.integers(0, cfg.N, 400))
+    _check_attn(msa, inp, dev, idx, cfg, rows, "32k")
 
 
 @pytest.mark.parametrize("N,H_q,H_kv,d_h,B_k,k", [
@@ -149,7 +212,7 @@ def test_attention_edge_shapes(msa, N, H_q, H_kv, d_h, B_k, k):
                            structure="iid", seed_index=23)
     inp = prefill_inputs_cached(cfg)
     dev = dev_inputs(inp)
-    idx = msa.index_topk(dev["q_idx"], dev["k_idx"], cfg.B_k, cfg.k)
+    idx = _index(msa, dev, cfg)
     _check_attn(msa, inp, dev, idx, cfg, np.arange(N), f"edge {N},{H_q},{H_kv},{d_h},{B_k},{k}")
 
 
@@ -160,8 +223,8 @@ def test_attention_dense_equivalence(msa):
                            seed_index=29)
     inp = prefill_inputs_cached(cfg)
     dev = dev_inputs(inp)
-    idx = msa.index_topk(dev["q_idx"], dev["k_idx"], B_k, 5)
-    o, lse = msa.sparse_attn_fwd(dev["q"], dev["k"], dev["v"], idx, B_k)
+    idx = _index(msa, dev, cfg)
+    o, lse = _attn(msa, dev, idx, B_k)
     rows = np.arange(N)
     ro, rlse = oracle.dense_attn(inp["q"], inp["k"], inp["v"], rows)
     compare.assert_attn_close(bf16_to_f64(o), ro, lse.cpu().numpy(), rlse, what="dense")
@@ -193,8 +256,7 @@ def test_attention_empty_and_future_entries(msa):
         b_i = i // cfg.B_k
         row = [b_i] + ([0] if b_i >= 2 else []) + ([b_i + 2] if b_i + 2 < B else [])
         idx[i, 0, : len(row)] = row  # group 1 stays empty
-    o, lse = msa.sparse_attn_fwd(dev["q"], dev["k"], dev["v"], torch.from_numpy(idx).cuda(),
-                                 cfg.B_k)
+    o, lse = _attn(msa, dev, torch.from_numpy(idx).cuda(), cfg.B_k)
     rows = np.arange(cfg.N)
     ro, rlse = oracle.sparse_attn(inp["q"], inp["k"], inp["v"], idx, cfg.B_k, rows)
     go = bf16_to_f64(o)
@@ -205,12 +267,14 @@ def test_attention_empty_and_future_entries(msa):
 
 
 def test_attention_128k_sampled(msa):
+    """Full 128K workload: every row of blocks 0, 1, B/2, B-1, the ends of
+    each group's block-0 list and random rows."""
     cfg = inputs.CONFIGS["128k"]
     inp = prefill_inputs_cached(cfg)
     dev = dev_inputs(inp)
-    idx = msa.index_topk(dev["q_idx"], dev["k_idx"], cfg.B_k, cfg.k)
+    idx = _index(msa, dev, cfg)
     rng = np.random.default_rng(3)
-    rows = np.unique(np.concatenate([rng.integers(0, cfg.N, 96), [0, 1, 127, 128, cfg.N - 1]]))
+    rows = structured_rows(cfg, idx.cpu().numpy(), extra=rng.integers(0, cfg.N, 96))
     _check_attn(msa, inp, dev, idx, cfg, rows, "128k")
 
 
@@ -259,7 +323,9 @@ def test_bounded_wait_times_out_reports_and_context_survives(msa):
 def _check_index_lse(msa, cfg, dev, inp, idx_dev, rows, what):
     """LSE_idx (Eq. 9's Index Branch normaliser) on the GPU against the oracle
     for the listed rows, from the same selection."""
-    lse_idx = msa.index_lse(dev["q_idx"], dev["k_idx"], idx_dev, cfg.B_k)
+    lse_idx = torch.full((dev["q_idx"].shape[0], cfg.H_kv), float("nan"), dtype=torch.float32,
+                         device="cuda")
+    msa.index_lse(dev["q_idx"], dev["k_idx"], idx_dev, cfg.B_k, lse_idx=lse_idx)
     torch.cuda.synchronize()
     rows = np.asarray(rows)
     sel = idx_dev.cpu().numpy()[rows]
@@ -274,7 +340,7 @@ def test_index_lse_tiny_all_rows(msa):
     cfg = inputs.CONFIGS["tiny"]
     inp = prefill_inputs_cached(cfg)
     dev = dev_inputs(inp)
-    idx = msa.index_topk(dev["q_idx"], dev["k_idx"], cfg.B_k, cfg.k)
+    idx = _index(msa, dev, cfg)
     _check_index_lse(msa, cfg, dev, inp, idx, np.arange(cfg.N), "tiny")
 
 
@@ -282,7 +348,7 @@ def test_index_lse_32k_recipe_and_128k_sampled(msa):
     for cfg, n_rand in ((_cfg("32k", N=8192), 200), (inputs.CONFIGS["128k"], 96)):
         inp = prefill_inputs_cached(cfg)
         dev = dev_inputs(inp)
-        idx = msa.index_topk(dev["q_idx"], dev["k_idx"], cfg.B_k, cfg.k)
+        idx = _index(msa, dev, cfg)
         rng = np.random.default_rng(7)
         rows = np.unique(np.concatenate([rng.integers(0, cfg.N, n_rand),
                                          [0, 1, 127, 128, cfg.N - 1]]))
@@ -299,7 +365,7 @@ def test_index_lse_edge_shapes_and_empty_rows(msa, N, H_kv, d_idx, B_k, k):
                            k=k, structure="iid", seed_index=43)
     inp = prefill_inputs_cached(cfg)
     dev = dev_inputs(inp)
-    idx = msa.index_topk(dev["q_idx"], dev["k_idx"], cfg.B_k, cfg.k)
+    idx = _index(msa, dev, cfg)
     idx[5, 0, :] = -1       # a row with no token: -inf
     idx[N - 1, H_kv - 1, 1:] = -1
     _check_index_lse(msa, cfg, dev, inp, idx, np.arange(N), "edge")
@@ -335,10 +401,13 @@ def _decode_run(msa, cfg, steps, check_seqs, seed=None):
     for step in range(steps):
         si = inputs.decode_step_inputs(cfg, step, st["sink"], seed)
         d = {k: to_dev(v) for k, v in si.items()}
-        idx_out = torch.empty((cfg.S, cfg.H_kv, cfg.k), dtype=torch.int32, device="cuda")
+        idx_out = torch.full((cfg.S, cfg.H_kv, cfg.k), SENTINEL, dtype=torch.int32,
+                             device="cuda")
+        o = torch.full((cfg.S, cfg.H_q, cfg.d_h), float("nan"), dtype=torch.bfloat16,
+                       device="cuda")
         o, _ = msa.sparse_decode(d["q"], d["q_idx"], d["k_new"], d["v_new"], d["k_idx_new"],
                                  dev["k_cache"], dev["v_cache"], dev["k_idx_cache"], seq_len,
-                                 cfg.B_k, cfg.k, idx_out=idx_out)
+                                 cfg.B_k, cfg.k, o=o, idx_out=idx_out)
         torch.cuda.synchronize()
         gidx = idx_out.cpu().numpy()
         ref = oracle.decode_reference(st, si, cfg.B_k, cfg.k, seqs=check_seqs,
@@ -408,18 +477,21 @@ def test_decode_full_size_sampled(msa):
 
 def test_forward_1m_sampled(msa):
     """The 1M-token sink-skewed workload through the whole forward (index +
-    attention, 128 query chunks); sampled rows checked against the oracle."""
+    attention in 8 query chunks of 131072); structured and sampled rows
+    checked against the oracle."""
     cfg = inputs.CONFIGS["1m"]
     inp = prefill_inputs_cached(cfg)
     dev = dev_inputs(inp)
-    o, lse, idx = msa.forward(dev["q"], dev["k"], dev["v"], dev["q_idx"], dev["k_idx"], cfg.B_k,
-                              cfg.k)
-    torch.cuda.synchronize()
+    idx = _index(msa, dev, cfg)
+    o, lse = _attn(msa, dev, idx, cfg.B_k)
     del dev
     rng = np.random.default_rng(5)
-    rows = np.unique(np.concatenate([rng.integers(0, cfg.N, 20),
-                                     [0, 129, 8191, 8192, cfg.N // 2, cfg.N - 1]]))
-    gidx = idx.cpu().numpy()[rows]
+    all_idx = idx.cpu().numpy()
+    # every row of blocks 0, 1, B/2, B-1 and the ends of each group's block-0
+    # list (chunks of 131072 queries: rows around a chunk boundary too)
+    rows = structured_rows(cfg, all_idx, extra=np.concatenate([
+        rng.integers(0, cfg.N, 20), [8191, 8192, 131071, 131072, cfg.N // 2 + 5]]))
+    gidx = all_idx[rows]
     ref, cut, nxt = oracle.index_topk(inp["q_idx"], inp["k_idx"], cfg.B_k, cfg.k, rows=rows)
     exact, band, fails = compare.check_topk(gidx, ref, cut, nxt, rows, cfg.B_k, cfg.k,
                                             q_idx_rows=inp["q_idx"][rows], k_idx=inp["k_idx"])
