@@ -54,6 +54,14 @@ def _load():
             P = ctypes.c_void_p
             I64, I32, D = ctypes.c_int64, ctypes.c_int, ctypes.c_double
             lib.oracle_max_threads.restype = I32
+            lib.oracle_e4m3_value.argtypes = [ctypes.c_uint8]
+            lib.oracle_e4m3_value.restype = D
+            lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
+            lib.oracle_e4m3_encode.restype = ctypes.c_uint8
+            lib.oracle_quantize_rows.argtypes = [P, I64, I32, P, P]
+            lib.oracle_paged_decode_fp8.argtypes = (
+                [P] * 5 + [P] * 6 + [P, I32, P] + [I32] * 6 + [D, D] + [P, I64] + [P] * 5
+                + [P] * 5)
             lib.oracle_block_scores.argtypes = [P, P, I64, I32, I32, I64, P]
             lib.oracle_index_topk.argtypes = [P, P, I64, I32, I32, I32, I32, P, I64, P, P, P, I32]
             lib.oracle_sparse_attn.argtypes = [P, P, P, P, I64, I32, I32, I32, I32, I32, D, P, I64,
@@ -251,3 +259,72 @@ def flops(N: float, H_q: int, H_kv: int, d_h: int, d_idx: int, B_k: int, k: int)
                          ctypes.byref(fi), ctypes.byref(fm))
     return {"gqa": g.value, "index": fi.value, "main": fm.value,
             "msa": fi.value + fm.value, "ratio": g.value / (fi.value + fm.value)}
+
+
+# ------------------------------------------------- FP8 (E4M3) paged decode --
+def e4m3_values() -> np.ndarray:
+    """Value of every E4M3 code 0..255 (float64; NaN for the two NaN codes)."""
+    lib = _load()
+    return np.array([lib.oracle_e4m3_value(c) for c in range(256)], dtype=np.float64)
+
+
+def e4m3_encode(x: np.ndarray) -> np.ndarray:
+    """float32 values -> E4M3 codes (nearest, ties to the even code, saturated)."""
+    lib = _load()
+    flat = np.asarray(x, dtype=np.float32).reshape(-1)
+    return np.array([lib.oracle_e4m3_encode(float(v)) for v in flat],
+                    dtype=np.uint8).reshape(np.shape(x))
+
+
+def quantize_rows(x_bf16: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:
+    """bf16 rows [..., dim] -> (E4M3 codes [..., dim] uint8, scales [...] float32),
+    scale = amax / 448 per row (1 for an all-zero row)."""
+    x = _c(x_bf16, np.uint16)
+    dim = x.shape[-1]
+    rows = x.size // dim
+    codes = np.empty(x.shape, dtype=np.uint8)
+    scales = np.empty(x.shape[:-1], dtype=np.float32)
+    _check(_load().oracle_quantize_rows(_p(x), rows, dim, _p(codes), _p(scales)),
+           "quantize_rows")
+    return codes, scales
+
+
+def paged_decode_fp8(pages: dict, step_in: dict, seq_len: np.ndarray, B_k: int, k: int,
+                     seqs=None, attn_scale: Optional[float] = None,
+                     idx_scale: Optional[float] = None) -> dict:
+    """One decode step on an FP8 paged cache for the listed sequences.
+
+    pages: k_pages/v_pages [P,B_k,H_kv,d_h] uint8, k_scale/v_scale [P,B_k,H_kv]
+    float32, kidx_pages [P,B_k,d_idx] uint8, kidx_scale [P,B_k] float32,
+    page_table [S,max_pages] int32.  step_in: q [S,H_q,d_h], q_idx
+    [S,H_kv,d_idx], k_new/v_new [S,H_kv,d_h], k_idx_new [S,d_idx] (bf16).
+    Returns idx, cut, next, o, lse and the new token's quantized rows
+    (new_k, new_v [n,H_kv,d_h], new_kv_scale [n,2,H_kv], new_kidx [n,d_idx],
+    new_kidx_scale [n])."""
+    S, H_q, d_h = step_in["q"].shape
+    H_kv, d_idx = step_in["q_idx"].shape[1], step_in["q_idx"].shape[2]
+    seqs = np.arange(S, dtype=np.int64) if seqs is None else np.asarray(seqs, dtype=np.int64)
+    n = seqs.size
+    pt = _c(pages["page_table"], np.int32)
+    a = {key: _c(step_in[key], np.uint16) for key in ("q", "q_idx", "k_new", "v_new",
+                                                        "k_idx_new")}
+    pg = {key: _c(pages[key], np.uint8) for key in ("k_pages", "v_pages", "kidx_pages")}
+    sc = {key: _c(pages[key], np.float32) for key in ("k_scale", "v_scale", "kidx_scale")}
+    out = {"idx": np.empty((n, H_kv, k), np.int32), "cut": np.empty((n, H_kv)),
+           "next": np.empty((n, H_kv)), "o": np.empty((n, H_q, d_h)), "lse": np.empty((n, H_q)),
+           "new_k": np.empty((n, H_kv, d_h), np.uint8), "new_v": np.empty((n, H_kv, d_h), np.uint8),
+           "new_kv_scale": np.empty((n, 2, H_kv), np.float32),
+           "new_kidx": np.empty((n, d_idx), np.uint8), "new_kidx_scale": np.empty(n, np.float32)}
+    sl = _c(seq_len, np.int32)
+    rc = _load().oracle_paged_decode_fp8(
+        _p(a["q"]), _p(a["q_idx"]), _p(a["k_new"]), _p(a["v_new"]), _p(a["k_idx_new"]),
+        _p(pg["k_pages"]), _p(sc["k_scale"]), _p(pg["v_pages"]), _p(sc["v_scale"]),
+        _p(pg["kidx_pages"]), _p(sc["kidx_scale"]), _p(pt), pt.shape[1], _p(sl),
+        H_q, H_kv, d_h, d_idx, B_k, k,
+        1.0 / np.sqrt(d_h) if attn_scale is None else attn_scale,
+        1.0 / np.sqrt(d_idx) if idx_scale is None else idx_scale,
+        _p(seqs), n, _p(out["idx"]), _p(out["cut"]), _p(out["next"]), _p(out["o"]),
+        _p(out["lse"]), _p(out["new_k"]), _p(out["new_v"]), _p(out["new_kv_scale"]),
+        _p(out["new_kidx"]), _p(out["new_kidx_scale"]))
+    _check(rc, "paged_decode_fp8")
+    return out

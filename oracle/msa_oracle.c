@@ -437,3 +437,226 @@ void oracle_flops(double N, double H_q, double H_kv, double d_h, double d_idx,
     if (f_index) *f_index = H_kv * d_idx * N * N;
     if (f_main) *f_main = 4.0 * H_q * d_h * N * k * B_k;
 }
+
+/* ------------------------------------------------------------------ */
+/* FP8 (E4M3) paged KV cache for decode.                               */
+/* ------------------------------------------------------------------ */
+
+/*
+ * The cached keys, values and index keys of the paged decode are stored as
+ * 8-bit floating point codes with one float32 scale per token (and per KV
+ * head for keys and values): value = e4m3(code) * scale.  The open
+ * implementation ships a "paged FP8 decode wrapper" ([chl] section 6, the
+ * system-configuration row); the pages give no encoding, so this is the
+ * plainest one: OCP E4M3 (1 sign bit, 4 exponent bits with bias 7, 3
+ * mantissa bits, subnormals, no infinities, S.1111.111 is NaN, largest
+ * finite 448), per-token absolute-maximum scaling scale = amax / 448, codes
+ * rounded to nearest with ties to the even code, saturated to +-448.
+ */
+
+/* E4M3 code -> value, from the format's definition (exact in double). */
+double oracle_e4m3_value(uint8_t code)
+{
+    const int s = code >> 7, e = (code >> 3) & 0xF, m = code & 7;
+    if (e == 0xF && m == 7) return NAN;
+    const double mag = (e == 0) ? ldexp((double)m / 8.0, -6) : ldexp(1.0 + (double)m / 8.0, e - 7);
+    return s ? -mag : mag;
+}
+
+/* float -> E4M3 code: round to the nearest representable value, ties to the
+ * code whose last mantissa bit is 0, magnitudes above 448 saturated to 448.
+ * The non-negative finite codes 0x00 .. 0x7E are ordered by value, so the
+ * rounding is a search for the bracketing pair. */
+uint8_t oracle_e4m3_encode(float x)
+{
+    if (isnan(x)) return 0x7F;
+    const uint8_t sign = signbit(x) ? 0x80 : 0x00;
+    double a = fabs((double)x);
+    if (a >= 448.0) return (uint8_t)(sign | 0x7E);
+    int lo = 0;
+    while (lo + 1 <= 0x7E && oracle_e4m3_value((uint8_t)(lo + 1)) <= a) ++lo;
+    const double vlo = oracle_e4m3_value((uint8_t)lo);
+    if (vlo == a || lo == 0x7E) return (uint8_t)(sign | lo);
+    const double vhi = oracle_e4m3_value((uint8_t)(lo + 1));
+    const double dlo = a - vlo, dhi = vhi - a;
+    int c;
+    if (dlo < dhi) c = lo;
+    else if (dhi < dlo) c = lo + 1;
+    else c = (lo & 1) ? lo + 1 : lo;  /* tie: the even code */
+    return (uint8_t)(sign | c);
+}
+
+/* Per-row quantization of bf16 rows: amax over the row (float32, exact),
+ * scale = amax / 448 in float32 (1 for an all-zero row), code[d] =
+ * encode(x[d] / scale) with the division in float32.  Every decision is
+ * taken in float32, as the GPU takes it.
+ * x: [n_rows, dim] bf16; codes: [n_rows, dim]; scales: [n_rows]. */
+int oracle_quantize_rows(const uint16_t *x, int64_t n_rows, int dim, uint8_t *codes,
+                         float *scales)
+{
+    if (!x || !codes || !scales || n_rows < 0 || dim <= 0) return -1;
+    for (int64_t t = 0; t < n_rows; ++t) {
+        const uint16_t *row = x + t * dim;
+        float amax = 0.0f;
+        for (int d = 0; d < dim; ++d) {
+            const float v = fabsf((float)bf(row[d]));
+            if (v > amax) amax = v;
+        }
+        const float sc = amax > 0.0f ? amax / 448.0f : 1.0f;
+        scales[t] = sc;
+        for (int d = 0; d < dim; ++d) {
+            const float y = (float)bf(row[d]) / sc;
+            codes[t * dim + d] = oracle_e4m3_encode(y);
+        }
+    }
+    return 0;
+}
+
+/*
+ * One decode step on an FP8 paged cache for the listed sequences (Eq. 1:
+ * the new token attends to itself; Eq. 6-8 for the single query i = L).
+ * Pages hold B_k consecutive tokens of one sequence; logical block b of
+ * sequence s lives in page page_table[s, b]:
+ *   k_pages, v_pages [P, B_k, H_kv, d_h] codes, k_scale, v_scale [P, B_k, H_kv],
+ *   kidx_pages [P, B_k, d_idx] codes, kidx_scale [P, B_k].
+ * For sequence s with L = seq_len[s] the new token's k, v (per KV head) and
+ * k_idx rows are quantized as oracle_quantize_rows does and take position L
+ * (page page_table[s, L / B_k], slot L % B_k); the caches themselves are not
+ * modified: new_* return the quantized rows so a caller can compare them.
+ * Then the selection (Eq. 6-7, decided in float32 as oracle_index_topk
+ * does) and the attention (Eq. 8, two passes in double) run on the
+ * dequantized values code * scale, exactly as the bf16 path runs on its
+ * widened bf16 values.
+ * Outputs per listed sequence n: idx [n, H_kv, k], cut/next [n, H_kv],
+ * o [n, H_q, d_h], lse [n, H_q]; new_k/new_v [n, H_kv, d_h] codes with
+ * new_kv_scale [n, 2, H_kv] (k then v), new_kidx [n, d_idx] codes with
+ * new_kidx_scale [n].
+ */
+int oracle_paged_decode_fp8(const uint16_t *q, const uint16_t *q_idx, const uint16_t *k_new,
+                            const uint16_t *v_new, const uint16_t *k_idx_new,
+                            const uint8_t *k_pages, const float *k_scale,
+                            const uint8_t *v_pages, const float *v_scale,
+                            const uint8_t *kidx_pages, const float *kidx_scale,
+                            const int32_t *page_table, int max_pages, const int32_t *seq_len,
+                            int H_q, int H_kv, int d_h, int d_idx, int B_k, int k,
+                            double attn_scale, double idx_scale,
+                            const int64_t *seqs, int64_t n_seqs,
+                            int32_t *idx_out, double *cut_out, double *next_out,
+                            double *o_out, double *lse_out,
+                            uint8_t *new_k, uint8_t *new_v, float *new_kv_scale,
+                            uint8_t *new_kidx, float *new_kidx_scale)
+{
+    if (!q || !q_idx || !k_new || !v_new || !k_idx_new || !k_pages || !k_scale || !v_pages ||
+        !v_scale || !kidx_pages || !kidx_scale || !page_table || !seq_len || !seqs ||
+        !idx_out || !o_out || H_q <= 0 || H_kv <= 0 || H_q % H_kv != 0 || d_h <= 0 ||
+        d_idx <= 0 || B_k <= 0 || k <= 0 || max_pages <= 0 || n_seqs < 0)
+        return -1;
+    const int G = H_q / H_kv;
+    for (int64_t n = 0; n < n_seqs; ++n) {
+        const int64_t s = seqs[n];
+        const int64_t L = seq_len[s];
+        if (L < 0 || L / B_k >= max_pages) return -2;
+        /* the new token, quantized as the append stores it */
+        uint8_t *nk = new_k + n * H_kv * d_h, *nv = new_v + n * H_kv * d_h;
+        float *nsc = new_kv_scale + n * 2 * H_kv;
+        oracle_quantize_rows(k_new + s * H_kv * d_h, H_kv, d_h, nk, nsc);
+        oracle_quantize_rows(v_new + s * H_kv * d_h, H_kv, d_h, nv, nsc + H_kv);
+        uint8_t *nki = new_kidx + n * d_idx;
+        oracle_quantize_rows(k_idx_new + s * d_idx, 1, d_idx, nki, new_kidx_scale + n);
+        const int32_t *pt = page_table + s * (int64_t)max_pages;
+        const int64_t b_i = L / B_k;
+        /* Eq. 6 over the dequantized index keys, per group r */
+        double *M = (double *)malloc(sizeof(double) * (size_t)(b_i + 1));
+        cand_t *scratch = (cand_t *)malloc(sizeof(cand_t) * (size_t)(b_i + 1));
+        if (!M || !scratch) {
+            free(M);
+            free(scratch);
+            return -3;
+        }
+        for (int r = 0; r < H_kv; ++r) {
+            const uint16_t *qr = q_idx + (s * H_kv + r) * (int64_t)d_idx;
+            for (int64_t b = 0; b <= b_i; ++b) M[b] = -INFINITY;
+            for (int64_t j = 0; j <= L; ++j) {
+                const uint8_t *code;
+                double sc;
+                if (j == L) {
+                    code = nki;
+                    sc = new_kidx_scale[n];
+                } else {
+                    const int64_t pg = pt[j / B_k], slot = j % B_k;
+                    code = kidx_pages + (pg * B_k + slot) * (int64_t)d_idx;
+                    sc = kidx_scale[pg * B_k + slot];
+                }
+                double dot = 0.0;
+                for (int d = 0; d < d_idx; ++d) dot += bf(qr[d]) * (oracle_e4m3_value(code[d]) * sc);
+                const double sj = dot * idx_scale;
+                if (sj > M[j / B_k]) M[j / B_k] = sj;
+            }
+            double cut, next;
+            select_row(M, b_i, k, scratch, idx_out + (n * H_kv + r) * k, &cut, &next);
+            if (cut_out) cut_out[n * H_kv + r] = cut;
+            if (next_out) next_out[n * H_kv + r] = next;
+        }
+        free(M);
+        free(scratch);
+        /* Eq. 8 over the selected blocks' tokens j <= L, dequantized */
+        const int64_t cap = (int64_t)k * B_k;
+        double *sv = (double *)malloc(sizeof(double) * (size_t)cap);
+        if (!sv) return -3;
+        for (int h = 0; h < H_q; ++h) {
+            const int r = h / G;
+            const uint16_t *qh = q + (s * H_q + h) * (int64_t)d_h;
+            const int32_t *sel = idx_out + (n * H_kv + r) * k;
+            /* pass 1: scores and their maximum */
+            double m = -INFINITY;
+            int64_t cnt = 0;
+            for (int sl = 0; sl < k; ++sl) {
+                if (sel[sl] < 0) continue;
+                for (int64_t j = (int64_t)sel[sl] * B_k; j < ((int64_t)sel[sl] + 1) * B_k && j <= L; ++j) {
+                    const uint8_t *code;
+                    double sc;
+                    if (j == L) {
+                        code = nk + r * d_h;
+                        sc = nsc[r];
+                    } else {
+                        const int64_t pg = pt[j / B_k], slot = j % B_k;
+                        code = k_pages + ((pg * B_k + slot) * H_kv + r) * (int64_t)d_h;
+                        sc = k_scale[(pg * B_k + slot) * H_kv + r];
+                    }
+                    double dot = 0.0;
+                    for (int d = 0; d < d_h; ++d) dot += bf(qh[d]) * (oracle_e4m3_value(code[d]) * sc);
+                    sv[cnt] = dot * attn_scale;
+                    if (sv[cnt] > m) m = sv[cnt];
+                    ++cnt;
+                }
+            }
+            /* pass 2: exp(s - m) weights over the values */
+            double *o = o_out + (n * H_q + h) * (int64_t)d_h;
+            for (int d = 0; d < d_h; ++d) o[d] = 0.0;
+            double l = 0.0;
+            int64_t c2 = 0;
+            for (int sl = 0; sl < k; ++sl) {
+                if (sel[sl] < 0) continue;
+                for (int64_t j = (int64_t)sel[sl] * B_k; j < ((int64_t)sel[sl] + 1) * B_k && j <= L; ++j) {
+                    const uint8_t *code;
+                    double sc;
+                    if (j == L) {
+                        code = nv + r * d_h;
+                        sc = nsc[H_kv + r];
+                    } else {
+                        const int64_t pg = pt[j / B_k], slot = j % B_k;
+                        code = v_pages + ((pg * B_k + slot) * H_kv + r) * (int64_t)d_h;
+                        sc = v_scale[(pg * B_k + slot) * H_kv + r];
+                    }
+                    const double w = exp(sv[c2++] - m);
+                    l += w;
+                    for (int d = 0; d < d_h; ++d) o[d] += w * (oracle_e4m3_value(code[d]) * sc);
+                }
+            }
+            for (int d = 0; d < d_h; ++d) o[d] /= l;
+            if (lse_out) lse_out[n * H_q + h] = m + log(l);
+        }
+        free(sv);
+    }
+    return 0;
+}

@@ -51,6 +51,26 @@ int oracle_dense_attn(const uint16_t *q_rows, const uint16_t *K, const uint16_t 
                       const int64_t *rows, int64_t n_rows, double *o_out,
                       double *lse_out, int n_threads);
 
+/* FP8 (E4M3) paged decode: code <-> value, per-row quantization, and one
+ * decode step on a paged FP8 cache (layouts in msa_oracle.c). */
+double oracle_e4m3_value(uint8_t code);
+uint8_t oracle_e4m3_encode(float x);
+int oracle_quantize_rows(const uint16_t *x, int64_t n_rows, int dim, uint8_t *codes,
+                         float *scales);
+int oracle_paged_decode_fp8(const uint16_t *q, const uint16_t *q_idx, const uint16_t *k_new,
+                            const uint16_t *v_new, const uint16_t *k_idx_new,
+                            const uint8_t *k_pages, const float *k_scale,
+                            const uint8_t *v_pages, const float *v_scale,
+                            const uint8_t *kidx_pages, const float *kidx_scale,
+                            const int32_t *page_table, int max_pages, const int32_t *seq_len,
+                            int H_q, int H_kv, int d_h, int d_idx, int B_k, int k,
+                            double attn_scale, double idx_scale,
+                            const int64_t *seqs, int64_t n_seqs,
+                            int32_t *idx_out, double *cut_out, double *next_out,
+                            double *o_out, double *lse_out,
+                            uint8_t *new_k, uint8_t *new_v, float *new_kv_scale,
+                            uint8_t *new_kidx, float *new_kidx_scale);
+
 /* Eq. 12 FLOP model. */
 void oracle_flops(double N, double H_q, double H_kv, double d_h, double d_idx,
                   double B_k, double k, double *f_gqa, double *f_index, double *f_main);
