@@ -7,12 +7,13 @@ synthetic inputs with a sink block and retrieval blocks).  Inputs (Q alone is
 1.07 GB) are larger than the 126 MB L2, so no flush is needed between steps.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl msa|reference]
-                    [--workload 128k|32k|1m|decode|decode8] [--no-also]
+                    [--workload 128k|32k|1m|decode|decode_fp8] [--no-also]
 
 On one GPU the 128K line also carries, under "also", the other two parts of
 the metric, each measured the same way: the 1M-token prefill ("1m", 3 steps
-after 2 warm-up steps) and the 64-sequence decode workload ("decode", 200
-steps after 10 warm-up steps, us per token).  For N > 1 each rank runs an
+after 2 warm-up steps), the 64-sequence decode workload ("decode", 200 steps
+after 10 warm-up steps, us per token) and the same decode on a paged FP8
+(E4M3) cache ("decode_fp8").  For N > 1 each rank runs an
 independent replica (its own sequence): the path has no exchange step, so
 there is no collective on the data path; timing is the max over ranks and
 ``value`` is the tokens of all ranks per second.  ``--impl reference`` times
@@ -231,18 +232,35 @@ def run_reference(args, cfg, rank, world):
     return 0
 
 
+def is_fp8(cfg) -> bool:
+    return cfg.name.startswith("decode_fp8")
+
+
+def decode_state_of(cfg, seed=None):
+    from block_sparse_gqa_idx_b200 import inputs
+
+    return (inputs.decode_fp8_state(cfg, seed=seed) if is_fp8(cfg)
+            else inputs.decode_state(cfg, seed=seed))
+
+
 def decode_oracle_sample(st, cfg, n_seq: int, step: int = 0):
     """Time the oracle's decode step (append + Eq. 6-8 for the new token) on
-    the first n_seq sequences of a decode state: (us per token, seconds, cores)."""
+    the first n_seq sequences of a decode state, bf16 or paged FP8:
+    (us per token, seconds, cores)."""
     import oracle
     from block_sparse_gqa_idx_b200 import inputs
 
     si = inputs.decode_step_inputs(cfg, step, st["sink"])
     seqs = list(range(min(n_seq, cfg.S)))
     t0 = time.perf_counter()
-    oracle.decode_reference(st, si, cfg.B_k, cfg.k, seqs=seqs)
+    if is_fp8(cfg):
+        oracle.paged_decode_fp8(st, si, st["seq_len"], cfg.B_k, cfg.k, seqs=seqs)
+        cores = 1  # the paged FP8 oracle runs on one thread
+    else:
+        oracle.decode_reference(st, si, cfg.B_k, cfg.k, seqs=seqs)
+        cores = oracle.max_threads()
     dt = time.perf_counter() - t0
-    return 1e6 * dt / len(seqs), dt, oracle.max_threads()
+    return 1e6 * dt / len(seqs), dt, cores
 
 
 def run_reference_decode(args, cfg, rank, world):
@@ -251,7 +269,7 @@ def run_reference_decode(args, cfg, rank, world):
         return 0
     from block_sparse_gqa_idx_b200 import inputs
 
-    st = inputs.decode_state(cfg)
+    st = decode_state_of(cfg)
     n_seq = args.ref_seqs
     times = []
     for it in range(args.warmup + args.steps):
@@ -504,14 +522,20 @@ def run_decode(args, cfg, rank, world, local, steps, warmup, e2e_steps, cpu_seqs
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream(dev)
+    fp8 = is_fp8(cfg)
     t0 = time.time()
-    st = inputs.decode_state(cfg, seed=cfg.seed + 1000 * rank)
+    st = decode_state_of(cfg, seed=cfg.seed + 1000 * rank)
     gen_s = time.time() - t0
 
     def dv(a):
         return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
 
-    caches = {k: dv(st[k]) for k in ("k_cache", "v_cache", "k_idx_cache")}
+    if fp8:
+        caches = {k: torch.from_numpy(np.ascontiguousarray(st[k])).to(dev)
+                  for k in ("k_pages", "v_pages", "kidx_pages", "k_scale", "v_scale", "kidx_scale",
+                            "page_table")}
+    else:
+        caches = {k: dv(st[k]) for k in ("k_cache", "v_cache", "k_idx_cache")}
     seq_len = torch.from_numpy(st["seq_len"]).to(dev)
     n_steps = warmup + steps + e2e_steps
     assert n_steps <= cfg.steps, "more steps than the cache has room for"
@@ -520,13 +544,25 @@ def run_decode(args, cfg, rank, world, local, steps, warmup, e2e_steps, cpu_seqs
     S, H_q, H_kv, d_h, d_idx, B_k, kk = cfg.S, cfg.H_q, cfg.H_kv, cfg.d_h, cfg.d_idx, cfg.B_k, cfg.k
     o = torch.empty((S, H_q, d_h), dtype=torch.bfloat16, device=dev)
     idx = torch.empty((S, H_kv, kk), dtype=torch.int32, device=dev)
-    dd = msa.decode_dims(S, cfg.L_max, H_q, H_kv, d_h, d_idx, B_k, kk)
-    ws = torch.empty(msa.sparse_decode_workspace_size(dd), dtype=torch.uint8, device=dev)
+    if fp8:
+        dd = msa.paged_dims(S, st["page_table"].shape[1], st["k_pages"].shape[0], H_q, H_kv, d_h,
+                            d_idx, B_k, kk)
+        ws = torch.empty(msa.paged_decode_fp8_workspace_size(dd), dtype=torch.uint8, device=dev)
+    else:
+        dd = msa.decode_dims(S, cfg.L_max, H_q, H_kv, d_h, d_idx, B_k, kk)
+        ws = torch.empty(msa.sparse_decode_workspace_size(dd), dtype=torch.uint8, device=dev)
 
     def step(x):
-        msa.sparse_decode(x["q"], x["q_idx"], x["k_new"], x["v_new"], x["k_idx_new"],
-                          caches["k_cache"], caches["v_cache"], caches["k_idx_cache"], seq_len,
-                          B_k, kk, o=o, idx_out=idx, workspace=ws, stream=stream)
+        if fp8:
+            c = caches
+            msa.paged_decode_fp8(x["q"], x["q_idx"], x["k_new"], x["v_new"], x["k_idx_new"],
+                                 c["k_pages"], c["k_scale"], c["v_pages"], c["v_scale"],
+                                 c["kidx_pages"], c["kidx_scale"], c["page_table"], seq_len, B_k,
+                                 kk, o=o, idx_out=idx, workspace=ws, stream=stream)
+        else:
+            msa.sparse_decode(x["q"], x["q_idx"], x["k_new"], x["v_new"], x["k_idx_new"],
+                              caches["k_cache"], caches["v_cache"], caches["k_idx_cache"], seq_len,
+                              B_k, kk, o=o, idx_out=idx, workspace=ws, stream=stream)
 
     def barrier():
         if world > 1:
@@ -570,8 +606,16 @@ def run_decode(args, cfg, rank, world, local, steps, warmup, e2e_steps, cpu_seqs
             for b in sel[s_, r]:
                 if b >= 0:
                     sel_rows += min(B_k, Li - int(b) * B_k)
-    bytes_step = (S * L * d_idx * 2 + sel_rows * d_h * 2 * 2
-                  + S * (H_q * d_h * 2 * 2 + H_kv * d_idx * 2 + H_kv * d_h * 2 * 2 * 2 + d_idx * 2 * 2))
+    if fp8:
+        # one byte per code plus a 4-byte scale per token (and head); the new
+        # rows arrive in bf16 and are written as codes and scales
+        bytes_step = (S * L * (d_idx + 4) + sel_rows * 2 * (d_h + 4)
+                      + S * (H_q * d_h * 2 * 2 + H_kv * d_idx * 2 + H_kv * d_h * 2 * 2
+                             + d_idx * 2 + 2 * H_kv * (d_h + 4) + d_idx + 4))
+    else:
+        bytes_step = (S * L * d_idx * 2 + sel_rows * d_h * 2 * 2
+                      + S * (H_q * d_h * 2 * 2 + H_kv * d_idx * 2 + H_kv * d_h * 2 * 2 * 2
+                             + d_idx * 2 * 2))
 
     # ---- end to end: each step's new rows from pinned host memory, the
     # step, and O and the selection back to pinned host memory
@@ -598,27 +642,32 @@ def run_decode(args, cfg, rank, world, local, steps, warmup, e2e_steps, cpu_seqs
         return None
     pk, pk_kind = peaks()
     gbs = bytes_step / (ms * 1e-3) / 1e9
-    cache_gb = S * cfg.L_max * (2 * H_kv * d_h + d_idx) * 2 / 1e9
+    cache_gb = (S * cfg.L_max * (2 * H_kv * (d_h + 4) + d_idx + 4) / 1e9 if fp8
+                else S * cfg.L_max * (2 * H_kv * d_h + d_idx) * 2 / 1e9)
     total_ms = sum(v[1] for v in prof.values())
     kernels = {n: {"launches": v[0], "ms_per_step": v[1] / steps,
                    "share": v[1] / total_ms if total_ms else None} for n, v in prof.items()}
-    scan_ms = prof.get("dec_scan", (1, 0.0))[1] / steps
-    scan_bytes = S * L * d_idx * 2
+    scan_ms = prof.get("dec8_scan" if fp8 else "dec_scan", (1, 0.0))[1] / steps
+    scan_bytes = S * L * (d_idx + 4) if fp8 else S * L * d_idx * 2
     cpu = None
     if world == 1 and cpu_seqs > 0:
         us_cpu, dt_cpu, cores = decode_oracle_sample(st, cfg, cpu_seqs)
         cpu = {"value": us_cpu, "unit": "us/token", "cores": cores, "kind": "oracle",
-               "sample": f"{cpu_seqs} of the {S} sequences, one decode step each (append, "
-                         f"full K_idx scan, Top-k, attention), {dt_cpu:.1f} s"}
+               "sample": f"{cpu_seqs} of the {S} sequences, one {'paged FP8 ' if fp8 else ''}"
+                         f"decode step each (append, full K_idx scan, Top-k, attention), "
+                         f"{dt_cpu:.1f} s"}
     idle = max(0.0, ms - total_ms / steps)
     return {
         "metric": METRIC, "value": 1e3 * ms / (S * world),
         "unit": "us/token", "n_gpus": world, "steps": steps, "warmup": warmup,
         "ms_per_step": ms, "us_per_step": 1e3 * ms, "higher_is_better": False,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None, "dtype": "e4m3 cache, bf16 math" if fp8 else "bf16",
+        "data": "synthetic",
         "config": {"workload": cfg.name, "S": S, "L": L, "H_q": H_q, "H_kv": H_kv, "d_h": d_h,
                    "d_idx": d_idx, "B_k": B_k, "k": kk,
-                   "l2": f"caches {cache_gb:.1f} GB (K, V, K_idx), larger than L2; no flush"},
+                   "l2": f"caches {cache_gb:.1f} GB (K, V, K_idx{' codes and scales' if fp8 else ''}), "
+                         f"larger than L2; no flush",
+                   **({"pages": int(st["k_pages"].shape[0]), "page_tokens": B_k} if fp8 else {})},
         "roofline": {"kernel": "decode step", "bound": "hbm", "achieved": gbs,
                      "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": gbs / pk["hbm_gbs"],
                      "traffic": None, "bytes_per_step": bytes_step, "peak_kind": pk_kind,
@@ -700,6 +749,10 @@ def main():
             cdec = workload("decode")
             also["decode"] = run_decode(args, cdec, rank, world, local, steps=200, warmup=10,
                                         e2e_steps=8, cpu_seqs=0 if args.no_cpu_baseline else 4)
+            free_device_memory()
+            also["decode_fp8"] = run_decode(args, workload("decode_fp8"), rank, world, local,
+                                            steps=200, warmup=10, e2e_steps=8,
+                                            cpu_seqs=0 if args.no_cpu_baseline else 4)
             line["also"] = also
         if rank == 0 and line is not None:
             print(json.dumps(line), flush=True)

@@ -7,6 +7,7 @@ of ``include/msa.h``); this package is its thin Python binding:
 * ``sparse_attn_fwd`` Main Branch, Eq. 8 (KV-outer sparse attention + merge)
 * ``forward``         both, for one prefill sequence
 * ``sparse_decode``   one decode step for a batch of sequences
+* ``paged_decode_fp8`` the same step on a paged FP8 (E4M3) KV cache
 
 ``inputs`` holds the seeded synthetic workload generators.  The binding is
 loaded on first use of one of the names above and raises if the CUDA library
@@ -16,7 +17,8 @@ _CAPI = ("index_topk", "sparse_attn_fwd", "forward", "sparse_decode", "device_st
          "version", "MSAError", "dims", "decode_dims", "index_topk_workspace_size",
          "sparse_attn_fwd_workspace_size", "sparse_decode_workspace_size", "EXPORTS", "LIB_PATH",
          "profile_enable", "profile_read", "sparse_decode_noalloc", "selftest_bounded_wait",
-         "index_lse", "index_lse_workspace_size")
+         "index_lse", "index_lse_workspace_size", "paged_dims", "paged_decode_fp8",
+         "paged_decode_fp8_workspace_size", "quantize_fp8_rows")
 
 __all__ = list(_CAPI) + ["inputs"]
 

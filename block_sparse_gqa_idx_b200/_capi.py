@@ -39,6 +39,13 @@ class msa_decode_dims(ctypes.Structure):
                 ("idx_scale", ctypes.c_float)]
 
 
+class msa_paged_dims(ctypes.Structure):
+    _fields_ = [("S", ctypes.c_int32), ("max_pages", ctypes.c_int32), ("n_pages", ctypes.c_int64),
+                ("H_q", ctypes.c_int32), ("H_kv", ctypes.c_int32), ("d_h", ctypes.c_int32),
+                ("d_idx", ctypes.c_int32), ("B_k", ctypes.c_int32), ("k", ctypes.c_int32),
+                ("attn_scale", ctypes.c_float), ("idx_scale", ctypes.c_float)]
+
+
 class msa_kernel_time(ctypes.Structure):
     _fields_ = [("name", ctypes.c_char * 48), ("launches", ctypes.c_int32),
                 ("total_ms", ctypes.c_double)]
@@ -49,7 +56,8 @@ EXPORTS = ("msa_index_topk_workspace", "msa_index_topk", "msa_sparse_attn_fwd_wo
            "msa_sparse_attn_fwd", "msa_sparse_decode_workspace", "msa_sparse_decode",
            "msa_get_device_status", "msa_profile_enable", "msa_profile_read",
            "msa_status_string", "msa_version", "msa_sparse_decode_noalloc", "msa_last_error",
-           "msa_selftest_bounded_wait", "msa_index_lse_workspace", "msa_index_lse")
+           "msa_selftest_bounded_wait", "msa_index_lse_workspace", "msa_index_lse",
+           "msa_paged_decode_fp8_workspace", "msa_paged_decode_fp8", "msa_quantize_fp8_rows")
 
 
 def _load() -> ctypes.CDLL:
@@ -81,6 +89,13 @@ def _load() -> ctypes.CDLL:
     lib.msa_index_lse_workspace.restype = Z
     lib.msa_index_lse.argtypes = [D, P, P, P, P, P, Z, P]
     lib.msa_index_lse.restype = I32
+    PD = ctypes.POINTER(msa_paged_dims)
+    lib.msa_paged_decode_fp8_workspace.argtypes = [PD]
+    lib.msa_paged_decode_fp8_workspace.restype = Z
+    lib.msa_paged_decode_fp8.argtypes = [PD] + [P] * 15 + [P, Z, P]
+    lib.msa_paged_decode_fp8.restype = I32
+    lib.msa_quantize_fp8_rows.argtypes = [P, ctypes.c_int64, I32, P, P, P]
+    lib.msa_quantize_fp8_rows.restype = I32
     lib.msa_selftest_bounded_wait.argtypes = [P, P]
     lib.msa_selftest_bounded_wait.restype = I32
     lib.msa_profile_enable.argtypes = [ctypes.c_int32]
@@ -345,3 +360,77 @@ def device_status(workspace: torch.Tensor, stream=None) -> Tuple[int, int]:
     LIB.msa_get_device_status(_ptr(workspace), _stream(stream), ctypes.byref(code),
                               ctypes.byref(where))
     return int(code.value), int(where.value)
+
+
+def paged_dims(S, max_pages, n_pages, H_q, H_kv, d_h, d_idx, B_k, k, attn_scale=0.0,
+               idx_scale=0.0) -> msa_paged_dims:
+    return msa_paged_dims(int(S), int(max_pages), int(n_pages), int(H_q), int(H_kv), int(d_h),
+                          int(d_idx), int(B_k), int(k), float(attn_scale), float(idx_scale))
+
+
+def paged_decode_fp8_workspace_size(d: msa_paged_dims) -> int:
+    return int(LIB.msa_paged_decode_fp8_workspace(ctypes.byref(d)))
+
+
+def paged_decode_fp8(q, q_idx, k_new, v_new, k_idx_new, k_pages, k_scale, v_pages, v_scale,
+                     kidx_pages, kidx_scale, page_table, seq_len, B_k: int, kk: int,
+                     attn_scale: float = 0.0, o: Optional[torch.Tensor] = None,
+                     idx_out: Optional[torch.Tensor] = None,
+                     workspace: Optional[torch.Tensor] = None, stream=None):
+    """One decode step on a paged FP8 (E4M3) cache: the new tokens are
+    quantized into their pages, then Eq. 6-8 run on the dequantized cache.
+    k_pages/v_pages [P,B_k,H_kv,d_h] uint8, k_scale/v_scale [P,B_k,H_kv] fp32,
+    kidx_pages [P,B_k,d_idx] uint8, kidx_scale [P,B_k] fp32, page_table
+    [S,max_pages] int32.  Returns (o [S,H_q,d_h] bf16, idx_out or None)."""
+    S, H_q, d_h = q.shape
+    H_kv, d_idx = q_idx.shape[1], q_idx.shape[2]
+    P = k_pages.shape[0]
+    max_pages = page_table.shape[1]
+    _want(q, "q", torch.bfloat16, (S, H_q, d_h))
+    _want(q_idx, "q_idx", torch.bfloat16, (S, H_kv, d_idx))
+    _want(k_new, "k_new", torch.bfloat16, (S, H_kv, d_h))
+    _want(v_new, "v_new", torch.bfloat16, (S, H_kv, d_h))
+    _want(k_idx_new, "k_idx_new", torch.bfloat16, (S, d_idx))
+    _want(k_pages, "k_pages", torch.uint8, (P, B_k, H_kv, d_h))
+    _want(v_pages, "v_pages", torch.uint8, (P, B_k, H_kv, d_h))
+    _want(k_scale, "k_scale", torch.float32, (P, B_k, H_kv))
+    _want(v_scale, "v_scale", torch.float32, (P, B_k, H_kv))
+    _want(kidx_pages, "kidx_pages", torch.uint8, (P, B_k, d_idx))
+    _want(kidx_scale, "kidx_scale", torch.float32, (P, B_k))
+    _want(page_table, "page_table", torch.int32, (S, max_pages))
+    _want(seq_len, "seq_len", torch.int32, (S,))
+    if o is None:
+        o = torch.empty((S, H_q, d_h), dtype=torch.bfloat16, device=q.device)
+    _want(o, "o", torch.bfloat16, (S, H_q, d_h))
+    if idx_out is not None:
+        _want(idx_out, "idx_out", torch.int32, (S, H_kv, kk))
+    d = paged_dims(S, max_pages, P, H_q, H_kv, d_h, d_idx, B_k, kk, attn_scale)
+    ws = _workspace(paged_decode_fp8_workspace_size(d), q.device, workspace)
+    _raise("msa_paged_decode_fp8",
+           LIB.msa_paged_decode_fp8(ctypes.byref(d), _ptr(q), _ptr(q_idx), _ptr(k_new),
+                                    _ptr(v_new), _ptr(k_idx_new), _ptr(k_pages), _ptr(k_scale),
+                                    _ptr(v_pages), _ptr(v_scale), _ptr(kidx_pages),
+                                    _ptr(kidx_scale), _ptr(page_table), _ptr(seq_len), _ptr(o),
+                                    _ptr(idx_out), _ptr(ws), ws.numel(), _stream(stream)))
+    return o, idx_out
+
+
+def quantize_fp8_rows(x: torch.Tensor, codes: Optional[torch.Tensor] = None,
+                      scales: Optional[torch.Tensor] = None, stream=None):
+    """bf16 rows [..., dim] -> (E4M3 codes [..., dim] uint8, scales [...] fp32)
+    with the FP8 decode's append rule (scale = amax / 448 per row)."""
+    if x.dtype != torch.bfloat16 or not x.is_cuda or not x.is_contiguous():
+        raise ValueError("x must be a contiguous bf16 CUDA tensor")
+    dim = x.shape[-1]
+    rows = x.numel() // dim
+    if codes is None:
+        codes = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty(x.shape[:-1], dtype=torch.float32, device=x.device)
+    _want(codes, "codes", torch.uint8, tuple(x.shape))
+    _want(scales, "scales", torch.float32, tuple(x.shape[:-1]))
+    _raise("msa_quantize_fp8_rows",
+           LIB.msa_quantize_fp8_rows(_ptr(x), rows, dim, _ptr(codes), _ptr(scales),
+                                     _stream(stream)))
+    return codes, scales
+

@@ -19,6 +19,8 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <cuda_fp8.h>
+
 #include "msa_internal.h"
 
 namespace msa {
@@ -567,6 +569,396 @@ cudaError_t launch_scan(const DecParams& p, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
+// ------------------------------------------------- FP8 paged KV-cache decode --
+// The same step on a paged cache of E4M3 codes with one float32 scale per
+// token (and KV head): value = e4m3(code) * scale.  Logical block b of
+// sequence s lives in page page_table[s, b] (pages hold B_k tokens):
+//   k_pages, v_pages [P, B_k, H_kv, d_h] codes, k_scale, v_scale [P, B_k, H_kv]
+//   kidx_pages [P, B_k, d_idx] codes, kidx_scale [P, B_k]
+// Every E4M3 value is exact in bf16, so the kernels feed the codes to the
+// bf16 tensor-core paths unchanged and apply the scales in float32: a key's
+// scale multiplies its scores, a value's scale multiplies its softmax
+// weight before P V.  The append quantizes the new token (amax / 448 per row,
+// the division and the E4M3 rounding in float32, saturated).
+struct Dec8Params {
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* q_idx;
+  const __nv_bfloat16* k_new;
+  const __nv_bfloat16* v_new;
+  const __nv_bfloat16* k_idx_new;
+  uint8_t* k_pages;
+  float* k_scale;
+  uint8_t* v_pages;
+  float* v_scale;
+  uint8_t* kidx_pages;
+  float* kidx_scale;
+  const int32_t* page_table;  // [S, max_pages]
+  int max_pages;
+  int64_t n_pages;
+};
+
+// Quantize one row of n bf16 values to E4M3 codes with scale amax / 448 (1
+// for an all-zero row), by one warp; returns the scale.
+__device__ __forceinline__ float quantize_row_warp(const __nv_bfloat16* x, int n, uint8_t* codes) {
+  const int lane = threadIdx.x & 31;
+  float amax = 0.0f;
+  for (int d = lane; d < n; d += 32) amax = fmaxf(amax, fabsf(__bfloat162float(x[d])));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+  const float sc = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+  for (int d = 2 * lane; d < n; d += 64) {
+    const float2 y = make_float2(__fdiv_rn(__bfloat162float(x[d]), sc),
+                                 __fdiv_rn(__bfloat162float(x[d + 1]), sc));
+    const __nv_fp8x2_storage_t c2 = __nv_cvt_float2_to_fp8x2(y, __NV_SATFINITE, __NV_E4M3);
+    *reinterpret_cast<uint16_t*>(codes + d) = static_cast<uint16_t>(c2);
+  }
+  return sc;
+}
+
+// Two E4M3 codes -> a bf16 pair (exact: every E4M3 value is a bf16 value).
+__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint16_t c2) {
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(c2), __NV_E4M3);
+  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h));
+  return pack_bf16(f.x, f.y);
+}
+
+// A page index of the table, or -1 (reported) when it is outside the pool.
+__device__ __forceinline__ int64_t page_of(const DecParams& p, const Dec8Params& q8, int s,
+                                           int64_t b) {
+  const int64_t pg = q8.page_table[static_cast<int64_t>(s) * q8.max_pages + b];
+  if (pg < 0 || pg >= q8.n_pages) {
+    report(p.status, DEV_ERR_BAD_INDEX, 88, s, static_cast<int>(pg));
+    return -1;
+  }
+  return pg;
+}
+
+// Scan (and append): as dec_scan_kernel, over the index-key pages.  Thread t
+// of a quad owns d in [t*D/4, (t+1)*D/4) of its two key rows; the codes are
+// widened to bf16 pairs in registers and each key's dot is scaled by the
+// key's scale before the block maximum.
+template <int D_IDX, int BK>
+__global__ void __launch_bounds__(256) dec8_scan_kernel(const DecParams p, const Dec8Params q8,
+                                                        int nsplit) {
+  constexpr int DT = D_IDX / 4;     // codes per thread and key row
+  constexpr int NMMA = D_IDX / 16;  // MMAs per 16-key tile
+  static_assert(DT % 16 == 0, "a thread's codes are whole 16-byte loads");
+  const int s = blockIdx.y;
+  const int64_t L = p.seq_len[s];  // written back (L + 1) only by the merge kernel
+  if (L < 0 || L / p.B_k >= q8.max_pages) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+      p.w.Lcur[s] = -1;
+      report(p.status, DEV_ERR_CACHE_FULL, 81, s, static_cast<int>(L));
+    }
+    return;
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (blockIdx.x == 0) {
+    // append: the new token quantized into slot L % B_k of its page, warp w
+    // taking K and V rows of head w (and warp H_kv the index key)
+    const int64_t pg = page_of(p, q8, s, L / p.B_k);
+    const int64_t slot = L % p.B_k;
+    if (pg >= 0) {
+      for (int r = warp; r < p.H_kv; r += 8) {
+        const int64_t tok = (pg * p.B_k + slot) * p.H_kv + r;
+        const float sk = quantize_row_warp(p.k_new + (static_cast<int64_t>(s) * p.H_kv + r) * p.d_h,
+                                           p.d_h, q8.k_pages + tok * p.d_h);
+        const float sv = quantize_row_warp(p.v_new + (static_cast<int64_t>(s) * p.H_kv + r) * p.d_h,
+                                           p.d_h, q8.v_pages + tok * p.d_h);
+        if (lane == 0) {
+          q8.k_scale[tok] = sk;
+          q8.v_scale[tok] = sv;
+        }
+      }
+      if (warp == 7) {
+        const float si = quantize_row_warp(p.k_idx_new + static_cast<int64_t>(s) * D_IDX, D_IDX,
+                                           q8.kidx_pages + (pg * p.B_k + slot) * D_IDX);
+        if (lane == 0) q8.kidx_scale[pg * p.B_k + slot] = si;
+      }
+    }
+    if (threadIdx.x == 0) p.w.Lcur[s] = static_cast<int32_t>(L);
+  }
+  const int64_t b_i = L / p.B_k;  // candidate blocks 0 .. b_i-1 (full, not the local one)
+  const int g = lane >> 2, t = lane & 3;
+  uint32_t bq[NMMA][2];
+  {
+    const __nv_bfloat16* qr = p.q_idx + (static_cast<int64_t>(s) * p.H_kv + (g < p.H_kv ? g : 0)) * D_IDX;
+#pragma unroll
+    for (int j = 0; j < NMMA; ++j) {
+      const int d0 = t * DT + 4 * j;
+      const uint32_t lo = *reinterpret_cast<const uint32_t*>(qr + d0);
+      const uint32_t hi = *reinterpret_cast<const uint32_t*>(qr + d0 + 2);
+      bq[j][0] = g < p.H_kv ? lo : 0u;
+      bq[j][1] = g < p.H_kv ? hi : 0u;
+    }
+  }
+  const int wstride = nsplit * 8;
+  for (int64_t b = blockIdx.x * 8 + warp; b < b_i; b += wstride) {
+    const int64_t pg = page_of(p, q8, s, b);
+    if (pg < 0) continue;
+    const uint8_t* kbase = q8.kidx_pages + pg * BK * D_IDX;
+    const float* sbase = q8.kidx_scale + pg * BK;
+    float mx0 = -INFINITY, mx1 = -INFINITY;  // columns 2t, 2t+1
+#pragma unroll
+    for (int tile = 0; tile < BK / 16; ++tile) {
+      const int row0 = tile * 16 + g;
+      const uint8_t* r0 = kbase + row0 * D_IDX + t * DT;
+      const uint8_t* r1 = r0 + 8 * D_IDX;
+      uint32_t w0[DT / 2], w1[DT / 2];  // bf16 pairs of rows g and g + 8
+#pragma unroll
+      for (int u = 0; u < DT / 16; ++u) {
+        const uint4 c0 = __ldg(reinterpret_cast<const uint4*>(r0) + u);
+        const uint4 c1 = __ldg(reinterpret_cast<const uint4*>(r1) + u);
+        const uint16_t* h0 = reinterpret_cast<const uint16_t*>(&c0);
+        const uint16_t* h1 = reinterpret_cast<const uint16_t*>(&c1);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          w0[u * 8 + e] = e4m3x2_to_bf16x2(h0[e]);
+          w1[u * 8 + e] = e4m3x2_to_bf16x2(h1[e]);
+        }
+      }
+      float c[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int j = 0; j < NMMA; ++j) {
+        // k-slots 2t,2t+1 <- d0,d0+1 ; 2t+8,2t+9 <- d0+2,d0+3 (d0 = t*DT + 4j)
+        const uint32_t a[4] = {w0[2 * j], w1[2 * j], w0[2 * j + 1], w1[2 * j + 1]};
+        mma_bf16_16816(c, a, bq[j][0], bq[j][1]);
+      }
+      const float s0 = __ldg(sbase + row0), s1 = __ldg(sbase + row0 + 8);
+      mx0 = fmax3(mx0, c[0] * s0, c[2] * s1);
+      mx1 = fmax3(mx1, c[1] * s0, c[3] * s1);
+    }
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xFFFFFFFFu, mx0, o));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xFFFFFFFFu, mx1, o));
+    }
+    if (g == 0) {
+      const int r0 = 2 * t, r1 = 2 * t + 1;
+      float* Mrow = p.w.M + static_cast<int64_t>(s) * p.H_kv * p.Bmax;
+      if (r0 < p.H_kv) Mrow[r0 * p.Bmax + b] = mx0;
+      if (r1 < p.H_kv) Mrow[r1 * p.Bmax + b] = mx1;
+    }
+  }
+}
+
+// Gathered attention: as dec_attend_kernel, with the selected page's K and V
+// codes of head r widened to bf16 into the swizzled tile layout by all
+// threads (plain loads: a key's d_h codes are one contiguous row), the keys'
+// scales staged in shared memory, S scaled per key and P per value.
+template <int D_H, int BK>
+__global__ void __launch_bounds__(128) dec8_attend_kernel(const DecParams p, const Dec8Params q8) {
+  constexpr int KW = BK / 4;          // keys per warp
+  constexpr int NT = KW / 8;          // S n-tiles per warp
+  constexpr int DT = D_H / 8;         // O n-tiles
+  constexpr int CPK = D_H / 16;       // 16-code pieces per key row
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sK = smem;
+  uint8_t* sV = smem + BK * D_H * 2;
+  float* red = reinterpret_cast<float*>(sV + BK * D_H * 2);  // [4][16] m, [4][16] l
+  float* ksc = red + 128;                                    // [BK] key scales
+  float* vsc = ksc + BK;                                     // [BK] value scales
+  float* obuf = reinterpret_cast<float*>(smem);  // [4][16][D_H], over K/V once both are used
+
+  const int item = blockIdx.x;  // (s, r, slot)
+  const int slot = item % p.kk;
+  const int r = (item / p.kk) % p.H_kv;
+  const int s = item / (p.kk * p.H_kv);
+  const int64_t L = p.w.Lcur[s];
+  if (L < 0) return;
+  const int b = p.w.sel[(static_cast<int64_t>(s) * p.H_kv + r) * p.kk + slot];
+  if (b < 0) return;
+  const int64_t pg = page_of(p, q8, s, b);
+  if (pg < 0) return;
+  const int64_t last = L;  // the new token's position: keys j <= last
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
+
+  // the block's codes -> bf16 tiles [d-chunk][key][64] with 128-byte swizzle
+  for (int c = threadIdx.x; c < BK * CPK; c += blockDim.x) {
+    const int key = c / CPK, piece = c - key * CPK;
+    const int64_t row = ((pg * BK + key) * p.H_kv + r) * D_H + piece * 16;
+    const uint4 kc = __ldg(reinterpret_cast<const uint4*>(q8.k_pages + row));
+    const uint4 vc = __ldg(reinterpret_cast<const uint4*>(q8.v_pages + row));
+    const uint16_t* hk = reinterpret_cast<const uint16_t*>(&kc);
+    const uint16_t* hv = reinterpret_cast<const uint16_t*>(&vc);
+    uint4 k0, k1, v0, v1;
+    uint32_t* pk0 = reinterpret_cast<uint32_t*>(&k0);
+    uint32_t* pk1 = reinterpret_cast<uint32_t*>(&k1);
+    uint32_t* pv0 = reinterpret_cast<uint32_t*>(&v0);
+    uint32_t* pv1 = reinterpret_cast<uint32_t*>(&v1);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      pk0[e] = e4m3x2_to_bf16x2(hk[e]);
+      pk1[e] = e4m3x2_to_bf16x2(hk[4 + e]);
+      pv0[e] = e4m3x2_to_bf16x2(hv[e]);
+      pv1[e] = e4m3x2_to_bf16x2(hv[4 + e]);
+    }
+    const int d = piece * 16;
+    const uint32_t o0 = sw_addr<BK>(0u, key, d), o1 = sw_addr<BK>(0u, key, d + 8);
+    *reinterpret_cast<uint4*>(sK + o0) = k0;
+    *reinterpret_cast<uint4*>(sK + o1) = k1;
+    *reinterpret_cast<uint4*>(sV + o0) = v0;
+    *reinterpret_cast<uint4*>(sV + o1) = v1;
+  }
+  for (int j = threadIdx.x; j < BK; j += blockDim.x) {
+    ksc[j] = __ldg(q8.k_scale + (pg * BK + j) * p.H_kv + r);
+    vsc[j] = __ldg(q8.v_scale + (pg * BK + j) * p.H_kv + r);
+  }
+  // Q fragments (rows = heads, zero beyond G)
+  uint32_t qa[D_H / 16][4];
+  {
+    const __nv_bfloat16* qb = p.q + (static_cast<int64_t>(s) * p.H_q + r * p.G) * D_H;
+#pragma unroll
+    for (int ks = 0; ks < D_H / 16; ++ks) {
+      const int d = ks * 16 + 2 * t;
+      qa[ks][0] = g < p.G ? *reinterpret_cast<const uint32_t*>(qb + g * D_H + d) : 0u;
+      qa[ks][1] = g + 8 < p.G ? *reinterpret_cast<const uint32_t*>(qb + (g + 8) * D_H + d) : 0u;
+      qa[ks][2] = g < p.G ? *reinterpret_cast<const uint32_t*>(qb + g * D_H + d + 8) : 0u;
+      qa[ks][3] = g + 8 < p.G ? *reinterpret_cast<const uint32_t*>(qb + (g + 8) * D_H + d + 8) : 0u;
+    }
+  }
+  __syncthreads();
+  const int kw0 = warp * KW;  // first key (within the block) of this warp
+  float sacc[NT][4];
+#pragma unroll
+  for (int n = 0; n < NT; ++n) sacc[n][0] = sacc[n][1] = sacc[n][2] = sacc[n][3] = 0.f;
+  {
+    const uint32_t kb = smem_u32(sK);
+#pragma unroll
+    for (int ks = 0; ks < D_H / 16; ++ks) {
+#pragma unroll
+      for (int n2 = 0; n2 < NT / 2; ++n2) {
+        const int mi = lane >> 3, rr = lane & 7;
+        const int key = kw0 + n2 * 16 + (mi >> 1) * 8 + rr;
+        const int d = ks * 16 + (mi & 1) * 8;
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(sw_addr<BK>(kb, key, d), b0, b1, b2, b3);
+        mma_bf16_16816(sacc[2 * n2], qa[ks], b0, b1);
+        mma_bf16_16816(sacc[2 * n2 + 1], qa[ks], b2, b3);
+      }
+    }
+  }
+  // key scale, softmax scale, causal mask (the block holding the new token)
+  const int64_t j0 = static_cast<int64_t>(b) * BK + kw0;
+  float m_lo = -INFINITY, m_hi = -INFINITY;
+#pragma unroll
+  for (int n = 0; n < NT; ++n) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int kl = kw0 + n * 8 + 2 * t + (e & 1);
+      const int64_t j = j0 + n * 8 + 2 * t + (e & 1);
+      float x = sacc[n][e] * ksc[kl] * p.scale_log2;
+      if (j > last) x = -INFINITY;
+      sacc[n][e] = x;
+    }
+    m_lo = fmax3(m_lo, sacc[n][0], sacc[n][1]);
+    m_hi = fmax3(m_hi, sacc[n][2], sacc[n][3]);
+  }
+#pragma unroll
+  for (int o = 1; o < 4; o <<= 1) {
+    m_lo = fmaxf(m_lo, __shfl_xor_sync(0xFFFFFFFFu, m_lo, o));
+    m_hi = fmaxf(m_hi, __shfl_xor_sync(0xFFFFFFFFu, m_hi, o));
+  }
+  const float ms_lo = m_lo == -INFINITY ? 0.f : m_lo;
+  const float ms_hi = m_hi == -INFINITY ? 0.f : m_hi;
+  float l_lo = 0.f, l_hi = 0.f;
+  uint32_t pa[NT / 2][4];
+#pragma unroll
+  for (int n = 0; n < NT; ++n) {
+    const float e0 = exp2f(sacc[n][0] - ms_lo), e1 = exp2f(sacc[n][1] - ms_lo);
+    const float e2 = exp2f(sacc[n][2] - ms_hi), e3 = exp2f(sacc[n][3] - ms_hi);
+    l_lo += e0 + e1;
+    l_hi += e2 + e3;
+    // the weights times the values' scales, so P V runs on the raw codes
+    const int kl = kw0 + n * 8 + 2 * t;
+    const float v0 = vsc[kl], v1 = vsc[kl + 1];
+    pa[n >> 1][(n & 1) * 2 + 0] = pack_bf16(e0 * v0, e1 * v1);
+    pa[n >> 1][(n & 1) * 2 + 1] = pack_bf16(e2 * v0, e3 * v1);
+  }
+#pragma unroll
+  for (int o = 1; o < 4; o <<= 1) {
+    l_lo += __shfl_xor_sync(0xFFFFFFFFu, l_lo, o);
+    l_hi += __shfl_xor_sync(0xFFFFFFFFu, l_hi, o);
+  }
+  float oacc[DT][4];
+#pragma unroll
+  for (int n = 0; n < DT; ++n) oacc[n][0] = oacc[n][1] = oacc[n][2] = oacc[n][3] = 0.f;
+  {
+    const uint32_t vb = smem_u32(sV);
+#pragma unroll
+    for (int ks = 0; ks < NT / 2; ++ks) {
+#pragma unroll
+      for (int n2 = 0; n2 < DT / 2; ++n2) {
+        const int mi = lane >> 3, rr = lane & 7;
+        const int key = kw0 + ks * 16 + (mi & 1) * 8 + rr;
+        const int d = n2 * 16 + (mi >> 1) * 8;
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(sw_addr<BK>(vb, key, d), b0, b1, b2, b3);
+        mma_bf16_16816(oacc[2 * n2], pa[ks], b0, b1);
+        mma_bf16_16816(oacc[2 * n2 + 1], pa[ks], b2, b3);
+      }
+    }
+  }
+  // merge the four warps' (m, l, O) through shared memory, as dec_attend_kernel
+  __syncthreads();
+  if (t == 0) {
+    red[warp * 16 + g] = m_lo;
+    red[warp * 16 + g + 8] = m_hi;
+    red[64 + warp * 16 + g] = l_lo;
+    red[64 + warp * 16 + g + 8] = l_hi;
+  }
+#pragma unroll
+  for (int n = 0; n < DT; ++n) {
+    float* o0 = obuf + (warp * 16 + g) * D_H + n * 8 + 2 * t;
+    float* o1 = obuf + (warp * 16 + g + 8) * D_H + n * 8 + 2 * t;
+    o0[0] = oacc[n][0];
+    o0[1] = oacc[n][1];
+    o1[0] = oacc[n][2];
+    o1[1] = oacc[n][3];
+  }
+  __syncthreads();
+  const int hr = threadIdx.x >> 3, part = threadIdx.x & 7;
+  if (hr < p.G) {
+    float M = -INFINITY;
+    for (int w = 0; w < 4; ++w) M = fmaxf(M, red[w * 16 + hr]);
+    const float Ms = M == -INFINITY ? 0.f : M;
+    float wsum = 0.f, wt[4];
+    for (int w = 0; w < 4; ++w) {
+      const float mw = red[w * 16 + hr];
+      wt[w] = mw == -INFINITY ? 0.f : exp2f(mw - Ms);
+      wsum += wt[w] * red[64 + w * 16 + hr];
+    }
+    const int64_t pslot = ((static_cast<int64_t>(s) * p.H_kv + r) * p.kk + slot) * p.G + hr;
+    float* dst = p.w.part_o + pslot * D_H;
+    const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+    for (int d = part; d < D_H; d += 8) {
+      float acc = 0.f;
+      for (int w = 0; w < 4; ++w) acc += wt[w] * obuf[(w * 16 + hr) * D_H + d];
+      dst[d] = acc * inv;
+    }
+    if (part == 0)
+      p.w.part_lse[pslot] = wsum > 0.f ? (M + log2f(wsum)) * 0.6931471805599453f : -INFINITY;
+  }
+}
+
+template <int D_H, int BK>
+size_t attend8_smem() {
+  static_assert(4 * 16 * D_H * 4 <= 2 * BK * D_H * 2, "warp-merge buffer must fit over K/V");
+  return 1024 + 2 * BK * D_H * 2 + 128 * 4 + 2 * BK * 4;
+}
+
+// Per-row E4M3 quantization of bf16 rows (for filling a cache): one warp per row.
+__global__ void __launch_bounds__(256) quantize_rows_kernel(const __nv_bfloat16* x, int64_t n_rows,
+                                                            int dim, uint8_t* codes, float* scales) {
+  const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  if (row >= n_rows) return;
+  const float sc = quantize_row_warp(x + row * dim, dim, codes + row * dim);
+  if ((threadIdx.x & 31) == 0) scales[row] = sc;
+}
+
 }  // namespace
 
 size_t decode_workspace_bytes(int S, int64_t L_max, int H_q, int H_kv, int d_h, int B_k, int kk) {
@@ -632,6 +1024,101 @@ cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t stream) {
   prof_begin("dec_merge", stream);
   if (a.d_h == 128) dec_merge_kernel<128><<<(rows * 32 + 255) / 256, 256, 0, stream>>>(p);
   else dec_merge_kernel<64><<<(rows * 32 + 255) / 256, 256, 0, stream>>>(p);
+  prof_end(stream);
+  return cudaGetLastError();
+}
+
+size_t paged_decode_workspace_bytes(int S, int max_pages, int H_q, int H_kv, int d_h, int B_k,
+                                    int kk) {
+  return decode_workspace_bytes(S, static_cast<int64_t>(max_pages) * B_k, H_q, H_kv, d_h, B_k, kk);
+}
+
+cudaError_t launch_paged_decode_fp8(const PagedLaunch& a, cudaStream_t stream) {
+  DecParams p;
+  p.q = static_cast<const __nv_bfloat16*>(a.q);
+  p.q_idx = static_cast<const __nv_bfloat16*>(a.q_idx);
+  p.k_new = static_cast<const __nv_bfloat16*>(a.k_new);
+  p.v_new = static_cast<const __nv_bfloat16*>(a.v_new);
+  p.k_idx_new = static_cast<const __nv_bfloat16*>(a.k_idx_new);
+  p.k_cache = nullptr;
+  p.v_cache = nullptr;
+  p.k_idx_cache = nullptr;
+  p.seq_len = a.seq_len;
+  p.o = static_cast<__nv_bfloat16*>(a.o);
+  p.idx_out = a.idx_out;
+  p.S = a.S;
+  p.L_max = static_cast<int64_t>(a.max_pages) * a.B_k;
+  p.Bmax = a.max_pages + 1;
+  p.H_q = a.H_q;
+  p.H_kv = a.H_kv;
+  p.d_h = a.d_h;
+  p.d_idx = a.d_idx;
+  p.B_k = a.B_k;
+  p.kk = a.kk;
+  p.G = a.H_q / a.H_kv;
+  p.scale = a.scale;
+  p.scale_log2 = a.scale * 1.4426950408889634f;
+  size_t need = 0;
+  p.w = carve(a.ws, a.S, p.L_max, a.H_q, a.H_kv, a.d_h, a.B_k, a.kk, &need);
+  if (need > a.ws_bytes) return cudaErrorInvalidValue;
+  p.status = a.status;
+  Dec8Params q8;
+  q8.k_pages = static_cast<uint8_t*>(a.k_pages);
+  q8.k_scale = a.k_scale;
+  q8.v_pages = static_cast<uint8_t*>(a.v_pages);
+  q8.v_scale = a.v_scale;
+  q8.kidx_pages = static_cast<uint8_t*>(a.kidx_pages);
+  q8.kidx_scale = a.kidx_scale;
+  q8.page_table = a.page_table;
+  q8.max_pages = a.max_pages;
+  q8.n_pages = a.n_pages;
+
+  const int nsplit = a.S >= 64 ? 8 : (a.S >= 16 ? 32 : 64);
+  const dim3 sgrid(nsplit, a.S);
+  prof_begin("dec8_scan", stream);
+  if (a.d_idx == 64 && a.B_k == 128) dec8_scan_kernel<64, 128><<<sgrid, 256, 0, stream>>>(p, q8, nsplit);
+  else if (a.d_idx == 64) dec8_scan_kernel<64, 64><<<sgrid, 256, 0, stream>>>(p, q8, nsplit);
+  else if (a.B_k == 128) dec8_scan_kernel<128, 128><<<sgrid, 256, 0, stream>>>(p, q8, nsplit);
+  else dec8_scan_kernel<128, 64><<<sgrid, 256, 0, stream>>>(p, q8, nsplit);
+  prof_end(stream);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int hs = a.kk - 1 > 0 ? a.kk - 1 : 1;
+  const size_t topk_smem = (8 * hs * 32 + 8 * hs) * sizeof(uint64_t);
+  e = cudaFuncSetAttribute(dec_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(topk_smem));
+  if (e != cudaSuccess) return e;
+  prof_begin("dec_topk", stream);
+  dec_topk_kernel<<<a.S * a.H_kv, 256, topk_smem, stream>>>(p);
+  prof_end(stream);
+  auto attend = [&](auto kern, size_t smem) -> cudaError_t {
+    cudaError_t r = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (r != cudaSuccess) return r;
+    prof_begin("dec8_attend", stream);
+    kern<<<a.S * a.H_kv * a.kk, 128, smem, stream>>>(p, q8);
+    prof_end(stream);
+    return cudaGetLastError();
+  };
+  if (a.d_h == 128 && a.B_k == 128) e = attend(dec8_attend_kernel<128, 128>, attend8_smem<128, 128>());
+  else if (a.d_h == 128) e = attend(dec8_attend_kernel<128, 64>, attend8_smem<128, 64>());
+  else if (a.B_k == 128) e = attend(dec8_attend_kernel<64, 128>, attend8_smem<64, 128>());
+  else e = attend(dec8_attend_kernel<64, 64>, attend8_smem<64, 64>());
+  if (e != cudaSuccess) return e;
+  const int rows = a.S * a.H_q;
+  prof_begin("dec_merge", stream);
+  if (a.d_h == 128) dec_merge_kernel<128><<<(rows * 32 + 255) / 256, 256, 0, stream>>>(p);
+  else dec_merge_kernel<64><<<(rows * 32 + 255) / 256, 256, 0, stream>>>(p);
+  prof_end(stream);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_fp8_rows(const void* x, int64_t n_rows, int dim, void* codes,
+                                     float* scales, cudaStream_t stream) {
+  const int64_t threads = n_rows * 32;
+  prof_begin("quantize_fp8_rows", stream);
+  quantize_rows_kernel<<<static_cast<unsigned>((threads + 255) / 256), 256, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(x), n_rows, dim, static_cast<uint8_t*>(codes), scales);
   prof_end(stream);
   return cudaGetLastError();
 }

@@ -374,6 +374,85 @@ msa_status msa_sparse_decode(const msa_decode_dims* d, const void* q, const void
   return from_cuda(msa::launch_decode(a, s));
 }
 
+// -------------------------------------------------- FP8 paged decode --
+namespace {
+msa_status check_paged_dims(const msa_paged_dims* d) {
+  if (d == nullptr || d->S < 1 || d->max_pages < 1 || d->n_pages < 1) return MSA_ERR_INVALID_ARG;
+  msa_status st = check_common(static_cast<int64_t>(d->max_pages) * (d->B_k > 0 ? d->B_k : 1),
+                               d->H_q, d->H_kv, d->d_h, d->d_idx, d->B_k, d->k, d->attn_scale,
+                               d->idx_scale, true, true);
+  if (st != MSA_OK) return st;
+  if (d->d_idx != 64 && d->d_idx != 128) return MSA_ERR_UNSUPPORTED;  // 16-byte code loads
+  const int G = d->H_q / d->H_kv;
+  if (G > 16 || d->H_kv > 8) return MSA_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(d->max_pages) * d->B_k >= (int64_t(1) << 31)) return MSA_ERR_UNSUPPORTED;
+  return MSA_OK;
+}
+}  // namespace
+
+size_t msa_paged_decode_fp8_workspace(const msa_paged_dims* d) {
+  if (check_paged_dims(d) != MSA_OK) return 0;
+  return kStatusBytes + msa::paged_decode_workspace_bytes(d->S, d->max_pages, d->H_q, d->H_kv,
+                                                          d->d_h, d->B_k, d->k);
+}
+
+msa_status msa_paged_decode_fp8(const msa_paged_dims* d, const void* q, const void* q_idx,
+                                const void* k_new, const void* v_new, const void* k_idx_new,
+                                void* k_pages, float* k_scale, void* v_pages, float* v_scale,
+                                void* kidx_pages, float* kidx_scale, const int32_t* page_table,
+                                int32_t* seq_len, void* o, int32_t* idx_out, void* ws,
+                                size_t ws_bytes, void* stream) {
+  msa_status st = check_paged_dims(d);
+  if (st != MSA_OK) return st;
+  const void* ptrs[] = {q, q_idx, k_new, v_new, k_idx_new, k_pages, k_scale, v_pages, v_scale,
+                        kidx_pages, kidx_scale, page_table, seq_len, o, ws};
+  for (const void* p : ptrs)
+    if (p == nullptr || !aligned16(p)) return MSA_ERR_INVALID_ARG;
+  if (idx_out != nullptr && !aligned16(idx_out)) return MSA_ERR_INVALID_ARG;
+  if (ws_bytes < msa_paged_decode_fp8_workspace(d)) return MSA_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (from_cuda(cudaMemsetAsync(ws, 0, sizeof(msa::DevStatus), s)) != MSA_OK) return MSA_ERR_CUDA;
+  msa::PagedLaunch a;
+  a.q = q;
+  a.q_idx = q_idx;
+  a.k_new = k_new;
+  a.v_new = v_new;
+  a.k_idx_new = k_idx_new;
+  a.k_pages = k_pages;
+  a.k_scale = k_scale;
+  a.v_pages = v_pages;
+  a.v_scale = v_scale;
+  a.kidx_pages = kidx_pages;
+  a.kidx_scale = kidx_scale;
+  a.page_table = page_table;
+  a.seq_len = seq_len;
+  a.o = o;
+  a.idx_out = idx_out;
+  a.S = d->S;
+  a.max_pages = d->max_pages;
+  a.n_pages = d->n_pages;
+  a.H_q = d->H_q;
+  a.H_kv = d->H_kv;
+  a.d_h = d->d_h;
+  a.d_idx = d->d_idx;
+  a.B_k = d->B_k;
+  a.kk = d->k;
+  a.scale = d->attn_scale > 0.0f ? d->attn_scale : 1.0f / sqrtf(static_cast<float>(d->d_h));
+  a.ws = static_cast<uint8_t*>(ws) + kStatusBytes;
+  a.ws_bytes = ws_bytes - kStatusBytes;
+  a.status = status_of(ws);
+  return from_cuda(msa::launch_paged_decode_fp8(a, s));
+}
+
+msa_status msa_quantize_fp8_rows(const void* x, int64_t n_rows, int32_t dim, void* codes,
+                                 float* scales, void* stream) {
+  if (x == nullptr || codes == nullptr || scales == nullptr || n_rows < 1 || dim < 2 ||
+      dim % 2 != 0 || dim > 4096 || !aligned16(x) || !aligned16(codes) || !aligned16(scales))
+    return MSA_ERR_INVALID_ARG;
+  return from_cuda(msa::launch_quantize_fp8_rows(x, n_rows, dim, codes, scales,
+                                                 reinterpret_cast<cudaStream_t>(stream)));
+}
+
 msa_status msa_profile_enable(int32_t on) {
   std::lock_guard<std::mutex> lk(msa::g_prof_mu);
   if (on) {

@@ -86,4 +86,34 @@ struct DecodeLaunch {
 size_t decode_workspace_bytes(int S, int64_t L_max, int H_q, int H_kv, int d_h, int B_k, int kk);
 cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t s);
 
+struct PagedLaunch {
+  const void* q;
+  const void* q_idx;
+  const void* k_new;
+  const void* v_new;
+  const void* k_idx_new;
+  void* k_pages;
+  float* k_scale;
+  void* v_pages;
+  float* v_scale;
+  void* kidx_pages;
+  float* kidx_scale;
+  const int32_t* page_table;
+  int32_t* seq_len;
+  void* o;
+  int32_t* idx_out;
+  int S, max_pages;
+  int64_t n_pages;
+  int H_q, H_kv, d_h, d_idx, B_k, kk;
+  float scale;
+  void* ws;
+  size_t ws_bytes;
+  DevStatus* status;
+};
+size_t paged_decode_workspace_bytes(int S, int max_pages, int H_q, int H_kv, int d_h, int B_k,
+                                    int kk);
+cudaError_t launch_paged_decode_fp8(const PagedLaunch& a, cudaStream_t s);
+cudaError_t launch_quantize_fp8_rows(const void* x, int64_t n_rows, int dim, void* codes,
+                                     float* scales, cudaStream_t s);
+
 }  // namespace msa

@@ -111,6 +111,9 @@ CONFIGS: Dict[str, object] = {
     # for counter captures of the decode kernels
     "decode8": DecodeConfig("decode8", S=8, L0=131072, steps=256, H_q=32, H_kv=4, d_h=128,
                             d_idx=64, B_k=128, k=16, seed_index=5),
+    # the decode workload on a paged FP8 (E4M3) cache (decode_fp8_state)
+    "decode_fp8": DecodeConfig("decode_fp8", S=64, L0=131072, steps=256, H_q=32, H_kv=4,
+                               d_h=128, d_idx=64, B_k=128, k=16, seed_index=6),
     # 1M-token prefill with a strong sink (block 0 picked by >= 90% of rows)
     "1m": MSAConfig("1m", N=1048576, H_q=32, H_kv=4, d_h=128, d_idx=64, B_k=128, k=16,
                     structure="sink_ar1", sink_strength=3.0, seed_index=4),
@@ -285,6 +288,70 @@ def decode_step_inputs(cfg: DecodeConfig, step: int, sink: np.ndarray,
         "v_new": _normal_bf16(r_v, (S, H_kv, d_h)),
         "k_idx_new": _normal_bf16(r_ki, (S, d_idx)),
     }
+
+
+def decode_fp8_state(cfg: DecodeConfig, seed: Optional[int] = None) -> Dict[str, np.ndarray]:
+    """A paged FP8 (E4M3) decode cache drawn directly as codes and scales.
+
+    Pages hold B_k tokens; page_table [S, n_blocks] is a seeded random
+    permutation of the n_pages = S * n_blocks pages (n_blocks = L_max / B_k,
+    rounded up), so every sequence's blocks are scattered over the pool.
+    Codes are uniform over the E4M3 bit patterns whose exponent field is at
+    most 9 (magnitude below 8, no NaN) with a random sign; scales are uniform
+    in [0.05, 0.15).  Sink: the index keys of every sequence's block 0 carry
+    the exponent-6 code 0x30 (value 0.5) with the sign of the sequence's unit
+    vector u, and scale 0.6, so index queries drawn around u score block 0
+    high.  Only the first L0 tokens are meaningful; seq_len = L0.
+    Returns k_pages/v_pages [P,B_k,H_kv,d_h] uint8, k_scale/v_scale
+    [P,B_k,H_kv] float32, kidx_pages [P,B_k,d_idx] uint8, kidx_scale [P,B_k]
+    float32, page_table [S,n_blocks] int32, seq_len [S] int32, sink [S,d_idx].
+    """
+    import os
+    from concurrent.futures import ThreadPoolExecutor
+
+    ss = np.random.SeedSequence((cfg.seed if seed is None else seed) + 77)
+    s_pt, s_k, s_v, s_ki, s_sc, s_sink = ss.spawn(6)
+    S, B_k, H_kv, d_h, d_idx = cfg.S, cfg.B_k, cfg.H_kv, cfg.d_h, cfg.d_idx
+    n_blocks = (cfg.L_max + B_k - 1) // B_k
+    P = S * n_blocks
+    page_table = np.random.default_rng(s_pt).permutation(P).astype(np.int32).reshape(S, n_blocks)
+
+    def codes(seq, shape):
+        n = int(np.prod(shape))
+        out = np.empty(n, dtype=np.uint8)
+        starts = list(range(0, n, _CHUNK))
+        kids = seq.spawn(len(starts))
+
+        def fill(j):
+            a, b = starts[j], min(n, starts[j] + _CHUNK)
+            r = np.random.default_rng(kids[j])
+            out[a:b] = (r.integers(0, 0x50, b - a, dtype=np.uint8)
+                        | (r.integers(0, 2, b - a, dtype=np.uint8) << 7))
+
+        with ThreadPoolExecutor(max_workers=min(len(starts), os.cpu_count() or 1)) as ex:
+            list(ex.map(fill, range(len(starts))))
+        return out.reshape(shape)
+
+    r_sc = np.random.default_rng(s_sc)
+    out = {
+        "k_pages": codes(s_k, (P, B_k, H_kv, d_h)),
+        "v_pages": codes(s_v, (P, B_k, H_kv, d_h)),
+        "kidx_pages": codes(s_ki, (P, B_k, d_idx)),
+        "k_scale": r_sc.uniform(0.05, 0.15, (P, B_k, H_kv)).astype(np.float32),
+        "v_scale": r_sc.uniform(0.05, 0.15, (P, B_k, H_kv)).astype(np.float32),
+        "kidx_scale": r_sc.uniform(0.05, 0.15, (P, B_k)).astype(np.float32),
+        "page_table": page_table,
+        "seq_len": np.full(S, cfg.L0, dtype=np.int32),
+    }
+    r_sink = np.random.default_rng(s_sink)
+    sink = np.stack([_unit(r_sink, d_idx) for _ in range(S)])
+    sign = (sink < 0).astype(np.uint8) << 7
+    for s_ in range(S):
+        pg = page_table[s_, 0]
+        out["kidx_pages"][pg] = (0x30 | sign[s_])[None, :]
+        out["kidx_scale"][pg] = np.float32(0.6)
+    out["sink"] = sink
+    return out
 
 
 def zipf_indices(N: int, H_kv: int, B_k: int, k: int, p_sink: float = 0.9,

@@ -205,6 +205,55 @@ MSA_API msa_status msa_index_lse(const msa_dims* dims, const void* q_idx, const 
                                  const int32_t* idx, float* lse_idx, void* workspace,
                                  size_t workspace_bytes, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * One decode step on a paged FP8 KV cache (the open implementation's "paged
+ * FP8 decode"; chlience notes, section 6, system-configuration row).  Same
+ * method as msa_sparse_decode (Eq. 1's i <= t, Eq. 6-8 for the new token of
+ * each sequence), on a cache of E4M3 codes with float32 scales:
+ *   value = e4m3(code) * scale  (OCP E4M3: bias 7, 3 mantissa bits, max 448)
+ * The cache is a pool of pages of B_k consecutive tokens; logical block b of
+ * sequence s lives in page page_table[s * max_pages + b]:
+ *   k_pages, v_pages  [n_pages, B_k, H_kv, d_h] uint8 codes
+ *   k_scale, v_scale  [n_pages, B_k, H_kv] fp32 (one per token and KV head)
+ *   kidx_pages        [n_pages, B_k, d_idx] uint8 codes
+ *   kidx_scale        [n_pages, B_k] fp32 (one per token)
+ *   page_table        [S, max_pages] int32 page indices (device); the pages
+ *                     of blocks 0 .. seq_len[s] / B_k must be assigned
+ * For each sequence with L = seq_len[s]: the new token's k_new, v_new (per KV
+ * head) and k_idx_new rows are quantized (scale = amax / 448 in fp32, 1 for
+ * an all-zero row; code = E4M3 of x / scale, nearest-even, saturated) into
+ * slot L % B_k of page page_table[s, L / B_k]; then the step runs on the
+ * dequantized cache and seq_len[s] becomes L + 1.  The other arguments are
+ * those of msa_sparse_decode.  A page index outside [0, n_pages) is skipped
+ * and recorded as MSA_DEV_BAD_INDEX; a sequence whose next token falls past
+ * max_pages * B_k is skipped and recorded as MSA_DEV_CACHE_FULL.
+ * Supported: d_h in {64,128}, d_idx in {64,128}, B_k in {64,128},
+ * H_q/H_kv <= 16, H_kv <= 8, 1 <= k <= 32.
+ * ------------------------------------------------------------------------- */
+typedef struct {
+  int32_t S;
+  int32_t max_pages;  /* page-table entries per sequence */
+  int64_t n_pages;    /* pages in the pool */
+  int32_t H_q, H_kv, d_h, d_idx, B_k, k;
+  float attn_scale;
+  float idx_scale;
+} msa_paged_dims;
+MSA_API size_t msa_paged_decode_fp8_workspace(const msa_paged_dims* dims);
+MSA_API msa_status msa_paged_decode_fp8(const msa_paged_dims* dims, const void* q,
+                                        const void* q_idx, const void* k_new, const void* v_new,
+                                        const void* k_idx_new, void* k_pages, float* k_scale,
+                                        void* v_pages, float* v_scale, void* kidx_pages,
+                                        float* kidx_scale, const int32_t* page_table,
+                                        int32_t* seq_len, void* o, int32_t* idx_out,
+                                        void* workspace, size_t ws_bytes, void* stream);
+
+/* Quantize n_rows bf16 rows of `dim` values (dim even, <= 4096) to E4M3
+ * codes [n_rows, dim] and one fp32 scale per row [n_rows], with the rule the
+ * FP8 decode uses for its appends (for filling a paged FP8 cache from bf16
+ * keys and values).  All pointers 16-byte aligned device memory. */
+MSA_API msa_status msa_quantize_fp8_rows(const void* x, int64_t n_rows, int32_t dim, void* codes,
+                                         float* scales, void* stream);
+
 /* Device status codes written into the workspace's status word. */
 #define MSA_DEV_OK 0
 #define MSA_DEV_TIMEOUT 1    /* a bounded on-device wait gave up; outputs invalid */
