@@ -11,7 +11,7 @@ synthetic inputs with a sink block and retrieval blocks).  Inputs (Q alone is
 
 On one GPU the 128K line also carries, under "also", the other two parts of
 the metric, each measured the same way: the 1M-token prefill ("1m", 3 steps
-after 2 warm-up steps), the 64-sequence decode workload ("decode", 200 steps
+after 2 warm-up steps), the 64-sequence decode workload ("decode", 1000 steps
 after 10 warm-up steps, us per token) and the same decode on a paged FP8
 (E4M3) cache ("decode_fp8").  For N > 1 each rank runs an
 independent replica (its own sequence): the path has no exchange step, so
@@ -747,11 +747,11 @@ def main():
                                  cpu_rows=0 if args.no_cpu_baseline else 32)
             free_device_memory()
             cdec = workload("decode")
-            also["decode"] = run_decode(args, cdec, rank, world, local, steps=200, warmup=10,
+            also["decode"] = run_decode(args, cdec, rank, world, local, steps=1000, warmup=10,
                                         e2e_steps=8, cpu_seqs=0 if args.no_cpu_baseline else 4)
             free_device_memory()
             also["decode_fp8"] = run_decode(args, workload("decode_fp8"), rank, world, local,
-                                            steps=200, warmup=10, e2e_steps=8,
+                                            steps=1000, warmup=10, e2e_steps=8,
                                             cpu_seqs=0 if args.no_cpu_baseline else 4)
             line["also"] = also
         if rank == 0 and line is not None:

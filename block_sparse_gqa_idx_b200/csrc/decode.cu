@@ -16,6 +16,8 @@
 //
 // Source: xllm-io paper review, "核心公式" Eq. 1, 6, 7, 8; chlience notes
 // 5.1.1 (selection steps) and 5.4 (exp-free selection on raw scores).
+#include <atomic>
+
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -622,6 +624,13 @@ __device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint16_t c2) {
   return pack_bf16(f.x, f.y);
 }
 
+// Two E4M3 codes -> an f16 pair (exact: E4M3's range and precision lie
+// inside f16's normal and subnormal values), one conversion instruction.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t c2) {
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(c2), __NV_E4M3);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
 // A page index of the table, or -1 (reported) when it is outside the pool.
 __device__ __forceinline__ int64_t page_of(const DecParams& p, const Dec8Params& q8, int s,
                                            int64_t b) {
@@ -635,10 +644,14 @@ __device__ __forceinline__ int64_t page_of(const DecParams& p, const Dec8Params&
 
 // Scan (and append): as dec_scan_kernel, over the index-key pages.  Thread t
 // of a quad owns d in [t*D/4, (t+1)*D/4) of its two key rows; the codes are
-// widened to bf16 pairs in registers and each key's dot is scaled by the
-// key's scale before the block maximum.
+// widened to f16 pairs in registers (one instruction per pair) and each
+// key's dot is scaled by the key's scale before the block maximum.  The
+// index query enters the f16 MMA multiplied by a power of two 2^e_r that
+// puts its largest magnitude in [2^13, 2^14): every bf16 value within 2^-30
+// of that maximum converts to f16 exactly, and the dot is multiplied by
+// 2^-e_r afterwards, so the scores are those of the bf16 query.
 template <int D_IDX, int BK>
-__global__ void __launch_bounds__(256) dec8_scan_kernel(const DecParams p, const Dec8Params q8,
+__global__ void __launch_bounds__(256, 4) dec8_scan_kernel(const DecParams p, const Dec8Params q8,
                                                         int nsplit) {
   constexpr int DT = D_IDX / 4;     // codes per thread and key row
   constexpr int NMMA = D_IDX / 16;  // MMAs per 16-key tile
@@ -681,52 +694,88 @@ __global__ void __launch_bounds__(256) dec8_scan_kernel(const DecParams p, const
   const int64_t b_i = L / p.B_k;  // candidate blocks 0 .. b_i-1 (full, not the local one)
   const int g = lane >> 2, t = lane & 3;
   uint32_t bq[NMMA][2];
+  float unscale0, unscale1;  // 2^-e of the heads in columns 2t and 2t+1
   {
     const __nv_bfloat16* qr = p.q_idx + (static_cast<int64_t>(s) * p.H_kv + (g < p.H_kv ? g : 0)) * D_IDX;
+    float qv[NMMA][4];
+    float amax = 0.f;
 #pragma unroll
     for (int j = 0; j < NMMA; ++j) {
       const int d0 = t * DT + 4 * j;
-      const uint32_t lo = *reinterpret_cast<const uint32_t*>(qr + d0);
-      const uint32_t hi = *reinterpret_cast<const uint32_t*>(qr + d0 + 2);
-      bq[j][0] = g < p.H_kv ? lo : 0u;
-      bq[j][1] = g < p.H_kv ? hi : 0u;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        qv[j][e] = g < p.H_kv ? __bfloat162float(qr[d0 + e]) : 0.f;
+        amax = fmaxf(amax, fabsf(qv[j][e]));
+      }
     }
+    amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
+    const int shift = amax > 0.f ? min(13 - ilogbf(amax), 126) : 0;
+#pragma unroll
+    for (int j = 0; j < NMMA; ++j) {
+      const __half2 lo = __floats2half2_rn(ldexpf(qv[j][0], shift), ldexpf(qv[j][1], shift));
+      const __half2 hi = __floats2half2_rn(ldexpf(qv[j][2], shift), ldexpf(qv[j][3], shift));
+      bq[j][0] = *reinterpret_cast<const uint32_t*>(&lo);
+      bq[j][1] = *reinterpret_cast<const uint32_t*>(&hi);
+    }
+    unscale0 = ldexpf(1.f, -__shfl_sync(0xFFFFFFFFu, shift, (2 * t) * 4));
+    unscale1 = ldexpf(1.f, -__shfl_sync(0xFFFFFFFFu, shift, (2 * t + 1) * 4));
   }
   const int wstride = nsplit * 8;
+  // the next block's page index is fetched while this block's codes load
+  const int* ptab = q8.page_table + static_cast<int64_t>(s) * q8.max_pages;
+  int pg_next = blockIdx.x * 8 + warp < b_i ? __ldg(ptab + blockIdx.x * 8 + warp) : 0;
   for (int64_t b = blockIdx.x * 8 + warp; b < b_i; b += wstride) {
-    const int64_t pg = page_of(p, q8, s, b);
-    if (pg < 0) continue;
+    const int64_t pg = pg_next;
+    if (b + wstride < b_i) pg_next = __ldg(ptab + b + wstride);
+    if (pg < 0 || pg >= q8.n_pages) {
+      report(p.status, DEV_ERR_BAD_INDEX, 88, s, static_cast<int>(pg));
+      continue;
+    }
     const uint8_t* kbase = q8.kidx_pages + pg * BK * D_IDX;
     const float* sbase = q8.kidx_scale + pg * BK;
     float mx0 = -INFINITY, mx1 = -INFINITY;  // columns 2t, 2t+1
+    // the block in two halves of NTILE/2 tiles: each half's codes are all
+    // loaded before its arithmetic, so they are in flight together
+    constexpr int NTILE = BK / 16, NU = DT / 16, HALF = NTILE / 2;
 #pragma unroll
-    for (int tile = 0; tile < BK / 16; ++tile) {
-      const int row0 = tile * 16 + g;
-      const uint8_t* r0 = kbase + row0 * D_IDX + t * DT;
-      const uint8_t* r1 = r0 + 8 * D_IDX;
-      uint32_t w0[DT / 2], w1[DT / 2];  // bf16 pairs of rows g and g + 8
+    for (int h = 0; h < 2; ++h) {
+      uint4 cr0[HALF][NU], cr1[HALF][NU];
 #pragma unroll
-      for (int u = 0; u < DT / 16; ++u) {
-        const uint4 c0 = __ldg(reinterpret_cast<const uint4*>(r0) + u);
-        const uint4 c1 = __ldg(reinterpret_cast<const uint4*>(r1) + u);
-        const uint16_t* h0 = reinterpret_cast<const uint16_t*>(&c0);
-        const uint16_t* h1 = reinterpret_cast<const uint16_t*>(&c1);
+      for (int i = 0; i < HALF; ++i) {
+        const uint8_t* r0 = kbase + ((h * HALF + i) * 16 + g) * D_IDX + t * DT;
+        const uint8_t* r1 = r0 + 8 * D_IDX;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          w0[u * 8 + e] = e4m3x2_to_bf16x2(h0[e]);
-          w1[u * 8 + e] = e4m3x2_to_bf16x2(h1[e]);
+        for (int u = 0; u < NU; ++u) {
+          cr0[i][u] = __ldg(reinterpret_cast<const uint4*>(r0) + u);
+          cr1[i][u] = __ldg(reinterpret_cast<const uint4*>(r1) + u);
         }
       }
-      float c[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int j = 0; j < NMMA; ++j) {
-        // k-slots 2t,2t+1 <- d0,d0+1 ; 2t+8,2t+9 <- d0+2,d0+3 (d0 = t*DT + 4j)
-        const uint32_t a[4] = {w0[2 * j], w1[2 * j], w0[2 * j + 1], w1[2 * j + 1]};
-        mma_bf16_16816(c, a, bq[j][0], bq[j][1]);
+      for (int i = 0; i < HALF; ++i) {
+        const int tile = h * HALF + i;
+        uint32_t w0[DT / 2], w1[DT / 2];  // f16 pairs of rows g and g + 8
+#pragma unroll
+        for (int u = 0; u < NU; ++u) {
+          const uint16_t* h0 = reinterpret_cast<const uint16_t*>(&cr0[i][u]);
+          const uint16_t* h1 = reinterpret_cast<const uint16_t*>(&cr1[i][u]);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            w0[u * 8 + e] = e4m3x2_to_f16x2(h0[e]);
+            w1[u * 8 + e] = e4m3x2_to_f16x2(h1[e]);
+          }
+        }
+        float c[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int j = 0; j < NMMA; ++j) {
+          // k-slots 2t,2t+1 <- d0,d0+1 ; 2t+8,2t+9 <- d0+2,d0+3 (d0 = t*DT + 4j)
+          const uint32_t a[4] = {w0[2 * j], w1[2 * j], w0[2 * j + 1], w1[2 * j + 1]};
+          mma_f16_16816(c, a, bq[j][0], bq[j][1]);
+        }
+        const float s0 = __ldg(sbase + tile * 16 + g), s1 = __ldg(sbase + tile * 16 + g + 8);
+        mx0 = fmax3(mx0, (c[0] * unscale0) * s0, (c[2] * unscale0) * s1);
+        mx1 = fmax3(mx1, (c[1] * unscale1) * s0, (c[3] * unscale1) * s1);
       }
-      const float s0 = __ldg(sbase + row0), s1 = __ldg(sbase + row0 + 8);
-      mx0 = fmax3(mx0, c[0] * s0, c[2] * s1);
-      mx1 = fmax3(mx1, c[1] * s0, c[3] * s1);
     }
 #pragma unroll
     for (int o = 4; o < 32; o <<= 1) {
@@ -766,24 +815,54 @@ __global__ void __launch_bounds__(128) dec8_attend_kernel(const DecParams p, con
   const int slot = item % p.kk;
   const int r = (item / p.kk) % p.H_kv;
   const int s = item / (p.kk * p.H_kv);
+  // both loads issue before either is tested (they do not depend on each other)
   const int64_t L = p.w.Lcur[s];
-  if (L < 0) return;
   const int b = p.w.sel[(static_cast<int64_t>(s) * p.H_kv + r) * p.kk + slot];
-  if (b < 0) return;
+  if (L < 0 || b < 0) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
+  // Q fragments (rows = heads, zero beyond G), in flight with the page lookup
+  uint32_t qa[D_H / 16][4];
+  {
+    const __nv_bfloat16* qb = p.q + (static_cast<int64_t>(s) * p.H_q + r * p.G) * D_H;
+#pragma unroll
+    for (int ks = 0; ks < D_H / 16; ++ks) {
+      const int d = ks * 16 + 2 * t;
+      qa[ks][0] = g < p.G ? *reinterpret_cast<const uint32_t*>(qb + g * D_H + d) : 0u;
+      qa[ks][1] = g + 8 < p.G ? *reinterpret_cast<const uint32_t*>(qb + (g + 8) * D_H + d) : 0u;
+      qa[ks][2] = g < p.G ? *reinterpret_cast<const uint32_t*>(qb + g * D_H + d + 8) : 0u;
+      qa[ks][3] = g + 8 < p.G ? *reinterpret_cast<const uint32_t*>(qb + (g + 8) * D_H + d + 8) : 0u;
+    }
+  }
   const int64_t pg = page_of(p, q8, s, b);
   if (pg < 0) return;
   const int64_t last = L;  // the new token's position: keys j <= last
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int g = lane >> 2, t = lane & 3;
 
-  // the block's codes -> bf16 tiles [d-chunk][key][64] with 128-byte swizzle
-  for (int c = threadIdx.x; c < BK * CPK; c += blockDim.x) {
+  // the block's codes -> bf16 tiles [d-chunk][key][64] with 128-byte swizzle;
+  // every load of the thread is issued before the first conversion, so the
+  // CTA has its whole 2*BK*D_H bytes in flight at once
+  constexpr int PER_T = BK * CPK / 128;  // 16-code pieces per thread and tensor
+  static_assert(BK * CPK % 128 == 0, "pieces divide over the 128 threads");
+  uint4 kcs[PER_T], vcs[PER_T];
+#pragma unroll
+  for (int i = 0; i < PER_T; ++i) {
+    const int c = threadIdx.x + i * 128;
     const int key = c / CPK, piece = c - key * CPK;
     const int64_t row = ((pg * BK + key) * p.H_kv + r) * D_H + piece * 16;
-    const uint4 kc = __ldg(reinterpret_cast<const uint4*>(q8.k_pages + row));
-    const uint4 vc = __ldg(reinterpret_cast<const uint4*>(q8.v_pages + row));
-    const uint16_t* hk = reinterpret_cast<const uint16_t*>(&kc);
-    const uint16_t* hv = reinterpret_cast<const uint16_t*>(&vc);
+    kcs[i] = __ldg(reinterpret_cast<const uint4*>(q8.k_pages + row));
+    vcs[i] = __ldg(reinterpret_cast<const uint4*>(q8.v_pages + row));
+  }
+  float ks_reg = 0.f, vs_reg = 0.f;
+  if (threadIdx.x < BK) {
+    ks_reg = __ldg(q8.k_scale + (pg * BK + threadIdx.x) * p.H_kv + r);
+    vs_reg = __ldg(q8.v_scale + (pg * BK + threadIdx.x) * p.H_kv + r);
+  }
+#pragma unroll
+  for (int i = 0; i < PER_T; ++i) {
+    const int c = threadIdx.x + i * 128;
+    const int key = c / CPK, piece = c - key * CPK;
+    const uint16_t* hk = reinterpret_cast<const uint16_t*>(&kcs[i]);
+    const uint16_t* hv = reinterpret_cast<const uint16_t*>(&vcs[i]);
     uint4 k0, k1, v0, v1;
     uint32_t* pk0 = reinterpret_cast<uint32_t*>(&k0);
     uint32_t* pk1 = reinterpret_cast<uint32_t*>(&k1);
@@ -803,22 +882,10 @@ __global__ void __launch_bounds__(128) dec8_attend_kernel(const DecParams p, con
     *reinterpret_cast<uint4*>(sV + o0) = v0;
     *reinterpret_cast<uint4*>(sV + o1) = v1;
   }
-  for (int j = threadIdx.x; j < BK; j += blockDim.x) {
-    ksc[j] = __ldg(q8.k_scale + (pg * BK + j) * p.H_kv + r);
-    vsc[j] = __ldg(q8.v_scale + (pg * BK + j) * p.H_kv + r);
-  }
-  // Q fragments (rows = heads, zero beyond G)
-  uint32_t qa[D_H / 16][4];
-  {
-    const __nv_bfloat16* qb = p.q + (static_cast<int64_t>(s) * p.H_q + r * p.G) * D_H;
-#pragma unroll
-    for (int ks = 0; ks < D_H / 16; ++ks) {
-      const int d = ks * 16 + 2 * t;
-      qa[ks][0] = g < p.G ? *reinterpret_cast<const uint32_t*>(qb + g * D_H + d) : 0u;
-      qa[ks][1] = g + 8 < p.G ? *reinterpret_cast<const uint32_t*>(qb + (g + 8) * D_H + d) : 0u;
-      qa[ks][2] = g < p.G ? *reinterpret_cast<const uint32_t*>(qb + g * D_H + d + 8) : 0u;
-      qa[ks][3] = g + 8 < p.G ? *reinterpret_cast<const uint32_t*>(qb + (g + 8) * D_H + d + 8) : 0u;
-    }
+  static_assert(BK <= 128, "one key scale per thread");
+  if (threadIdx.x < BK) {
+    ksc[threadIdx.x] = ks_reg;
+    vsc[threadIdx.x] = vs_reg;
   }
   __syncthreads();
   const int kw0 = warp * KW;  // first key (within the block) of this warp
@@ -942,6 +1009,25 @@ __global__ void __launch_bounds__(128) dec8_attend_kernel(const DecParams p, con
     if (part == 0)
       p.w.part_lse[pslot] = wsum > 0.f ? (M + log2f(wsum)) * 0.6931471805599453f : -INFINITY;
   }
+}
+
+// CTAs per sequence of the FP8 scan: the S sequences share one wave of the
+// CTAs the device holds at once (resident CTAs per SM from the kernel's
+// registers, times the SMs), at most 64.
+template <int D_IDX, int BK>
+int scan8_split(int S) {
+  static std::atomic<int> slots{0};
+  int n = slots.load(std::memory_order_relaxed);
+  if (n == 0) {
+    int dev = 0, sms = 0, occ = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, dec8_scan_kernel<D_IDX, BK>, 256, 0);
+    n = (occ > 0 ? occ : 1) * (sms > 0 ? sms : 1);
+    slots.store(n, std::memory_order_relaxed);
+  }
+  const int per = n / (S > 0 ? S : 1);
+  return per < 1 ? 1 : (per > 64 ? 64 : per);
 }
 
 template <int D_H, int BK>
@@ -1073,7 +1159,11 @@ cudaError_t launch_paged_decode_fp8(const PagedLaunch& a, cudaStream_t stream) {
   q8.max_pages = a.max_pages;
   q8.n_pages = a.n_pages;
 
-  const int nsplit = a.S >= 64 ? 8 : (a.S >= 16 ? 32 : 64);
+  int nsplit;
+  if (a.d_idx == 64 && a.B_k == 128) nsplit = scan8_split<64, 128>(a.S);
+  else if (a.d_idx == 64) nsplit = scan8_split<64, 64>(a.S);
+  else if (a.B_k == 128) nsplit = scan8_split<128, 128>(a.S);
+  else nsplit = scan8_split<128, 64>(a.S);
   const dim3 sgrid(nsplit, a.S);
   prof_begin("dec8_scan", stream);
   if (a.d_idx == 64 && a.B_k == 128) dec8_scan_kernel<64, 128><<<sgrid, 256, 0, stream>>>(p, q8, nsplit);

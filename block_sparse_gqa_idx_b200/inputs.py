@@ -105,14 +105,14 @@ CONFIGS: Dict[str, object] = {
     "128k": MSAConfig("128k", N=131072, H_q=32, H_kv=4, d_h=128, d_idx=64, B_k=128, k=16,
                       structure="sink_ar1_retrieval", seed_index=2),
     # decode: 64 sequences of 131072 cached tokens, 256 appended steps
-    "decode": DecodeConfig("decode", S=64, L0=131072, steps=256, H_q=32, H_kv=4, d_h=128,
+    "decode": DecodeConfig("decode", S=64, L0=131072, steps=1152, H_q=32, H_kv=4, d_h=128,
                            d_idx=64, B_k=128, k=16, seed_index=3),
     # the decode step at 8 sequences (2.3 GB of caches): a case small enough
     # for counter captures of the decode kernels
     "decode8": DecodeConfig("decode8", S=8, L0=131072, steps=256, H_q=32, H_kv=4, d_h=128,
                             d_idx=64, B_k=128, k=16, seed_index=5),
     # the decode workload on a paged FP8 (E4M3) cache (decode_fp8_state)
-    "decode_fp8": DecodeConfig("decode_fp8", S=64, L0=131072, steps=256, H_q=32, H_kv=4,
+    "decode_fp8": DecodeConfig("decode_fp8", S=64, L0=131072, steps=1152, H_q=32, H_kv=4,
                                d_h=128, d_idx=64, B_k=128, k=16, seed_index=6),
     # 1M-token prefill with a strong sink (block 0 picked by >= 90% of rows)
     "1m": MSAConfig("1m", N=1048576, H_q=32, H_kv=4, d_h=128, d_idx=64, B_k=128, k=16,

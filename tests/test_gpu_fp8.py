@@ -42,9 +42,11 @@ def _dev_pages(st):
     return {k: torch.from_numpy(np.ascontiguousarray(st[k])).cuda() for k in keys}
 
 
-def _run(msa, cfg, st, steps, seqs):
+def _run(msa, cfg, st, steps, seqs, q_idx_pow2=None):
     """`steps` decode steps on the GPU and on the oracle (which carries the
-    oracle's own quantized appends forward), comparing the listed sequences."""
+    oracle's own quantized appends forward), comparing the listed sequences.
+    q_idx_pow2: per index head, a power of two the index queries are
+    multiplied by (exact in bf16) before both sides see them."""
     dev = _dev_pages(st)
     seq_len = torch.from_numpy(st["seq_len"].copy()).cuda()
     host = {k: st[k].copy() for k in ("k_pages", "v_pages", "kidx_pages", "k_scale", "v_scale",
@@ -52,6 +54,10 @@ def _run(msa, cfg, st, steps, seqs):
     L = st["seq_len"].copy()
     for step in range(steps):
         si = inputs.decode_step_inputs(cfg, step, st["sink"])
+        if q_idx_pow2 is not None:
+            f = np.asarray(q_idx_pow2, dtype=np.float32)[None, :, None]
+            qf = (si["q_idx"].astype(np.uint32) << 16).view(np.float32) * f
+            si["q_idx"] = inputs.bf16_bits(qf)
         d = {k: to_dev(v) for k, v in si.items()}
         o = torch.full((cfg.S, cfg.H_q, cfg.d_h), float("nan"), dtype=torch.bfloat16,
                        device="cuda")
@@ -112,6 +118,15 @@ def test_paged_fp8_decode_full_size_sampled(msa):
     cfg = inputs.CONFIGS["decode_fp8"]
     st = inputs.decode_fp8_state(cfg)
     _run(msa, cfg, st, 2, np.array([0, 31, 63]))
+
+
+def test_paged_fp8_decode_index_query_magnitudes(msa):
+    """Index queries from 2^-24 to 2^24 times the recipe's (beyond f16's
+    range at both ends): the selection and outputs still match the oracle."""
+    cfg = inputs.DecodeConfig("fp8mag", S=4, L0=2000, steps=2, H_q=32, H_kv=4, d_h=128,
+                              d_idx=64, B_k=128, k=8, seed_index=68)
+    st = inputs.decode_fp8_state(cfg)
+    _run(msa, cfg, st, 2, np.arange(cfg.S), q_idx_pow2=[2.0 ** 24, 2.0 ** -24, 1.0, 2.0 ** 10])
 
 
 def test_paged_fp8_bad_page_is_reported(msa):
