@@ -46,6 +46,9 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # reported only while that code is unchanged.
 # kernel -> (source, kernel function, sha256, bytes per unit, unit)
 NCU_TRAFFIC = {
+    "attn_phase1": ("sparse_attn.cu", "attn_phase1_kernel",
+                    "f8cd4b0892d910c11d79d609f62236528ec32731aed1994bac70d3557c7e182a",
+                    (3.571552e9 + 4.184725e9) / 32768, "query"),
     "attn_merge": ("sparse_attn.cu", "attn_merge_kernel",
                    "beaa021d56c8173edcff10bc3f30370f75c95031da3075c63dc4e1054a981835",
                    (4.243224e9 + 0.269582e9) / 32768, "query"),

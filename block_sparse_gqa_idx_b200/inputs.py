@@ -114,6 +114,10 @@ CONFIGS: Dict[str, object] = {
     # the decode workload on a paged FP8 (E4M3) cache (decode_fp8_state)
     "decode_fp8": DecodeConfig("decode_fp8", S=64, L0=131072, steps=1152, H_q=32, H_kv=4,
                                d_h=128, d_idx=64, B_k=128, k=16, seed_index=6),
+    # the FP8 decode at 8 sequences (1.2 GB of pages): the case its kernels
+    # are profiled on
+    "decode_fp8_s8": DecodeConfig("decode_fp8_s8", S=8, L0=131072, steps=256, H_q=32, H_kv=4,
+                                  d_h=128, d_idx=64, B_k=128, k=16, seed_index=7),
     # 1M-token prefill with a strong sink (block 0 picked by >= 90% of rows)
     "1m": MSAConfig("1m", N=1048576, H_q=32, H_kv=4, d_h=128, d_idx=64, B_k=128, k=16,
                     structure="sink_ar1", sink_strength=3.0, seed_index=4),

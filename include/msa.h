@@ -16,7 +16,10 @@
  *     argument; "bf16" arguments hold IEEE bfloat16 values.  All tensor
  *     pointers are DEVICE pointers, 16-byte aligned, owned by the caller; the
  *     library never allocates or frees memory and keeps no pointer after the
- *     call returns.
+ *     call returns.  Its one piece of device memory of its own is a fixed
+ *     MSA_DECODE_NOALLOC_SCRATCH_BYTES array, resident on every device where
+ *     the library's module is loaded, which only msa_sparse_decode_noalloc
+ *     uses.
  *   - Every call is asynchronous on `stream` (a cudaStream_t, NULL = the
  *     legacy default stream).  Arguments are validated on the host first; on
  *     a validation error nothing is launched and the outputs are untouched.
