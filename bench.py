@@ -47,11 +47,11 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # kernel -> (source, kernel function, sha256, bytes per unit, unit)
 NCU_TRAFFIC = {
     "attn_phase1": ("sparse_attn.cu", "attn_phase1_kernel",
-                    "f8cd4b0892d910c11d79d609f62236528ec32731aed1994bac70d3557c7e182a",
-                    (3.571552e9 + 4.184725e9) / 32768, "query"),
+                    "91ddfb0015a1d8d22df128a8656c1976787bd4a09264ceab50825a78cac785c1",
+                    (3575268352 + 4186103552) / 32768, "query"),
     "attn_merge": ("sparse_attn.cu", "attn_merge_kernel",
-                   "beaa021d56c8173edcff10bc3f30370f75c95031da3075c63dc4e1054a981835",
-                   (4.243224e9 + 0.269582e9) / 32768, "query"),
+                   "b3995bc06ce2e51f1d1aca2b258c6c448bf62dd831be86d2dab58401aca75b38",
+                   (4243319552 + 265582848) / 32768, "query"),
 }
 
 

@@ -6,6 +6,7 @@ of ``include/msa.h``); this package is its thin Python binding:
 * ``index_topk``      Index Branch, Eq. 6-7 (fused scores, block max, Top-k)
 * ``sparse_attn_fwd`` Main Branch, Eq. 8 (KV-outer sparse attention + merge)
 * ``forward``         both, for one prefill sequence
+* ``forward_varlen``  both, for a packed batch of sequences of any lengths
 * ``sparse_decode``   one decode step for a batch of sequences
 * ``paged_decode_fp8`` the same step on a paged FP8 (E4M3) KV cache
 
@@ -18,7 +19,8 @@ _CAPI = ("index_topk", "sparse_attn_fwd", "forward", "sparse_decode", "device_st
          "sparse_attn_fwd_workspace_size", "sparse_decode_workspace_size", "EXPORTS", "LIB_PATH",
          "profile_enable", "profile_read", "sparse_decode_noalloc", "selftest_bounded_wait",
          "index_lse", "index_lse_workspace_size", "paged_dims", "paged_decode_fp8",
-         "paged_decode_fp8_workspace_size", "quantize_fp8_rows")
+         "paged_decode_fp8_workspace_size", "quantize_fp8_rows", "index_topk_varlen",
+         "sparse_attn_fwd_varlen", "forward_varlen", "varlen_dims")
 
 __all__ = list(_CAPI) + ["inputs"]
 

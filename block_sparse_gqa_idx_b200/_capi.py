@@ -46,6 +46,13 @@ class msa_paged_dims(ctypes.Structure):
                 ("attn_scale", ctypes.c_float), ("idx_scale", ctypes.c_float)]
 
 
+class msa_varlen_dims(ctypes.Structure):
+    _fields_ = [("n_seqs", ctypes.c_int32), ("N", ctypes.c_int64), ("H_q", ctypes.c_int32),
+                ("H_kv", ctypes.c_int32), ("d_h", ctypes.c_int32), ("d_idx", ctypes.c_int32),
+                ("B_k", ctypes.c_int32), ("k", ctypes.c_int32), ("attn_scale", ctypes.c_float),
+                ("idx_scale", ctypes.c_float)]
+
+
 class msa_kernel_time(ctypes.Structure):
     _fields_ = [("name", ctypes.c_char * 48), ("launches", ctypes.c_int32),
                 ("total_ms", ctypes.c_double)]
@@ -57,7 +64,9 @@ EXPORTS = ("msa_index_topk_workspace", "msa_index_topk", "msa_sparse_attn_fwd_wo
            "msa_get_device_status", "msa_profile_enable", "msa_profile_read",
            "msa_status_string", "msa_version", "msa_sparse_decode_noalloc", "msa_last_error",
            "msa_selftest_bounded_wait", "msa_index_lse_workspace", "msa_index_lse",
-           "msa_paged_decode_fp8_workspace", "msa_paged_decode_fp8", "msa_quantize_fp8_rows")
+           "msa_paged_decode_fp8_workspace", "msa_paged_decode_fp8", "msa_quantize_fp8_rows",
+           "msa_index_topk_varlen_workspace", "msa_index_topk_varlen",
+           "msa_sparse_attn_fwd_varlen_workspace", "msa_sparse_attn_fwd_varlen")
 
 
 def _load() -> ctypes.CDLL:
@@ -96,6 +105,15 @@ def _load() -> ctypes.CDLL:
     lib.msa_paged_decode_fp8.restype = I32
     lib.msa_quantize_fp8_rows.argtypes = [P, ctypes.c_int64, I32, P, P, P]
     lib.msa_quantize_fp8_rows.restype = I32
+    VD, CU = ctypes.POINTER(msa_varlen_dims), ctypes.POINTER(ctypes.c_int64)
+    lib.msa_index_topk_varlen_workspace.argtypes = [VD, CU]
+    lib.msa_index_topk_varlen_workspace.restype = Z
+    lib.msa_index_topk_varlen.argtypes = [VD, CU, P, P, P, P, P, Z, P]
+    lib.msa_index_topk_varlen.restype = I32
+    lib.msa_sparse_attn_fwd_varlen_workspace.argtypes = [VD, CU]
+    lib.msa_sparse_attn_fwd_varlen_workspace.restype = Z
+    lib.msa_sparse_attn_fwd_varlen.argtypes = [VD, CU, P, P, P, P, P, P, P, Z, P]
+    lib.msa_sparse_attn_fwd_varlen.restype = I32
     lib.msa_selftest_bounded_wait.argtypes = [P, P]
     lib.msa_selftest_bounded_wait.restype = I32
     lib.msa_profile_enable.argtypes = [ctypes.c_int32]
@@ -263,6 +281,87 @@ def forward(q, k, v, q_idx, k_idx, B_k: int, kk: int, attn_scale: float = 0.0, s
     """Whole MSA forward (Eq. 6-8): returns (o, lse, idx)."""
     idx = index_topk(q_idx, k_idx, B_k, kk, workspace=workspace, stream=stream)
     o, lse = sparse_attn_fwd(q, k, v, idx, B_k, attn_scale, workspace=workspace, stream=stream)
+    return o, lse, idx
+
+
+def _cu(cu_seqlens, N: int):
+    """cu_seqlens (a list, numpy array or CPU tensor of n + 1 ints) as a host
+    int64 array for the C ABI, with the count of sequences."""
+    vals = [int(x) for x in (cu_seqlens.tolist() if hasattr(cu_seqlens, "tolist")
+                             else cu_seqlens)]
+    if len(vals) < 2 or vals[0] != 0 or vals[-1] != N:
+        raise ValueError(f"cu_seqlens must run from 0 to N={N}")
+    return (ctypes.c_int64 * len(vals))(*vals), len(vals) - 1
+
+
+def varlen_dims(n_seqs, N, H_q, H_kv, d_h, d_idx, B_k, k, attn_scale=0.0,
+                idx_scale=0.0) -> msa_varlen_dims:
+    return msa_varlen_dims(int(n_seqs), int(N), int(H_q), int(H_kv), int(d_h), int(d_idx),
+                           int(B_k), int(k), float(attn_scale), float(idx_scale))
+
+
+def index_topk_varlen(q_idx: torch.Tensor, k_idx: torch.Tensor, cu_seqlens, B_k: int, k: int,
+                      idx_out: Optional[torch.Tensor] = None,
+                      score_out: Optional[torch.Tensor] = None, idx_scale: float = 0.0,
+                      workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Eq. 6-7 per sequence of a packed batch: q_idx [N,H_kv,d_idx], k_idx
+    [N,d_idx] bf16, sequence s = tokens cu_seqlens[s] .. cu_seqlens[s+1]-1 ->
+    idx [N,H_kv,k] int32 with block indices local to each token's sequence."""
+    N, H_kv, d_idx = q_idx.shape
+    _want(q_idx, "q_idx", torch.bfloat16, (N, H_kv, d_idx))
+    _want(k_idx, "k_idx", torch.bfloat16, (N, d_idx))
+    if idx_out is None:
+        idx_out = torch.empty((N, H_kv, k), dtype=torch.int32, device=q_idx.device)
+    _want(idx_out, "idx_out", torch.int32, (N, H_kv, k))
+    if score_out is not None:
+        _want(score_out, "score_out", torch.float32, (N, H_kv, k))
+    cu, n = _cu(cu_seqlens, N)
+    d = varlen_dims(n, N, H_kv, H_kv, 64, d_idx, B_k, k, idx_scale=idx_scale)
+    ws = _workspace(int(LIB.msa_index_topk_varlen_workspace(ctypes.byref(d), cu)), q_idx.device,
+                    workspace)
+    _raise("msa_index_topk_varlen",
+           LIB.msa_index_topk_varlen(ctypes.byref(d), cu, _ptr(q_idx), _ptr(k_idx), _ptr(idx_out),
+                                     _ptr(score_out), _ptr(ws), ws.numel(), _stream(stream)))
+    return idx_out
+
+
+def sparse_attn_fwd_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                           idx: torch.Tensor, cu_seqlens, B_k: int, attn_scale: float = 0.0,
+                           o: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                           want_lse: bool = True, workspace: Optional[torch.Tensor] = None,
+                           stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Eq. 8 per sequence of a packed batch (idx local to each sequence):
+    o [N,H_q,d_h] bf16 and lse [N,H_q] fp32."""
+    N, H_q, d_h = q.shape
+    H_kv = k.shape[1]
+    kk = idx.shape[2]
+    _want(q, "q", torch.bfloat16, (N, H_q, d_h))
+    _want(k, "k", torch.bfloat16, (N, H_kv, d_h))
+    _want(v, "v", torch.bfloat16, (N, H_kv, d_h))
+    _want(idx, "idx", torch.int32, (N, H_kv, kk))
+    if o is None:
+        o = torch.empty((N, H_q, d_h), dtype=torch.bfloat16, device=q.device)
+    _want(o, "o", torch.bfloat16, (N, H_q, d_h))
+    if lse is None and want_lse:
+        lse = torch.empty((N, H_q), dtype=torch.float32, device=q.device)
+    if lse is not None:
+        _want(lse, "lse", torch.float32, (N, H_q))
+    cu, n = _cu(cu_seqlens, N)
+    d = varlen_dims(n, N, H_q, H_kv, d_h, 64, B_k, kk, attn_scale)
+    ws = _workspace(int(LIB.msa_sparse_attn_fwd_varlen_workspace(ctypes.byref(d), cu)), q.device,
+                    workspace)
+    _raise("msa_sparse_attn_fwd_varlen",
+           LIB.msa_sparse_attn_fwd_varlen(ctypes.byref(d), cu, _ptr(q), _ptr(k), _ptr(v),
+                                          _ptr(idx), _ptr(o), _ptr(lse), _ptr(ws), ws.numel(),
+                                          _stream(stream)))
+    return o, lse
+
+
+def forward_varlen(q, k, v, q_idx, k_idx, cu_seqlens, B_k: int, kk: int, attn_scale: float = 0.0,
+                   stream=None):
+    """Whole MSA forward (Eq. 6-8) of a packed batch of sequences: (o, lse, idx)."""
+    idx = index_topk_varlen(q_idx, k_idx, cu_seqlens, B_k, kk, stream=stream)
+    o, lse = sparse_attn_fwd_varlen(q, k, v, idx, cu_seqlens, B_k, attn_scale, stream=stream)
     return o, lse, idx
 
 

@@ -54,6 +54,13 @@ struct IndexParams {
   int64_t N;
   int H_kv, B_k, k;
   int n_mtiles;
+  // several sequences packed along the token axis: one record per M-tile,
+  // longest first, {first Q_idx row, first token of the tile's sequence,
+  // local block of its queries, valid rows}; and per token {first token of
+  // its sequence, first global block of its sequence}.  Both null for one
+  // sequence.
+  const int4* tiles;
+  const int2* qinfo;
   int32_t* idx_out;
   float* score_out;  // [N, H_kv, k] or null: the selected blocks' Eq. 6 scores
   float scale;       // Eq. 6 scale applied to score_out
@@ -82,17 +89,35 @@ __device__ __forceinline__ int unit_of(int round, int cta, int nctas) {
   return round * nctas + ((round & 1) ? (nctas - 1 - cta) : cta);
 }
 
-// The block c of an M-tile's queries and the number of 256-key tiles holding
-// its candidate blocks 0..c-1 (0 if the M-tile does not exist or c = 0).
-__device__ __forceinline__ int mtile_ntiles(const IndexParams& p, int m, int* c_out) {
-  if (m >= p.n_mtiles) {
-    *c_out = 0;
-    return 0;
+// Work unit u (longest first): the M-tile's first Q_idx row, the first key
+// row of its sequence, the local block c of its queries (relative to the
+// sequence) and its valid rows.  Its candidate blocks 0..c-1 of the sequence
+// are keys key0 .. key0 + c*B_k - 1.
+struct MTile {
+  int64_t row0, key0;
+  int c, nrows;
+};
+__device__ __forceinline__ MTile mtile_of(const IndexParams& p, int u) {
+  MTile t;
+  if (p.tiles != nullptr) {
+    const int4 r = p.tiles[u];
+    t.row0 = r.x;
+    t.key0 = r.y;
+    t.c = r.z;
+    t.nrows = r.w;
+  } else {
+    const int m = p.n_mtiles - 1 - u;
+    t.row0 = static_cast<int64_t>(m) * kRows;
+    t.key0 = 0;
+    t.c = static_cast<int>(t.row0 / p.H_kv / p.B_k);
+    const int64_t left = p.N * p.H_kv - t.row0;
+    t.nrows = left < kRows ? static_cast<int>(left) : kRows;
   }
-  const int64_t i0 = (static_cast<int64_t>(m) * kRows) / p.H_kv;
-  const int c = static_cast<int>(i0 / p.B_k);
-  *c_out = c;
-  return static_cast<int>((static_cast<int64_t>(c) * p.B_k + kKeys - 1) / kKeys);
+  return t;
+}
+// 256-key tiles holding the candidate blocks 0..c-1 (0 when c = 0).
+__device__ __forceinline__ int mtile_ntiles(const IndexParams& p, const MTile& t) {
+  return static_cast<int>((static_cast<int64_t>(t.c) * p.B_k + kKeys - 1) / kKeys);
 }
 
 // Top-k keys: the score's order-preserving bits above the inverted block
@@ -190,14 +215,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int round = 0;; ++round) {
         const int u = unit_of(round, cta, nctas);
         if (u >= p.n_mtiles || *abort_flag) break;
-        const int m = p.n_mtiles - 1 - u;  // longest first
-        int c;
-        const int nt = mtile_ntiles(p, m, &c);
+        const MTile mt = mtile_of(p, u);  // longest first
+        const int nt = mtile_ntiles(p, mt);
         if (nt == 0) continue;
         if (!mbar_wait(a_empty, (ua & 1) ^ 1, abort_flag, p.status, 10)) break;
         mbar_arrive_expect_tx(a_full, S::A_BYTES);
         for (int ch = 0; ch < S::CH; ++ch)
-          tma_load_2d(sA + ch * kRows * S::SWB, &tm_q, a_full, ch * S::CHE, m * kRows);
+          tma_load_2d(sA + ch * kRows * S::SWB, &tm_q, a_full, ch * S::CHE,
+                      static_cast<int>(mt.row0));
         ++ua;
         bool ok = true;
         for (int t = 0; t < nt; ++t, ++g) {
@@ -209,7 +234,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_expect_tx(&b_full[st], S::B_BYTES);
           for (int ch = 0; ch < S::CH; ++ch)
             tma_load_2d(sB + st * S::B_BYTES + ch * kKeys * S::SWB, &tm_k, &b_full[st],
-                        ch * S::CHE, t * kKeys);
+                        ch * S::CHE, static_cast<int>(mt.key0) + t * kKeys);
         }
         if (!ok) break;
       }
@@ -222,9 +247,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int round = 0;; ++round) {
         const int u = unit_of(round, cta, nctas);
         if (u >= p.n_mtiles || *abort_flag) break;
-        const int m = p.n_mtiles - 1 - u;
-        int c;
-        const int nt = mtile_ntiles(p, m, &c);
+        const int nt = mtile_ntiles(p, mtile_of(p, u));
         if (nt == 0) continue;
         if (!mbar_wait(a_full, ua & 1, abort_flag, p.status, 20)) break;
         tc_fence_after();
@@ -274,9 +297,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int round = 0;; ++round, ++ucnt) {
       const int u = unit_of(round, cta, nctas);
       if (u >= p.n_mtiles || *abort_flag) break;
-      const int m = p.n_mtiles - 1 - u;
-      int c;
-      const int nt = mtile_ntiles(p, m, &c);
+      const MTile mt = mtile_of(p, u);
+      const int c = mt.c;
+      const int nt = mtile_ntiles(p, mt);
       // group 1 reuses its keys[] column once group 0 has merged the last unit
       if (grp == 1 && ucnt > 0 &&
           !mbar_wait(xch_empty, (ucnt - 1) & 1, abort_flag, p.status, 31))
@@ -441,8 +464,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(xch_empty);
-      const int64_t row_glob = static_cast<int64_t>(m) * kRows + row;
-      if (row_glob < p.N * p.H_kv) {
+      const int64_t row_glob = mt.row0 + row;
+      if (row < mt.nrows) {
         for (int a = 1; a < n; ++a) {  // ascending
           const int x = sel[a];
           const float xs = scr[a];
@@ -487,7 +510,8 @@ __global__ void __launch_bounds__(256) local_block_score_kernel(const __nv_bfloa
   const int lane = threadIdx.x & 31;
   if (row >= p.N * p.H_kv) return;
   const int64_t i = row / p.H_kv;
-  const int64_t b_i = i / p.B_k;
+  const int64_t i0 = p.qinfo != nullptr ? p.qinfo[i].x : 0;  // first token of i's sequence
+  const int64_t b_i = (i - i0) / p.B_k;
   float q[D_IDX];
   const __nv_bfloat16* qr = q_idx + row * D_IDX;
 #pragma unroll
@@ -497,7 +521,7 @@ __global__ void __launch_bounds__(256) local_block_score_kernel(const __nv_bfloa
     q[d + 1] = f.y;
   }
   float m = -INFINITY;
-  for (int64_t j = b_i * p.B_k + lane; j <= i; j += 32) {
+  for (int64_t j = i0 + b_i * p.B_k + lane; j <= i; j += 32) {
     const __nv_bfloat16* kr = k_idx + j * D_IDX;
     float dot = 0.0f;
 #pragma unroll
@@ -550,7 +574,10 @@ cudaError_t launch_typed(const IndexLaunch& a, cudaStream_t stream) {
   p.H_kv = a.H_kv;
   p.B_k = a.B_k;
   p.k = a.k;
-  p.n_mtiles = static_cast<int>((a.N * a.H_kv + kRows - 1) / kRows);
+  p.n_mtiles = a.tiles != nullptr ? a.n_tiles
+                                  : static_cast<int>((a.N * a.H_kv + kRows - 1) / kRows);
+  p.tiles = a.tiles;
+  p.qinfo = a.qinfo;
   p.idx_out = a.idx_out;
   p.score_out = a.score_out;
   p.scale = a.scale;

@@ -230,7 +230,7 @@ msa_status msa_index_topk(const msa_dims* d, const void* q_idx, const void* k_id
   if (ws_bytes < msa_index_topk_workspace(d)) return MSA_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (from_cuda(cudaMemsetAsync(ws, 0, sizeof(msa::DevStatus), s)) != MSA_OK) return MSA_ERR_CUDA;
-  msa::IndexLaunch a;
+  msa::IndexLaunch a{};
   a.q_idx = q_idx;
   a.k_idx = k_idx;
   a.idx_out = idx_out;
@@ -302,7 +302,7 @@ msa_status msa_sparse_attn_fwd(const msa_dims* d, const void* q, const void* k, 
   if (ws_bytes < msa_sparse_attn_fwd_workspace(d)) return MSA_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (from_cuda(cudaMemsetAsync(ws, 0, sizeof(msa::DevStatus), s)) != MSA_OK) return MSA_ERR_CUDA;
-  msa::AttnLaunch a;
+  msa::AttnLaunch a{};
   a.q = q;
   a.k = k;
   a.v = v;
@@ -318,6 +318,152 @@ msa_status msa_sparse_attn_fwd(const msa_dims* d, const void* q, const void* k, 
   a.scale = d->attn_scale > 0.0f ? d->attn_scale : 1.0f / sqrtf(static_cast<float>(d->d_h));
   a.ws = static_cast<uint8_t*>(ws) + kStatusBytes;
   a.ws_bytes = ws_bytes - kStatusBytes;
+  a.status = status_of(ws);
+  return from_cuda(msa::launch_sparse_attn(a, s));
+}
+
+// ------------------------------------------------ packed sequences (varlen) --
+namespace {
+
+// cu_seqlens: n + 1 host values from 0 to N, non-decreasing.
+msa_status check_cu(const msa_varlen_dims* d, const int64_t* cu) {
+  if (d == nullptr || cu == nullptr || d->n_seqs < 1) return MSA_ERR_INVALID_ARG;
+  if (cu[0] != 0 || cu[d->n_seqs] != d->N) return MSA_ERR_INVALID_ARG;
+  for (int s = 0; s < d->n_seqs; ++s)
+    if (cu[s + 1] < cu[s]) return MSA_ERR_INVALID_ARG;
+  return MSA_OK;
+}
+
+msa_dims flat_dims(const msa_varlen_dims* d) {
+  msa_dims f;
+  f.N = d->N;
+  f.H_q = d->H_q;
+  f.H_kv = d->H_kv;
+  f.d_h = d->d_h;
+  f.d_idx = d->d_idx;
+  f.B_k = d->B_k;
+  f.k = d->k;
+  f.attn_scale = d->attn_scale;
+  f.idx_scale = d->idx_scale;
+  return f;
+}
+
+msa_status check_index_varlen(const msa_varlen_dims* d, const int64_t* cu) {
+  msa_status st = check_cu(d, cu);
+  if (st != MSA_OK) return st;
+  st = check_common(d->N, d->H_q, d->H_kv, 64, d->d_idx, d->B_k, d->k, d->attn_scale,
+                    d->idx_scale, false, true);
+  if (st != MSA_OK) return st;
+  if (!pow2_in(d->H_kv, 1, 8) || 128 / d->H_kv > d->B_k) return MSA_ERR_UNSUPPORTED;
+  if (d->N * d->H_kv >= (int64_t(1) << 31) - 256) return MSA_ERR_UNSUPPORTED;
+  return MSA_OK;
+}
+
+msa_status check_attn_varlen(const msa_varlen_dims* d, const int64_t* cu) {
+  msa_status st = check_cu(d, cu);
+  if (st != MSA_OK) return st;
+  const msa_dims f = flat_dims(d);
+  return check_attn_dims(&f);
+}
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+}  // namespace
+
+size_t msa_index_topk_varlen_workspace(const msa_varlen_dims* d, const int64_t* cu_seqlens) {
+  if (check_index_varlen(d, cu_seqlens) != MSA_OK) return 0;
+  return kStatusBytes + msa::varlen_table_bytes(cu_seqlens, d->n_seqs, d->B_k, d->H_kv, true);
+}
+
+msa_status msa_index_topk_varlen(const msa_varlen_dims* d, const int64_t* cu_seqlens,
+                                 const void* q_idx, const void* k_idx, int32_t* idx_out,
+                                 float* score_out, void* ws, size_t ws_bytes, void* stream) {
+  if (q_idx == nullptr || k_idx == nullptr || idx_out == nullptr || ws == nullptr)
+    return MSA_ERR_INVALID_ARG;
+  msa_status st = check_index_varlen(d, cu_seqlens);
+  if (st != MSA_OK) return st;
+  if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(idx_out) || !aligned16(ws) ||
+      (score_out != nullptr && !aligned16(score_out)))
+    return MSA_ERR_INVALID_ARG;
+  if (ws_bytes < msa_index_topk_varlen_workspace(d, cu_seqlens))
+    return MSA_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (from_cuda(cudaMemsetAsync(ws, 0, sizeof(msa::DevStatus), s)) != MSA_OK) return MSA_ERR_CUDA;
+  msa::VarlenTables vt;
+  if (from_cuda(msa::build_varlen_tables(cu_seqlens, d->n_seqs, d->B_k, d->H_kv, true,
+                                         static_cast<uint8_t*>(ws) + kStatusBytes, &vt, s)) !=
+      MSA_OK)
+    return MSA_ERR_CUDA;
+  if (vt.n_tiles == 0) return MSA_OK;  // every sequence empty
+  msa::IndexLaunch a{};
+  a.q_idx = q_idx;
+  a.k_idx = k_idx;
+  a.idx_out = idx_out;
+  a.score_out = score_out;
+  a.scale = d->idx_scale > 0.0f ? d->idx_scale : 1.0f / sqrtf(static_cast<float>(d->d_idx));
+  a.N = d->N;
+  a.H_kv = d->H_kv;
+  a.d_idx = d->d_idx;
+  a.B_k = d->B_k;
+  a.k = d->k;
+  a.tiles = vt.tiles;
+  a.n_tiles = vt.n_tiles;
+  a.qinfo = vt.qinfo;
+  a.status = status_of(ws);
+  return from_cuda(msa::launch_index_topk(a, s));
+}
+
+size_t msa_sparse_attn_fwd_varlen_workspace(const msa_varlen_dims* d, const int64_t* cu_seqlens) {
+  if (check_attn_varlen(d, cu_seqlens) != MSA_OK) return 0;
+  const int64_t B_tot = msa::varlen_blocks(cu_seqlens, d->n_seqs, d->B_k);
+  return kStatusBytes +
+         align256(msa::varlen_table_bytes(cu_seqlens, d->n_seqs, d->B_k, d->H_kv, false)) +
+         msa::attn_workspace_bytes(d->N, d->H_q, d->H_kv, d->d_h, d->B_k, d->k,
+                                   B_tot > 0 ? B_tot : 1);
+}
+
+msa_status msa_sparse_attn_fwd_varlen(const msa_varlen_dims* d, const int64_t* cu_seqlens,
+                                      const void* q, const void* k, const void* v,
+                                      const int32_t* idx, void* o, float* lse, void* ws,
+                                      size_t ws_bytes, void* stream) {
+  if (q == nullptr || k == nullptr || v == nullptr || idx == nullptr || o == nullptr ||
+      ws == nullptr)
+    return MSA_ERR_INVALID_ARG;
+  msa_status st = check_attn_varlen(d, cu_seqlens);
+  if (st != MSA_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(idx) || !aligned16(o) ||
+      !aligned16(ws) || (lse != nullptr && !aligned16(lse)))
+    return MSA_ERR_INVALID_ARG;
+  if (ws_bytes < msa_sparse_attn_fwd_varlen_workspace(d, cu_seqlens))
+    return MSA_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (from_cuda(cudaMemsetAsync(ws, 0, sizeof(msa::DevStatus), s)) != MSA_OK) return MSA_ERR_CUDA;
+  msa::VarlenTables vt;
+  uint8_t* tables = static_cast<uint8_t*>(ws) + kStatusBytes;
+  if (from_cuda(msa::build_varlen_tables(cu_seqlens, d->n_seqs, d->B_k, d->H_kv, false, tables,
+                                         &vt, s)) != MSA_OK)
+    return MSA_ERR_CUDA;
+  const size_t tb = align256(msa::varlen_table_bytes(cu_seqlens, d->n_seqs, d->B_k, d->H_kv,
+                                                     false));
+  msa::AttnLaunch a{};
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.idx = idx;
+  a.o = o;
+  a.lse = lse;
+  a.N = d->N;
+  a.H_q = d->H_q;
+  a.H_kv = d->H_kv;
+  a.d_h = d->d_h;
+  a.B_k = d->B_k;
+  a.kk = d->k;
+  a.scale = d->attn_scale > 0.0f ? d->attn_scale : 1.0f / sqrtf(static_cast<float>(d->d_h));
+  a.ws = tables + tb;
+  a.ws_bytes = ws_bytes - kStatusBytes - tb;
+  a.qinfo = vt.qinfo;
+  a.blk_row = vt.blk_row;
+  a.B_tot = vt.B_tot > 0 ? vt.B_tot : 1;
   a.status = status_of(ws);
   return from_cuda(msa::launch_sparse_attn(a, s));
 }

@@ -27,9 +27,36 @@ struct IndexLaunch {
   float scale;       // Eq. 6 scale for score_out
   int64_t N;
   int H_kv, d_idx, B_k, k;
+  // packed sequences (VarlenTables); null / 0 for one sequence
+  const int4* tiles;
+  int n_tiles;
+  const int2* qinfo;
   DevStatus* status;
 };
 cudaError_t launch_index_topk(const IndexLaunch& a, cudaStream_t s);
+
+// Several sequences packed along the token axis (cu_seqlens on the host:
+// sequence s holds tokens cu[s] .. cu[s+1]-1).  Blocks are numbered per
+// sequence (block b of sequence s starts at token cu[s] + b*B_k) and, in the
+// attention's inverse index, globally: g = blk_base[s] + b.
+struct VarlenTables {
+  const int2* qinfo;     // [N] per token: {cu[s], blk_base[s]} of its sequence
+  const int32_t* blk_row;  // [B_tot] first token of each global block
+  const int4* tiles;     // [n_tiles] index M-tiles, longest first (or null)
+  int n_tiles;
+  int64_t B_tot;
+};
+// Device bytes of the tables for the n sequences of cu (tiles: with the
+// index kernel's tile list).
+size_t varlen_table_bytes(const int64_t* cu, int n, int B_k, int H_kv, bool tiles);
+// Global blocks of the n sequences of cu.
+int64_t varlen_blocks(const int64_t* cu, int n, int B_k);
+// Fill the tables at `dst` (varlen_table_bytes of device memory) from the
+// host cu_seqlens: the per-sequence bases and the tile list are written on
+// the host and copied (cudaMemcpyAsync from pageable memory, staged before
+// the call returns), the per-token and per-block tables by a kernel.
+cudaError_t build_varlen_tables(const int64_t* cu, int n, int B_k, int H_kv, bool tiles,
+                                void* dst, VarlenTables* out, cudaStream_t s);
 
 struct AttnLaunch {
   const void* q;
@@ -43,9 +70,16 @@ struct AttnLaunch {
   float scale;
   void* ws;  // device workspace after the status word
   size_t ws_bytes;
+  // packed sequences: per-token and per-block tables, B_tot global blocks
+  // (null / 0 for one sequence)
+  const int2* qinfo;
+  const int32_t* blk_row;
+  int64_t B_tot;
   DevStatus* status;
 };
-size_t attn_workspace_bytes(int64_t N, int H_q, int H_kv, int d_h, int B_k, int kk);
+// B_tot: global blocks (0 for one sequence of N tokens)
+size_t attn_workspace_bytes(int64_t N, int H_q, int H_kv, int d_h, int B_k, int kk,
+                            int64_t B_tot = 0);
 cudaError_t launch_sparse_attn(const AttnLaunch& a, cudaStream_t s);
 
 struct IdxLseLaunch {

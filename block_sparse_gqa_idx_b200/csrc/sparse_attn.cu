@@ -116,7 +116,10 @@ struct InvParams {
   const int32_t* idx;
   int64_t q0, nq;  // chunk [q0, q0 + nq)
   int H_kv, B_k, kk;
-  int64_t B;
+  int64_t B;  // blocks (all sequences' blocks, numbered globally, when qinfo is set)
+  // packed sequences: per token {first token, first global block} of its
+  // sequence; null for one sequence
+  const int2* qinfo;
   int Tq;
   int Cw, W;  // queries per window, windows in the chunk
   ChunkBufs c;
@@ -133,9 +136,15 @@ inline int64_t inv_nkeys(int64_t nq, int Cw, int H_kv, int64_t B) {
 }
 inline int64_t scan_blocks(int64_t nkeys) { return (nkeys + kScanBlockKeys - 1) / kScanBlockKeys; }
 
-// The window-local key (r * B + b) of entry e of the chunk, or -1 when the
-// entry selects nothing (-1 padding, or a block after the query's own).
-// Entry e is (query, group, slot) in the layout of I, so e is also the
+// Query i's sequence: its first token and the global number of its block 0
+// ({0, 0} for one sequence).
+__device__ __forceinline__ int2 seq_of(const int2* qinfo, int64_t i) {
+  return qinfo != nullptr ? qinfo[i] : make_int2(0, 0);
+}
+
+// The window-local key (r * B + global block) of entry e of the chunk, or -1
+// when the entry selects nothing (-1 padding, or a block after the query's
+// own).  Entry e is (query, group, slot) in the layout of I, so e is also the
 // entry's output slot id and I is read contiguously.
 __device__ __forceinline__ int inv_key(const InvParams& p, int64_t e, bool report_bad) {
   const int64_t per_q = static_cast<int64_t>(p.H_kv) * p.kk;
@@ -147,7 +156,8 @@ __device__ __forceinline__ int inv_key(const InvParams& p, int64_t e, bool repor
     if (report_bad) report(p.status, DEV_ERR_BAD_INDEX, 40, static_cast<int>(i), b);
     return -1;
   }
-  return (b >= 0 && b <= i / p.B_k) ? r * static_cast<int>(p.B) + b : -1;
+  const int2 sq = seq_of(p.qinfo, i);
+  return (b >= 0 && b <= (i - sq.x) / p.B_k) ? r * static_cast<int>(p.B) + sq.y + b : -1;
 }
 
 // Inverse index with a per-CTA histogram of one window's keys in shared
@@ -213,11 +223,12 @@ __global__ void inv_index_kernel(const InvParams p) {
       const int64_t il = rem % p.nq;
       const int64_t i = p.q0 + il;
       const int32_t b = p.idx[(i * p.H_kv + r) * p.kk + s];
-      const int64_t b_i = i / p.B_k;
+      const int2 sq = seq_of(p.qinfo, i);
+      const int64_t b_i = (i - sq.x) / p.B_k;
       if (b < -1 || b >= p.B) {
         if (!SCATTER) report(p.status, DEV_ERR_BAD_INDEX, 40, static_cast<int>(i), b);
       } else if (b >= 0 && b <= b_i) {
-        key = ((il / p.Cw) * p.H_kv + r) * p.B + b;
+        key = ((il / p.Cw) * p.H_kv + r) * p.B + sq.y + b;
         slot = static_cast<uint32_t>((il * p.H_kv + r) * p.kk + s);
       }
     }
@@ -429,8 +440,9 @@ struct P1Params {
   int64_t q0;
   int q4d;  // 1: one 4-D TMA box per gathered query ([d-chunk][head] rows, 8 heads)
   int H_q, H_kv, B_k, kk, G, R, Tq;
-  int B;          // blocks of the sequence
+  int B;          // blocks of the sequence (of all sequences, numbered globally)
   int64_t nkeys;  // (window, group, block) keys
+  const int32_t* blk_row;  // first token of each global block; null: block b at b * B_k
   float scale_log2;  // softmax scale * log2(e)
   float scale;
   ChunkBufs c;
@@ -466,6 +478,7 @@ constexpr int kMaxTq = 16;  // queries per tile (128 rows / at least 8 rows per 
 
 struct TileInfo {
   int r, b, len, gen;  // group, block, queries in the tile, K/V generation
+  int jb;              // the block's first token
   uint32_t slot[kMaxTq];  // each query's output slot
   int qi[kMaxTq];         // each query's position i
 };
@@ -606,8 +619,9 @@ __global__ void __launch_bounds__(kP1Threads, 1)
         if (lane == 0) mbar_arrive_expect_tx(&kv_full[slot], SH::K_BYTES + SH::V_BYTES);
         __syncwarp();
         if (lane < SH::DCH) {
-          tma_load_3d(sK + lane * B_K * 128, &tm_k, &kv_full[slot], lane * 64, r, b * B_K);
-          tma_load_3d(sV + lane * B_K * 128, &tm_v, &kv_full[slot], lane * 64, r, b * B_K);
+          const int row = p.blk_row != nullptr ? p.blk_row[b] : b * B_K;
+          tma_load_3d(sK + lane * B_K * 128, &tm_k, &kv_full[slot], lane * 64, r, row);
+          tma_load_3d(sV + lane * B_K * 128, &tm_v, &kv_full[slot], lane * 64, r, row);
         }
       };
       int kv_key = -1, kvgen = 0;
@@ -634,6 +648,7 @@ __global__ void __launch_bounds__(kP1Threads, 1)
           ti.b = b;
           ti.len = len;
           ti.gen = gen;
+          ti.jb = p.blk_row != nullptr ? p.blk_row[b] : b * B_K;
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&i_full[is]);
@@ -876,7 +891,7 @@ __global__ void __launch_bounds__(kP1Threads, 1)
       // a padding row (past the tile's queries) is never masked
       const int iA = liveA ? ti.qi[qA] : INT_MAX;
       const int iB = liveB ? ti.qi[qB] : INT_MAX;
-      const int jb = ti.b * B_K;  // the block's first key
+      const int jb = ti.jb;  // the block's first key
       tmem_wait_ld();
       if (jb + B_K - 1 > (iA < iB ? iA : iB)) {  // a query's own block: j <= i
 #pragma unroll
@@ -975,6 +990,7 @@ struct MergeParams {
   float* lse;
   int64_t q0, nq;
   int H_q, H_kv, kk, G, B_k;
+  const int2* qinfo;  // packed sequences (per token), or null
   ChunkBufs c;
 };
 
@@ -999,7 +1015,7 @@ __global__ void __launch_bounds__(256, 2) attn_merge_kernel(const MergeParams p)
   const int e0 = (wq * 32 + lane) * E;  // element offset inside the [G, D_H] block
   const int g = e0 / D_H, d0 = e0 - g * D_H;
   const int64_t i = p.q0 + il;
-  const int64_t b_i = i / p.B_k;
+  const int64_t b_i = (i - seq_of(p.qinfo, i).x) / p.B_k;
   const int64_t slot0 = (il * p.H_kv + r) * p.kk;
   int32_t myb = -1;
   if (lane < p.kk) myb = p.idx[(i * p.H_kv + r) * p.kk + lane];
@@ -1079,7 +1095,7 @@ __global__ void __launch_bounds__(256) attn_merge_small_kernel(const MergeParams
   const int64_t il = unit / p.H_kv;
   const int r = static_cast<int>(unit - il * p.H_kv);
   const int64_t i = p.q0 + il;
-  const int64_t b_i = i / p.B_k;
+  const int64_t b_i = (i - seq_of(p.qinfo, i).x) / p.B_k;
   const int64_t slot0 = (il * p.H_kv + r) * p.kk;
   const int32_t* sel = p.idx + (i * p.H_kv + r) * p.kk;
   const float* lse_h = p.c.part_lse + slot0 * p.G + g;
@@ -1133,7 +1149,7 @@ cudaError_t launch_typed(const AttnLaunch& a, cudaStream_t stream) {
   const int G = a.H_q / a.H_kv;
   const int R = rows_per_query(G);
   const int Tq = kRowsPerTile / R;
-  const int64_t B = (a.N + a.B_k - 1) / a.B_k;
+  const int64_t B = a.B_tot > 0 ? a.B_tot : (a.N + a.B_k - 1) / a.B_k;
   const int64_t Nc = chunk_len(a.N, a.B_k);
   const int64_t nkeys_max = inv_nkeys(Nc, kWindow, a.H_kv, B);  // per chunk, at most
   size_t need = 0;
@@ -1185,7 +1201,7 @@ cudaError_t launch_typed(const AttnLaunch& a, cudaStream_t stream) {
     const int64_t nkeys = inv_nkeys(nq, kWindow, a.H_kv, B);
     e = cudaMemsetAsync(c.counts, 0, sizeof(int32_t) * nkeys, stream);
     if (e != cudaSuccess) return e;
-    InvParams ip;
+    InvParams ip{};
     ip.idx = a.idx;
     ip.q0 = q0;
     ip.nq = nq;
@@ -1193,6 +1209,7 @@ cudaError_t launch_typed(const AttnLaunch& a, cudaStream_t stream) {
     ip.B_k = a.B_k;
     ip.kk = a.kk;
     ip.B = B;
+    ip.qinfo = a.qinfo;
     ip.Tq = Tq;
     ip.Cw = kWindow;
     ip.W = static_cast<int>((nq + kWindow - 1) / kWindow);
@@ -1200,7 +1217,7 @@ cudaError_t launch_typed(const AttnLaunch& a, cudaStream_t stream) {
     ip.status = a.status;
     launch_inv_index(ip, hist_bytes, hist_grid, sms, stream);
 
-    P1Params pp;
+    P1Params pp{};
     pp.q0 = q0;
     pp.q4d = q4d;
     pp.H_q = a.H_q;
@@ -1212,6 +1229,7 @@ cudaError_t launch_typed(const AttnLaunch& a, cudaStream_t stream) {
     pp.Tq = Tq;
     pp.B = static_cast<int>(B);
     pp.nkeys = nkeys;
+    pp.blk_row = a.blk_row;
     pp.scale = a.scale;
     pp.scale_log2 = a.scale * 1.4426950408889634f;
     pp.c = c;
@@ -1220,7 +1238,7 @@ cudaError_t launch_typed(const AttnLaunch& a, cudaStream_t stream) {
     attn_phase1_kernel<D_H, B_K><<<sms, kP1Threads, smem, stream>>>(tq, tk, tv, pp);
     prof_end(stream);
 
-    MergeParams mp;
+    MergeParams mp{};
     mp.idx = a.idx;
     mp.o = static_cast<__nv_bfloat16*>(a.o);
     mp.lse = a.lse;
@@ -1231,6 +1249,7 @@ cudaError_t launch_typed(const AttnLaunch& a, cudaStream_t stream) {
     mp.kk = a.kk;
     mp.G = G;
     mp.B_k = a.B_k;
+    mp.qinfo = a.qinfo;
     mp.c = c;
     prof_begin("attn_merge", stream);
     if (G * D_H < 256) {
@@ -1452,7 +1471,7 @@ cudaError_t launch_idx_lse_typed(const IdxLseLaunch& a, cudaStream_t stream) {
     const int64_t nq = (a.N - q0) < Nc ? (a.N - q0) : Nc;
     e = cudaMemsetAsync(c.counts, 0, sizeof(int32_t) * nkeys, stream);
     if (e != cudaSuccess) return e;
-    InvParams ip;
+    InvParams ip{};
     ip.idx = a.idx;
     ip.q0 = q0;
     ip.nq = nq;
@@ -1509,8 +1528,9 @@ cudaError_t launch_idx_lse(const IdxLseLaunch& a, cudaStream_t s) {
   return cudaErrorInvalidValue;
 }
 
-size_t attn_workspace_bytes(int64_t N, int H_q, int H_kv, int d_h, int B_k, int kk) {
-  const int64_t B = (N + B_k - 1) / B_k;
+size_t attn_workspace_bytes(int64_t N, int H_q, int H_kv, int d_h, int B_k, int kk,
+                            int64_t B_tot) {
+  const int64_t B = B_tot > 0 ? B_tot : (N + B_k - 1) / B_k;
   size_t total = 0;
   const int64_t Nc = chunk_len(N, B_k);
   carve(nullptr, Nc, H_q, H_kv, d_h, kk, inv_nkeys(Nc, kWindow, H_kv, B), &total);

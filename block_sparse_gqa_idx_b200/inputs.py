@@ -94,6 +94,39 @@ class DecodeConfig:
         return SEED_BASE + self.seed_index
 
 
+@dataclasses.dataclass(frozen=True)
+class VarlenConfig:
+    """A packed batch of prefill sequences: n_seqs lengths drawn by
+    ``varlen_lengths`` (log-uniform in [len_lo, len_hi], summing to N), each
+    sequence with ``prefill_inputs``' recipe for ``structure``."""
+    name: str
+    n_seqs: int
+    N: int
+    len_lo: int
+    len_hi: int
+    H_q: int
+    H_kv: int
+    d_h: int
+    d_idx: int
+    B_k: int
+    k: int
+    structure: str = "sink_ar1"
+    seed_index: int = 0
+
+    @property
+    def seed(self) -> int:
+        return SEED_BASE + self.seed_index
+
+    @property
+    def prefill(self) -> "MSAConfig":
+        """The per-sequence heads and recipe (N = 0: each sequence sets its own)."""
+        return MSAConfig(self.name, 0, self.H_q, self.H_kv, self.d_h, self.d_idx, self.B_k,
+                         self.k, self.structure, 1.0, self.seed_index)
+
+    def lengths(self) -> np.ndarray:
+        return varlen_lengths(self.n_seqs, self.N, self.len_lo, self.len_hi, self.seed)
+
+
 CONFIGS: Dict[str, object] = {
     # tiny prefill: the oracle finishes in seconds
     "tiny": MSAConfig("tiny", N=2048, H_q=8, H_kv=2, d_h=64, d_idx=32, B_k=64, k=4,
@@ -118,10 +151,48 @@ CONFIGS: Dict[str, object] = {
     # are profiled on
     "decode_fp8_s8": DecodeConfig("decode_fp8_s8", S=8, L0=131072, steps=256, H_q=32, H_kv=4,
                                   d_h=128, d_idx=64, B_k=128, k=16, seed_index=7),
+    # a packed batch of 32 prefill sequences, 131072 tokens in all, lengths
+    # log-uniform in [512, 16384], pages' heads
+    "varlen": VarlenConfig("varlen", n_seqs=32, N=131072, len_lo=512, len_hi=16384, H_q=32,
+                           H_kv=4, d_h=128, d_idx=64, B_k=128, k=16, structure="sink_ar1",
+                           seed_index=8),
     # 1M-token prefill with a strong sink (block 0 picked by >= 90% of rows)
     "1m": MSAConfig("1m", N=1048576, H_q=32, H_kv=4, d_h=128, d_idx=64, B_k=128, k=16,
                     structure="sink_ar1", sink_strength=3.0, seed_index=4),
 }
+
+
+def varlen_lengths(n_seqs: int, total: int, lo: int, hi: int, seed: int) -> np.ndarray:
+    """A seeded mix of n_seqs sequence lengths, log-uniform in [lo, hi] and
+    rescaled to sum to ``total`` (the last one takes the rounding)."""
+    r = np.random.default_rng(np.random.SeedSequence(seed + 901))
+    x = np.exp(r.uniform(np.log(lo), np.log(hi), n_seqs))
+    L = np.maximum(1, np.floor(x * total / x.sum())).astype(np.int64)
+    L[-1] += total - L.sum()
+    return L
+
+
+def varlen_inputs(cfg: MSAConfig, lengths, seed: Optional[int] = None):
+    """A packed batch: sequence s is ``prefill_inputs`` of cfg's heads and
+    structure at N = lengths[s] (its own seed), the sequences concatenated
+    along the token axis.  Returns (inputs, cu_seqlens int64 [n+1])."""
+    lengths = [int(x) for x in lengths]
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int64)
+    base = cfg.seed if seed is None else seed
+    parts = []
+    for s, n in enumerate(lengths):
+        if n == 0:
+            continue
+        sub = MSAConfig(f"{cfg.name}/{s}", n, cfg.H_q, cfg.H_kv, cfg.d_h, cfg.d_idx, cfg.B_k, cfg.k,
+                        cfg.structure, cfg.sink_strength, cfg.seed_index)
+        parts.append(prefill_inputs(sub, seed=base + 7919 * (s + 1)))
+    out = {}
+    for key, shape in (("q", (cfg.H_q, cfg.d_h)), ("k", (cfg.H_kv, cfg.d_h)),
+                       ("v", (cfg.H_kv, cfg.d_h)), ("q_idx", (cfg.H_kv, cfg.d_idx)),
+                       ("k_idx", (cfg.d_idx,))):
+        out[key] = (np.concatenate([p[key] for p in parts]) if parts
+                    else np.zeros((0,) + shape, np.uint16))
+    return out, cu
 
 
 def bf16_bits(x: np.ndarray) -> np.ndarray:

@@ -118,6 +118,41 @@ MSA_API msa_status msa_sparse_attn_fwd(const msa_dims* dims, const void* q, cons
                                void* workspace, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Several prefill sequences packed along the token axis (variable length):
+ * sequence s holds tokens cu_seqlens[s] .. cu_seqlens[s+1]-1 of every tensor
+ * (any lengths, empty ones allowed, no padding), and the method runs inside
+ * each sequence on its own (Eq. 6-8 per sequence: a query's candidate blocks
+ * are the earlier blocks of its sequence, block b of sequence s covers tokens
+ * cu_seqlens[s] + b*B_k .. and its local block is (i - cu_seqlens[s]) / B_k).
+ *   cu_seqlens  HOST array of n_seqs + 1 int64 values, 0 = cu[0] <= cu[1] <=
+ *               ... <= cu[n_seqs] = N; read during the call only
+ * Tensors are those of the single-sequence calls with N = all tokens; idx
+ * holds block indices local to each token's sequence.  The calls copy small
+ * per-sequence tables from the host into the workspace (cudaMemcpyAsync from
+ * pageable memory), so they cannot be captured into a CUDA graph.
+ * ------------------------------------------------------------------------- */
+typedef struct {
+  int32_t n_seqs;
+  int64_t N;  /* cu_seqlens[n_seqs] */
+  int32_t H_q, H_kv, d_h, d_idx, B_k, k;
+  float attn_scale;
+  float idx_scale;
+} msa_varlen_dims;
+MSA_API size_t msa_index_topk_varlen_workspace(const msa_varlen_dims* dims,
+                                               const int64_t* cu_seqlens);
+MSA_API msa_status msa_index_topk_varlen(const msa_varlen_dims* dims, const int64_t* cu_seqlens,
+                                         const void* q_idx, const void* k_idx, int32_t* idx_out,
+                                         float* score_out, void* workspace, size_t ws_bytes,
+                                         void* stream);
+MSA_API size_t msa_sparse_attn_fwd_varlen_workspace(const msa_varlen_dims* dims,
+                                                    const int64_t* cu_seqlens);
+MSA_API msa_status msa_sparse_attn_fwd_varlen(const msa_varlen_dims* dims,
+                                              const int64_t* cu_seqlens, const void* q,
+                                              const void* k, const void* v, const int32_t* idx,
+                                              void* o, float* lse, void* workspace,
+                                              size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
  * One decode step for S sequences (Eq. 1's i <= t: the new token attends to
  * itself).  For each sequence s with L = seq_len[s] (read on the device):
  * append k_new/v_new/k_idx_new at row L, then run Eq. 6-8 for the single query

@@ -222,6 +222,36 @@ def forward(inp: dict, B_k: int, k: int, rows: Optional[np.ndarray] = None,
     return {"idx": idx, "cut": cut, "next": nxt, "o": o, "lse": lse, "rows": rows}
 
 
+def forward_varlen(inp: dict, cu_seqlens, B_k: int, k: int, rows: Optional[np.ndarray] = None,
+                   idx_rows: Optional[np.ndarray] = None, threads: int = 0) -> dict:
+    """Eq. 6-8 for a batch of sequences packed along the token axis: sequence
+    s is tokens cu_seqlens[s] .. cu_seqlens[s+1]-1 of every input, and each
+    sequence is its own prefill (``forward`` on its slice; block indices in
+    ``idx`` are local to the sequence).  Returns the fields of ``forward`` for
+    ``rows`` (global token indices, default all) plus each row's sequence.
+    ``idx_rows`` (one selection per row, local block indices) replaces the
+    oracle's own selection in the attention step, as in ``forward``."""
+    cu = [int(x) for x in cu_seqlens]
+    N = cu[-1]
+    rows = np.arange(N, dtype=np.int64) if rows is None else np.asarray(rows, dtype=np.int64)
+    n = rows.size
+    H_kv, H_q, d_h = inp["q_idx"].shape[1], inp["q"].shape[1], inp["q"].shape[2]
+    out = {"idx": np.empty((n, H_kv, k), np.int32), "cut": np.empty((n, H_kv)),
+           "next": np.empty((n, H_kv)), "o": np.empty((n, H_q, d_h)), "lse": np.empty((n, H_q)),
+           "rows": rows, "seq": np.searchsorted(np.asarray(cu[1:]), rows, side="right")}
+    for s in range(len(cu) - 1):
+        a, b = cu[s], cu[s + 1]
+        pick = np.nonzero((rows >= a) & (rows < b))[0]
+        if pick.size == 0:
+            continue
+        sub = {key: inp[key][a:b] for key in ("q", "k", "v", "q_idx", "k_idx")}
+        r = forward(sub, B_k, k, rows[pick] - a,
+                    idx_rows=None if idx_rows is None else idx_rows[pick], threads=threads)
+        for key in ("idx", "cut", "next", "o", "lse"):
+            out[key][pick] = r[key]
+    return out
+
+
 def decode_reference(state: dict, step_in: dict, B_k: int, k: int, seqs=None,
                      idx_rows: Optional[np.ndarray] = None, threads: int = 0) -> dict:
     """One decode step for the listed sequences, on host copies of the caches.

@@ -142,3 +142,32 @@ def test_prefill_workspace_queries_reject_bad_dims(capi):
         d = capi.dims(4096, 8, 4, 128, 64, 128, 16)
         setattr(d, field, value)
         assert capi.LIB.msa_index_lse_workspace(ctypes.byref(d)) == 0, field
+
+
+def test_varlen_rejects_bad_cu_seqlens_on_host(capi):
+    """cu_seqlens must run from 0 to N without decreasing; the workspace
+    queries return 0 and the calls INVALID_ARG, launching nothing."""
+    FAKE = ctypes.c_void_p(1 << 20)
+    d = capi.varlen_dims(3, 500, 8, 2, 64, 32, 64, 4)
+
+    def cu(vals):
+        return (ctypes.c_int64 * len(vals))(*vals)
+
+    good = cu([0, 200, 200, 500])
+    assert capi.LIB.msa_index_topk_varlen_workspace(ctypes.byref(d), good) > 0
+    assert capi.LIB.msa_sparse_attn_fwd_varlen_workspace(ctypes.byref(d), good) > 0
+    for bad in ([1, 200, 300, 500], [0, 300, 200, 500], [0, 200, 300, 499]):
+        c = cu(bad)
+        assert capi.LIB.msa_index_topk_varlen_workspace(ctypes.byref(d), c) == 0, bad
+        assert capi.LIB.msa_sparse_attn_fwd_varlen_workspace(ctypes.byref(d), c) == 0, bad
+        assert capi.LIB.msa_index_topk_varlen(ctypes.byref(d), c, FAKE, FAKE, FAKE, None, FAKE,
+                                              1 << 30, None) == 1, bad
+        assert capi.LIB.msa_sparse_attn_fwd_varlen(ctypes.byref(d), c, FAKE, FAKE, FAKE, FAKE,
+                                                   FAKE, None, FAKE, 1 << 30, None) == 1, bad
+    assert capi.LIB.msa_index_topk_varlen(ctypes.byref(d), None, FAKE, FAKE, FAKE, None, FAKE,
+                                          1 << 30, None) == 1
+    # a workspace below the query's size
+    assert capi.LIB.msa_index_topk_varlen(ctypes.byref(d), good, FAKE, FAKE, FAKE, None, FAKE,
+                                          8, None) == 3
+    with pytest.raises(ValueError):
+        capi._cu([0, 10, 20], 30)
