@@ -7,13 +7,15 @@ synthetic inputs with a sink block and retrieval blocks).  Inputs (Q alone is
 1.07 GB) are larger than the 126 MB L2, so no flush is needed between steps.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl msa|reference]
-                    [--workload 128k|32k|1m|decode|decode_fp8] [--no-also]
+                    [--workload 128k|32k|1m|varlen|decode|decode_fp8] [--no-also]
 
-On one GPU the 128K line also carries, under "also", the other two parts of
-the metric, each measured the same way: the 1M-token prefill ("1m", 3 steps
-after 2 warm-up steps), the 64-sequence decode workload ("decode", 1000 steps
-after 10 warm-up steps, us per token) and the same decode on a paged FP8
-(E4M3) cache ("decode_fp8").  For N > 1 each rank runs an
+On one GPU the 128K line also carries, under "also", the other parts of the
+metric and the path's other workloads, each measured the same way: the
+1M-token prefill ("1m", 3 steps after 2 warm-up steps), a packed batch of 32
+prefill sequences of mixed lengths, 131072 tokens in all ("varlen"), the
+64-sequence decode workload ("decode", 1000 steps after 10 warm-up steps, us
+per token) and the same decode on a paged FP8 (E4M3) cache ("decode_fp8").
+For N > 1 each rank runs an
 independent replica (its own sequence): the path has no exchange step, so
 there is no collective on the data path; timing is the max over ranks and
 ``value`` is the tokens of all ranks per second.  ``--impl reference`` times
@@ -190,10 +192,26 @@ def workload(name: str):
 
 
 def flops_of(cfg):
-    """Eq. 12 (xllm-io review): index term H_kv*d_idx*N^2, main term 4*N*H_q*k*B_k*d_h."""
-    f_idx = cfg.H_kv * cfg.d_idx * float(cfg.N) ** 2
+    """Eq. 12 (xllm-io review): index term H_kv*d_idx*N^2, main term 4*N*H_q*k*B_k*d_h,
+    summed over the sequences of a packed batch."""
+    lengths = cfg.lengths() if hasattr(cfg, "lengths") else [cfg.N]
+    f_idx = cfg.H_kv * cfg.d_idx * float(sum(float(n) ** 2 for n in lengths))
     f_main = 4.0 * cfg.N * cfg.H_q * cfg.k * cfg.B_k * cfg.d_h
     return f_idx, f_main
+
+
+def selected_key_flops(cfg) -> float:
+    """The main term without Eq. 12's k full blocks per query: 4*H_q*d_h per
+    visible selected key, where query i (position within its sequence) sees
+    min(k-1, i // B_k) earlier full blocks and the i % B_k + 1 keys of its
+    own block.  Below Eq. 12 for the first k blocks of every sequence, so it
+    is the count a batch of short sequences is measured against."""
+    lengths = cfg.lengths() if hasattr(cfg, "lengths") else [cfg.N]
+    keys = 0
+    for n in lengths:
+        i = np.arange(int(n), dtype=np.int64)
+        keys += int((np.minimum(cfg.k - 1, i // cfg.B_k) * cfg.B_k + i % cfg.B_k + 1).sum())
+    return 4.0 * cfg.H_q * cfg.d_h * float(keys)
 
 
 # ------------------------------------------------------------ reference arm --
@@ -204,14 +222,21 @@ def run_reference(args, cfg, rank, world):
     import oracle
     from block_sparse_gqa_idx_b200 import inputs
 
-    inp = inputs.prefill_inputs(cfg)
+    varlen = isinstance(cfg, inputs.VarlenConfig)
+    if varlen:
+        inp, cu = inputs.varlen_inputs(cfg.prefill, cfg.lengths())
+    else:
+        inp = inputs.prefill_inputs(cfg)
     rng = np.random.default_rng(7)
     n_rows = args.ref_rows
     times = []
     for it in range(args.warmup + args.steps):
         rows = np.sort(rng.choice(cfg.N, size=n_rows, replace=False))
         t0 = time.perf_counter()
-        oracle.forward(inp, cfg.B_k, cfg.k, rows=rows)
+        if varlen:
+            oracle.forward_varlen(inp, cu, cfg.B_k, cfg.k, rows=rows)
+        else:
+            oracle.forward(inp, cfg.B_k, cfg.k, rows=rows)
         dt = time.perf_counter() - t0
         if it >= args.warmup:
             times.append(dt)
@@ -325,9 +350,13 @@ def run_msa(args, cfg, rank, world, local, steps, warmup, e2e_steps, cpu_rows):
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream(dev)
 
-    # every replica gets its own seeded sequence
+    # every replica gets its own seeded sequence (or packed batch)
+    varlen = isinstance(cfg, inputs.VarlenConfig)
     t_gen = time.time()
-    inp = inputs.prefill_inputs(cfg, seed=cfg.seed + 1000 * rank)
+    if varlen:
+        inp, cu = inputs.varlen_inputs(cfg.prefill, cfg.lengths(), seed=cfg.seed + 1000 * rank)
+    else:
+        inp = inputs.prefill_inputs(cfg, seed=cfg.seed + 1000 * rank)
     gen_s = time.time() - t_gen
     host = {k: torch.from_numpy(np.ascontiguousarray(v).view(np.int16)).view(torch.bfloat16)
             for k, v in inp.items()}
@@ -337,12 +366,23 @@ def run_msa(args, cfg, rank, world, local, steps, warmup, e2e_steps, cpu_rows):
     o = torch.empty((N, H_q, d_h), dtype=torch.bfloat16, device=dev)
     lse = torch.empty((N, H_q), dtype=torch.float32, device=dev)
     dims = msa.dims(N, H_q, H_kv, d_h, d_idx, B_k, kk)
-    ws = torch.empty(max(msa.sparse_attn_fwd_workspace_size(dims),
-                         msa.index_topk_workspace_size(dims),
-                         msa.index_lse_workspace_size(dims)), dtype=torch.uint8, device=dev)
+    if varlen:
+        if args.kl_lse:
+            raise SystemExit("--kl-lse runs on one sequence per replica, not a packed batch")
+        ws_bytes = msa.varlen_workspace_size(cu, N, H_q, H_kv, d_h, d_idx, B_k, kk)
+    else:
+        ws_bytes = max(msa.sparse_attn_fwd_workspace_size(dims), msa.index_topk_workspace_size(dims),
+                       msa.index_lse_workspace_size(dims))
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     lse_idx = torch.empty((N, H_kv), dtype=torch.float32, device=dev) if args.kl_lse else None
 
     def step(src, o_, idx_, lse_):
+        if varlen:
+            msa.index_topk_varlen(src["q_idx"], src["k_idx"], cu, B_k, kk, idx_out=idx_,
+                                  workspace=ws, stream=stream)
+            msa.sparse_attn_fwd_varlen(src["q"], src["k"], src["v"], idx_, cu, B_k, o=o_,
+                                       lse=lse_, workspace=ws, stream=stream)
+            return
         msa.index_topk(src["q_idx"], src["k_idx"], B_k, kk, idx_out=idx_, workspace=ws,
                        stream=stream)
         msa.sparse_attn_fwd(src["q"], src["k"], src["v"], idx_, B_k, o=o_, lse=lse_,
@@ -443,6 +483,9 @@ def run_msa(args, cfg, rank, world, local, steps, warmup, e2e_steps, cpu_rows):
     # ---- roofline of the dominant kernel (live CUDA-event durations)
     pk, pk_kind = peaks()
     f_idx, f_main = flops_of(cfg)
+    if varlen:
+        # short sequences select fewer than k blocks: count the keys selected
+        f_main = selected_key_flops(cfg)
     total_ms = sum(v[1] for v in prof.values())
     dom = max(prof, key=lambda n: prof[n][1])
     launches, dom_ms = prof[dom]
@@ -473,7 +516,10 @@ def run_msa(args, cfg, rank, world, local, steps, warmup, e2e_steps, cpu_rows):
         rng = np.random.default_rng(11)
         rows = np.sort(rng.choice(N, size=cpu_rows, replace=False))
         t0 = time.perf_counter()
-        oracle.forward(inp, B_k, kk, rows=rows)
+        if varlen:
+            oracle.forward_varlen(inp, cu, B_k, kk, rows=rows)
+        else:
+            oracle.forward(inp, B_k, kk, rows=rows)
         dt = time.perf_counter() - t0
         cpu = {"value": cpu_rows / dt, "unit": "tokens/s", "cores": oracle.max_threads(),
                "kind": "oracle",
@@ -493,8 +539,13 @@ def run_msa(args, cfg, rank, world, local, steps, warmup, e2e_steps, cpu_rows):
                    "d_idx": d_idx, "B_k": B_k, "k": kk, "parallelism": f"replicas x{world}",
                    "l2": "inputs larger than L2 (Q alone %.2f GB); no flush"
                          % (N * H_q * d_h * 2 / 1e9),
-                   "kl_lse": bool(args.kl_lse)},
+                   "kl_lse": bool(args.kl_lse),
+                   **({"n_seqs": cfg.n_seqs, "lengths": f"log-uniform in [{cfg.len_lo}, "
+                       f"{cfg.len_hi}], min {int(np.min(np.diff(cu)))}, max "
+                       f"{int(np.max(np.diff(cu)))}"} if varlen else {})},
         "tc_frac_eq12": (f_idx + f_main) / (ms * 1e-3) / 1e12 / pk["bf16_tflops"],
+        "main_flops": ("selected visible keys, 4*H_q*d_h each" if varlen
+                       else "Eq. 12 main term, 4*N*H_q*k*B_k*d_h"),
         "roofline": roofline,
         "roofline_per_kernel": per_kernel,
         "cpu_baseline": cpu,
@@ -749,8 +800,11 @@ def main():
             also["1m"] = run_msa(args, c1m, rank, world, local, steps=3, warmup=2, e2e_steps=2,
                                  cpu_rows=0 if args.no_cpu_baseline else 32)
             free_device_memory()
-            cdec = workload("decode")
-            also["decode"] = run_decode(args, cdec, rank, world, local, steps=1000, warmup=10,
+            also["varlen"] = run_msa(args, workload("varlen"), rank, world, local, steps=10,
+                                     warmup=3, e2e_steps=4,
+                                     cpu_rows=0 if args.no_cpu_baseline else 128)
+            free_device_memory()
+            also["decode"] = run_decode(args, workload("decode"), rank, world, local, steps=1000, warmup=10,
                                         e2e_steps=8, cpu_seqs=0 if args.no_cpu_baseline else 4)
             free_device_memory()
             also["decode_fp8"] = run_decode(args, workload("decode_fp8"), rank, world, local,

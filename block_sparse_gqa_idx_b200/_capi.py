@@ -53,6 +53,11 @@ class msa_varlen_dims(ctypes.Structure):
                 ("idx_scale", ctypes.c_float)]
 
 
+class msa_proj_dims(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int64), ("d_model", ctypes.c_int32), ("H_q", ctypes.c_int32),
+                ("H_kv", ctypes.c_int32), ("d_h", ctypes.c_int32), ("d_idx", ctypes.c_int32)]
+
+
 class msa_kernel_time(ctypes.Structure):
     _fields_ = [("name", ctypes.c_char * 48), ("launches", ctypes.c_int32),
                 ("total_ms", ctypes.c_double)]
@@ -66,7 +71,8 @@ EXPORTS = ("msa_index_topk_workspace", "msa_index_topk", "msa_sparse_attn_fwd_wo
            "msa_selftest_bounded_wait", "msa_index_lse_workspace", "msa_index_lse",
            "msa_paged_decode_fp8_workspace", "msa_paged_decode_fp8", "msa_quantize_fp8_rows",
            "msa_index_topk_varlen_workspace", "msa_index_topk_varlen",
-           "msa_sparse_attn_fwd_varlen_workspace", "msa_sparse_attn_fwd_varlen")
+           "msa_sparse_attn_fwd_varlen_workspace", "msa_sparse_attn_fwd_varlen",
+           "msa_project_workspace", "msa_project")
 
 
 def _load() -> ctypes.CDLL:
@@ -114,6 +120,11 @@ def _load() -> ctypes.CDLL:
     lib.msa_sparse_attn_fwd_varlen_workspace.restype = Z
     lib.msa_sparse_attn_fwd_varlen.argtypes = [VD, CU, P, P, P, P, P, P, P, Z, P]
     lib.msa_sparse_attn_fwd_varlen.restype = I32
+    PJ = ctypes.POINTER(msa_proj_dims)
+    lib.msa_project_workspace.argtypes = [PJ]
+    lib.msa_project_workspace.restype = Z
+    lib.msa_project.argtypes = [PJ] + [P] * 12 + [Z, P]
+    lib.msa_project.restype = I32
     lib.msa_selftest_bounded_wait.argtypes = [P, P]
     lib.msa_selftest_bounded_wait.restype = I32
     lib.msa_profile_enable.argtypes = [ctypes.c_int32]
@@ -284,6 +295,38 @@ def forward(q, k, v, q_idx, k_idx, B_k: int, kk: int, attn_scale: float = 0.0, s
     return o, lse, idx
 
 
+def project(x: torch.Tensor, w_q: torch.Tensor, w_k: torch.Tensor, w_v: torch.Tensor,
+            w_qidx: torch.Tensor, w_kidx: torch.Tensor, H_q: int, H_kv: int,
+            workspace: Optional[torch.Tensor] = None, stream=None) -> dict:
+    """The projections upstream of the path: x [T,d_model] bf16 and the five
+    weights [d_model, out] bf16 -> q [T,H_q,d_h], k, v [T,H_kv,d_h], q_idx
+    [T,H_kv,d_idx], k_idx [T,d_idx] (x W for each; the index branch's
+    stopgrad(x) is x forward)."""
+    T, d_model = x.shape
+    d_h = w_q.shape[1] // H_q
+    d_idx = w_kidx.shape[1]
+    _want(x, "x", torch.bfloat16, (T, d_model))
+    _want(w_q, "w_q", torch.bfloat16, (d_model, H_q * d_h))
+    _want(w_k, "w_k", torch.bfloat16, (d_model, H_kv * d_h))
+    _want(w_v, "w_v", torch.bfloat16, (d_model, H_kv * d_h))
+    _want(w_qidx, "w_qidx", torch.bfloat16, (d_model, H_kv * d_idx))
+    _want(w_kidx, "w_kidx", torch.bfloat16, (d_model, d_idx))
+    dev = x.device
+    out = {"q": torch.empty((T, H_q, d_h), dtype=torch.bfloat16, device=dev),
+           "k": torch.empty((T, H_kv, d_h), dtype=torch.bfloat16, device=dev),
+           "v": torch.empty((T, H_kv, d_h), dtype=torch.bfloat16, device=dev),
+           "q_idx": torch.empty((T, H_kv, d_idx), dtype=torch.bfloat16, device=dev),
+           "k_idx": torch.empty((T, d_idx), dtype=torch.bfloat16, device=dev)}
+    d = msa_proj_dims(int(T), int(d_model), int(H_q), int(H_kv), int(d_h), int(d_idx))
+    ws = _workspace(int(LIB.msa_project_workspace(ctypes.byref(d))), dev, workspace)
+    _raise("msa_project",
+           LIB.msa_project(ctypes.byref(d), _ptr(x), _ptr(w_q), _ptr(w_k), _ptr(w_v), _ptr(w_qidx),
+                           _ptr(w_kidx), _ptr(out["q"]), _ptr(out["k"]), _ptr(out["v"]),
+                           _ptr(out["q_idx"]), _ptr(out["k_idx"]), _ptr(ws), ws.numel(),
+                           _stream(stream)))
+    return out
+
+
 def _cu(cu_seqlens, N: int):
     """cu_seqlens (a list, numpy array or CPU tensor of n + 1 ints) as a host
     int64 array for the C ABI, with the count of sequences."""
@@ -298,6 +341,14 @@ def varlen_dims(n_seqs, N, H_q, H_kv, d_h, d_idx, B_k, k, attn_scale=0.0,
                 idx_scale=0.0) -> msa_varlen_dims:
     return msa_varlen_dims(int(n_seqs), int(N), int(H_q), int(H_kv), int(d_h), int(d_idx),
                            int(B_k), int(k), float(attn_scale), float(idx_scale))
+
+
+def varlen_workspace_size(cu_seqlens, N, H_q, H_kv, d_h, d_idx, B_k, k) -> int:
+    """Bytes of one workspace that serves both packed-batch calls."""
+    cu, n = _cu(cu_seqlens, N)
+    d = varlen_dims(n, N, H_q, H_kv, d_h, d_idx, B_k, k)
+    return max(int(LIB.msa_index_topk_varlen_workspace(ctypes.byref(d), cu)),
+               int(LIB.msa_sparse_attn_fwd_varlen_workspace(ctypes.byref(d), cu)))
 
 
 def index_topk_varlen(q_idx: torch.Tensor, k_idx: torch.Tensor, cu_seqlens, B_k: int, k: int,

@@ -322,6 +322,62 @@ msa_status msa_sparse_attn_fwd(const msa_dims* d, const void* q, const void* k, 
   return from_cuda(msa::launch_sparse_attn(a, s));
 }
 
+// ------------------------------------------------- upstream projections --
+namespace {
+constexpr size_t kCublasWorkspace = size_t(32) << 20;
+
+msa_status check_proj(const msa_proj_dims* d) {
+  if (d == nullptr || d->T < 1 || d->d_model < 1 || d->H_q < 1 || d->H_kv < 1 || d->d_h < 1 ||
+      d->d_idx < 1)
+    return MSA_ERR_INVALID_ARG;
+  if (d->T >= (int64_t(1) << 31)) return MSA_ERR_UNSUPPORTED;
+  const int64_t widths[4] = {int64_t(d->H_q) * d->d_h, int64_t(d->H_kv) * d->d_h,
+                             int64_t(d->H_kv) * d->d_idx, d->d_idx};
+  if (d->d_model % 8 != 0) return MSA_ERR_UNSUPPORTED;
+  for (int64_t w : widths)
+    if (w % 8 != 0 || w >= (int64_t(1) << 31)) return MSA_ERR_UNSUPPORTED;
+  return MSA_OK;
+}
+}  // namespace
+
+size_t msa_project_workspace(const msa_proj_dims* d) {
+  if (check_proj(d) != MSA_OK) return 0;
+  return kStatusBytes + kCublasWorkspace;
+}
+
+msa_status msa_project(const msa_proj_dims* d, const void* x, const void* w_q, const void* w_k,
+                       const void* w_v, const void* w_qidx, const void* w_kidx, void* q, void* k,
+                       void* v, void* q_idx, void* k_idx, void* ws, size_t ws_bytes,
+                       void* stream) {
+  const void* ptrs[12] = {x, w_q, w_k, w_v, w_qidx, w_kidx, q, k, v, q_idx, k_idx, ws};
+  for (const void* p : ptrs)
+    if (p == nullptr || !aligned16(p)) return MSA_ERR_INVALID_ARG;
+  msa_status st = check_proj(d);
+  if (st != MSA_OK) return st;
+  if (ws_bytes < msa_project_workspace(d)) return MSA_ERR_WORKSPACE_TOO_SMALL;
+  msa::ProjectLaunch a{};
+  a.x = x;
+  a.w_q = w_q;
+  a.w_k = w_k;
+  a.w_v = w_v;
+  a.w_qidx = w_qidx;
+  a.w_kidx = w_kidx;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.q_idx = q_idx;
+  a.k_idx = k_idx;
+  a.T = d->T;
+  a.d_model = d->d_model;
+  a.H_q = d->H_q;
+  a.H_kv = d->H_kv;
+  a.d_h = d->d_h;
+  a.d_idx = d->d_idx;
+  a.ws = static_cast<uint8_t*>(ws) + kStatusBytes;
+  a.ws_bytes = ws_bytes - kStatusBytes;
+  return from_cuda(msa::launch_project(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 // ------------------------------------------------ packed sequences (varlen) --
 namespace {
 

@@ -58,6 +58,26 @@ int64_t varlen_blocks(const int64_t* cu, int n, int B_k);
 cudaError_t build_varlen_tables(const int64_t* cu, int n, int B_k, int H_kv, bool tiles,
                                 void* dst, VarlenTables* out, cudaStream_t s);
 
+// The projections upstream of the path (five GEMMs through cuBLAS).
+struct ProjectLaunch {
+  const void* x;  // [T, d_model] bf16
+  const void* w_q;
+  const void* w_k;
+  const void* w_v;
+  const void* w_qidx;
+  const void* w_kidx;  // [d_model, out] bf16 each
+  void* q;
+  void* k;
+  void* v;
+  void* q_idx;
+  void* k_idx;
+  int64_t T;
+  int d_model, H_q, H_kv, d_h, d_idx;
+  void* ws;  // cuBLAS workspace
+  size_t ws_bytes;
+};
+cudaError_t launch_project(const ProjectLaunch& a, cudaStream_t s);
+
 struct AttnLaunch {
   const void* q;
   const void* k;

@@ -118,6 +118,32 @@ MSA_API msa_status msa_sparse_attn_fwd(const msa_dims* dims, const void* q, cons
                                void* workspace, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * The projections upstream of the path (xllm-io review, Algorithm 1, lines
+ * 1-2): Q = X W_q, K = X W_k, V = X W_v, Q_idx = stopgrad(X) W_qidx, K_idx =
+ * stopgrad(X) W_kidx (stopgrad acts on gradients only: forward, X itself).
+ *   x       [T, d_model] bf16 (T tokens; one sequence or a packed batch)
+ *   w_q     [d_model, H_q * d_h]     w_k, w_v  [d_model, H_kv * d_h]
+ *   w_qidx  [d_model, H_kv * d_idx]  w_kidx    [d_model, d_idx]      (bf16)
+ *   q [T, H_q, d_h], k, v [T, H_kv, d_h], q_idx [T, H_kv, d_idx],
+ *   k_idx [T, d_idx]: bf16, written, fp32 accumulation rounded to nearest
+ * Five GEMMs through cuBLAS (libcublas.so.12, opened on first use;
+ * MSA_ERR_CUDA with msa_last_error "shared object initialization failed" if
+ * it cannot be loaded).  The workspace is handed to cuBLAS as its scratch;
+ * cuBLAS's handle (one per thread and device, created on the first call)
+ * holds cuBLAS's own small device state.  Supported: T < 2^31, d_model and
+ * every output width a multiple of 8.
+ * ------------------------------------------------------------------------- */
+typedef struct {
+  int64_t T;
+  int32_t d_model, H_q, H_kv, d_h, d_idx;
+} msa_proj_dims;
+MSA_API size_t msa_project_workspace(const msa_proj_dims* dims);
+MSA_API msa_status msa_project(const msa_proj_dims* dims, const void* x, const void* w_q,
+                               const void* w_k, const void* w_v, const void* w_qidx,
+                               const void* w_kidx, void* q, void* k, void* v, void* q_idx,
+                               void* k_idx, void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
  * Several prefill sequences packed along the token axis (variable length):
  * sequence s holds tokens cu_seqlens[s] .. cu_seqlens[s+1]-1 of every tensor
  * (any lengths, empty ones allowed, no padding), and the method runs inside

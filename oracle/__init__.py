@@ -222,6 +222,16 @@ def forward(inp: dict, B_k: int, k: int, rows: Optional[np.ndarray] = None,
     return {"idx": idx, "cut": cut, "next": nxt, "o": o, "lse": lse, "rows": rows}
 
 
+def project(x: np.ndarray, w: np.ndarray) -> np.ndarray:
+    """One projection of Algorithm 1, lines 1-2 (xllm-io review): x W in fp64
+    from the exactly widened bf16 operands.  x [T, d_model], w [d_model, n]
+    (bf16 bits) -> [T, n] float64.  The index projections take stopgrad(x),
+    which is x itself in a forward pass."""
+    xf = (np.ascontiguousarray(x, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
+    wf = (np.ascontiguousarray(w, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
+    return xf.astype(np.float64) @ wf.astype(np.float64)
+
+
 def forward_varlen(inp: dict, cu_seqlens, B_k: int, k: int, rows: Optional[np.ndarray] = None,
                    idx_rows: Optional[np.ndarray] = None, threads: int = 0) -> dict:
     """Eq. 6-8 for a batch of sequences packed along the token axis: sequence
