@@ -67,6 +67,9 @@ def _load():
             lib.oracle_sparse_attn.argtypes = [P, P, P, P, I64, I32, I32, I32, I32, I32, D, P, I64,
                                                P, P, I32]
             lib.oracle_dense_attn.argtypes = [P, P, P, I64, I32, I32, I32, D, P, I64, P, P, I32]
+            lib.oracle_sparse_attn_bwd.argtypes = [P, P, P, P, P, I64, I32, I32, I32, I32, I32, D,
+                                                   P, P, P, I32]
+            lib.oracle_sparse_attn_bwd.restype = I32
             lib.oracle_index_lse.argtypes = [P, P, P, I64, I32, I32, I32, I32, D, P, I64, P, I32]
             lib.oracle_flops.argtypes = [D] * 7 + [P, P, P]
             for f in ("oracle_block_scores", "oracle_index_topk", "oracle_sparse_attn",
@@ -165,6 +168,26 @@ def sparse_attn(q_rows: np.ndarray, k: np.ndarray, v: np.ndarray, idx_rows: np.n
                                       ir.shape[2], float(scale), _p(rows), n, _p(o), _p(lse),
                                       threads), "sparse_attn")
     return o, lse
+
+
+def sparse_attn_bwd(q: np.ndarray, k: np.ndarray, v: np.ndarray, idx: np.ndarray,
+                    d_o: np.ndarray, B_k: int, scale: Optional[float] = None,
+                    threads: int = 0) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """Gradients of Eq. 8 with the selection fixed, all rows of one sequence:
+    q, d_o [N,H_q,d_h], k/v [N,H_kv,d_h] (bf16 bits), idx [N,H_kv,kk] ->
+    dQ [N,H_q,d_h], dK, dV [N,H_kv,d_h] (float64)."""
+    qq, kk_, vv, gg = (_c(a, np.uint16) for a in (q, k, v, d_o))
+    ir = _c(idx, np.int32)
+    N, H_q, d_h = qq.shape
+    H_kv = kk_.shape[1]
+    scale = 1.0 / np.sqrt(d_h) if scale is None else scale
+    dq = np.empty((N, H_q, d_h), dtype=np.float64)
+    dk = np.empty((N, H_kv, d_h), dtype=np.float64)
+    dv = np.empty((N, H_kv, d_h), dtype=np.float64)
+    _check(_load().oracle_sparse_attn_bwd(_p(qq), _p(kk_), _p(vv), _p(ir), _p(gg), N, H_q, H_kv,
+                                          d_h, B_k, ir.shape[2], float(scale), _p(dq), _p(dk),
+                                          _p(dv), threads), "sparse_attn_bwd")
+    return dq, dk, dv
 
 
 def index_lse(q_idx_rows: np.ndarray, k_idx: np.ndarray, idx_rows: np.ndarray, B_k: int,

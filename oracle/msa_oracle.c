@@ -231,6 +231,110 @@ static void attend(const uint16_t *q, const uint16_t *K, const uint16_t *V,
 }
 
 /*
+ * Gradients of Eq. 8 for every row of one sequence (the backward pass of the
+ * Main Branch with the selection held fixed: the Index Branch is not
+ * differentiated through the Top-k).  With s_j = scale <q_i,h, k_j>, p the
+ * softmax of s over the row's selected tokens j <= i, o = sum_j p_j v_j and
+ * dO the gradient arriving at o:
+ *   dp_j = <dO, v_j>,  D = <dO, o>,  ds_j = p_j (dp_j - D)
+ *   dQ[i,h]  = scale sum_j ds_j k_j
+ *   dK[j,r] += scale ds_j q_i,h       dV[j,r] += p_j dO   (r = h / G)
+ * q, dO: [N, H_q, d_h]; K, V: [N, H_kv, d_h]; idx: [N, H_kv, k];
+ * dq_out: [N, H_q, d_h]; dk_out, dv_out: [N, H_kv, d_h] (float64).
+ * Threads split the KV groups: group r's rows write only dK/dV of group r.
+ */
+int oracle_sparse_attn_bwd(const uint16_t *q, const uint16_t *K, const uint16_t *V,
+                           const int32_t *idx, const uint16_t *dO, int64_t N, int H_q,
+                           int H_kv, int d_h, int B_k, int k, double scale, double *dq_out,
+                           double *dk_out, double *dv_out, int n_threads)
+{
+    if (!q || !K || !V || !idx || !dO || !dq_out || !dk_out || !dv_out || N <= 0 || H_q <= 0 ||
+        H_kv <= 0 || H_q % H_kv != 0 || d_h <= 0 || B_k <= 0 || k <= 0)
+        return -1;
+    const int G = H_q / H_kv;
+    const int64_t B = (N + B_k - 1) / B_k;
+    for (int64_t e = 0; e < N * H_kv * k; ++e)
+        if (idx[e] >= B || idx[e] < -1) return -4;
+    const int64_t kv_stride = (int64_t)H_kv * d_h;
+    for (int64_t e = 0; e < N * H_q * d_h; ++e) dq_out[e] = 0.0;
+    for (int64_t e = 0; e < N * kv_stride; ++e) {
+        dk_out[e] = 0.0;
+        dv_out[e] = 0.0;
+    }
+    set_threads(n_threads);
+    int err = 0;
+#pragma omp parallel
+    {
+        const int64_t cap = (int64_t)k * B_k;
+        int64_t *keys = (int64_t *)malloc(sizeof(int64_t) * (size_t)cap);
+        double *p = (double *)malloc(sizeof(double) * (size_t)cap);
+        double *o = (double *)malloc(sizeof(double) * (size_t)d_h);
+        if (!keys || !p || !o) {
+#pragma omp atomic write
+            err = -3;
+        } else {
+#pragma omp for schedule(static, 1)
+            for (int r = 0; r < H_kv; ++r) {
+                for (int64_t i = 0; i < N; ++i) {
+                    int64_t n = 0;
+                    for (int sl = 0; sl < k; ++sl) {
+                        const int32_t b = idx[(i * H_kv + r) * k + sl];
+                        if (b < 0) continue;
+                        const int64_t j0 = (int64_t)b * B_k;
+                        int64_t j1 = j0 + B_k;
+                        if (j1 > N) j1 = N;
+                        for (int64_t j = j0; j < j1 && j <= i; ++j) keys[n++] = j;
+                    }
+                    if (n == 0) continue;
+                    for (int g = 0; g < G; ++g) {
+                        const int h = r * G + g;
+                        const uint16_t *qh = q + (i * H_q + h) * d_h;
+                        const uint16_t *gh = dO + (i * H_q + h) * d_h;
+                        double m = -INFINITY;
+                        for (int64_t t = 0; t < n; ++t) {
+                            const uint16_t *kr = K + keys[t] * kv_stride + (int64_t)r * d_h;
+                            double dot = 0.0;
+                            for (int d = 0; d < d_h; ++d) dot += bf(qh[d]) * bf(kr[d]);
+                            p[t] = dot * scale;
+                            if (p[t] > m) m = p[t];
+                        }
+                        double l = 0.0;
+                        for (int64_t t = 0; t < n; ++t) {
+                            p[t] = exp(p[t] - m);
+                            l += p[t];
+                        }
+                        for (int d = 0; d < d_h; ++d) o[d] = 0.0;
+                        for (int64_t t = 0; t < n; ++t) {
+                            p[t] /= l;
+                            const uint16_t *vr = V + keys[t] * kv_stride + (int64_t)r * d_h;
+                            for (int d = 0; d < d_h; ++d) o[d] += p[t] * bf(vr[d]);
+                        }
+                        double D = 0.0;
+                        for (int d = 0; d < d_h; ++d) D += bf(gh[d]) * o[d];
+                        double *dq = dq_out + (i * H_q + h) * d_h;
+                        for (int64_t t = 0; t < n; ++t) {
+                            const int64_t row = keys[t] * kv_stride + (int64_t)r * d_h;
+                            double dp = 0.0;
+                            for (int d = 0; d < d_h; ++d) dp += bf(gh[d]) * bf(V[row + d]);
+                            const double ds = p[t] * (dp - D);
+                            for (int d = 0; d < d_h; ++d) {
+                                dq[d] += scale * ds * bf(K[row + d]);
+                                dk_out[row + d] += scale * ds * bf(qh[d]);
+                                dv_out[row + d] += p[t] * bf(gh[d]);
+                            }
+                        }
+                    }
+                }
+            }
+        }
+        free(keys);
+        free(p);
+        free(o);
+    }
+    return err;
+}
+
+/*
  * Eq. 8 [xllm], [chl] 5.1: for each requested query row i and head h
  * (group r = h / G, adjacent heads share one KV head, Eq. 1 note) attend to
  * the tokens of the blocks in idx[row, r, :] (entries < 0 are empty slots),

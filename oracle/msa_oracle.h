@@ -29,6 +29,14 @@ int oracle_index_topk(const uint16_t *q_idx_rows, const uint16_t *k_idx,
                       int32_t *idx_out, double *cut_out, double *next_out,
                       int n_threads);
 
+/* Gradients of Eq. 8 (selection fixed) for all N rows of one sequence:
+ * q, dO: [N, H_q, d_h]; K, V: [N, H_kv, d_h]; idx: [N, H_kv, k];
+ * dq_out: [N, H_q, d_h]; dk_out, dv_out: [N, H_kv, d_h] (float64). */
+int oracle_sparse_attn_bwd(const uint16_t *q, const uint16_t *K, const uint16_t *V,
+                           const int32_t *idx, const uint16_t *dO, int64_t N, int H_q,
+                           int H_kv, int d_h, int B_k, int k, double scale, double *dq_out,
+                           double *dk_out, double *dv_out, int n_threads);
+
 /* Eq. 8 for the listed rows with the given selection.
  * q_rows: [n_rows, H_q, d_h]; K, V: [N, H_kv, d_h]; idx: [n_rows, H_kv, k];
  * o_out: [n_rows, H_q, d_h]; lse_out: [n_rows, H_q] or NULL. */
