@@ -8,6 +8,7 @@ of ``include/msa.h``); this package is its thin Python binding:
 * ``forward``         both, for one prefill sequence
 * ``forward_varlen``  both, for a packed batch of sequences of any lengths
 * ``project``         the Q, K, V and index projections upstream of the path
+* ``sparse_attn_bwd`` the backward of the Main Branch (dQ, dK, dV)
 * ``sparse_decode``   one decode step for a batch of sequences
 * ``paged_decode_fp8`` the same step on a paged FP8 (E4M3) KV cache
 
@@ -22,7 +23,7 @@ _CAPI = ("index_topk", "sparse_attn_fwd", "forward", "sparse_decode", "device_st
          "index_lse", "index_lse_workspace_size", "paged_dims", "paged_decode_fp8",
          "paged_decode_fp8_workspace_size", "quantize_fp8_rows", "index_topk_varlen",
          "sparse_attn_fwd_varlen", "forward_varlen", "varlen_dims", "project",
-         "varlen_workspace_size")
+         "varlen_workspace_size", "sparse_attn_bwd")
 
 __all__ = list(_CAPI) + ["inputs"]
 

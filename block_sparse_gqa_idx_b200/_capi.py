@@ -72,7 +72,8 @@ EXPORTS = ("msa_index_topk_workspace", "msa_index_topk", "msa_sparse_attn_fwd_wo
            "msa_paged_decode_fp8_workspace", "msa_paged_decode_fp8", "msa_quantize_fp8_rows",
            "msa_index_topk_varlen_workspace", "msa_index_topk_varlen",
            "msa_sparse_attn_fwd_varlen_workspace", "msa_sparse_attn_fwd_varlen",
-           "msa_project_workspace", "msa_project")
+           "msa_project_workspace", "msa_project", "msa_sparse_attn_bwd_workspace",
+           "msa_sparse_attn_bwd")
 
 
 def _load() -> ctypes.CDLL:
@@ -120,6 +121,10 @@ def _load() -> ctypes.CDLL:
     lib.msa_sparse_attn_fwd_varlen_workspace.restype = Z
     lib.msa_sparse_attn_fwd_varlen.argtypes = [VD, CU, P, P, P, P, P, P, P, Z, P]
     lib.msa_sparse_attn_fwd_varlen.restype = I32
+    lib.msa_sparse_attn_bwd_workspace.argtypes = [D]
+    lib.msa_sparse_attn_bwd_workspace.restype = Z
+    lib.msa_sparse_attn_bwd.argtypes = [D] + [P] * 11 + [Z, P]
+    lib.msa_sparse_attn_bwd.restype = I32
     PJ = ctypes.POINTER(msa_proj_dims)
     lib.msa_project_workspace.argtypes = [PJ]
     lib.msa_project_workspace.restype = Z
@@ -285,6 +290,35 @@ def sparse_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, idx: torc
            LIB.msa_sparse_attn_fwd(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(idx), _ptr(o),
                                    _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)))
     return o, lse
+
+
+def sparse_attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, idx: torch.Tensor,
+                    o: torch.Tensor, lse: torch.Tensor, d_o: torch.Tensor, B_k: int,
+                    attn_scale: float = 0.0, workspace: Optional[torch.Tensor] = None,
+                    stream=None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """Backward of Eq. 8 with the selection fixed: (dq, dk, dv) bf16 from the
+    forward's o [N,H_q,d_h], lse [N,H_q] and d_o [N,H_q,d_h]."""
+    N, H_q, d_h = q.shape
+    H_kv = k.shape[1]
+    kk = idx.shape[2]
+    for t, name, dt, sh in ((q, "q", torch.bfloat16, (N, H_q, d_h)),
+                            (k, "k", torch.bfloat16, (N, H_kv, d_h)),
+                            (v, "v", torch.bfloat16, (N, H_kv, d_h)),
+                            (idx, "idx", torch.int32, (N, H_kv, kk)),
+                            (o, "o", torch.bfloat16, (N, H_q, d_h)),
+                            (lse, "lse", torch.float32, (N, H_q)),
+                            (d_o, "d_o", torch.bfloat16, (N, H_q, d_h))):
+        _want(t, name, dt, sh)
+    dq = torch.empty_like(q)
+    dk = torch.empty_like(k)
+    dv = torch.empty_like(v)
+    d = dims(N, H_q, H_kv, d_h, 64, B_k, kk, attn_scale)
+    ws = _workspace(int(LIB.msa_sparse_attn_bwd_workspace(ctypes.byref(d))), q.device, workspace)
+    _raise("msa_sparse_attn_bwd",
+           LIB.msa_sparse_attn_bwd(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(idx), _ptr(o),
+                                   _ptr(lse), _ptr(d_o), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws),
+                                   ws.numel(), _stream(stream)))
+    return dq, dk, dv
 
 
 def forward(q, k, v, q_idx, k_idx, B_k: int, kk: int, attn_scale: float = 0.0, stream=None,

@@ -322,6 +322,51 @@ msa_status msa_sparse_attn_fwd(const msa_dims* d, const void* q, const void* k, 
   return from_cuda(msa::launch_sparse_attn(a, s));
 }
 
+// ------------------------------------------- backward of the Main Branch --
+size_t msa_sparse_attn_bwd_workspace(const msa_dims* d) {
+  if (d == nullptr || check_attn_dims(d) != MSA_OK) return 0;
+  return kStatusBytes +
+         msa::attn_bwd_workspace_bytes(d->N, d->H_q, d->H_kv, d->d_h, d->B_k, d->k);
+}
+
+msa_status msa_sparse_attn_bwd(const msa_dims* d, const void* q, const void* k, const void* v,
+                               const int32_t* idx, const void* o, const float* lse,
+                               const void* d_o, void* dq, void* dk, void* dv, void* ws,
+                               size_t ws_bytes, void* stream) {
+  const void* ptrs[12] = {q, k, v, idx, o, lse, d_o, dq, dk, dv, ws, d};
+  for (const void* p : ptrs)
+    if (p == nullptr) return MSA_ERR_INVALID_ARG;
+  for (int j = 0; j < 11; ++j)
+    if (!aligned16(ptrs[j])) return MSA_ERR_INVALID_ARG;
+  msa_status st = check_attn_dims(d);
+  if (st != MSA_OK) return st;
+  if (ws_bytes < msa_sparse_attn_bwd_workspace(d)) return MSA_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (from_cuda(cudaMemsetAsync(ws, 0, sizeof(msa::DevStatus), s)) != MSA_OK) return MSA_ERR_CUDA;
+  msa::BwdLaunch a{};
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.idx = idx;
+  a.o = o;
+  a.lse = lse;
+  a.dO = d_o;
+  a.dq = dq;
+  a.dk = dk;
+  a.dv = dv;
+  a.N = d->N;
+  a.H_q = d->H_q;
+  a.H_kv = d->H_kv;
+  a.d_h = d->d_h;
+  a.B_k = d->B_k;
+  a.kk = d->k;
+  a.scale = d->attn_scale > 0.0f ? d->attn_scale : 1.0f / sqrtf(static_cast<float>(d->d_h));
+  a.ws = static_cast<uint8_t*>(ws) + kStatusBytes;
+  a.ws_bytes = ws_bytes - kStatusBytes;
+  a.status = status_of(ws);
+  return from_cuda(msa::launch_sparse_attn_bwd(a, s));
+}
+
 // ------------------------------------------------- upstream projections --
 namespace {
 constexpr size_t kCublasWorkspace = size_t(32) << 20;

@@ -102,6 +102,29 @@ size_t attn_workspace_bytes(int64_t N, int H_q, int H_kv, int d_h, int B_k, int 
                             int64_t B_tot = 0);
 cudaError_t launch_sparse_attn(const AttnLaunch& a, cudaStream_t s);
 
+// Backward of Eq. 8 (selection fixed): dQ, dK, dV from dO, the forward's O
+// and LSE.
+struct BwdLaunch {
+  const void* q;
+  const void* k;
+  const void* v;
+  const int32_t* idx;
+  const void* o;
+  const float* lse;
+  const void* dO;
+  void* dq;
+  void* dk;
+  void* dv;
+  int64_t N;
+  int H_q, H_kv, d_h, B_k, kk;
+  float scale;
+  void* ws;
+  size_t ws_bytes;
+  DevStatus* status;
+};
+size_t attn_bwd_workspace_bytes(int64_t N, int H_q, int H_kv, int d_h, int B_k, int kk);
+cudaError_t launch_sparse_attn_bwd(const BwdLaunch& a, cudaStream_t s);
+
 struct IdxLseLaunch {
   const void* q_idx;
   const void* k_idx;

@@ -118,6 +118,28 @@ MSA_API msa_status msa_sparse_attn_fwd(const msa_dims* dims, const void* q, cons
                                void* workspace, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Backward of the Main Branch, Eq. 8, with the selection held fixed (the
+ * Index Branch is not differentiated through its Top-k): given dO, the
+ * gradient arriving at O, and the forward's O and LSE,
+ *   P = softmax over the selected tokens j <= i (from LSE),  D = rowsum(dO*O),
+ *   dS = P (dO V^T - D),  dQ = scale dS K,  dK = scale dS^T Q,  dV = P^T dO
+ * (xllm-io review, §四 "Dynamic load balancing" and §五 4.3: the backward
+ * runs over the forward's KV-outer schedule, hot blocks split by a global
+ * atomic work counter).
+ *   q, o, d_o  [N, H_q, d_h] bf16     k, v [N, H_kv, d_h] bf16
+ *   idx        [N, H_kv, k] int32 (the forward's selection)
+ *   lse        [N, H_q] fp32 (the forward's natural-log LSE)
+ *   dq [N, H_q, d_h], dk, dv [N, H_kv, d_h]: bf16, written (fp32 sums
+ *   rounded to nearest); keys no query selected get zero gradients.
+ * Supported: as msa_sparse_attn_fwd.  One sequence (batch 1).
+ * ------------------------------------------------------------------------- */
+MSA_API size_t msa_sparse_attn_bwd_workspace(const msa_dims* dims);
+MSA_API msa_status msa_sparse_attn_bwd(const msa_dims* dims, const void* q, const void* k,
+                                       const void* v, const int32_t* idx, const void* o,
+                                       const float* lse, const void* d_o, void* dq, void* dk,
+                                       void* dv, void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
  * The projections upstream of the path (xllm-io review, Algorithm 1, lines
  * 1-2): Q = X W_q, K = X W_k, V = X W_v, Q_idx = stopgrad(X) W_qidx, K_idx =
  * stopgrad(X) W_kidx (stopgrad acts on gradients only: forward, X itself).
