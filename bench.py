@@ -528,6 +528,9 @@ def run_msa(args, cfg, rank, world, local, steps, warmup, e2e_steps, cpu_rows):
 
     kernels = {n: {"launches": v[0], "ms_per_step": v[1] / steps,
                    "share": v[1] / total_ms if total_ms else None} for n, v in prof.items()}
+    backward = None
+    if world == 1 and not varlen and getattr(args, "backward", False) and cfg.name == args.workload:
+        backward = time_backward(msa, d, idx, o, lse, cfg, stream, f_main, pk, pk_kind)
     # time between kernels: the step time minus the kernels' summed event time
     idle = max(0.0, ms - total_ms / steps)
     return {
@@ -559,7 +562,51 @@ def run_msa(args, cfg, rank, world, local, steps, warmup, e2e_steps, cpu_rows):
         "idle_ms_per_step": idle, "idle_frac": idle / ms if ms else None,
         "clocks": clk,
         "input_generation_s": gen_s,
+        **({"backward": backward} if backward is not None else {}),
     }
+
+
+def time_backward(msa, d, idx, o, lse, cfg, stream, f_main, pk, pk_kind, steps=3, warmup=1):
+    """The backward of the Main Branch (dQ, dK, dV with the selection fixed)
+    after the timed forward steps: seeded dO, the last forward's O, LSE and
+    selection; CUDA events on the stream.  Its work is the five GEMMs per
+    selected key (S recomputed, dP, dQ, dK, dV): 2.5x the forward's main term."""
+    import torch
+
+    gen = torch.Generator(device=o.device).manual_seed(1234)
+    d_o = torch.randn(o.shape, generator=gen, device=o.device, dtype=torch.float32).to(o.dtype)
+    ws = torch.empty(msa.sparse_attn_bwd_workspace_size(
+        msa.dims(cfg.N, cfg.H_q, cfg.H_kv, cfg.d_h, cfg.d_idx, cfg.B_k, cfg.k)),
+        dtype=torch.uint8, device=o.device)
+
+    def run():
+        return msa.sparse_attn_bwd(d["q"], d["k"], d["v"], idx, o, lse, d_o, cfg.B_k,
+                                   workspace=ws, stream=stream)
+
+    for _ in range(warmup):
+        run()
+    torch.cuda.synchronize()
+    msa.profile_enable(True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        run()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    msa.profile_enable(False)
+    prof = msa.profile_read()
+    code, where = msa.device_status(ws)
+    if code != 0:
+        raise RuntimeError(f"device status {code} at {where} in the backward")
+    ms = e0.elapsed_time(e1) / steps
+    flops = 2.5 * f_main
+    return {"ms_per_step": ms, "value": cfg.N / (ms * 1e-3), "unit": "tokens/s",
+            "steps": steps, "warmup": warmup,
+            "achieved_tflops": flops / (ms * 1e-3) / 1e12,
+            "frac": flops / (ms * 1e-3) / 1e12 / pk["bf16_tflops"], "peak_kind": pk_kind,
+            "flops": "2.5x the Eq. 12 main term (S, dP, dQ, dK, dV per selected key)",
+            "kernels": {n: {"launches": v[0], "ms_per_step": v[1] / steps}
+                        for n, v in prof.items()}}
 
 
 # -------------------------------------------------------------- decode arm --
@@ -761,9 +808,14 @@ def main():
     ap.add_argument("--no-also", action="store_true",
                     help="time only --workload (by default the 128K line also carries the "
                          "1M prefill and the decode workload)")
+    ap.add_argument("--backward", action="store_true",
+                    help="also time the backward of the Main Branch on the 128K/32K line "
+                         "(on by default for the 128K workload)")
     ap.add_argument("--kl-lse", action="store_true",
                     help="add the KL-loss fusion's LSE_idx to every step (a training forward)")
     args = ap.parse_args()
+    if args.workload == "128k" and not args.kl_lse:
+        args.backward = True
     world, rank, local = dist_init()
     cfg = workload(args.workload)
     is_decode = args.workload.startswith("decode")

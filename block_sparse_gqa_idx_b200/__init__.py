@@ -23,7 +23,8 @@ _CAPI = ("index_topk", "sparse_attn_fwd", "forward", "sparse_decode", "device_st
          "index_lse", "index_lse_workspace_size", "paged_dims", "paged_decode_fp8",
          "paged_decode_fp8_workspace_size", "quantize_fp8_rows", "index_topk_varlen",
          "sparse_attn_fwd_varlen", "forward_varlen", "varlen_dims", "project",
-         "varlen_workspace_size", "sparse_attn_bwd")
+         "varlen_workspace_size", "sparse_attn_bwd",
+         "sparse_attn_bwd_workspace_size")
 
 __all__ = list(_CAPI) + ["inputs"]
 

@@ -292,6 +292,10 @@ def sparse_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, idx: torc
     return o, lse
 
 
+def sparse_attn_bwd_workspace_size(d: msa_dims) -> int:
+    return int(LIB.msa_sparse_attn_bwd_workspace(ctypes.byref(d)))
+
+
 def sparse_attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, idx: torch.Tensor,
                     o: torch.Tensor, lse: torch.Tensor, d_o: torch.Tensor, B_k: int,
                     attn_scale: float = 0.0, workspace: Optional[torch.Tensor] = None,

@@ -1561,8 +1561,13 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool v
                "r"(valid ? 16 : 0)
                : "memory");
 }
-__device__ __forceinline__ void cp_async_wait_all() {
-  asm volatile("cp.async.wait_all;" ::: "memory");
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+// wait until at most N of this thread's most recent groups are pending
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 // Per-row scalars of the tile in shared memory.
@@ -1578,16 +1583,17 @@ template <int D_H, int B_K>
 struct BwdSmem {
   static constexpr int Q_BYTES = kBwdRows * D_H * 2;
   static constexpr int K_BYTES = B_K * D_H * 2;
+  // two stages of the tile's Q and dO rows (the next tile's land while the
+  // current one computes), one K/V block
   static constexpr size_t bytes() {
-    return 128 + 2 * Q_BYTES + 2 * K_BYTES + sizeof(BwdRows);
+    return 128 + 4 * Q_BYTES + 2 * K_BYTES + 2 * sizeof(BwdRows);
   }
 };
 
-// The tile's rows: scalars first (threads 0..127), then Q and dO rows by
-// 16-byte async copies (padding rows zero-filled).
-template <int D_H>
-__device__ __forceinline__ void bwd_load_rows(const BwdParams& p, int4 meta, int r, BwdRows* rows,
-                                              uint8_t* sQ, uint8_t* sdO) {
+// The tile's per-row scalars (threads 0..127); the caller synchronises
+// before bwd_issue_rows reads them.
+__device__ __forceinline__ void bwd_row_scalars(const BwdParams& p, int4 meta, int r,
+                                                BwdRows* rows) {
   const int per_q = p.H_kv * p.kk;
   const int t = threadIdx.x;
   if (t < kBwdRows) {
@@ -1609,8 +1615,15 @@ __device__ __forceinline__ void bwd_load_rows(const BwdParams& p, int4 meta, int
       rows->Drow[t] = 0.f;
     }
   }
-  __syncthreads();
+}
+
+// The tile's Q and dO rows by 16-byte async copies (padding rows
+// zero-filled), one commit group.
+template <int D_H>
+__device__ __forceinline__ void bwd_issue_rows(const BwdParams& p, const BwdRows* rows,
+                                               uint8_t* sQ, uint8_t* sdO) {
   constexpr int CPR = D_H / 8;  // 16-byte chunks per row
+  const int t = threadIdx.x;
   const uint32_t q_base = smem_u32(sQ), g_base = smem_u32(sdO);
   for (int c = t; c < kBwdRows * CPR; c += kBwdThreads) {
     const int row = c / CPR, ch = c - row * CPR;
@@ -1620,6 +1633,17 @@ __device__ __forceinline__ void bwd_load_rows(const BwdParams& p, int4 meta, int
     cp_async16(q_base + bsw<kBwdRows>(row, ch * 8), p.q + off, ok);
     cp_async16(g_base + bsw<kBwdRows>(row, ch * 8), p.dO + off, ok);
   }
+  cp_async_commit();
+}
+
+// Start loading tile `tile` into stage st: its scalars, then its rows.
+template <int D_H>
+__device__ __forceinline__ void bwd_prefetch(const BwdParams& p, int tile, BwdRows* rows,
+                                             uint8_t* sQ, uint8_t* sdO) {
+  const int4 meta = p.c.tile_meta[tile];
+  bwd_row_scalars(p, meta, (meta.x / p.B) % p.H_kv, rows);
+  __syncthreads();
+  bwd_issue_rows<D_H>(p, rows, sQ, sdO);
 }
 
 // The K and V rows of block b of group r (rows past N zero-filled).
@@ -1636,6 +1660,7 @@ __device__ __forceinline__ void bwd_load_kv(const BwdParams& p, int r, int b, ui
     cp_async16(k_base + bsw<B_K>(key, ch * 8), p.k + off, ok);
     cp_async16(v_base + bsw<B_K>(key, ch * 8), p.v + off, ok);
   }
+  cp_async_commit();
 }
 
 // dQ: each CTA walks a contiguous range of tiles; warp w owns rows
@@ -1647,28 +1672,38 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const BwdParams 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) &
                                              ~static_cast<uintptr_t>(127));
-  uint8_t* sQ = smem;
-  uint8_t* sdO = sQ + SM::Q_BYTES;
-  uint8_t* sK = sdO + SM::Q_BYTES;
+  // stage s: Q rows at smem + 2s Q_BYTES, dO rows right after
+  auto sQs = [&](int st) { return smem + st * 2 * SM::Q_BYTES; };
+  auto sdOs = [&](int st) { return smem + st * 2 * SM::Q_BYTES + SM::Q_BYTES; };
+  uint8_t* sK = smem + 4 * SM::Q_BYTES;
   uint8_t* sV = sK + SM::K_BYTES;
-  BwdRows* rows = reinterpret_cast<BwdRows*>(sV + SM::K_BYTES);
+  BwdRows* rows_s = reinterpret_cast<BwdRows*>(sV + SM::K_BYTES);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t4 = lane & 3, mi = lane >> 3, rr = lane & 7;
   const int n_tiles = p.c.n_tiles[0];
   const int t_beg = static_cast<int>(static_cast<int64_t>(n_tiles) * blockIdx.x / gridDim.x);
   const int t_end = static_cast<int>(static_cast<int64_t>(n_tiles) * (blockIdx.x + 1) / gridDim.x);
   int kv_key = -1;
+  if (t_beg < t_end) bwd_prefetch<D_H>(p, t_beg, &rows_s[0], sQs(0), sdOs(0));
   for (int tile = t_beg; tile < t_end; ++tile) {
+    const int st = (tile - t_beg) & 1;
     const int4 meta = p.c.tile_meta[tile];
     const int r = (meta.x / p.B) % p.H_kv, b = meta.x % p.B;
-    if (meta.x != kv_key) {
+    if (meta.x != kv_key) {  // every warp finished the previous tile (barrier below)
       bwd_load_kv<D_H, B_K>(p, r, b, sK, sV);
       kv_key = meta.x;
     }
-    bwd_load_rows<D_H>(p, meta, r, rows, sQ, sdO);
-    cp_async_wait_all();
+    // the next tile's rows land while this one computes
+    if (tile + 1 < t_end) {
+      bwd_prefetch<D_H>(p, tile + 1, &rows_s[st ^ 1], sQs(st ^ 1), sdOs(st ^ 1));
+      cp_async_wait_group<1>();
+    } else {
+      cp_async_wait_group<0>();
+    }
     __syncthreads();
-    const uint32_t qb = smem_u32(sQ), gb = smem_u32(sdO), kb = smem_u32(sK), vb = smem_u32(sV);
+    const BwdRows* rows = &rows_s[st];
+    const uint32_t qb = smem_u32(sQs(st)), gb = smem_u32(sdOs(st)), kb = smem_u32(sK),
+                   vb = smem_u32(sV);
     // S = Q K^T and dP = dO V^T for the warp's 16 rows
     float sacc[NT][4], pacc[NT][4];
 #pragma unroll
@@ -1757,11 +1792,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const BwdParam
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) &
                                              ~static_cast<uintptr_t>(127));
-  uint8_t* sQ = smem;
-  uint8_t* sdO = sQ + SM::Q_BYTES;
-  uint8_t* sK = sdO + SM::Q_BYTES;
+  // stage s: Q rows at smem + 2s Q_BYTES, dO rows right after
+  auto sQs = [&](int st) { return smem + st * 2 * SM::Q_BYTES; };
+  auto sdOs = [&](int st) { return smem + st * 2 * SM::Q_BYTES + SM::Q_BYTES; };
+  uint8_t* sK = smem + 4 * SM::Q_BYTES;
   uint8_t* sV = sK + SM::K_BYTES;
-  BwdRows* rows = reinterpret_cast<BwdRows*>(sV + SM::K_BYTES);
+  BwdRows* rows_s = reinterpret_cast<BwdRows*>(sV + SM::K_BYTES);
   __shared__ int s_unit;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t4 = lane & 3, mi = lane >> 3, rr = lane & 7;
@@ -1804,7 +1840,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const BwdParam
     const int t1 = t0 + kBwdUnit < n_tiles ? t0 + kBwdUnit : n_tiles;
     int cur = -1, cr = 0, cb = 0;
     zero();
+    bwd_prefetch<D_H>(p, t0, &rows_s[0], sQs(0), sdOs(0));
     for (int tile = t0; tile < t1; ++tile) {
+      const int st = (tile - t0) & 1;
       const int4 meta = p.c.tile_meta[tile];
       const int r = (meta.x / p.B) % p.H_kv, b = meta.x % p.B;
       if (meta.x != cur) {
@@ -1815,11 +1853,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const BwdParam
         cb = b;
         bwd_load_kv<D_H, B_K>(p, r, b, sK, sV);
       }
-      bwd_load_rows<D_H>(p, meta, r, rows, sQ, sdO);
-      cp_async_wait_all();
+      if (tile + 1 < t1) {
+        bwd_prefetch<D_H>(p, tile + 1, &rows_s[st ^ 1], sQs(st ^ 1), sdOs(st ^ 1));
+        cp_async_wait_group<1>();
+      } else {
+        cp_async_wait_group<0>();
+      }
       __syncthreads();
+      const BwdRows* rows = &rows_s[st];
       if (keys_warp) {
-        const uint32_t qb = smem_u32(sQ), gb = smem_u32(sdO), kb = smem_u32(sK),
+        const uint32_t qb = smem_u32(sQs(st)), gb = smem_u32(sdOs(st)), kb = smem_u32(sK),
                        vb = smem_u32(sV);
         const int jA = b * B_K + warp * 16 + g, jB = jA + 8;  // the thread's two keys
 #pragma unroll 1
