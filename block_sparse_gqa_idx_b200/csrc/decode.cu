@@ -1236,6 +1236,7 @@ extern "C" msa_status msa_sparse_decode_noalloc(const msa_decode_dims* d, const 
                                                 void* k_cache, void* v_cache, void* k_idx_cache,
                                                 int32_t* seq_len, void* o, int32_t* idx_out,
                                                 void* stream) {
+  msa::NvtxRange nvtx_range("msa_sparse_decode_noalloc");
   // the dims are checked before the scratch size is computed from them
   const msa_status dims_ok = msa_check_decode_dims(d);
   if (dims_ok != MSA_OK) return dims_ok;

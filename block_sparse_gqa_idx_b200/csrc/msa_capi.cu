@@ -217,6 +217,7 @@ size_t msa_index_topk_workspace(const msa_dims* d) {
 msa_status msa_index_topk(const msa_dims* d, const void* q_idx, const void* k_idx,
                           int32_t* idx_out, float* score_out, void* ws, size_t ws_bytes,
                           void* stream) {
+  msa::NvtxRange nvtx_range("msa_index_topk");
   if (d == nullptr || q_idx == nullptr || k_idx == nullptr || idx_out == nullptr || ws == nullptr)
     return MSA_ERR_INVALID_ARG;
   msa_status st = check_common(d->N, d->H_q, d->H_kv, 64, d->d_idx, d->B_k, d->k, d->attn_scale,
@@ -254,6 +255,7 @@ size_t msa_index_lse_workspace(const msa_dims* d) {
 msa_status msa_index_lse(const msa_dims* d, const void* q_idx, const void* k_idx,
                          const int32_t* idx, float* lse_idx, void* ws, size_t ws_bytes,
                          void* stream) {
+  msa::NvtxRange nvtx_range("msa_index_lse");
   if (d == nullptr || q_idx == nullptr || k_idx == nullptr || idx == nullptr ||
       lse_idx == nullptr || ws == nullptr)
     return MSA_ERR_INVALID_ARG;
@@ -291,6 +293,7 @@ size_t msa_sparse_attn_fwd_workspace(const msa_dims* d) {
 msa_status msa_sparse_attn_fwd(const msa_dims* d, const void* q, const void* k, const void* v,
                                const int32_t* idx, void* o, float* lse, void* ws, size_t ws_bytes,
                                void* stream) {
+  msa::NvtxRange nvtx_range("msa_sparse_attn_fwd");
   if (d == nullptr || q == nullptr || k == nullptr || v == nullptr || idx == nullptr ||
       o == nullptr || ws == nullptr)
     return MSA_ERR_INVALID_ARG;
@@ -333,6 +336,7 @@ msa_status msa_sparse_attn_bwd(const msa_dims* d, const void* q, const void* k, 
                                const int32_t* idx, const void* o, const float* lse,
                                const void* d_o, void* dq, void* dk, void* dv, void* ws,
                                size_t ws_bytes, void* stream) {
+  msa::NvtxRange nvtx_range("msa_sparse_attn_bwd");
   const void* ptrs[12] = {q, k, v, idx, o, lse, d_o, dq, dk, dv, ws, d};
   for (const void* p : ptrs)
     if (p == nullptr) return MSA_ERR_INVALID_ARG;
@@ -394,6 +398,7 @@ msa_status msa_project(const msa_proj_dims* d, const void* x, const void* w_q, c
                        const void* w_v, const void* w_qidx, const void* w_kidx, void* q, void* k,
                        void* v, void* q_idx, void* k_idx, void* ws, size_t ws_bytes,
                        void* stream) {
+  msa::NvtxRange nvtx_range("msa_project");
   const void* ptrs[12] = {x, w_q, w_k, w_v, w_qidx, w_kidx, q, k, v, q_idx, k_idx, ws};
   for (const void* p : ptrs)
     if (p == nullptr || !aligned16(p)) return MSA_ERR_INVALID_ARG;
@@ -479,6 +484,7 @@ size_t msa_index_topk_varlen_workspace(const msa_varlen_dims* d, const int64_t* 
 msa_status msa_index_topk_varlen(const msa_varlen_dims* d, const int64_t* cu_seqlens,
                                  const void* q_idx, const void* k_idx, int32_t* idx_out,
                                  float* score_out, void* ws, size_t ws_bytes, void* stream) {
+  msa::NvtxRange nvtx_range("msa_index_topk_varlen");
   if (q_idx == nullptr || k_idx == nullptr || idx_out == nullptr || ws == nullptr)
     return MSA_ERR_INVALID_ARG;
   msa_status st = check_index_varlen(d, cu_seqlens);
@@ -527,6 +533,7 @@ msa_status msa_sparse_attn_fwd_varlen(const msa_varlen_dims* d, const int64_t* c
                                       const void* q, const void* k, const void* v,
                                       const int32_t* idx, void* o, float* lse, void* ws,
                                       size_t ws_bytes, void* stream) {
+  msa::NvtxRange nvtx_range("msa_sparse_attn_fwd_varlen");
   if (q == nullptr || k == nullptr || v == nullptr || idx == nullptr || o == nullptr ||
       ws == nullptr)
     return MSA_ERR_INVALID_ARG;
@@ -580,6 +587,7 @@ msa_status msa_sparse_decode(const msa_decode_dims* d, const void* q, const void
                              const void* k_new, const void* v_new, const void* k_idx_new,
                              void* k_cache, void* v_cache, void* k_idx_cache, int32_t* seq_len,
                              void* o, int32_t* idx_out, void* ws, size_t ws_bytes, void* stream) {
+  msa::NvtxRange nvtx_range("msa_sparse_decode");
   if (d == nullptr || q == nullptr || q_idx == nullptr || k_new == nullptr || v_new == nullptr ||
       k_idx_new == nullptr || k_cache == nullptr || v_cache == nullptr ||
       k_idx_cache == nullptr || seq_len == nullptr || o == nullptr || ws == nullptr)
@@ -649,6 +657,7 @@ msa_status msa_paged_decode_fp8(const msa_paged_dims* d, const void* q, const vo
                                 void* kidx_pages, float* kidx_scale, const int32_t* page_table,
                                 int32_t* seq_len, void* o, int32_t* idx_out, void* ws,
                                 size_t ws_bytes, void* stream) {
+  msa::NvtxRange nvtx_range("msa_paged_decode_fp8");
   msa_status st = check_paged_dims(d);
   if (st != MSA_OK) return st;
   const void* ptrs[] = {q, q_idx, k_new, v_new, k_idx_new, k_pages, k_scale, v_pages, v_scale,
@@ -693,6 +702,7 @@ msa_status msa_paged_decode_fp8(const msa_paged_dims* d, const void* q, const vo
 
 msa_status msa_quantize_fp8_rows(const void* x, int64_t n_rows, int32_t dim, void* codes,
                                  float* scales, void* stream) {
+  msa::NvtxRange nvtx_range("msa_quantize_fp8_rows");
   if (x == nullptr || codes == nullptr || scales == nullptr || n_rows < 1 || dim < 2 ||
       dim % 2 != 0 || dim > 4096 || !aligned16(x) || !aligned16(codes) || !aligned16(scales))
     return MSA_ERR_INVALID_ARG;

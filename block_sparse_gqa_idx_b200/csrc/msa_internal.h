@@ -4,9 +4,20 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "msa_common.cuh"
 
 namespace msa {
+
+// An NVTX range around one C-ABI call (header-only NVTX 3: a no-op unless a
+// profiler is attached), so a timeline shows each call with its kernels.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 // Host: encode a 2D/3D bf16 tiled tensor map (dims/strides innermost first).
 bool make_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
