@@ -406,7 +406,6 @@ def run_msa(args, cfg, rank, world, local, steps, warmup, e2e_steps, cpu_rows):
     barrier()
     torch.cuda.synchronize()
     clocks.start()
-    msa.profile_enable(True)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(steps):
@@ -414,10 +413,17 @@ def run_msa(args, cfg, rank, world, local, steps, warmup, e2e_steps, cpu_rows):
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    msa.profile_enable(False)
     clk = clocks.stop()
-    prof = msa.profile_read()
     ms = max_over_ranks(e0.elapsed_time(e1) / steps, dev, world)
+    # the per-kernel split from a second pass with an event pair around
+    # every launch (kept out of the timed pass: events between the kernels
+    # would stand in the way of overlapped launches)
+    msa.profile_enable(True)
+    for _ in range(steps):
+        step(d, o, idx, lse)
+    torch.cuda.synchronize()
+    msa.profile_enable(False)
+    prof = msa.profile_read()
     value = aggregate_tokens_per_s(world, N, ms)
     code, where = msa.device_status(ws)
     if code != 0:
@@ -531,7 +537,8 @@ def run_msa(args, cfg, rank, world, local, steps, warmup, e2e_steps, cpu_rows):
     backward = None
     if world == 1 and not varlen and getattr(args, "backward", False) and cfg.name == args.workload:
         backward = time_backward(msa, d, idx, o, lse, cfg, stream, f_main, pk, pk_kind)
-    # time between kernels: the step time minus the kernels' summed event time
+    # time between kernels: the timed step minus the kernels' summed event
+    # times from the profiled pass
     idle = max(0.0, ms - total_ms / steps)
     return {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
@@ -638,10 +645,11 @@ def run_decode(args, cfg, rank, world, local, steps, warmup, e2e_steps, cpu_seqs
     else:
         caches = {k: dv(st[k]) for k in ("k_cache", "v_cache", "k_idx_cache")}
     seq_len = torch.from_numpy(st["seq_len"]).to(dev)
-    n_steps = warmup + steps + e2e_steps
+    prof_steps = max(1, min(steps, 100))
+    n_steps = warmup + steps + prof_steps + e2e_steps
     assert n_steps <= cfg.steps, "more steps than the cache has room for"
     host_in = [inputs.decode_step_inputs(cfg, j, st["sink"]) for j in range(n_steps)]
-    steps_in = [{k: dv(v) for k, v in h.items()} for h in host_in[:warmup + steps]]
+    steps_in = [{k: dv(v) for k, v in h.items()} for h in host_in[:warmup + steps + prof_steps]]
     S, H_q, H_kv, d_h, d_idx, B_k, kk = cfg.S, cfg.H_q, cfg.H_kv, cfg.d_h, cfg.d_idx, cfg.B_k, cfg.k
     o = torch.empty((S, H_q, d_h), dtype=torch.bfloat16, device=dev)
     idx = torch.empty((S, H_kv, kk), dtype=torch.int32, device=dev)
@@ -679,7 +687,6 @@ def run_decode(args, cfg, rank, world, local, steps, warmup, e2e_steps, cpu_seqs
     barrier()
     torch.cuda.synchronize()
     clocks.start()
-    msa.profile_enable(True)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for j in range(warmup, warmup + steps):
@@ -687,9 +694,7 @@ def run_decode(args, cfg, rank, world, local, steps, warmup, e2e_steps, cpu_seqs
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    msa.profile_enable(False)
     clk = clocks.stop()
-    prof = msa.profile_read()
     # the slowest replica's step time; every rank's S sequences got a token
     ms = max_over_ranks(e0.elapsed_time(e1) / steps, dev, world)
     code, where = msa.device_status(ws)
@@ -707,6 +712,14 @@ def run_decode(args, cfg, rank, world, local, steps, warmup, e2e_steps, cpu_seqs
             for b in sel[s_, r]:
                 if b >= 0:
                     sel_rows += min(B_k, Li - int(b) * B_k)
+    # the per-kernel split from a second, shorter pass with an event pair
+    # around every launch (kept out of the timed pass)
+    msa.profile_enable(True)
+    for j in range(warmup + steps, warmup + steps + prof_steps):
+        step(steps_in[j])
+    torch.cuda.synchronize()
+    msa.profile_enable(False)
+    prof = msa.profile_read()
     if fp8:
         # one byte per code plus a 4-byte scale per token (and head); the new
         # rows arrive in bf16 and are written as codes and scales
@@ -721,7 +734,7 @@ def run_decode(args, cfg, rank, world, local, steps, warmup, e2e_steps, cpu_seqs
     # ---- end to end: each step's new rows from pinned host memory, the
     # step, and O and the selection back to pinned host memory
     pinned = [{k: torch.from_numpy(np.ascontiguousarray(v).view(np.int16)).view(torch.bfloat16)
-               .pin_memory() for k, v in h.items()} for h in host_in[warmup + steps:]]
+               .pin_memory() for k, v in h.items()} for h in host_in[warmup + steps + prof_steps:]]
     dev_in = {k: torch.empty_like(v, device=dev) for k, v in pinned[0].items()}
     o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
     idx_host = torch.empty(idx.shape, dtype=idx.dtype).pin_memory()
@@ -746,9 +759,9 @@ def run_decode(args, cfg, rank, world, local, steps, warmup, e2e_steps, cpu_seqs
     cache_gb = (S * cfg.L_max * (2 * H_kv * (d_h + 4) + d_idx + 4) / 1e9 if fp8
                 else S * cfg.L_max * (2 * H_kv * d_h + d_idx) * 2 / 1e9)
     total_ms = sum(v[1] for v in prof.values())
-    kernels = {n: {"launches": v[0], "ms_per_step": v[1] / steps,
+    kernels = {n: {"launches": v[0], "ms_per_step": v[1] / prof_steps,
                    "share": v[1] / total_ms if total_ms else None} for n, v in prof.items()}
-    scan_ms = prof.get("dec8_scan" if fp8 else "dec_scan", (1, 0.0))[1] / steps
+    scan_ms = prof.get("dec8_scan" if fp8 else "dec_scan", (1, 0.0))[1] / prof_steps
     scan_bytes = S * L * (d_idx + 4) if fp8 else S * L * d_idx * 2
     cpu = None
     if world == 1 and cpu_seqs > 0:
@@ -757,7 +770,7 @@ def run_decode(args, cfg, rank, world, local, steps, warmup, e2e_steps, cpu_seqs
                "sample": f"{cpu_seqs} of the {S} sequences, one {'paged FP8 ' if fp8 else ''}"
                          f"decode step each (append, full K_idx scan, Top-k, attention), "
                          f"{dt_cpu:.1f} s"}
-    idle = max(0.0, ms - total_ms / steps)
+    idle = max(0.0, ms - total_ms / prof_steps)
     return {
         "metric": METRIC, "value": 1e3 * ms / (S * world),
         "unit": "us/token", "n_gpus": world, "steps": steps, "warmup": warmup,
@@ -779,7 +792,8 @@ def run_decode(args, cfg, rank, world, local, steps, warmup, e2e_steps, cpu_seqs
                 "us_per_step": 1e3 * e2e_ms, "steps": len(pinned),
                 "note": "each step's new rows from pinned host memory, the step, and O and "
                         "the selection back to pinned host memory, in stream order"},
-        "gpu_launches": sum(v[0] for v in prof.values()), "kernels": kernels,
+        "gpu_launches": sum(v[0] for v in prof.values()) * steps // prof_steps,
+        "kernels": kernels, "kernel_split_steps": prof_steps,
         "idle_ms_per_step": idle, "clocks": clk, "input_generation_s": gen_s,
     }
 

@@ -186,6 +186,7 @@ __device__ __forceinline__ uint64_t pack_key(float v, int b) {
 // warps' winners against each other (count of larger keys), keeps the k-1
 // best, adds the local block and writes the set in ascending block order.
 __global__ void __launch_bounds__(256) dec_topk_kernel(const DecParams p) {
+  griddep_wait();  // the previous kernel of the step has finished
   extern __shared__ uint64_t lists[];  // [8 warps][k-1][32 lanes] + winners [8][k-1]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int pair = blockIdx.x;
@@ -276,6 +277,7 @@ template <int D_H, int BK>
 __global__ void __launch_bounds__(128) dec_attend_kernel(const __grid_constant__ CUtensorMap tm_k,
                                                          const __grid_constant__ CUtensorMap tm_v,
                                                          const DecParams p) {
+  griddep_wait();  // the previous kernel of the step has finished
   constexpr int KW = BK / 4;          // keys per warp
   constexpr int NT = KW / 8;          // S n-tiles per warp
   constexpr int DT = D_H / 8;         // O n-tiles
@@ -458,6 +460,7 @@ __global__ void __launch_bounds__(128) dec_attend_kernel(const __grid_constant__
 // D_H/32 consecutive floats) is fetched with all loads in flight.
 template <int D_H>
 __global__ void __launch_bounds__(256) dec_merge_kernel(const DecParams p) {
+  griddep_wait();  // the previous kernel of the step has finished
   constexpr int PER = D_H / 32;
   const int lane = threadIdx.x & 31;
   const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;  // (s, h)
@@ -538,9 +541,10 @@ cudaError_t launch_attend(const DecParams& p, cudaStream_t stream) {
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   prof_begin("dec_attend", stream);
-  dec_attend_kernel<D_H, BK><<<p.S * p.H_kv * p.kk, 128, smem, stream>>>(tk, tv, p);
+  e = launch_pdl(dec_attend_kernel<D_H, BK>, dim3(p.S * p.H_kv * p.kk), dim3(128), smem, stream,
+                 tk, tv, p);
   prof_end(stream);
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 template <int D_IDX>
@@ -780,6 +784,7 @@ __global__ void __launch_bounds__(256, 4) dec8_scan_kernel(const DecParams p, co
 // scales staged in shared memory, S scaled per key and P per value.
 template <int D_H, int BK>
 __global__ void __launch_bounds__(128) dec8_attend_kernel(const DecParams p, const Dec8Params q8) {
+  griddep_wait();  // the previous kernel of the step has finished
   constexpr int KW = BK / 4;          // keys per warp
   constexpr int NT = KW / 8;          // S n-tiles per warp
   constexpr int DT = D_H / 8;         // O n-tiles
@@ -1080,9 +1085,8 @@ cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t stream) {
                            static_cast<int>(topk_smem));
   if (e != cudaSuccess) return e;
   prof_begin("dec_topk", stream);
-  dec_topk_kernel<<<a.S * a.H_kv, 256, topk_smem, stream>>>(p);
+  e = launch_pdl(dec_topk_kernel, dim3(a.S * a.H_kv), dim3(256), topk_smem, stream, p);
   prof_end(stream);
-  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (a.d_h == 128 && a.B_k == 128) e = launch_attend<128, 128>(p, stream);
   else if (a.d_h == 128 && a.B_k == 64) e = launch_attend<128, 64>(p, stream);
@@ -1091,10 +1095,10 @@ cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   const int rows = a.S * a.H_q;
   prof_begin("dec_merge", stream);
-  if (a.d_h == 128) dec_merge_kernel<128><<<(rows * 32 + 255) / 256, 256, 0, stream>>>(p);
-  else dec_merge_kernel<64><<<(rows * 32 + 255) / 256, 256, 0, stream>>>(p);
+  e = launch_pdl(a.d_h == 128 ? dec_merge_kernel<128> : dec_merge_kernel<64>,
+                 dim3((rows * 32 + 255) / 256), dim3(256), 0, stream, p);
   prof_end(stream);
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 size_t paged_decode_workspace_bytes(int S, int max_pages, int H_q, int H_kv, int d_h, int B_k,
@@ -1162,16 +1166,17 @@ cudaError_t launch_paged_decode_fp8(const PagedLaunch& a, cudaStream_t stream) {
                            static_cast<int>(topk_smem));
   if (e != cudaSuccess) return e;
   prof_begin("dec_topk", stream);
-  dec_topk_kernel<<<a.S * a.H_kv, 256, topk_smem, stream>>>(p);
+  e = launch_pdl(dec_topk_kernel, dim3(a.S * a.H_kv), dim3(256), topk_smem, stream, p);
   prof_end(stream);
+  if (e != cudaSuccess) return e;
   auto attend = [&](auto kern, size_t smem) -> cudaError_t {
     cudaError_t r = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (r != cudaSuccess) return r;
     prof_begin("dec8_attend", stream);
-    kern<<<a.S * a.H_kv * a.kk, 128, smem, stream>>>(p, q8);
+    r = launch_pdl(kern, dim3(a.S * a.H_kv * a.kk), dim3(128), smem, stream, p, q8);
     prof_end(stream);
-    return cudaGetLastError();
+    return r != cudaSuccess ? r : cudaGetLastError();
   };
   if (a.d_h == 128 && a.B_k == 128) e = attend(dec8_attend_kernel<128, 128>, attend8_smem<128, 128>());
   else if (a.d_h == 128) e = attend(dec8_attend_kernel<128, 64>, attend8_smem<128, 64>());
@@ -1180,10 +1185,10 @@ cudaError_t launch_paged_decode_fp8(const PagedLaunch& a, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   const int rows = a.S * a.H_q;
   prof_begin("dec_merge", stream);
-  if (a.d_h == 128) dec_merge_kernel<128><<<(rows * 32 + 255) / 256, 256, 0, stream>>>(p);
-  else dec_merge_kernel<64><<<(rows * 32 + 255) / 256, 256, 0, stream>>>(p);
+  e = launch_pdl(a.d_h == 128 ? dec_merge_kernel<128> : dec_merge_kernel<64>,
+                 dim3((rows * 32 + 255) / 256), dim3(256), 0, stream, p);
   prof_end(stream);
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t launch_quantize_fp8_rows(const void* x, int64_t n_rows, int dim, void* codes,

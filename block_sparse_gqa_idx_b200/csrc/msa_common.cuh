@@ -121,6 +121,12 @@ MSA_DEVI void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// Programmatic dependent launch: a kernel launched with the programmatic
+// stream serialization attribute may start while the previous kernel in the
+// stream finishes; griddepcontrol.wait blocks until that kernel has completed
+// and its memory operations are visible (a no-op for an ordinary launch).
+MSA_DEVI void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ldmatrix: four 8x8 b16 matrices; lanes 8j..8j+7 give the row addresses of
 // matrix j, and each lane receives one 32-bit element pair of every matrix
 // (register j from matrix j).  The .trans form delivers each matrix

@@ -25,6 +25,25 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t
 
 int num_sms();
 
+// Launch `kern` so that it may start while the previous kernel of the stream
+// finishes (programmatic stream serialization); the kernel must call
+// griddep_wait() before it reads anything the previous kernel writes.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 // Optional per-kernel timing (msa_profile_enable): when on, prof_begin/prof_end
 // record a CUDA event pair around each kernel launch on its stream.
 void prof_begin(const char* name, cudaStream_t s);
