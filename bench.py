@@ -504,7 +504,9 @@ def run_msa(args, cfg, rank, world, local, steps, warmup, e2e_steps, cpu_rows):
     else:
         roofline = {"bound": "hbm", "achieved": None, "peak": pk["hbm_gbs"], "unit": "GB/s",
                     "frac": None, "peak_kind": pk_kind}
-    traffic, traffic_src = ncu_traffic(dom, N / (launches / steps))
+    # the captured bytes scale with N k; a packed batch of short sequences
+    # selects fewer blocks per query, so it gets no figure
+    traffic, traffic_src = (None, None) if varlen else ncu_traffic(dom, N / (launches / steps))
     roofline = {"kernel": dom, **roofline, "traffic": traffic, "traffic_source": traffic_src,
                 "share": dom_ms / total_ms if total_ms else None}
     # each tensor-bound kernel against the same peak
