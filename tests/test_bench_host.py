@@ -22,8 +22,10 @@ def test_traffic_figures_match_the_current_kernels():
 def test_kernel_hash_ignores_comments_and_other_code():
     text = open(SRC, encoding="utf-8").read()
     h = bench.kernel_code_hash(text, "attn_phase1_kernel")
-    commented = text.replace("const int nb = static_cast<int>(p.nkeys / p.H_kv);",
-                             "const int nb = static_cast<int>(p.nkeys / p.H_kv);  // keys per group", 1)
+    line = "const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;"
+    i = text.index("attn_phase1_kernel(")
+    j = text.index(line, i)  # a line inside the kernel
+    commented = text[:j] + line + "  // warp and lane" + text[j + len(line):]
     assert commented != text
     assert bench.kernel_code_hash(commented, "attn_phase1_kernel") == h
     elsewhere = text + "\n__global__ void unrelated_kernel() {}\n"
