@@ -49,8 +49,8 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # kernel -> (source, kernel function, sha256, bytes per unit, unit)
 NCU_TRAFFIC = {
     "attn_phase1": ("sparse_attn.cu", "attn_phase1_kernel",
-                    "91ddfb0015a1d8d22df128a8656c1976787bd4a09264ceab50825a78cac785c1",
-                    (3575268352 + 4186103552) / 32768, "query"),
+                    "f1b0fc93e3f2bf85ed14c4b8f528f468a9d3856cb1a9f7aeea45eaeb627e8f25",
+                    (3576701184 + 4184357120) / 32768, "query"),
     "attn_merge": ("sparse_attn.cu", "attn_merge_kernel",
                    "b3995bc06ce2e51f1d1aca2b258c6c448bf62dd831be86d2dab58401aca75b38",
                    (4243319552 + 265582848) / 32768, "query"),

@@ -354,6 +354,40 @@ MSA_DEVI float fmax3(float a, float b, float c) {
   return r;
 }
 
+// Packed pairs of fp32 (sm_100 PTX .f32x2): one instruction applies the
+// operation to both halves, each rounded as the scalar op would round it.
+// A pair is carried in a 64-bit register, low half first.
+MSA_DEVI uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+MSA_DEVI float f2_lo(uint64_t x) {
+  float lo, hi;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(x));
+  return lo;
+}
+MSA_DEVI float f2_hi(uint64_t x) {
+  float lo, hi;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(x));
+  return hi;
+}
+MSA_DEVI uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+MSA_DEVI uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+MSA_DEVI uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
 MSA_DEVI bool elect_lane0() { return (threadIdx.x & 31) == 0; }
 
 }  // namespace msa

@@ -496,38 +496,45 @@ __global__ void __launch_bounds__(kP1Threads, 1)
         mB = fmaxf(mB, __shfl_xor_sync(0xFFFFFFFFu, mB, o));
       }
       const float msA = mA * p.scale_log2, msB = mB * p.scale_log2;
-      float lA0 = 0.0f, lA1 = 0.0f, lB0 = 0.0f, lB1 = 0.0f;
+      // scale, exponent, row sums and 1/l on packed pairs of a row's two keys
+      // (the halves of lA2 and lB2 are the row's two running sums)
+      const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2);
+      const uint64_t nmA = f2_pack(-msA, -msA), nmB = f2_pack(-msB, -msB);
+      uint64_t lA2 = f2_pack(0.0f, 0.0f), lB2 = lA2;
 #pragma unroll
       for (int r = 0; r < B_K / 8; ++r) {
-        const float a0 = ex2_ftz(fmaf(__uint_as_float(v[4 * r]), p.scale_log2, -msA));
-        const float a1 = ex2_ftz(fmaf(__uint_as_float(v[4 * r + 1]), p.scale_log2, -msA));
-        const float b0 = ex2_ftz(fmaf(__uint_as_float(v[4 * r + 2]), p.scale_log2, -msB));
-        const float b1 = ex2_ftz(fmaf(__uint_as_float(v[4 * r + 3]), p.scale_log2, -msB));
-        lA0 += a0;
-        lA1 += a1;
-        lB0 += b0;
-        lB1 += b1;
+        const uint64_t xa = f2_fma(
+            f2_pack(__uint_as_float(v[4 * r]), __uint_as_float(v[4 * r + 1])), sc2, nmA);
+        const uint64_t xb = f2_fma(
+            f2_pack(__uint_as_float(v[4 * r + 2]), __uint_as_float(v[4 * r + 3])), sc2, nmB);
+        const float a0 = ex2_ftz(f2_lo(xa)), a1 = ex2_ftz(f2_hi(xa));
+        const float b0 = ex2_ftz(f2_lo(xb)), b1 = ex2_ftz(f2_hi(xb));
+        lA2 = f2_add(lA2, f2_pack(a0, a1));
+        lB2 = f2_add(lB2, f2_pack(b0, b1));
         v[4 * r] = __float_as_uint(a0);
         v[4 * r + 1] = __float_as_uint(a1);
         v[4 * r + 2] = __float_as_uint(b0);
         v[4 * r + 3] = __float_as_uint(b1);
       }
-      float lA = lA0 + lA1, lB = lB0 + lB1;
+      float lA = f2_lo(lA2) + f2_hi(lA2), lB = f2_lo(lB2) + f2_hi(lB2);
 #pragma unroll
       for (int o = 1; o < 4; o <<= 1) {
         lA += __shfl_xor_sync(0xFFFFFFFFu, lA, o);
         lB += __shfl_xor_sync(0xFFFFFFFFu, lB, o);
       }
       const float invA = 1.0f / lA, invB = 1.0f / lB;
+      const uint64_t invA2 = f2_pack(invA, invA), invB2 = f2_pack(invB, invB);
       // P / l as bf16 pairs: the pair of keys (8r + 2c, 8r + 2c + 1) is P
       // column 4r + c
       uint32_t pk[B_K / 4];
 #pragma unroll
       for (int r = 0; r < B_K / 8; ++r) {
-        __nv_bfloat162 xa = __floats2bfloat162_rn(__uint_as_float(v[4 * r]) * invA,
-                                                  __uint_as_float(v[4 * r + 1]) * invA);
-        __nv_bfloat162 xb = __floats2bfloat162_rn(__uint_as_float(v[4 * r + 2]) * invB,
-                                                  __uint_as_float(v[4 * r + 3]) * invB);
+        const uint64_t na = f2_mul(
+            f2_pack(__uint_as_float(v[4 * r]), __uint_as_float(v[4 * r + 1])), invA2);
+        const uint64_t nb = f2_mul(
+            f2_pack(__uint_as_float(v[4 * r + 2]), __uint_as_float(v[4 * r + 3])), invB2);
+        __nv_bfloat162 xa = __floats2bfloat162_rn(f2_lo(na), f2_hi(na));
+        __nv_bfloat162 xb = __floats2bfloat162_rn(f2_lo(nb), f2_hi(nb));
         pk[2 * r] = *reinterpret_cast<uint32_t*>(&xa);
         pk[2 * r + 1] = *reinterpret_cast<uint32_t*>(&xb);
       }
