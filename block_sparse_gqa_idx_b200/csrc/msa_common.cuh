@@ -362,16 +362,8 @@ MSA_DEVI uint64_t f2_pack(float lo, float hi) {
   asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
   return r;
 }
-MSA_DEVI float f2_lo(uint64_t x) {
-  float lo, hi;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(x));
-  return lo;
-}
-MSA_DEVI float f2_hi(uint64_t x) {
-  float lo, hi;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(x));
-  return hi;
-}
+MSA_DEVI float f2_lo(uint64_t x) { return __uint_as_float(static_cast<uint32_t>(x)); }
+MSA_DEVI float f2_hi(uint64_t x) { return __uint_as_float(static_cast<uint32_t>(x >> 32)); }
 MSA_DEVI uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
   uint64_t r;
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
