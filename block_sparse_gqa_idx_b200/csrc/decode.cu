@@ -778,13 +778,26 @@ __global__ void __launch_bounds__(256, 4) dec8_scan_kernel(const DecParams p, co
   }
 }
 
+// Shared memory of the FP8 attend: one bf16 tile (K, then V over it) that
+// later also holds the warps' O rows for their merge.
+template <int D_H, int BK>
+struct Attend8Smem {
+  static constexpr int TILE = BK * D_H * 2;
+  static constexpr int OBUF = 4 * 16 * D_H * 4;
+  static constexpr int REGION = TILE > OBUF ? TILE : OBUF;
+};
+
 // Gathered attention: as dec_attend_kernel, with the selected page's K and V
 // codes of head r widened to bf16 into the swizzled tile layout by all
 // threads (plain loads: a key's d_h codes are one contiguous row), the keys'
-// scales staged in shared memory, S scaled per key and P per value.
+// scales staged in shared memory, S scaled per key and P per value.  K and V
+// share one tile: the V codes wait in registers (all loads are issued at the
+// start) and are widened over K once every warp has computed S, which halves
+// the shared memory of a CTA so that more CTAs (items) run on an SM at once.
 template <int D_H, int BK>
 __global__ void __launch_bounds__(128) dec8_attend_kernel(const DecParams p, const Dec8Params q8) {
   griddep_wait();  // the previous kernel of the step has finished
+  using SM = Attend8Smem<D_H, BK>;
   constexpr int KW = BK / 4;          // keys per warp
   constexpr int NT = KW / 8;          // S n-tiles per warp
   constexpr int DT = D_H / 8;         // O n-tiles
@@ -792,12 +805,11 @@ __global__ void __launch_bounds__(128) dec8_attend_kernel(const DecParams p, con
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint8_t* sK = smem;
-  uint8_t* sV = smem + BK * D_H * 2;
-  float* red = reinterpret_cast<float*>(sV + BK * D_H * 2);  // [4][16] m, [4][16] l
+  uint8_t* sT = smem;                                          // K tile, then V tile
+  float* red = reinterpret_cast<float*>(smem + SM::REGION);  // [4][16] m, [4][16] l
   float* ksc = red + 128;                                    // [BK] key scales
   float* vsc = ksc + BK;                                     // [BK] value scales
-  float* obuf = reinterpret_cast<float*>(smem);  // [4][16][D_H], over K/V once both are used
+  float* obuf = reinterpret_cast<float*>(smem);  // [4][16][D_H], over the V tile once it is used
 
   const int item = blockIdx.x;  // (s, r, slot)
   const int slot = item % p.kk;
@@ -845,31 +857,27 @@ __global__ void __launch_bounds__(128) dec8_attend_kernel(const DecParams p, con
     ks_reg = __ldg(q8.k_scale + (pg * BK + threadIdx.x) * p.H_kv + r);
     vs_reg = __ldg(q8.v_scale + (pg * BK + threadIdx.x) * p.H_kv + r);
   }
+  // 16-code pieces -> bf16 pieces of the swizzled tile
+  auto widen = [&](const uint4 (&codes)[PER_T]) {
 #pragma unroll
-  for (int i = 0; i < PER_T; ++i) {
-    const int c = threadIdx.x + i * 128;
-    const int key = c / CPK, piece = c - key * CPK;
-    const uint16_t* hk = reinterpret_cast<const uint16_t*>(&kcs[i]);
-    const uint16_t* hv = reinterpret_cast<const uint16_t*>(&vcs[i]);
-    uint4 k0, k1, v0, v1;
-    uint32_t* pk0 = reinterpret_cast<uint32_t*>(&k0);
-    uint32_t* pk1 = reinterpret_cast<uint32_t*>(&k1);
-    uint32_t* pv0 = reinterpret_cast<uint32_t*>(&v0);
-    uint32_t* pv1 = reinterpret_cast<uint32_t*>(&v1);
+    for (int i = 0; i < PER_T; ++i) {
+      const int c = threadIdx.x + i * 128;
+      const int key = c / CPK, piece = c - key * CPK;
+      const uint16_t* h = reinterpret_cast<const uint16_t*>(&codes[i]);
+      uint4 x0, x1;
+      uint32_t* p0 = reinterpret_cast<uint32_t*>(&x0);
+      uint32_t* p1 = reinterpret_cast<uint32_t*>(&x1);
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      pk0[e] = e4m3x2_to_bf16x2(hk[e]);
-      pk1[e] = e4m3x2_to_bf16x2(hk[4 + e]);
-      pv0[e] = e4m3x2_to_bf16x2(hv[e]);
-      pv1[e] = e4m3x2_to_bf16x2(hv[4 + e]);
+      for (int e = 0; e < 4; ++e) {
+        p0[e] = e4m3x2_to_bf16x2(h[e]);
+        p1[e] = e4m3x2_to_bf16x2(h[4 + e]);
+      }
+      const int d = piece * 16;
+      *reinterpret_cast<uint4*>(sT + sw_addr<BK>(0u, key, d)) = x0;
+      *reinterpret_cast<uint4*>(sT + sw_addr<BK>(0u, key, d + 8)) = x1;
     }
-    const int d = piece * 16;
-    const uint32_t o0 = sw_addr<BK>(0u, key, d), o1 = sw_addr<BK>(0u, key, d + 8);
-    *reinterpret_cast<uint4*>(sK + o0) = k0;
-    *reinterpret_cast<uint4*>(sK + o1) = k1;
-    *reinterpret_cast<uint4*>(sV + o0) = v0;
-    *reinterpret_cast<uint4*>(sV + o1) = v1;
-  }
+  };
+  widen(kcs);
   static_assert(BK <= 128, "one key scale per thread");
   if (threadIdx.x < BK) {
     ksc[threadIdx.x] = ks_reg;
@@ -881,7 +889,7 @@ __global__ void __launch_bounds__(128) dec8_attend_kernel(const DecParams p, con
 #pragma unroll
   for (int n = 0; n < NT; ++n) sacc[n][0] = sacc[n][1] = sacc[n][2] = sacc[n][3] = 0.f;
   {
-    const uint32_t kb = smem_u32(sK);
+    const uint32_t kb = smem_u32(sT);
 #pragma unroll
     for (int ks = 0; ks < D_H / 16; ++ks) {
 #pragma unroll
@@ -938,11 +946,14 @@ __global__ void __launch_bounds__(128) dec8_attend_kernel(const DecParams p, con
     l_lo += __shfl_xor_sync(0xFFFFFFFFu, l_lo, o);
     l_hi += __shfl_xor_sync(0xFFFFFFFFu, l_hi, o);
   }
+  __syncthreads();  // every warp has read K
+  widen(vcs);
+  __syncthreads();
   float oacc[DT][4];
 #pragma unroll
   for (int n = 0; n < DT; ++n) oacc[n][0] = oacc[n][1] = oacc[n][2] = oacc[n][3] = 0.f;
   {
-    const uint32_t vb = smem_u32(sV);
+    const uint32_t vb = smem_u32(sT);
 #pragma unroll
     for (int ks = 0; ks < NT / 2; ++ks) {
 #pragma unroll
@@ -1020,8 +1031,7 @@ int scan8_split(int S) {
 
 template <int D_H, int BK>
 size_t attend8_smem() {
-  static_assert(4 * 16 * D_H * 4 <= 2 * BK * D_H * 2, "warp-merge buffer must fit over K/V");
-  return 1024 + 2 * BK * D_H * 2 + 128 * 4 + 2 * BK * 4;
+  return 1024 + Attend8Smem<D_H, BK>::REGION + 128 * 4 + 2 * BK * 4;
 }
 
 // Per-row E4M3 quantization of bf16 rows (for filling a cache): one warp per row.
