@@ -228,21 +228,20 @@ __global__ void __launch_bounds__(256) dec_topk_kernel(const DecParams p) {
     if (lane == 0) win[warp * hs1 + round] = best;
   }
   __syncthreads();
-  if (warp != 0) return;
-  // rank the 8 warps' winners: a key is kept if fewer than HS keys beat it
+  // rank the 8 warps' winners, one thread per winner: a key is kept if fewer
+  // than HS keys beat it (keys are distinct: each carries its block)
   const int T = 8 * HS;
-  int nkept = 0;
-  for (int base = 0; base < T; base += 32) {
-    const int j = base + lane;
-    const uint64_t mine = j < T ? win[j] : 0ull;
+  bool keep = false;
+  if (static_cast<int>(threadIdx.x) < T) {
+    const uint64_t mine = win[threadIdx.x];
     int rank = 0;
     if (mine != 0ull)
       for (int m = 0; m < T; ++m) rank += win[m] > mine ? 1 : 0;
-    const bool keep = mine != 0ull && rank < HS;
+    keep = mine != 0ull && rank < HS;
     if (keep) chosen[rank] = static_cast<int32_t>(0xFFFFFFFFu - static_cast<uint32_t>(mine));
-    nkept += __popc(__ballot_sync(0xFFFFFFFFu, keep));
   }
-  __syncwarp();
+  const int nkept = __syncthreads_count(keep);
+  if (warp != 0) return;
   if (lane == 0) chosen[nkept] = b_i;  // the local block (Eq. 7: always kept)
   __syncwarp();
   const int nsel = nkept + 1;

@@ -104,6 +104,8 @@ def _run(msa, cfg, st, steps, seqs, q_idx_pow2=None):
     (1279, 128, 128, 64, 8),   # the second step starts a new page
     (700, 64, 64, 128, 5),     # B_k = 64, d_h = 64, d_idx = 128
     (300, 128, 128, 64, 16),   # fewer visible blocks than k
+    (900, 64, 128, 64, 8),     # B_k = 64 with d_h = 128
+    (900, 128, 64, 64, 8),     # B_k = 128 with d_h = 64
 ])
 def test_paged_fp8_decode_small(msa, L0, B_k, d_h, d_idx, k):
     cfg = inputs.DecodeConfig("fp8", S=5, L0=L0, steps=3, H_q=32, H_kv=4, d_h=d_h, d_idx=d_idx,
