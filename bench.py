@@ -51,9 +51,6 @@ NCU_TRAFFIC = {
     "attn_phase1": ("sparse_attn.cu", "attn_phase1_kernel",
                     "f1b0fc93e3f2bf85ed14c4b8f528f468a9d3856cb1a9f7aeea45eaeb627e8f25",
                     (3576701184 + 4184357120) / 32768, "query"),
-    "attn_merge": ("sparse_attn.cu", "attn_merge_kernel",
-                   "b3995bc06ce2e51f1d1aca2b258c6c448bf62dd831be86d2dab58401aca75b38",
-                   (4243319552 + 265582848) / 32768, "query"),
 }
 
 

@@ -607,13 +607,18 @@ __global__ void __launch_bounds__(256, 2) attn_merge_kernel(const MergeParams p)
   const int64_t slot0 = (il * p.H_kv + r) * p.kk;
   int32_t myb = -1;
   if (lane < p.kk) myb = p.idx[(i * p.H_kv + r) * p.kk + lane];
-  const unsigned use = __ballot_sync(0xFFFFFFFFu, lane < p.kk && myb >= 0 && myb <= b_i);
-  // this lane's head: the largest LSE of its used slots (read again below,
-  // from L1, rather than held in registers)
+  // this lane's head: the largest LSE of its used slots.  All of the row's
+  // LSEs are loaded together with the selection (a slot that turns out
+  // unused is never read into the arithmetic), then kept in registers only
+  // for the maximum; the weights read them again below, from L1.
   const float* lse_h = p.c.part_lse + slot0 * p.G + g;
+  float lv[32];
+#pragma unroll
+  for (int s = 0; s < 32; ++s) lv[s] = s < p.kk ? lse_h[s * p.G] : -INFINITY;
+  const unsigned use = __ballot_sync(0xFFFFFFFFu, lane < p.kk && myb >= 0 && myb <= b_i);
   float m = -INFINITY;
-  for (int s = 0; s < p.kk; ++s)
-    if ((use >> s) & 1u) m = fmaxf(m, lse_h[s * p.G]);
+#pragma unroll
+  for (int s = 0; s < 32; ++s) m = ((use >> s) & 1u) ? fmaxf(m, lv[s]) : m;
   float acc[E];
 #pragma unroll
   for (int e = 0; e < E; ++e) acc[e] = 0.0f;
