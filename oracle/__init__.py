@@ -29,17 +29,24 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "msa_oracle.c")
 _HDR = os.path.join(_HERE, "msa_oracle.h")
-_LIB = os.path.join(_HERE, "liboracle.so")
+# MSA_ORACLE_SANITIZE=1 selects a copy built with AddressSanitizer and
+# UndefinedBehaviorSanitizer (the process must preload libasan and libubsan),
+# to check the oracle's own memory accesses and arithmetic.
+_SANITIZE = os.environ.get("MSA_ORACLE_SANITIZE") == "1"
+_LIB = os.path.join(_HERE, "liboracle_san.so" if _SANITIZE else "liboracle.so")
 _lock = threading.Lock()
 _lib = None
 
 
 def build(force: bool = False) -> str:
-    """Compile msa_oracle.c into liboracle.so (gcc, -O2, no fast-math)."""
+    """Compile msa_oracle.c into liboracle.so (gcc, -O2, no fast-math), or the
+    sanitized copy (-O1 with -fsanitize=address,undefined) when selected."""
     newest = max(os.path.getmtime(_SRC), os.path.getmtime(_HDR))
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < newest:
         tmp = _LIB + f".{os.getpid()}.tmp"
-        cmd = ["gcc", "-std=c11", "-O2", "-fno-fast-math", "-ffp-contract=off", "-fopenmp",
+        opt = (["-O1", "-g", "-fsanitize=address,undefined", "-fno-omit-frame-pointer"]
+               if _SANITIZE else ["-O2"])
+        cmd = ["gcc", "-std=c11", *opt, "-fno-fast-math", "-ffp-contract=off", "-fopenmp",
                "-fPIC", "-shared", "-Wall", "-Wextra", "-o", tmp, _SRC, "-lm"]
         subprocess.run(cmd, check=True)
         os.replace(tmp, _LIB)
